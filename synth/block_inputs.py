@@ -1,0 +1,117 @@
+"""Seeded draws of the block's weights and activations.
+
+Distributions (the workload description): activations, text tokens, latents
+and the timestep embedding ~ N(0, 1); linear weights ~ N(0, 1/fan_in); the
+AdaLN projections ~ N(0, 0.02^2); biases 0; QK-norm weights 1.  ``stress=True``
+draws non-trivial biases (N(0, 0.1^2)) and QK-norm weights (1 + N(0, 0.2^2))
+so that a dropped bias or norm weight shows up in parity.
+
+FP8 weights use the release format: E4M3 ("fn", max 448) codes with a
+per-output-channel fp32 scale s[n] = max_k |W[n, k]| / 448, codes rounded to
+nearest even from W / s.  Everything is returned as CPU torch tensors.
+"""
+
+from __future__ import annotations
+
+import zlib
+
+import numpy as np
+import torch
+
+from .configs import Config
+
+E4M3_MAX = 448.0
+
+
+def tensor_rng(seed: int, block: int, name: str) -> np.random.Generator:
+    """One independent numpy stream per (seed, block, tensor name)."""
+    return np.random.default_rng([int(seed), int(block), zlib.crc32(name.encode())])
+
+
+def _normal(seed, block, name, shape, std=1.0) -> np.ndarray:
+    a = tensor_rng(seed, block, name).standard_normal(size=shape, dtype=np.float32)
+    if std != 1.0:
+        a *= np.float32(std)
+    return a
+
+
+def quantize_e4m3_per_channel(w: np.ndarray):
+    """fp32 [N, K] -> (E4M3 codes as torch.float8_e4m3fn [N, K], fp32 scale [N])."""
+    w = torch.from_numpy(np.ascontiguousarray(w, dtype=np.float32))
+    amax = w.abs().amax(dim=1)
+    scale = torch.where(amax > 0, amax / E4M3_MAX, torch.ones_like(amax))
+    q = (w / scale[:, None]).clamp_(-E4M3_MAX, E4M3_MAX).to(torch.float8_e4m3fn)
+    return q, scale.to(torch.float32)
+
+
+def _linear(seed, block, name, n_out, n_in, w_dtype, std=None):
+    """Weight [n_out, n_in] (+ scale for E4M3, else None)."""
+    std = (1.0 / np.sqrt(n_in)) if std is None else std
+    w = _normal(seed, block, name, (n_out, n_in), std)
+    if w_dtype == "bf16":
+        return torch.from_numpy(w).to(torch.bfloat16), None
+    if w_dtype == "e4m3":
+        return quantize_e4m3_per_channel(w)
+    raise ValueError(f"w_dtype {w_dtype!r}")
+
+
+def _bias(seed, block, name, n, stress):
+    if stress:
+        return torch.from_numpy(_normal(seed, block, name, (n,), 0.1))
+    return torch.zeros(n, dtype=torch.float32)
+
+
+def make_block_weights(cfg: Config, seed: int = 0, block: int = 0, stress: bool = False,
+                       zero_adaln: bool = False) -> dict:
+    """Weights of one block: w_* [out, in] (bf16 or E4M3 codes), s_* fp32 scales
+    (E4M3 only, else None), b_ada fp32 [6D], g_q / g_k fp32 [head_dim]."""
+    D, I, A, dh = cfg.D, cfg.I, cfg.adaln_dim, cfg.head_dim
+    wd = cfg.w_dtype
+    out = {}
+    out["w_ada"], out["s_ada"] = _linear(seed, block, "w_ada", 6 * D, A, wd, std=0.02)
+    if zero_adaln:
+        out["w_ada"] = torch.zeros_like(out["w_ada"])
+    out["b_ada"] = torch.zeros(6 * D) if zero_adaln else _bias(seed, block, "b_ada", 6 * D, stress)
+    out["w_qkv"], out["s_qkv"] = _linear(seed, block, "w_qkv", 3 * D, D, wd)
+    out["w_o"], out["s_o"] = _linear(seed, block, "w_o", D, D, wd)
+    out["w_gate"], out["s_gate"] = _linear(seed, block, "w_gate", I, D, wd)
+    out["w_up"], out["s_up"] = _linear(seed, block, "w_up", I, D, wd)
+    out["w_down"], out["s_down"] = _linear(seed, block, "w_down", D, I, wd)
+    if stress:
+        out["g_q"] = torch.from_numpy(1.0 + _normal(seed, block, "g_q", (dh,), 0.2))
+        out["g_k"] = torch.from_numpy(1.0 + _normal(seed, block, "g_k", (dh,), 0.2))
+    else:
+        out["g_q"] = torch.ones(dh, dtype=torch.float32)
+        out["g_k"] = torch.ones(dh, dtype=torch.float32)
+    return out
+
+
+def make_block_activations(cfg: Config, seed: int = 0) -> dict:
+    """x [B, L, D] (fp32 or bf16 per cfg.x_dtype) and temb [B, adaln_dim] fp32."""
+    x = torch.from_numpy(_normal(seed, 0, "x", (cfg.B, cfg.L, cfg.D)))
+    if cfg.x_dtype == "bf16":
+        x = x.to(torch.bfloat16)
+    elif cfg.x_dtype != "f32":
+        raise ValueError(f"x_dtype {cfg.x_dtype!r}")
+    temb = torch.from_numpy(_normal(seed, 0, "temb", (cfg.B, cfg.adaln_dim)))
+    return {"x": x, "temb": temb}
+
+
+def make_stack_inputs(cfg: Config, seed: int = 0, stress: bool = False) -> dict:
+    """Stack-level inputs: latents [B, N, C] and text [B, T, D] (x_dtype), temb fp32,
+    in-proj w_in [D, C] / b_in, final AdaLN w_f [2D, A] / b_f, out-proj w_out [C, D] /
+    b_out (weights in cfg.w_dtype with scales for E4M3).  Block weights come from
+    make_block_weights(cfg, seed, block=i)."""
+    D, A, C = cfg.D, cfg.adaln_dim, cfg.latent_ch
+    xd = torch.bfloat16 if cfg.x_dtype == "bf16" else torch.float32
+    out = {}
+    out["x_latent"] = torch.from_numpy(_normal(seed, 0, "x_latent", (cfg.B, cfg.n_img, C))).to(xd)
+    out["text"] = torch.from_numpy(_normal(seed, 0, "text", (cfg.B, cfg.T_text, D))).to(xd)
+    out["temb"] = torch.from_numpy(_normal(seed, 0, "temb", (cfg.B, A)))
+    out["w_in"], out["s_in"] = _linear(seed, 0, "w_in", D, C, cfg.w_dtype)
+    out["b_in"] = _bias(seed, 0, "b_in", D, stress)
+    out["w_f"], out["s_f"] = _linear(seed, 0, "w_f", 2 * D, A, cfg.w_dtype, std=0.02)
+    out["b_f"] = _bias(seed, 0, "b_f", 2 * D, stress)
+    out["w_out"], out["s_out"] = _linear(seed, 0, "w_out", C, D, cfg.w_dtype)
+    out["b_out"] = _bias(seed, 0, "b_out", C, stress)
+    return out
