@@ -1,0 +1,459 @@
+#!/usr/bin/env python
+"""Benchmark of the Ideogram 4 DiT block forward on B200 (sm_100a).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1024px] [--impl ours|reference]
+
+One step = one full Ideogram4TransformerBlock forward (AdaLN, norm, QKV +
+QK-norm + MRoPE, joint attention, gated out-projection, norm, SwiGLU, gated
+down-projection) over one batch of synthetic inputs, weights resident in HBM.
+Prints one JSON line (rank 0).  For N > 1 (torchrun) every rank runs an
+independent replica on its own GPU (the block has no data-path exchange);
+time is the max over ranks, value the whole-job TFLOP/s.
+
+--impl reference times the fp64 CPU oracle on the host cores instead (the
+slow baseline): each step evaluates the block for a fixed sample of token
+rows of the same workload, which needs k and v of every token.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("DiT block fwd TFLOP/s & ms at 1024px (4608d, 4096+512 tok), % of B200 tensor peak")
+KERNEL_NAMES = ["adaln", "rope_table", "norm1", "qkv_norm_rope", "attention", "out_proj_residual",
+                "norm2", "gate_up_swiglu", "down_residual"]
+KERNEL_NAMES_FP8 = ["adaln", "rope_table", "norm1", "qkv_norm_rope", "attention", "quantize_o",
+                    "out_proj_residual", "norm2", "gate_up_swiglu", "quantize_u", "down_residual"]
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+REFERENCE_ROWS = 32
+KERNEL_SOURCES = ["ig4_api.cu", "ig4_ptx.cuh", "ig4_gemm.cuh", "ig4_attention.cuh", "ig4_small.cuh"]
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--config", default="1024px")
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)),
+            int(os.environ.get("WORLD_SIZE", 1)))
+
+
+def block_work(cfg):
+    """Algorithmic FLOPs of one block call (2 per multiply-add)."""
+    B, L, D, I, A = cfg.B, cfg.L, cfg.D, cfg.I, cfg.adaln_dim
+    M = B * L
+    per_kernel = {
+        "qkv_norm_rope": 2.0 * M * D * 3 * D,
+        "attention": 4.0 * B * L * L * D,
+        "out_proj_residual": 2.0 * M * D * D,
+        "gate_up_swiglu": 2.0 * M * D * 2 * I,
+        "down_residual": 2.0 * M * I * D,
+        "adaln": 12.0 * B * A * D,
+    }
+    return sum(per_kernel.values()), per_kernel
+
+
+def kernel_bytes(cfg, name):
+    """Algorithmic HBM bytes of the memory-bound kernels (one launch)."""
+    M, D, L = cfg.M, cfg.D, cfg.L
+    xs = 4 if cfg.x_dtype == "f32" else 2
+    ws = 1 if cfg.w_dtype == "e4m3" else 2
+    hs = 1 if cfg.w_dtype == "e4m3" else 2
+    if name == "adaln":
+        return 6 * D * cfg.adaln_dim * ws + 6 * D * 4 * (1 + cfg.B)
+    if name in ("norm1", "norm2"):
+        return M * D * (xs + hs)
+    if name == "rope_table":
+        return L * (3 * 4 + 2 * 64 * 4)
+    if name == "quantize_o":
+        return M * D * 3
+    if name == "quantize_u":
+        return M * cfg.I * 3
+    return None
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "stream_diffusion_transformer_fwd_b200", "csrc", name),
+                  "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    ent = rec.get(workload, {}).get(kernel)
+    if not ent or ent.get("source_hash") != kernel_source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples of one GPU while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "20"], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.3)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sms, maxes, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sms.append(float(parts[1]))
+                maxes.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sms:
+            return None
+        loaded = [s for s in sms if s > 0.5 * max(sms)] or sms
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(maxes),
+                "reasons": sorted(reasons), "samples": len(sms)}
+
+
+# ----------------------------------------------------------------- our arm
+
+def run_ours(args, rank, local_rank, world):
+    import torch
+    import torch.distributed as dist
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    from stream_diffusion_transformer_fwd_b200.build import build
+    if rank == 0:
+        build()
+    if world > 1:
+        dist.barrier()
+    import stream_diffusion_transformer_fwd_b200 as ig4
+    from synth import CONFIGS, make_block_activations, make_block_weights
+
+    cfg = CONFIGS[args.config]
+    fp8 = cfg.w_dtype == "e4m3"
+    names = KERNEL_NAMES_FP8 if fp8 else KERNEL_NAMES
+    acts = make_block_activations(cfg, seed=rank)
+    wts = make_block_weights(cfg, seed=rank)
+    wd = {k: (None if v is None else v.to(dev)) for k, v in wts.items()}
+    bw = ig4.block_weights(wd)
+    c = ig4.config_from(cfg)
+    x = acts["x"].to(dev)
+    temb = acts["temb"].to(dev)
+    pos = ig4.ig4_mrope_positions(cfg.T_text, cfg.grid_t, cfg.grid_h, cfg.grid_w, device=dev)
+    y = torch.empty_like(x)
+    ws = torch.empty(ig4.ig4_workspace_size(c), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    n_ev = ig4.IG4_BLOCK_TRACE_EVENTS
+    K, W = args.steps, args.warmup
+
+    for _ in range(W):
+        ig4.ig4_block_forward(c, bw, x, y, pos, temb, ws)
+    torch.cuda.synchronize()
+    assert ig4.ig4_last_device_error() == ig4.IG4_OK
+
+    # ---- device-timed region: K traced block calls (events between kernels)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(K)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(K):
+        ig4.ig4_block_forward(c, bw, x, y, pos, temb, ws, events=evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    err = ig4.ig4_last_device_error()
+    ms_total = start.elapsed_time(end)
+    n_launch = len(names)
+    per_kernel_ms = [0.0] * n_launch
+    for i in range(K):
+        for j in range(n_launch):
+            per_kernel_ms[j] += evs[i][j].elapsed_time(evs[i][j + 1])
+    per_kernel_ms = [t / K for t in per_kernel_ms]
+
+    # ---- end-to-end region: pinned host buffers, H2D inputs and D2H result each step
+    x_h = acts["x"].pin_memory()
+    temb_h = acts["temb"].pin_memory()
+    pos_h = ig4.ig4_mrope_positions(cfg.T_text, cfg.grid_t, cfg.grid_h, cfg.grid_w).pin_memory()
+    y_h = torch.empty_like(x_h).pin_memory()
+    x_d, temb_d, pos_d = torch.empty_like(x), torch.empty_like(temb), torch.empty_like(pos)
+    for _ in range(max(1, W // 2)):
+        x_d.copy_(x_h, non_blocking=True)
+        ig4.ig4_block_forward(c, bw, x_d, y, pos_d.copy_(pos_h, non_blocking=True),
+                              temb_d.copy_(temb_h, non_blocking=True), ws)
+        y_h.copy_(y, non_blocking=True)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(K):
+        x_d.copy_(x_h, non_blocking=True)
+        temb_d.copy_(temb_h, non_blocking=True)
+        pos_d.copy_(pos_h, non_blocking=True)
+        ig4.ig4_block_forward(c, bw, x_d, y, pos_d, temb_d, ws)
+        y_h.copy_(y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = e0.elapsed_time(e1)
+    h2d = x_h.numel() * x_h.element_size() + temb_h.numel() * 4 + pos_h.numel() * 4
+    d2h = y_h.numel() * y_h.element_size()
+
+    if world > 1:
+        t = torch.tensor([ms_total, ms_e2e], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total, ms_e2e = t.tolist()
+
+    flops, per_kernel_flops = block_work(cfg)
+    ms_step = ms_total / K
+    value = world * flops * K / (ms_total * 1e-3) / 1e12
+    e2e_value = world * flops * K / (ms_e2e * 1e-3) / 1e12
+
+    # dominant kernel and its roofline
+    peaks, peak_src = load_peaks()
+    dom = max(range(n_launch), key=lambda j: per_kernel_ms[j])
+    dom_name = names[dom]
+    dom_ms = per_kernel_ms[dom]
+    if dom_name in per_kernel_flops and dom_name != "adaln":
+        achieved = per_kernel_flops[dom_name] / (dom_ms * 1e-3) / 1e12
+        if fp8 and dom_name != "attention":
+            peak = 2.0 * peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+            peak_note = f"2 x bf16 sustained ({peak_src}): nominal fp8/bf16 ratio"
+        else:
+            peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+            peak_note = f"bf16 sustained ({peak_src})"
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "traffic": recorded_traffic(dom_name, cfg.name), "kernel": dom_name,
+                "peak_source": peak_note}
+    else:
+        b = kernel_bytes(cfg, dom_name)
+        achieved = b / (dom_ms * 1e-3) / 1e9
+        peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": recorded_traffic(dom_name, cfg.name),
+                "kernel": dom_name, "peak_source": f"hbm copy ({peak_src})"}
+
+    cpu_base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu_base = cpu_baseline(cfg, acts, wts)
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    breakdown = {names[j]: round(per_kernel_ms[j], 4) for j in range(n_launch)}
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "fp8-e4m3 weights, bf16 activations" if fp8 else "bf16",
+        "data": "synthetic (seeded N(0,1) activations, N(0,1/fan_in) weights, random init)",
+        "config": {
+            "workload": (f"{cfg.name} Ideogram4 block: B={cfg.B}, {cfg.T_text} text + "
+                         f"{cfg.grid_h}x{cfg.grid_w} image = {cfg.L} tokens, D={cfg.D}, "
+                         f"{cfg.H}x{cfg.head_dim} heads, I={cfg.I}, w={cfg.w_dtype}, "
+                         f"x={cfg.x_dtype}"),
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "inputs larger than L2 (block weights alone are "
+                  f"{(8 * cfg.D * cfg.D + 6 * cfg.D * cfg.I) * (1 if fp8 else 2) / 1e6:.0f} MB per step)",
+            "gflop_per_step": round(flops / 1e9, 1),
+        },
+        "pct_of_peak": round(100.0 * value / world / peaks.get(
+            "bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]), 2),
+        "pct_of_peak_basis": f"bf16 sustained cuBLAS ({peak_src})",
+        "roofline": roof,
+        "kernel_ms": breakdown,
+        "clocks": clocks,
+        "device_error": ig4.ig4_status_string(err),
+        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e / K, 4)},
+        "gpu_launches": n_launch * K,
+        "cpu_baseline": cpu_base,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _cores():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        for ent in info:
+            if ent.get("user_api") == "blas":
+                return int(ent.get("num_threads"))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def cpu_baseline(cfg, acts, wts):
+    """The oracle, as it stands, on the host cores: one full block forward of the
+    same workload (the whole step)."""
+    import oracle as O
+    from oracle.inputs import block_weights_f64, to_f64
+
+    W = block_weights_f64(wts)
+    x = to_f64(acts["x"])
+    temb = to_f64(acts["temb"])
+    pos = O.mrope_positions(cfg.T_text, cfg.grid_t, cfg.grid_h, cfg.grid_w)
+    t0 = time.perf_counter()
+    O.block_forward(x, temb, pos, W, cfg.H, cfg.rope_theta, cfg.sections, cfg.eps)
+    dt = time.perf_counter() - t0
+    flops, _ = block_work(cfg)
+    return {"value": round(flops / dt / 1e12, 4), "unit": "TFLOP/s", "cores": _cores(),
+            "kind": "oracle", "sample": f"one full block forward of the {cfg.name} workload "
+            f"({flops / 1e9:.0f} GFLOP), fp64 numpy, {dt:.1f} s"}
+
+
+# ----------------------------------------------------------- reference arm
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    import numpy as np
+
+    import oracle as O
+    from oracle.inputs import block_weights_f64, to_f64
+    from synth import CONFIGS, make_block_activations, make_block_weights
+
+    cfg = CONFIGS[args.config]
+    acts = make_block_activations(cfg, seed=0)
+    W = block_weights_f64(make_block_weights(cfg, seed=0))
+    x = to_f64(acts["x"])
+    temb = to_f64(acts["temb"])
+    pos = O.mrope_positions(cfg.T_text, cfg.grid_t, cfg.grid_h, cfg.grid_w)
+    rng = np.random.default_rng(0)
+    S = min(REFERENCE_ROWS, cfg.L)
+    D, I, L, A = cfg.D, cfg.I, cfg.L, cfg.adaln_dim
+    # work of one sample: k, v of all L tokens of the sample, then q, attention,
+    # out-projection and MLP for the S rows, plus the AdaLN projection
+    sample_flops = (2.0 * 2 * L * D * D + 2.0 * S * D * D + 4.0 * S * L * D + 2.0 * S * D * D +
+                    6.0 * S * D * I + 12.0 * A * D)
+    times = []
+    for i in range(args.warmup + args.steps):
+        rows = rng.choice(L, size=S, replace=False)  # rows of sample 0
+        t0 = time.perf_counter()
+        O.block_forward_rows(x, temb, pos, W, cfg.H, rows, cfg.rope_theta, cfg.sections, cfg.eps)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = sample_flops * len(times) / total / 1e12
+    flops, _ = block_work(cfg)
+    cores = _cores()
+    line = {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 4),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(1e3 * total / len(times), 2),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded, same generator as the GPU arm)",
+        "config": {"workload": f"{cfg.name} Ideogram4 block (fp64 CPU oracle, sampled rows)",
+                   "gflop_per_step": round(sample_flops / 1e9, 1),
+                   "full_block_gflop": round(flops / 1e9, 1)},
+        "cpu_baseline": {"value": round(value, 4), "unit": "TFLOP/s", "cores": cores,
+                         "kind": "oracle",
+                         "sample": f"{S} token rows per step (k, v of all {L} tokens), "
+                                   f"{sample_flops / 1e9:.0f} GFLOP per step"},
+        "e2e": {"value": round(value, 4), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    rank, local_rank, world = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    return run_ours(args, rank, local_rank, world)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,265 @@
+/*
+ * ig4.h - C ABI of a B200 (sm_100a) implementation of the Ideogram 4
+ * single-stream DiT block forward and of the 34-block stack.
+ *
+ * The operation is the one described on the Ideogram 4.0 survey page
+ * ("Ideogram 4.0", section "模型架构", subsections "单 block 内部",
+ * "Model spec" and "条件注入方式"):  one sequence [text tokens | image latent
+ * tokens] of width emb_dim (4608) flows through Ideogram4TransformerBlock
+ * layers, each an AdaLN-modulated self-attention with QK-RMSNorm and 3D
+ * multimodal RoPE (mrope_section (24, 20, 20), rope_theta 5e6; text tokens use
+ * a 1D position broadcast to the 3 axes, image tokens use (t, h, w)), followed
+ * by an AdaLN-modulated SwiGLU MLP (intermediate 12288), both with gated
+ * residuals driven by a 512-d timestep embedding (adaln_dim 512).  The weights
+ * are released in FP8 E4M3 (SimpleTuner quickstart page, "硬件和精度").
+ *
+ * Conventions fixed where the pages are silent (they match the CPU oracle):
+ *   AdaLN: mod = SiLU(temb) W_ada^T + b_ada, chunks of D in the order
+ *     shift_msa, scale_msa, gate_msa, shift_mlp, scale_mlp, gate_mlp;
+ *   pre-norm: RMSNorm over D (weightless, eps), then (1 + scale) and + shift;
+ *   QK-RMSNorm: per head over head_dim with weights g_q, g_k [head_dim];
+ *   rotary: the 64 frequency pairs act on dims [0,128) of each head, pair j
+ *     joining dims j and j+64; pairs [0,24) follow t, [24,44) h, [44,64) w;
+ *     inv_freq[j] = theta^(-2j/128);
+ *   positions: text token l -> (l, l, l); image token (t, i, j) of a
+ *     row-major grid -> (T+t, T+i, T+j) after T text tokens;
+ *   attention: softmax(q k^T / sqrt(head_dim)) v, no mask;
+ *   SwiGLU: u = silu(h W_gate^T) * (h W_up^T);  no biases on the block linears.
+ *
+ * Memory: every pointer argument documented as "device" must be device
+ * memory of the current device; the caller owns every buffer.  The library
+ * never allocates, frees, or synchronises a stream, except
+ * ig4_last_device_error, which synchronises the stream it is given.
+ * Linear weights are row-major [out, in] (K contiguous).  All calls are
+ * asynchronous on the given cudaStream_t (passed as void*, NULL = legacy
+ * default stream); argument errors are returned synchronously and nothing is
+ * launched.  A device-side wait that runs past its limit (about 2 s) sets a
+ * device error word that ig4_last_device_error reports as IG4_ERR_TIMEOUT.
+ * Calls that share a workspace or output buffer must be ordered by the caller.
+ */
+#ifndef IG4_H
+#define IG4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum ig4_status {
+  IG4_OK = 0,
+  IG4_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned pointer */
+  IG4_ERR_UNSUPPORTED = 2,  /* a shape or dtype outside what the kernels support */
+  IG4_ERR_WORKSPACE = 3,    /* workspace too small or misaligned */
+  IG4_ERR_CUDA = 4,         /* a CUDA runtime / driver call failed */
+  IG4_ERR_TIMEOUT = 5       /* a device-side wait ran past its limit */
+} ig4_status;
+
+typedef enum ig4_dtype {
+  IG4_F32 = 0,
+  IG4_BF16 = 1,
+  IG4_E4M3 = 2   /* FP8 E4M3 "fn" (max 448), with an fp32 scale array */
+} ig4_dtype;
+
+/* Shape and precision of one block call.  L = T_text + grid_t*grid_h*grid_w.
+ * Supported: head_dim == 256, D == H*256, D % 256 == 0, I % 128 == 0,
+ * adaln_dim % 8 == 0 and <= 1024, B*L >= 1, x_dtype F32 or BF16,
+ * w_dtype BF16 or E4M3. */
+typedef struct ig4_config {
+  int B, T_text, grid_t, grid_h, grid_w;
+  int D, H, head_dim, I, adaln_dim;
+  double rope_theta;   /* 5e6 */
+  int sections[3];     /* (24, 20, 20): must sum to 64 */
+  float eps;           /* RMSNorm epsilon, 1e-6 */
+  int x_dtype;         /* residual stream storage: IG4_F32 or IG4_BF16 */
+  int w_dtype;         /* linear weights: IG4_BF16, or IG4_E4M3 with s_* scales */
+} ig4_config;
+
+/* One block's weights (device pointers).  w_* are [out, in] row-major in
+ * w_dtype: w_ada [6D, adaln_dim], w_qkv [3D, D] (rows: q | k | v, head-major,
+ * column n = head*256 + d), w_o [D, D], w_gate [I, D], w_up [I, D],
+ * w_down [D, I].  s_* are fp32 per-output-channel scales [out] (E4M3 only,
+ * else ignored).  b_ada fp32 [6D], g_q / g_k fp32 [head_dim]. */
+typedef struct ig4_block_weights {
+  const void *w_ada, *w_qkv, *w_o, *w_gate, *w_up, *w_down;
+  const float *s_ada, *s_qkv, *s_o, *s_gate, *s_up, *s_down;
+  const float *b_ada, *g_q, *g_k;
+} ig4_block_weights;
+
+/* Stack weights: a host array of n_blocks block weight structs, the latent
+ * in-projection w_in [D, C] + b_in [D], the final AdaLN w_f [2D, adaln_dim] +
+ * b_f [2D] (chunks shift, scale), the out-projection w_out [C, D] + b_out [C].
+ * Weights in cfg->w_dtype, s_* scales for E4M3.  C = latent_ch (128). */
+typedef struct ig4_stack_weights {
+  int n_blocks;
+  int latent_ch;
+  const ig4_block_weights *blocks;   /* HOST array of n_blocks entries */
+  const void *w_in;  const float *s_in;  const float *b_in;
+  const void *w_f;   const float *s_f;   const float *b_f;
+  const void *w_out; const float *s_out; const float *b_out;
+} ig4_stack_weights;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *ig4_status_string(int status);
+
+/* ABI revision of this header (increases on any incompatible change). */
+int ig4_abi_version(void);
+
+/* ---------------------------------------------------------------- a-11 ---
+ * MRoPE position table (survey page, "单 block 内部": text tokens use a 1D
+ * position broadcast to the 3 axes, image tokens use (t, h, w); "条件注入方式":
+ * text precedes the image).  Writes int32 pos[3][L] (rows t, h, w), with
+ * text token l at (l, l, l) and image token (t, i, j), row-major over the
+ * grid, at (T+t, T+i, T+j).  out_on_device = 0: pos_out is host memory and the
+ * table is written by host code before the call returns (stream unused);
+ * 1: pos_out is device memory, written by a kernel launched on `stream`.
+ * Errors: INVALID_ARG for negative sizes, L == 0, L > 2^24, or NULL pos_out. */
+ig4_status ig4_mrope_positions(int T_text, int grid_t, int grid_h, int grid_w,
+                               int32_t *pos_out, int out_on_device, void *stream);
+
+/* ----------------------------------------------------------------- a-5 ---
+ * Rotary tables for a position table: cos_out[l][j] = cos(pos[axis(j)][l] *
+ * theta^(-2j/128)), sin_out likewise, fp32 [L][64], angles evaluated in fp64.
+ * axis(j) follows `sections` (contiguous chunks t, h, w).  pos: device int32
+ * [3][L]; outputs device.  Errors: INVALID_ARG (NULL, L < 1, sections not
+ * summing to 64, theta <= 0). */
+ig4_status ig4_rope_table(int L, const int32_t *pos, double rope_theta, const int sections[3],
+                          float *cos_out, float *sin_out, void *stream);
+
+/* ----------------------------------------------------------------- a-1 ---
+ * AdaLN modulation (survey page, "单 block 内部": AdaLN from the timestep
+ * embedding gives the per-block modulation): mod[b][n] = sum_k SiLU(temb[b][k])
+ * * W[n][k] (* w_scale[n] for E4M3) + bias[n], fp32 out [B][N].  temb fp32
+ * [B][A]; W [N][A] in w_dtype (BF16 or E4M3); bias fp32 [N] or NULL.
+ * Errors: INVALID_ARG (NULL, B < 1, B > 8, A % 8, A > 1024, N < 1). */
+ig4_status ig4_adaln_modulation(int B, int A, int N, const float *temb, const void *w,
+                                int w_dtype, const float *w_scale, const float *bias,
+                                float *mod_out, void *stream);
+
+/* ----------------------------------------------------------------- a-2 ---
+ * Pre-norm + modulate: h[r] = x[r] * rsqrt(mean(x[r]^2) + eps) * (1 + scale[b])
+ * + shift[b] for each token row r of sample b = r / L.  x [B*L][D] in x_dtype
+ * (F32 or BF16); shift / scale fp32 with sample stride mod_stride (pointers into
+ * an AdaLN output, e.g. mod + 0*D and mod + 1*D with stride 6D).  Output h in
+ * h_dtype: BF16, or E4M3 with a per-row fp32 scale written to h_scale_out
+ * (h = code * scale, scale = max|h| / 448).  D % 8 == 0, D <= 8192. */
+ig4_status ig4_norm_modulate(int B, int L, int D, const void *x, int x_dtype,
+                             const float *shift, const float *scale, int mod_stride, float eps,
+                             void *h_out, int h_dtype, float *h_scale_out, void *stream);
+
+/* ------------------------------------------------------- a-3, a-4, a-5 ---
+ * Fused QKV projection with per-head QK-RMSNorm and MRoPE (survey page,
+ * "单 block 内部": self-attention with QK-RMSNorm and 3D MRoPE).
+ * qkv = h W_qkv^T; q and k are RMS-normalised per (token, head) with g_q / g_k
+ * and rotated with the tables of ig4_rope_table; v passes through.
+ * h [B*L][D] in h_dtype (BF16; or E4M3 with per-row scale h_scale when
+ * w_dtype is E4M3).  Outputs (bf16, device): q_out, k_out [B][H][L][256],
+ * vt_out [B][H][256][vt_ld] (v transposed, keys contiguous), vt_ld >= L and
+ * vt_ld % 8 == 0.  Errors: UNSUPPORTED unless head_dim == 256 and D == 256*H. */
+ig4_status ig4_qkv_project(int B, int L, int D, int H, const void *h, int h_dtype,
+                           const float *h_scale, const void *w_qkv, int w_dtype,
+                           const float *w_scale, const float *g_q, const float *g_k, float eps,
+                           const float *rope_cos, const float *rope_sin, void *q_out,
+                           void *k_out, void *vt_out, int vt_ld, void *stream);
+
+/* ----------------------------------------------------------------- a-6 ---
+ * Joint bidirectional attention over [text | image] (survey page: one
+ * self-attention over the single sequence, no separate branches):
+ * o[b, l, h*256 + d] = sum_m softmax_m(q[b,h,l] . k[b,h,m] / 16) v[b,h,m,d].
+ * q, k bf16 [B][H][L][256]; vt bf16 [B][H][256][vt_ld]; o_out bf16 [B*L][H*256].
+ * Errors: INVALID_ARG (NULL, L < 1, vt_ld < L or vt_ld % 8). */
+ig4_status ig4_joint_attention(int B, int H, int L, const void *q, const void *k,
+                               const void *vt, int vt_ld, void *o_out, void *stream);
+
+/* ----------------------------------------------------------- a-7, a-9 ---
+ * Gated residual linear (survey page, "单 block 内部": AdaLN gates modulate
+ * the attention and MLP residual paths): x_out[r][n] = x_res[r][n] +
+ * gate[b*gate_stride + n] * sum_k a[r][k] W[n][k] (scaled by a_scale[r] *
+ * w_scale[n] in E4M3), b = r / L.  a [B*L][K] in a_dtype (BF16, or E4M3 +
+ * a_scale when w_dtype is E4M3); x_res / x_out [B*L][N] in x_dtype and may be
+ * the same buffer.  N % 256 == 0, K % 64 == 0 (bf16) / % 128 == 0 (E4M3). */
+ig4_status ig4_gated_residual_linear(int B, int L, int N, int K, const void *a, int a_dtype,
+                                     const float *a_scale, const void *w, int w_dtype,
+                                     const float *w_scale, const float *gate, int gate_stride,
+                                     const void *x_res, void *x_out, int x_dtype, void *stream);
+
+/* ----------------------------------------------------------------- a-8 ---
+ * SwiGLU hidden state (survey page, "单 block 内部": SwiGLU MLP with a SiLU
+ * gate): u[r][i] = silu(sum_k h[r][k] Wg[i][k]) * sum_k h[r][k] Wu[i][k]
+ * (E4M3: each sum times h_scale[r] * s_gate[i] or s_up[i]).  h [M][K];
+ * w_gate, w_up [I][K]; u_out bf16 [M][I].  I % 128 == 0, K % 64 == 0 (bf16) /
+ * % 128 == 0 (E4M3). */
+ig4_status ig4_swiglu(int M, int I, int K, const void *h, int h_dtype, const float *h_scale,
+                      const void *w_gate, const void *w_up, int w_dtype, const float *s_gate,
+                      const float *s_up, void *u_out, void *stream);
+
+/* ---------------------------------------------------------------- a-10 ---
+ * Row quantisation of an activation to FP8 E4M3 for the FP8-weight path:
+ * scale[r] = max_k |x[r][k]| / 448 (1 if the row is zero), q[r][k] =
+ * RNE(x[r][k] / scale[r]) saturated to +-448.  x bf16 [M][K]; q_out E4M3
+ * [M][K]; scale_out fp32 [M].  K % 8 == 0, K <= 16384. */
+ig4_status ig4_quantize_rows(int M, int K, const void *x, void *q_out, float *scale_out,
+                             void *stream);
+
+/* --------------------------------------------------------- whole block ---
+ * Bytes of workspace ig4_block_forward needs for cfg (0 if cfg is invalid). */
+size_t ig4_workspace_size(const ig4_config *cfg);
+
+/* One Ideogram4TransformerBlock forward: x_out = block(x_in).  x_in, x_out
+ * [B][L][D] in cfg->x_dtype (device, must not overlap); pos device int32
+ * [3][L] (see ig4_mrope_positions); temb device fp32 [B][adaln_dim];
+ * workspace device, 256-byte aligned, >= ig4_workspace_size(cfg).
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE (checked before any launch). */
+ig4_status ig4_block_forward(const ig4_config *cfg, const ig4_block_weights *w,
+                             const void *x_in, void *x_out, const int32_t *pos,
+                             const float *temb, void *workspace, size_t ws_bytes, void *stream);
+
+/* ig4_block_forward that also records the caller's CUDA events (cudaEvent_t
+ * handles passed as void*) on `stream` around each kernel: events[0] before
+ * the first launch and events[i+1] after launch i.  n_events must be 0 (no
+ * tracing) or IG4_BLOCK_TRACE_EVENTS.  Launch order: 0 AdaLN, 1 rotary table,
+ * 2 norm1, 3 QKV+norm+rope, 4 attention, 5 out-proj+residual, 6 norm2,
+ * 7 gate/up+SwiGLU, 8 down+residual; the E4M3 path adds 9 quantise(o) and
+ * 10 quantise(u), recorded in launch order (quantise(o) before out-proj). */
+#define IG4_BLOCK_TRACE_EVENTS 12
+ig4_status ig4_block_forward_traced(const ig4_config *cfg, const ig4_block_weights *w,
+                                    const void *x_in, void *x_out, const int32_t *pos,
+                                    const float *temb, void *workspace, size_t ws_bytes,
+                                    void *stream, void *const *events, int n_events);
+
+/* ---------------------------------------------------------------- a-12 ---
+ * Bytes of workspace ig4_stack_forward needs (0 if invalid). */
+size_t ig4_stack_workspace_size(const ig4_config *cfg, int latent_ch);
+
+/* One denoiser step of the stack (survey page: 34 single-stream layers over
+ * [text | image]; 128-channel latent tokens, a 1024 px image = 64 x 64 grid):
+ * s = [text | x_latent W_in^T + b_in]; s = block_i(s) for each block;
+ * out_latent = (RMSNorm(s) (1 + scale_f) + shift_f)[:, T:] W_out^T + b_out,
+ * (shift_f, scale_f) = SiLU(temb) W_f^T + b_f.  x_latent [B][N][C], text
+ * [B][T][D], out_latent [B][N][C], all in cfg->x_dtype (device); N = grid_t *
+ * grid_h * grid_w; pos and temb as for ig4_block_forward. */
+ig4_status ig4_stack_forward(const ig4_config *cfg, const ig4_stack_weights *sw,
+                             const void *x_latent, const void *text, void *out_latent,
+                             const int32_t *pos, const float *temb, void *workspace,
+                             size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------ failure ---
+ * Synchronises `stream`, then reads and clears the device error word that the
+ * kernels set when a bounded wait times out: IG4_ERR_TIMEOUT if set,
+ * IG4_ERR_CUDA if the synchronisation itself failed, else IG4_OK. */
+ig4_status ig4_last_device_error(void *stream);
+
+/* Failure-detection self test: launches a one-CTA kernel that waits on an
+ * mbarrier nothing will ever complete, with a wait limit of wait_us
+ * microseconds (1 .. 5,000,000).  The kernel gives up at the limit, sets the
+ * device error word and returns, so a following ig4_last_device_error()
+ * returns IG4_ERR_TIMEOUT and the context stays usable.  No paper
+ * counterpart: it exercises the timeout path every other kernel relies on. */
+ig4_status ig4_selftest_timeout(int wait_us, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* IG4_H */

@@ -1,0 +1,825 @@
+// ig4_api.cu - C ABI of the Ideogram 4 DiT block library (see include/ig4.h).
+//
+// Host side: argument validation (before anything is launched), TMA
+// descriptor encoding, the workspace layout, and the launch sequence of the
+// block and of the stack on the caller's stream.  The device code lives in
+// the ig4_*.cuh headers.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "ig4.h"
+#include "ig4_attention.cuh"
+#include "ig4_gemm.cuh"
+#include "ig4_small.cuh"
+
+using namespace ig4;
+
+namespace {
+
+constexpr int ABI_VERSION = 1;
+
+// ------------------------------------------------------------------ utils
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
+
+ig4_status last_launch_status() {
+  return cudaGetLastError() == cudaSuccess ? IG4_OK : IG4_ERR_CUDA;
+}
+
+#define IG4_TRY(expr)                       \
+  do {                                      \
+    const ig4_status st_ = (expr);          \
+    if (st_ != IG4_OK) return st_;          \
+  } while (0)
+
+// Per-device facts queried once.
+struct DeviceInfo {
+  int sms = 0;
+};
+constexpr int MAX_DEVICES = 64;
+DeviceInfo g_dev[MAX_DEVICES];
+std::mutex g_dev_mu;
+
+ig4_status device_info(DeviceInfo **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return IG4_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (g_dev[dev].sms == 0) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return IG4_ERR_CUDA;
+    g_dev[dev].sms = sms;
+  }
+  *out = &g_dev[dev];
+  return IG4_OK;
+}
+
+// Raise a kernel's dynamic shared-memory limit (idempotent, cheap).
+template <typename K>
+ig4_status allow_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
+                 cudaSuccess
+             ? IG4_OK
+             : IG4_ERR_CUDA;
+}
+
+// --------------------------------------------------------- tensor maps
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Row-major matrix [rows][cols] of esize-byte elements (row stride ld
+// elements), box [box_rows][box_cols] with box_cols * esize == 128 bytes.
+ig4_status map_2d(CUtensorMap *m, const void *base, int esize, long rows, long cols, long ld,
+                  int box_rows, int box_cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return IG4_ERR_CUDA;
+  const CUtensorMapDataType dt =
+      esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * esize};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? IG4_OK : IG4_ERR_CUDA;
+}
+
+// bf16 tensor [d2][d1][d0] (d0 contiguous, row stride ld0 elements, plane
+// stride ld1 elements), box [1][b1][b0], b0 * 2 == 128 bytes.
+ig4_status map_3d_bf16(CUtensorMap *m, const void *base, long d0, long d1, long d2, long ld0,
+                       long ld1, int b0, int b1) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return IG4_ERR_CUDA;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d0), static_cast<cuuint64_t>(d1),
+                        static_cast<cuuint64_t>(d2)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld0) * 2, static_cast<cuuint64_t>(ld1) * 2};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(b0), static_cast<cuuint32_t>(b1), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? IG4_OK : IG4_ERR_CUDA;
+}
+
+// -------------------------------------------------------------- GEMMs
+
+template <int BN, bool FP8, bool DUAL_B, class Epi>
+ig4_status launch_gemm(const CUtensorMap &A, const CUtensorMap &B, const CUtensorMap &B2, int M,
+                       int n_tiles_n, int K, const Epi &epi, cudaStream_t st) {
+  DeviceInfo *di = nullptr;
+  IG4_TRY(device_info(&di));
+  auto kern = gemm_tc_kernel<BN, FP8, DUAL_B, Epi>;
+  constexpr int SMEM = GemmShape<BN>::SMEM_BYTES;
+  IG4_TRY(allow_smem(kern, SMEM));
+  const long tiles = static_cast<long>((M + GEMM_BM - 1) / GEMM_BM) * n_tiles_n;
+  const int grid = static_cast<int>(std::min<long>(tiles, di->sms));
+  kern<<<grid, GEMM_THREADS, SMEM, st>>>(A, B, B2, M, n_tiles_n, K, epi);
+  return last_launch_status();
+}
+
+// A [M][K] and W [N][K] maps for one GEMM (esize 2 = bf16, 1 = e4m3).
+ig4_status gemm_maps(CUtensorMap *ma, CUtensorMap *mb, const void *a, const void *w, int esize,
+                     long M, long N, long K, int b_rows) {
+  const int bk = 128 / esize;
+  IG4_TRY(map_2d(ma, a, esize, M, K, K, GEMM_BM, bk));
+  IG4_TRY(map_2d(mb, w, esize, N, K, K, b_rows, bk));
+  return IG4_OK;
+}
+
+bool is_fp8(int dt) { return dt == IG4_E4M3; }
+
+// ------------------------------------------------------------ validation
+
+bool valid_dtype_x(int d) { return d == IG4_F32 || d == IG4_BF16; }
+bool valid_dtype_w(int d) { return d == IG4_BF16 || d == IG4_E4M3; }
+
+ig4_status check_config(const ig4_config *c) {
+  if (!c) return IG4_ERR_INVALID_ARG;
+  if (c->B < 1 || c->T_text < 0 || c->grid_t < 0 || c->grid_h < 0 || c->grid_w < 0)
+    return IG4_ERR_INVALID_ARG;
+  const long L = static_cast<long>(c->T_text) + static_cast<long>(c->grid_t) * c->grid_h * c->grid_w;
+  if (L < 1 || L > (1L << 24)) return IG4_ERR_INVALID_ARG;
+  if (static_cast<long>(c->B) * L > (1L << 26)) return IG4_ERR_UNSUPPORTED;
+  if (c->H < 1 || c->D < 1 || c->I < 1 || c->adaln_dim < 1) return IG4_ERR_INVALID_ARG;
+  if (c->sections[0] < 0 || c->sections[1] < 0 || c->sections[2] < 0 ||
+      c->sections[0] + c->sections[1] + c->sections[2] != 64)
+    return IG4_ERR_INVALID_ARG;
+  if (!(c->rope_theta > 0.0) || !(c->eps > 0.0f)) return IG4_ERR_INVALID_ARG;
+  if (!valid_dtype_x(c->x_dtype) || !valid_dtype_w(c->w_dtype)) return IG4_ERR_INVALID_ARG;
+  if (c->head_dim != 256 || c->D != 256 * c->H) return IG4_ERR_UNSUPPORTED;
+  if (c->D > 6144) return IG4_ERR_UNSUPPORTED;
+  if (c->I % 128 != 0) return IG4_ERR_UNSUPPORTED;
+  if (c->adaln_dim % 16 != 0 || c->adaln_dim > 1024 || c->B > 8) return IG4_ERR_UNSUPPORTED;
+  return IG4_OK;
+}
+
+// ------------------------------------------------------------- launchers
+
+ig4_status launch_adaln(int B, int A, int N, const float *temb, const void *w, int w_dtype,
+                        const float *w_scale, const float *bias, float *mod, cudaStream_t st) {
+  const int rows_per_cta = (ADALN_THREADS / 32) * ADALN_ROWS_PER_WARP;
+  const int grid = (N + rows_per_cta - 1) / rows_per_cta;
+  const int smem = B * A * 4;
+  if (is_fp8(w_dtype))
+    adaln_kernel<true><<<grid, ADALN_THREADS, smem, st>>>(temb, w, w_scale, bias, mod, B, A, N);
+  else
+    adaln_kernel<false><<<grid, ADALN_THREADS, smem, st>>>(temb, w, w_scale, bias, mod, B, A, N);
+  return last_launch_status();
+}
+
+template <typename XT, bool FP8>
+ig4_status launch_norm_t(int rows, int L, int D, const void *x, const float *shift,
+                         const float *scale, int mod_stride, float eps, void *h, float *hs,
+                         int remap_n, int remap_L, int remap_off, cudaStream_t st) {
+  const int grid = (rows + NORM_THREADS / 32 - 1) / (NORM_THREADS / 32);
+  const int nv = (D / 8 + 31) / 32;
+  const XT *xp = static_cast<const XT *>(x);
+#define IG4_NORM_CASE(NV)                                                                        \
+  if (nv <= NV) {                                                                                \
+    norm_modulate_kernel<XT, FP8, NV><<<grid, NORM_THREADS, 0, st>>>(                            \
+        xp, shift, scale, mod_stride, rows, L, D, eps, h, hs, remap_n, remap_L, remap_off);      \
+    return last_launch_status();                                                                 \
+  }
+  IG4_NORM_CASE(2)
+  IG4_NORM_CASE(4)
+  IG4_NORM_CASE(8)
+  IG4_NORM_CASE(12)
+  IG4_NORM_CASE(18)
+  IG4_NORM_CASE(24)
+#undef IG4_NORM_CASE
+  return IG4_ERR_UNSUPPORTED;
+}
+
+ig4_status launch_norm(int rows, int L, int D, const void *x, int x_dtype, const float *shift,
+                       const float *scale, int mod_stride, float eps, void *h, int h_dtype,
+                       float *hs, int remap_n, int remap_L, int remap_off, cudaStream_t st) {
+  const bool f8 = is_fp8(h_dtype);
+  if (x_dtype == IG4_F32)
+    return f8 ? launch_norm_t<float, true>(rows, L, D, x, shift, scale, mod_stride, eps, h, hs,
+                                           remap_n, remap_L, remap_off, st)
+              : launch_norm_t<float, false>(rows, L, D, x, shift, scale, mod_stride, eps, h, hs,
+                                            remap_n, remap_L, remap_off, st);
+  return f8 ? launch_norm_t<__nv_bfloat16, true>(rows, L, D, x, shift, scale, mod_stride, eps, h,
+                                                 hs, remap_n, remap_L, remap_off, st)
+            : launch_norm_t<__nv_bfloat16, false>(rows, L, D, x, shift, scale, mod_stride, eps, h,
+                                                  hs, remap_n, remap_L, remap_off, st);
+}
+
+ig4_status launch_rope_table(int L, const int32_t *pos, double theta, const int sec[3], float *c,
+                             float *s, cudaStream_t st) {
+  const int n = L * 64;
+  rope_table_kernel<<<(n + 255) / 256, 256, 0, st>>>(pos, L, theta, sec[0], sec[1], c, s);
+  return last_launch_status();
+}
+
+ig4_status launch_quantize(int M, int K, const void *x, void *q, float *scale, cudaStream_t st) {
+  const int nv = (K / 8 + QUANT_THREADS - 1) / QUANT_THREADS;
+  const __nv_bfloat16 *xp = static_cast<const __nv_bfloat16 *>(x);
+  uint8_t *qp = static_cast<uint8_t *>(q);
+#define IG4_Q_CASE(NV)                                                                   \
+  if (nv <= NV) {                                                                        \
+    quantize_rows_kernel<NV><<<M, QUANT_THREADS, 0, st>>>(xp, qp, scale, K);             \
+    return last_launch_status();                                                         \
+  }
+  IG4_Q_CASE(1)
+  IG4_Q_CASE(2)
+  IG4_Q_CASE(4)
+  IG4_Q_CASE(6)
+  IG4_Q_CASE(8)
+#undef IG4_Q_CASE
+  return IG4_ERR_UNSUPPORTED;
+}
+
+ig4_status launch_qkv(int B, int L, int D, int H, const void *h, int h_dtype, const float *h_scale,
+                      const void *w, const float *w_scale, const float *g_q, const float *g_k,
+                      float eps, const float *cs, const float *sn, void *q, void *k, void *vt,
+                      int vt_ld, cudaStream_t st) {
+  const int M = B * L;
+  const bool f8 = is_fp8(h_dtype);
+  const int esize = f8 ? 1 : 2;
+  CUtensorMap ma, mb;
+  IG4_TRY(gemm_maps(&ma, &mb, h, w, esize, M, 3L * D, D, 256));
+  const int ntn = 3 * H;
+  if (f8) {
+    EpiQKV<true> e{static_cast<__nv_bfloat16 *>(q), static_cast<__nv_bfloat16 *>(k),
+                   static_cast<__nv_bfloat16 *>(vt), vt_ld, L, H, M, g_q, g_k, eps, cs, sn,
+                   h_scale, w_scale};
+    return launch_gemm<256, true, false>(ma, mb, mb, M, ntn, D, e, st);
+  }
+  EpiQKV<false> e{static_cast<__nv_bfloat16 *>(q), static_cast<__nv_bfloat16 *>(k),
+                  static_cast<__nv_bfloat16 *>(vt), vt_ld, L, H, M, g_q, g_k, eps, cs, sn,
+                  nullptr, nullptr};
+  return launch_gemm<256, false, false>(ma, mb, mb, M, ntn, D, e, st);
+}
+
+ig4_status launch_attention(int B, int H, int L, const void *q, const void *k, const void *vt,
+                            int vt_ld, void *o, cudaStream_t st) {
+  CUtensorMap mq, mk, mv;
+  const long BH = static_cast<long>(B) * H;
+  IG4_TRY(map_3d_bf16(&mq, q, 256, L, BH, 256, static_cast<long>(L) * 256, 64, ATT_BM));
+  IG4_TRY(map_3d_bf16(&mk, k, 256, L, BH, 256, static_cast<long>(L) * 256, 64, ATT_BN));
+  IG4_TRY(map_3d_bf16(&mv, vt, L, 256, BH, vt_ld, 256L * vt_ld, ATT_BN, 256));
+  IG4_TRY(allow_smem(attention_kernel, ATT_SMEM_BYTES));
+  dim3 grid((L + ATT_BM - 1) / ATT_BM, H, B);
+  attention_kernel<<<grid, ATT_THREADS, ATT_SMEM_BYTES, st>>>(
+      mq, mk, mv, static_cast<__nv_bfloat16 *>(o), L, H);
+  return last_launch_status();
+}
+
+template <typename XT>
+ig4_status launch_resid_t(int B, int L, int N, int K, const void *a, bool f8, const float *a_scale,
+                          const void *w, const float *w_scale, const float *gate, int gate_stride,
+                          const void *x_res, void *x_out, cudaStream_t st) {
+  const int M = B * L;
+  CUtensorMap ma, mb;
+  IG4_TRY(gemm_maps(&ma, &mb, a, w, f8 ? 1 : 2, M, N, K, 256));
+  if (f8) {
+    EpiResidGate<256, true, XT> e{static_cast<const XT *>(x_res), static_cast<XT *>(x_out), gate,
+                                   gate_stride, L, M, N, a_scale, w_scale};
+    return launch_gemm<256, true, false>(ma, mb, mb, M, N / 256, K, e, st);
+  }
+  EpiResidGate<256, false, XT> e{static_cast<const XT *>(x_res), static_cast<XT *>(x_out), gate,
+                                  gate_stride, L, M, N, nullptr, nullptr};
+  return launch_gemm<256, false, false>(ma, mb, mb, M, N / 256, K, e, st);
+}
+
+ig4_status launch_resid(int B, int L, int N, int K, const void *a, bool f8, const float *a_scale,
+                        const void *w, const float *w_scale, const float *gate, int gate_stride,
+                        const void *x_res, void *x_out, int x_dtype, cudaStream_t st) {
+  if (x_dtype == IG4_F32)
+    return launch_resid_t<float>(B, L, N, K, a, f8, a_scale, w, w_scale, gate, gate_stride, x_res,
+                                 x_out, st);
+  return launch_resid_t<__nv_bfloat16>(B, L, N, K, a, f8, a_scale, w, w_scale, gate, gate_stride,
+                                       x_res, x_out, st);
+}
+
+ig4_status launch_swiglu(int M, int I, int K, const void *h, bool f8, const float *h_scale,
+                         const void *wg, const void *wu, const float *sg, const float *su, void *u,
+                         cudaStream_t st) {
+  const int esize = f8 ? 1 : 2;
+  CUtensorMap ma, mg, mu;
+  IG4_TRY(map_2d(&ma, h, esize, M, K, K, GEMM_BM, 128 / esize));
+  IG4_TRY(map_2d(&mg, wg, esize, I, K, K, 128, 128 / esize));
+  IG4_TRY(map_2d(&mu, wu, esize, I, K, K, 128, 128 / esize));
+  if (f8) {
+    EpiSwiGLU<true> e{static_cast<__nv_bfloat16 *>(u), I, M, h_scale, sg, su};
+    return launch_gemm<256, true, true>(ma, mg, mu, M, I / 128, K, e, st);
+  }
+  EpiSwiGLU<false> e{static_cast<__nv_bfloat16 *>(u), I, M, nullptr, nullptr, nullptr};
+  return launch_gemm<256, false, true>(ma, mg, mu, M, I / 128, K, e, st);
+}
+
+// E4M3 weight [N][K] with per-row scale -> bf16 [N][K].  K % 16 == 0.
+ig4_status launch_dequant(int N, int K, const void *q, const float *s, void *out, cudaStream_t st) {
+  const long total16 = static_cast<long>(N) * K / 16;
+  const int grid = static_cast<int>(std::min<long>((total16 + 255) / 256, 148L * 16));
+  dequant_e4m3_rows_kernel<<<grid, 256, 0, st>>>(static_cast<const uint8_t *>(q), s,
+                                                 static_cast<__nv_bfloat16 *>(out), K, total16);
+  return last_launch_status();
+}
+
+// Plain linear with bias (stack in/out projections).  N % 128 == 0.
+ig4_status launch_linear_store(int M, int N, int K, const void *a, bool f8, const float *a_scale,
+                               const void *w, const float *w_scale, const float *bias, void *out,
+                               int out_dtype, int ldo, int remap_n, int remap_L, int remap_off,
+                               cudaStream_t st) {
+  CUtensorMap ma, mb;
+  IG4_TRY(gemm_maps(&ma, &mb, a, w, f8 ? 1 : 2, M, N, K, 128));
+  if (out_dtype == IG4_F32) {
+    if (f8) {
+      EpiStore<128, true, float> e{static_cast<float *>(out), ldo, M, N, bias, a_scale, w_scale,
+                                   remap_n, remap_L, remap_off};
+      return launch_gemm<128, true, false>(ma, mb, mb, M, N / 128, K, e, st);
+    }
+    EpiStore<128, false, float> e{static_cast<float *>(out), ldo, M, N, bias, nullptr, nullptr,
+                                  remap_n, remap_L, remap_off};
+    return launch_gemm<128, false, false>(ma, mb, mb, M, N / 128, K, e, st);
+  }
+  if (f8) {
+    EpiStore<128, true, __nv_bfloat16> e{static_cast<__nv_bfloat16 *>(out), ldo, M, N, bias,
+                                         a_scale, w_scale, remap_n, remap_L, remap_off};
+    return launch_gemm<128, true, false>(ma, mb, mb, M, N / 128, K, e, st);
+  }
+  EpiStore<128, false, __nv_bfloat16> e{static_cast<__nv_bfloat16 *>(out), ldo, M, N, bias,
+                                        nullptr, nullptr, remap_n, remap_L, remap_off};
+  return launch_gemm<128, false, false>(ma, mb, mb, M, N / 128, K, e, st);
+}
+
+// ------------------------------------------------------- workspace layout
+
+struct BlockWs {
+  float *mod, *cos, *sin;
+  void *h;        // bf16 [M][D] or e4m3 [M][D]
+  float *h_scale; // [M] (E4M3)
+  void *q, *k, *vt;
+  void *o;        // bf16 [M][D]
+  void *oq;       // e4m3 [M][D]
+  float *o_scale;
+  void *u;        // bf16 [M][I]
+  void *uq;       // e4m3 [M][I]
+  float *u_scale;
+  int vt_ld;
+  size_t bytes;
+};
+
+// Lays the block's buffers out from `base` (nullptr: only count bytes).
+BlockWs block_ws_layout(const ig4_config *c, uint8_t *base) {
+  BlockWs w{};
+  const long L = c->T_text + static_cast<long>(c->grid_t) * c->grid_h * c->grid_w;
+  const long M = c->B * L;
+  const long D = c->D, I = c->I, H = c->H;
+  const bool f8 = is_fp8(c->w_dtype);
+  w.vt_ld = static_cast<int>(round_up(L, 8));
+  size_t off = 0;
+  auto take = [&](size_t n) -> uint8_t * {
+    uint8_t *p = base ? base + off : nullptr;
+    off += round_up(n, 256);
+    return p;
+  };
+  w.mod = reinterpret_cast<float *>(take(sizeof(float) * c->B * 6 * D));
+  w.cos = reinterpret_cast<float *>(take(sizeof(float) * L * 64));
+  w.sin = reinterpret_cast<float *>(take(sizeof(float) * L * 64));
+  w.h = take((f8 ? 1 : 2) * M * D);
+  w.h_scale = reinterpret_cast<float *>(take(f8 ? sizeof(float) * M : 0));
+  w.q = take(2 * c->B * H * L * 256);
+  w.k = take(2 * c->B * H * L * 256);
+  w.vt = take(2 * c->B * H * 256 * static_cast<long>(w.vt_ld));
+  w.o = take(2 * M * D);
+  w.oq = take(f8 ? M * D : 0);
+  w.o_scale = reinterpret_cast<float *>(take(f8 ? sizeof(float) * M : 0));
+  w.u = take(2 * M * I);
+  w.uq = take(f8 ? M * I : 0);
+  w.u_scale = reinterpret_cast<float *>(take(f8 ? sizeof(float) * M : 0));
+  w.bytes = off;
+  return w;
+}
+
+ig4_status check_block_weights(const ig4_config *c, const ig4_block_weights *w) {
+  if (!w) return IG4_ERR_INVALID_ARG;
+  const void *ptrs[] = {w->w_ada, w->w_qkv, w->w_o, w->w_gate, w->w_up, w->w_down,
+                        w->b_ada, w->g_q, w->g_k};
+  for (const void *p : ptrs)
+    if (!p || !aligned16(p)) return IG4_ERR_INVALID_ARG;
+  if (is_fp8(c->w_dtype)) {
+    const void *s[] = {w->s_ada, w->s_qkv, w->s_o, w->s_gate, w->s_up, w->s_down};
+    for (const void *p : s)
+      if (!p || !aligned16(p)) return IG4_ERR_INVALID_ARG;
+  }
+  return IG4_OK;
+}
+
+// Event recording for the traced block forward.
+struct Tracer {
+  void *const *ev;
+  int n;
+  int next;
+  cudaStream_t st;
+  ig4_status mark() {
+    if (!ev || next >= n) return IG4_OK;
+    return cudaEventRecord(reinterpret_cast<cudaEvent_t>(ev[next++]), st) == cudaSuccess
+               ? IG4_OK
+               : IG4_ERR_CUDA;
+  }
+};
+
+// The block on already validated arguments.
+ig4_status block_forward_impl(const ig4_config *c, const ig4_block_weights *w, const void *x_in,
+                              void *x_out, const int32_t *pos, const float *temb,
+                              const BlockWs &ws, cudaStream_t st, Tracer *tr) {
+  const int L = c->T_text + c->grid_t * c->grid_h * c->grid_w;
+  const int M = c->B * L;
+  const int D = c->D, I = c->I, H = c->H;
+  const bool f8 = is_fp8(c->w_dtype);
+  const int hdt = f8 ? IG4_E4M3 : IG4_BF16;
+  const int ms = 6 * D;
+  Tracer none{nullptr, 0, 0, st};
+  Tracer &t = tr ? *tr : none;
+
+  IG4_TRY(t.mark());
+  IG4_TRY(launch_adaln(c->B, c->adaln_dim, 6 * D, temb, w->w_ada, c->w_dtype, w->s_ada, w->b_ada,
+                       ws.mod, st));
+  IG4_TRY(t.mark());
+  IG4_TRY(launch_rope_table(L, pos, c->rope_theta, c->sections, ws.cos, ws.sin, st));
+  IG4_TRY(t.mark());
+  IG4_TRY(launch_norm(M, L, D, x_in, c->x_dtype, ws.mod + 0 * D, ws.mod + 1 * D, ms, c->eps, ws.h,
+                      hdt, ws.h_scale, 0, 0, 0, st));
+  IG4_TRY(t.mark());
+  IG4_TRY(launch_qkv(c->B, L, D, H, ws.h, hdt, ws.h_scale, w->w_qkv, w->s_qkv, w->g_q, w->g_k,
+                     c->eps, ws.cos, ws.sin, ws.q, ws.k, ws.vt, ws.vt_ld, st));
+  IG4_TRY(t.mark());
+  IG4_TRY(launch_attention(c->B, H, L, ws.q, ws.k, ws.vt, ws.vt_ld, ws.o, st));
+  IG4_TRY(t.mark());
+  if (f8) {
+    IG4_TRY(launch_quantize(M, D, ws.o, ws.oq, ws.o_scale, st));
+    IG4_TRY(t.mark());
+  }
+  IG4_TRY(launch_resid(c->B, L, D, D, f8 ? ws.oq : ws.o, f8, ws.o_scale, w->w_o, w->s_o,
+                       ws.mod + 2 * D, ms, x_in, x_out, c->x_dtype, st));
+  IG4_TRY(t.mark());
+  IG4_TRY(launch_norm(M, L, D, x_out, c->x_dtype, ws.mod + 3 * D, ws.mod + 4 * D, ms, c->eps,
+                      ws.h, hdt, ws.h_scale, 0, 0, 0, st));
+  IG4_TRY(t.mark());
+  IG4_TRY(launch_swiglu(M, I, D, ws.h, f8, ws.h_scale, w->w_gate, w->w_up, w->s_gate, w->s_up,
+                        ws.u, st));
+  IG4_TRY(t.mark());
+  if (f8) {
+    IG4_TRY(launch_quantize(M, I, ws.u, ws.uq, ws.u_scale, st));
+    IG4_TRY(t.mark());
+  }
+  IG4_TRY(launch_resid(c->B, L, D, I, f8 ? ws.uq : ws.u, f8, ws.u_scale, w->w_down, w->s_down,
+                       ws.mod + 5 * D, ms, x_out, x_out, c->x_dtype, st));
+  IG4_TRY(t.mark());
+  return IG4_OK;
+}
+
+// Stack workspace: two sequence buffers, the block workspace, final-layer buffers.
+struct StackWs {
+  void *s0, *s1;
+  BlockWs blk;
+  float *mod_f;
+  void *hf;  // bf16 [B*N][D]
+  void *w_in16, *w_out16;  // bf16 copies of E4M3 in/out projection weights
+  size_t bytes;
+};
+
+StackWs stack_ws_layout(const ig4_config *c, int C, uint8_t *base) {
+  StackWs w{};
+  const long L = c->T_text + static_cast<long>(c->grid_t) * c->grid_h * c->grid_w;
+  const long N = static_cast<long>(c->grid_t) * c->grid_h * c->grid_w;
+  const long M = c->B * L;
+  const bool f8 = is_fp8(c->w_dtype);
+  const long xs = c->x_dtype == IG4_F32 ? 4 : 2;
+  size_t off = 0;
+  auto take = [&](size_t n) -> uint8_t * {
+    uint8_t *p = base ? base + off : nullptr;
+    off += round_up(n, 256);
+    return p;
+  };
+  w.s0 = take(xs * M * c->D);
+  w.s1 = take(xs * M * c->D);
+  w.mod_f = reinterpret_cast<float *>(take(sizeof(float) * c->B * 2 * c->D));
+  w.hf = take(2 * c->B * N * c->D);
+  w.w_in16 = take(f8 ? 2L * c->D * C : 0);
+  w.w_out16 = take(f8 ? 2L * C * c->D : 0);
+  uint8_t *blk_base = base ? base + off : nullptr;
+  w.blk = block_ws_layout(c, blk_base);
+  off += w.blk.bytes;
+  w.bytes = off;
+  return w;
+}
+
+}  // namespace
+
+// =================================================================== C ABI
+
+extern "C" {
+
+const char *ig4_status_string(int s) {
+  switch (s) {
+    case IG4_OK: return "IG4_OK";
+    case IG4_ERR_INVALID_ARG: return "IG4_ERR_INVALID_ARG";
+    case IG4_ERR_UNSUPPORTED: return "IG4_ERR_UNSUPPORTED";
+    case IG4_ERR_WORKSPACE: return "IG4_ERR_WORKSPACE";
+    case IG4_ERR_CUDA: return "IG4_ERR_CUDA";
+    case IG4_ERR_TIMEOUT: return "IG4_ERR_TIMEOUT";
+    default: return "IG4_ERR_UNKNOWN";
+  }
+}
+
+int ig4_abi_version(void) { return ABI_VERSION; }
+
+ig4_status ig4_mrope_positions(int T, int gt, int gh, int gw, int32_t *pos, int on_device,
+                               void *stream) {
+  if (!pos || T < 0 || gt < 0 || gh < 0 || gw < 0) return IG4_ERR_INVALID_ARG;
+  const long L = static_cast<long>(T) + static_cast<long>(gt) * gh * gw;
+  if (L < 1 || L > (1L << 24)) return IG4_ERR_INVALID_ARG;
+  if (on_device) {
+    if (!aligned16(pos)) return IG4_ERR_INVALID_ARG;
+    mrope_positions_kernel<<<static_cast<int>((L + 255) / 256), 256, 0, as_stream(stream)>>>(
+        T, gt, gh, gw, pos);
+    return last_launch_status();
+  }
+  for (long l = 0; l < T; ++l) pos[l] = pos[L + l] = pos[2 * L + l] = static_cast<int32_t>(l);
+  long n = T;
+  for (int t = 0; t < gt; ++t)
+    for (int i = 0; i < gh; ++i)
+      for (int j = 0; j < gw; ++j, ++n) {
+        pos[n] = T + t;
+        pos[L + n] = T + i;
+        pos[2 * L + n] = T + j;
+      }
+  return IG4_OK;
+}
+
+ig4_status ig4_rope_table(int L, const int32_t *pos, double theta, const int sections[3],
+                          float *cos_out, float *sin_out, void *stream) {
+  if (L < 1 || !pos || !sections || !cos_out || !sin_out || !(theta > 0.0))
+    return IG4_ERR_INVALID_ARG;
+  if (sections[0] < 0 || sections[1] < 0 || sections[2] < 0 ||
+      sections[0] + sections[1] + sections[2] != 64)
+    return IG4_ERR_INVALID_ARG;
+  return launch_rope_table(L, pos, theta, sections, cos_out, sin_out, as_stream(stream));
+}
+
+ig4_status ig4_adaln_modulation(int B, int A, int N, const float *temb, const void *w, int w_dtype,
+                                const float *w_scale, const float *bias, float *mod_out,
+                                void *stream) {
+  if (!temb || !w || !mod_out || B < 1 || B > 8 || A < 16 || A % 16 || A > 1024 || N < 1)
+    return IG4_ERR_INVALID_ARG;
+  if (!valid_dtype_w(w_dtype) || (is_fp8(w_dtype) && !w_scale) || !aligned16(w))
+    return IG4_ERR_INVALID_ARG;
+  return launch_adaln(B, A, N, temb, w, w_dtype, w_scale, bias, mod_out, as_stream(stream));
+}
+
+ig4_status ig4_norm_modulate(int B, int L, int D, const void *x, int x_dtype, const float *shift,
+                             const float *scale, int mod_stride, float eps, void *h_out,
+                             int h_dtype, float *h_scale_out, void *stream) {
+  if (!x || !shift || !scale || !h_out || B < 1 || L < 1 || D < 8 || D % 8 || D > 6144 ||
+      !(eps > 0.0f) || mod_stride < D)
+    return IG4_ERR_INVALID_ARG;
+  if (!valid_dtype_x(x_dtype) || (h_dtype != IG4_BF16 && h_dtype != IG4_E4M3))
+    return IG4_ERR_INVALID_ARG;
+  if (h_dtype == IG4_E4M3 && !h_scale_out) return IG4_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(shift) || !aligned16(scale) || !aligned16(h_out) ||
+      mod_stride % 4)
+    return IG4_ERR_INVALID_ARG;
+  return launch_norm(B * L, L, D, x, x_dtype, shift, scale, mod_stride, eps, h_out, h_dtype,
+                     h_scale_out, 0, 0, 0, as_stream(stream));
+}
+
+ig4_status ig4_qkv_project(int B, int L, int D, int H, const void *h, int h_dtype,
+                           const float *h_scale, const void *w_qkv, int w_dtype,
+                           const float *w_scale, const float *g_q, const float *g_k, float eps,
+                           const float *rope_cos, const float *rope_sin, void *q_out, void *k_out,
+                           void *vt_out, int vt_ld, void *stream) {
+  if (B < 1 || L < 1 || H < 1 || !h || !w_qkv || !g_q || !g_k || !rope_cos || !rope_sin ||
+      !q_out || !k_out || !vt_out || !(eps > 0.0f) || vt_ld < L || vt_ld % 8)
+    return IG4_ERR_INVALID_ARG;
+  if (D != 256 * H) return IG4_ERR_UNSUPPORTED;
+  if (!valid_dtype_w(w_dtype) || h_dtype != (is_fp8(w_dtype) ? IG4_E4M3 : IG4_BF16))
+    return IG4_ERR_UNSUPPORTED;
+  if (is_fp8(w_dtype) && (!h_scale || !w_scale)) return IG4_ERR_INVALID_ARG;
+  const void *al[] = {h, w_qkv, g_q, g_k, rope_cos, rope_sin, q_out, k_out, vt_out};
+  for (const void *p : al)
+    if (!aligned16(p)) return IG4_ERR_INVALID_ARG;
+  return launch_qkv(B, L, D, H, h, h_dtype, h_scale, w_qkv, w_scale, g_q, g_k, eps, rope_cos,
+                    rope_sin, q_out, k_out, vt_out, vt_ld, as_stream(stream));
+}
+
+ig4_status ig4_joint_attention(int B, int H, int L, const void *q, const void *k, const void *vt,
+                               int vt_ld, void *o_out, void *stream) {
+  if (B < 1 || H < 1 || L < 1 || !q || !k || !vt || !o_out || vt_ld < L || vt_ld % 8)
+    return IG4_ERR_INVALID_ARG;
+  if (H > 65535 || B > 65535) return IG4_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(vt) || !aligned16(o_out))
+    return IG4_ERR_INVALID_ARG;
+  return launch_attention(B, H, L, q, k, vt, vt_ld, o_out, as_stream(stream));
+}
+
+ig4_status ig4_gated_residual_linear(int B, int L, int N, int K, const void *a, int a_dtype,
+                                     const float *a_scale, const void *w, int w_dtype,
+                                     const float *w_scale, const float *gate, int gate_stride,
+                                     const void *x_res, void *x_out, int x_dtype, void *stream) {
+  if (B < 1 || L < 1 || N < 1 || K < 1 || !a || !w || !gate || !x_res || !x_out ||
+      gate_stride < N || gate_stride % 4)
+    return IG4_ERR_INVALID_ARG;
+  if (!valid_dtype_w(w_dtype) || !valid_dtype_x(x_dtype)) return IG4_ERR_INVALID_ARG;
+  const bool f8 = is_fp8(w_dtype);
+  if (a_dtype != (f8 ? IG4_E4M3 : IG4_BF16)) return IG4_ERR_UNSUPPORTED;
+  if (f8 && (!a_scale || !w_scale)) return IG4_ERR_INVALID_ARG;
+  if (N % 256 || K % (f8 ? 128 : 64)) return IG4_ERR_UNSUPPORTED;
+  if (!aligned16(a) || !aligned16(w) || !aligned16(gate) || !aligned16(x_res) ||
+      !aligned16(x_out))
+    return IG4_ERR_INVALID_ARG;
+  return launch_resid(B, L, N, K, a, f8, a_scale, w, w_scale, gate, gate_stride, x_res, x_out,
+                      x_dtype, as_stream(stream));
+}
+
+ig4_status ig4_swiglu(int M, int I, int K, const void *h, int h_dtype, const float *h_scale,
+                      const void *w_gate, const void *w_up, int w_dtype, const float *s_gate,
+                      const float *s_up, void *u_out, void *stream) {
+  if (M < 1 || I < 1 || K < 1 || !h || !w_gate || !w_up || !u_out) return IG4_ERR_INVALID_ARG;
+  if (!valid_dtype_w(w_dtype)) return IG4_ERR_INVALID_ARG;
+  const bool f8 = is_fp8(w_dtype);
+  if (h_dtype != (f8 ? IG4_E4M3 : IG4_BF16)) return IG4_ERR_UNSUPPORTED;
+  if (f8 && (!h_scale || !s_gate || !s_up)) return IG4_ERR_INVALID_ARG;
+  if (I % 128 || K % (f8 ? 128 : 64)) return IG4_ERR_UNSUPPORTED;
+  if (!aligned16(h) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(u_out))
+    return IG4_ERR_INVALID_ARG;
+  return launch_swiglu(M, I, K, h, f8, h_scale, w_gate, w_up, s_gate, s_up, u_out,
+                       as_stream(stream));
+}
+
+ig4_status ig4_quantize_rows(int M, int K, const void *x, void *q_out, float *scale_out,
+                             void *stream) {
+  if (M < 1 || K < 8 || K % 8 || K > 16384 || !x || !q_out || !scale_out)
+    return IG4_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(q_out)) return IG4_ERR_INVALID_ARG;
+  return launch_quantize(M, K, x, q_out, scale_out, as_stream(stream));
+}
+
+size_t ig4_workspace_size(const ig4_config *cfg) {
+  if (check_config(cfg) != IG4_OK) return 0;
+  return block_ws_layout(cfg, nullptr).bytes;
+}
+
+static ig4_status block_forward_checked(const ig4_config *cfg, const ig4_block_weights *w,
+                                        const void *x_in, void *x_out, const int32_t *pos,
+                                        const float *temb, void *workspace, size_t ws_bytes,
+                                        void *stream, void *const *events, int n_events) {
+  IG4_TRY(check_config(cfg));
+  IG4_TRY(check_block_weights(cfg, w));
+  if (!x_in || !x_out || !pos || !temb || !workspace) return IG4_ERR_INVALID_ARG;
+  if (!aligned16(x_in) || !aligned16(x_out) || !aligned16(temb)) return IG4_ERR_INVALID_ARG;
+  if (n_events != 0 && (n_events != IG4_BLOCK_TRACE_EVENTS || !events)) return IG4_ERR_INVALID_ARG;
+  const long L = cfg->T_text + static_cast<long>(cfg->grid_t) * cfg->grid_h * cfg->grid_w;
+  const size_t xbytes = (cfg->x_dtype == IG4_F32 ? 4 : 2) * static_cast<size_t>(cfg->B) * L * cfg->D;
+  const uint8_t *xi = static_cast<const uint8_t *>(x_in);
+  const uint8_t *xo = static_cast<const uint8_t *>(x_out);
+  if (xi < xo + xbytes && xo < xi + xbytes) return IG4_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return IG4_ERR_WORKSPACE;
+  const BlockWs ws = block_ws_layout(cfg, static_cast<uint8_t *>(workspace));
+  if (ws_bytes < ws.bytes) return IG4_ERR_WORKSPACE;
+  Tracer tr{events, n_events, 0, as_stream(stream)};
+  return block_forward_impl(cfg, w, x_in, x_out, pos, temb, ws, as_stream(stream),
+                            n_events ? &tr : nullptr);
+}
+
+ig4_status ig4_block_forward(const ig4_config *cfg, const ig4_block_weights *w, const void *x_in,
+                             void *x_out, const int32_t *pos, const float *temb, void *workspace,
+                             size_t ws_bytes, void *stream) {
+  return block_forward_checked(cfg, w, x_in, x_out, pos, temb, workspace, ws_bytes, stream,
+                               nullptr, 0);
+}
+
+ig4_status ig4_block_forward_traced(const ig4_config *cfg, const ig4_block_weights *w,
+                                    const void *x_in, void *x_out, const int32_t *pos,
+                                    const float *temb, void *workspace, size_t ws_bytes,
+                                    void *stream, void *const *events, int n_events) {
+  return block_forward_checked(cfg, w, x_in, x_out, pos, temb, workspace, ws_bytes, stream,
+                               events, n_events);
+}
+
+size_t ig4_stack_workspace_size(const ig4_config *cfg, int latent_ch) {
+  if (check_config(cfg) != IG4_OK || latent_ch < 128 || latent_ch % 128 ||
+      cfg->x_dtype != IG4_BF16)
+    return 0;
+  return stack_ws_layout(cfg, latent_ch, nullptr).bytes;
+}
+
+ig4_status ig4_stack_forward(const ig4_config *cfg, const ig4_stack_weights *sw,
+                             const void *x_latent, const void *text, void *out_latent,
+                             const int32_t *pos, const float *temb, void *workspace,
+                             size_t ws_bytes, void *stream) {
+  IG4_TRY(check_config(cfg));
+  if (!sw || !x_latent || !out_latent || !pos || !temb || !workspace) return IG4_ERR_INVALID_ARG;
+  if (cfg->x_dtype != IG4_BF16) return IG4_ERR_UNSUPPORTED;
+  const int C = sw->latent_ch;
+  if (C < 128 || C % 128 || sw->n_blocks < 0 || (sw->n_blocks > 0 && !sw->blocks))
+    return IG4_ERR_INVALID_ARG;
+  const int N = cfg->grid_t * cfg->grid_h * cfg->grid_w;
+  const int T = cfg->T_text;
+  if (N < 1 || (T > 0 && !text)) return IG4_ERR_INVALID_ARG;
+  const bool f8 = is_fp8(cfg->w_dtype);
+  const void *need[] = {sw->w_in, sw->b_in, sw->w_f, sw->b_f, sw->w_out, sw->b_out};
+  for (const void *p : need)
+    if (!p || !aligned16(p)) return IG4_ERR_INVALID_ARG;
+  if (f8 && (!sw->s_in || !sw->s_f || !sw->s_out)) return IG4_ERR_INVALID_ARG;
+  for (int i = 0; i < sw->n_blocks; ++i) IG4_TRY(check_block_weights(cfg, &sw->blocks[i]));
+  if (!aligned16(x_latent) || !aligned16(out_latent) || !aligned16(temb) ||
+      (text && !aligned16(text)))
+    return IG4_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return IG4_ERR_WORKSPACE;
+  const StackWs ws = stack_ws_layout(cfg, C, static_cast<uint8_t *>(workspace));
+  if (ws_bytes < ws.bytes) return IG4_ERR_WORKSPACE;
+
+  cudaStream_t st = as_stream(stream);
+  const int L = T + N;
+  const int D = cfg->D;
+  const int B = cfg->B;
+  // [text | image] sequence in s0: the text prefix, then the latent in-projection.
+  if (T > 0) {
+    const int vpr = D * 2 / 16;
+    const long total = static_cast<long>(B) * T * vpr;
+    const int grid = static_cast<int>(std::min<long>((total + 255) / 256, 148L * 8));
+    copy_rows_kernel<<<grid, 256, 0, st>>>(static_cast<const uint4 *>(text),
+                                           static_cast<uint4 *>(ws.s0), T, L, 0, vpr, total);
+    IG4_TRY(last_launch_status());
+  }
+  // The latent in/out projections are 0.01% of the step's work: they run in
+  // bf16 (E4M3 weights decoded into the workspace) so that they add no
+  // activation-quantisation error.
+  const void *w_in = sw->w_in;
+  const void *w_out = sw->w_out;
+  if (f8) {
+    IG4_TRY(launch_dequant(D, C, sw->w_in, sw->s_in, ws.w_in16, st));
+    IG4_TRY(launch_dequant(C, D, sw->w_out, sw->s_out, ws.w_out16, st));
+    w_in = ws.w_in16;
+    w_out = ws.w_out16;
+  }
+  IG4_TRY(launch_linear_store(B * N, D, C, x_latent, false, nullptr, w_in, nullptr, sw->b_in,
+                              ws.s0, IG4_BF16, D, N, L, T, st));
+  void *cur = ws.s0;
+  void *nxt = ws.s1;
+  for (int i = 0; i < sw->n_blocks; ++i) {
+    IG4_TRY(block_forward_impl(cfg, &sw->blocks[i], cur, nxt, pos, temb, ws.blk, st, nullptr));
+    std::swap(cur, nxt);
+  }
+  // Final layer on the image tokens: RMSNorm + (shift, scale), then D -> C.
+  IG4_TRY(launch_adaln(B, cfg->adaln_dim, 2 * D, temb, sw->w_f, cfg->w_dtype, sw->s_f, sw->b_f,
+                       ws.mod_f, st));
+  IG4_TRY(launch_norm(B * N, L, D, cur, IG4_BF16, ws.mod_f, ws.mod_f + D, 2 * D, cfg->eps, ws.hf,
+                      IG4_BF16, nullptr, N, L, T, st));
+  IG4_TRY(launch_linear_store(B * N, C, D, ws.hf, false, nullptr, w_out, nullptr, sw->b_out,
+                              out_latent, IG4_BF16, C, 0, 0, 0, st));
+  return IG4_OK;
+}
+
+ig4_status ig4_last_device_error(void *stream) {
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return IG4_ERR_CUDA;
+  unsigned int word = 0;
+  if (cudaMemcpyFromSymbol(&word, g_device_error, sizeof(word)) != cudaSuccess)
+    return IG4_ERR_CUDA;
+  if (word) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess)
+      return IG4_ERR_CUDA;
+    return IG4_ERR_TIMEOUT;
+  }
+  return IG4_OK;
+}
+
+ig4_status ig4_selftest_timeout(int wait_us, void *stream) {
+  if (wait_us < 1 || wait_us > 5000000) return IG4_ERR_INVALID_ARG;
+  selftest_timeout_kernel<<<1, 32, 0, as_stream(stream)>>>(
+      static_cast<unsigned long long>(wait_us) * 1000ull);
+  return last_launch_status();
+}
+
+}  // extern "C"

@@ -1,0 +1,503 @@
+// ig4_gemm.cuh - persistent tcgen05 GEMM C = A B^T for sm_100a with fused
+// epilogues for the block's linears.
+//
+// A [M, K] and B [N, K] are K-major (row-major, K contiguous) in bf16, or both
+// in FP8 E4M3 for the FP8-weight path (activation codes + per-row scale,
+// weight codes + per-output-channel scale).  One CTA per SM walks the output
+// tiles (128 x BN) in m-fastest order so that the CTAs in flight share the
+// same few B column blocks and all of A through L2.
+//
+// Warp roles (192 threads):
+//   warp 4      TMA producer: A and B tiles (128-byte swizzle) into a STAGES
+//               deep shared-memory ring, one mbarrier per stage;
+//   warp 5      TMEM allocator and MMA issuer (one thread): 4 tcgen05.mma per
+//               stage into one of two TMEM accumulators (2 x BN fp32 columns),
+//               tcgen05.commit frees the stage / publishes the accumulator;
+//   warps 0-3   epilogue: each warp owns 32 accumulator rows (TMEM lanes
+//               32*(warp%4) ..), reads 32 columns at a time with tcgen05.ld,
+//               applies the fused epilogue and stores to global memory, then
+//               releases the accumulator so the MMA of tile t+2 can reuse it.
+#pragma once
+
+#include "ig4_ptx.cuh"
+
+namespace ig4 {
+
+constexpr int GEMM_BM = 128;
+constexpr int GEMM_THREADS = 192;
+
+template <int BN>
+struct GemmShape {
+  static constexpr int A_BYTES = GEMM_BM * 128;
+  static constexpr int B_BYTES = BN * 128;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = (BN == 256) ? 4 : 6;
+  static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+};
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
+  const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+  return reinterpret_cast<uint8_t *>((a + 1023) & ~static_cast<uintptr_t>(1023));
+}
+
+// ----------------------------------------------------------- store helpers
+
+__device__ __forceinline__ void store32_bf16(__nv_bfloat16 *dst, const float (&v)[32]) {
+  uint4 *d = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 w;
+    w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+    w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+    w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+    w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+    d[q] = w;
+  }
+}
+
+__device__ __forceinline__ void store32_f32(float *dst, const float (&v)[32]) {
+  float4 *d = reinterpret_cast<float4 *>(dst);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+}
+
+__device__ __forceinline__ void load32_bf16(const __nv_bfloat16 *src, float (&v)[32]) {
+  const uint4 *s = reinterpret_cast<const uint4 *>(src);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 w = s[q];
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v[8 * q + 2 * e] = __uint_as_float(u[e] << 16);
+      v[8 * q + 2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
+    }
+  }
+}
+
+__device__ __forceinline__ void load32_f32(const float *src, float (&v)[32]) {
+  const float4 *s = reinterpret_cast<const float4 *>(src);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const float4 w = s[q];
+    v[4 * q] = w.x;
+    v[4 * q + 1] = w.y;
+    v[4 * q + 2] = w.z;
+    v[4 * q + 3] = w.w;
+  }
+}
+
+__device__ __forceinline__ void load32_f32_ldg(const float *src, float (&v)[32]) {
+  const float4 *s = reinterpret_cast<const float4 *>(src);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const float4 w = __ldg(s + q);
+    v[4 * q] = w.x;
+    v[4 * q + 1] = w.y;
+    v[4 * q + 2] = w.z;
+    v[4 * q + 3] = w.w;
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ void load32_x(const T *src, float (&v)[32]);
+template <>
+__device__ __forceinline__ void load32_x<float>(const float *src, float (&v)[32]) {
+  load32_f32(src, v);
+}
+template <>
+__device__ __forceinline__ void load32_x<__nv_bfloat16>(const __nv_bfloat16 *src, float (&v)[32]) {
+  load32_bf16(src, v);
+}
+template <typename T>
+__device__ __forceinline__ void store32_x(T *dst, const float (&v)[32]);
+template <>
+__device__ __forceinline__ void store32_x<float>(float *dst, const float (&v)[32]) {
+  store32_f32(dst, v);
+}
+template <>
+__device__ __forceinline__ void store32_x<__nv_bfloat16>(__nv_bfloat16 *dst, const float (&v)[32]) {
+  store32_bf16(dst, v);
+}
+
+// Dequantisation factors of the FP8 path: acc * a_scale[row] * b_scale[col].
+template <bool FP8>
+__device__ __forceinline__ void apply_scales(float (&v)[32], float rs, const float *bs) {
+  if constexpr (FP8) {
+    float s[32];
+    load32_f32_ldg(bs, s);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] *= rs * s[i];
+  }
+}
+
+// ------------------------------------------------------------- epilogues
+// Each epilogue is called by the 128 epilogue threads for one output tile;
+// `tacc` is the TMEM address of this warp's 32 lanes at column 0 of the
+// tile's accumulator and `r` the thread's row inside the tile.
+
+// out[row', col] = acc (* scales) (+ bias[col]); row' = row, or, with
+// remap_n > 0, (row / remap_n) * remap_L + remap_off + row % remap_n (writes
+// the latent in-projection straight into the image part of the sequence).
+template <int BN, bool FP8, typename OT>
+struct EpiStore {
+  OT *out;
+  int ldo;
+  int M, N;
+  const float *bias;
+  const float *a_scale, *b_scale;
+  int remap_n, remap_L, remap_off;
+
+  __device__ __forceinline__ void operator()(int m0, int n0, uint32_t tacc, int r) const {
+    const int row = m0 + r;
+    const bool valid = row < M;
+    long orow = row;
+    if (remap_n > 0) orow = static_cast<long>(row / remap_n) * remap_L + remap_off + row % remap_n;
+    const float rs = (FP8 && valid) ? __ldg(a_scale + row) : 1.0f;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      float v[32];
+      tmem_ld32(tacc + c, v);
+      tmem_ld_wait();
+      if (n0 + c >= N) continue;
+      apply_scales<FP8>(v, rs, b_scale + n0 + c);
+      if (bias != nullptr) {
+        float bb[32];
+        load32_f32_ldg(bias + n0 + c, bb);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] += bb[i];
+      }
+      if (valid) store32_x<OT>(out + orow * ldo + n0 + c, v);
+    }
+  }
+};
+
+// Gated residual: x_out[row, col] = x_res[row, col] + gate[b, col] * acc,
+// b = row / L (the AdaLN gate of the row's sample).
+template <int BN, bool FP8, typename XT>
+struct EpiResidGate {
+  const XT *x_res;
+  XT *x_out;
+  const float *gate;
+  int gate_stride;
+  int L, M, N;
+  const float *a_scale, *b_scale;
+
+  __device__ __forceinline__ void operator()(int m0, int n0, uint32_t tacc, int r) const {
+    const int row = m0 + r;
+    const bool valid = row < M;
+    const int b = valid ? row / L : 0;
+    const float rs = (FP8 && valid) ? __ldg(a_scale + row) : 1.0f;
+    const float *grow = gate + static_cast<long>(b) * gate_stride + n0;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      float v[32];
+      tmem_ld32(tacc + c, v);
+      tmem_ld_wait();
+      if (!valid) continue;
+      apply_scales<FP8>(v, rs, b_scale + n0 + c);
+      float g[32], x[32];
+      load32_f32_ldg(grow + c, g);
+      const long off = static_cast<long>(row) * N + n0 + c;
+      load32_x<XT>(x_res + off, x);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) x[i] = fmaf(g[i], v[i], x[i]);
+      store32_x<XT>(x_out + off, x);
+    }
+  }
+};
+
+// SwiGLU: the 256-column tile holds gate rows [n, n+128) in columns [0,128)
+// and up rows [n, n+128) in columns [128,256); u[row, n + c] =
+// silu(gate) * up.  (Two TMA loads fill the two halves of the B tile.)
+template <bool FP8>
+struct EpiSwiGLU {
+  __nv_bfloat16 *u;
+  int I, M;
+  const float *a_scale, *s_gate, *s_up;
+
+  __device__ __forceinline__ void operator()(int m0, int n0, uint32_t tacc, int r) const {
+    const int row = m0 + r;
+    const bool valid = row < M;
+    const float rs = (FP8 && valid) ? __ldg(a_scale + row) : 1.0f;
+    const int n = n0 / 2;  // tile index * 128
+#pragma unroll 1
+    for (int c = 0; c < 128; c += 32) {
+      float g[32], up[32];
+      tmem_ld32(tacc + c, g);
+      tmem_ld32(tacc + 128 + c, up);
+      tmem_ld_wait();
+      if (!valid) continue;
+      apply_scales<FP8>(g, rs, s_gate + n + c);
+      apply_scales<FP8>(up, rs, s_up + n + c);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) g[i] = silu_f(g[i]) * up[i];
+      store32_bf16(u + static_cast<long>(row) * I + n + c, g);
+    }
+  }
+};
+
+// QKV projection with per-head QK-RMSNorm and MRoPE.  Tile columns
+// [n0, n0+256) are one head of q (n-tile < H), k (< 2H) or v.  q, k are
+// normalised over the 256 values, scaled by g, and the pairs (j, j+64),
+// j < 64, are rotated by the row's table angle; they are stored as
+// [B, H, L, 256].  v is stored transposed, [B, H, 256, vt_ld].
+template <bool FP8>
+struct EpiQKV {
+  __nv_bfloat16 *q, *k, *vt;
+  int vt_ld;
+  int L, H, M;
+  const float *g_q, *g_k;
+  float eps;
+  const float *rope_cos, *rope_sin;
+  const float *a_scale, *b_scale;
+
+  __device__ __forceinline__ void operator()(int m0, int n0, uint32_t tacc, int r) const {
+    const int row = m0 + r;
+    const bool valid = row < M;
+    const int b = valid ? row / L : 0;
+    const int l = valid ? row - b * L : 0;
+    const int nt = n0 >> 8;
+    const int sec = nt / H;
+    const int h = nt - sec * H;
+    const float rs = (FP8 && valid) ? __ldg(a_scale + row) : 1.0f;
+    const float *bs = b_scale + n0;
+
+    if (sec == 2) {
+      __nv_bfloat16 *dst = vt + static_cast<long>(b * H + h) * 256 * vt_ld + l;
+#pragma unroll 1
+      for (int c = 0; c < 256; c += 32) {
+        float v[32];
+        tmem_ld32(tacc + c, v);
+        tmem_ld_wait();
+        if (!valid) continue;
+        apply_scales<FP8>(v, rs, bs + c);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) dst[static_cast<long>(c + i) * vt_ld] = __float2bfloat16_rn(v[i]);
+      }
+      return;
+    }
+
+    float ss = 0.0f;
+#pragma unroll 1
+    for (int c = 0; c < 256; c += 32) {
+      float v[32];
+      tmem_ld32(tacc + c, v);
+      tmem_ld_wait();
+      apply_scales<FP8>(v, rs, bs + c);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
+    }
+    const float rstd = rsqrtf(ss * (1.0f / 256.0f) + eps);
+    const float *g = (sec == 0) ? g_q : g_k;
+    __nv_bfloat16 *dst = ((sec == 0) ? q : k) + (static_cast<long>(b * H + h) * L + l) * 256;
+    const float *cs = rope_cos + static_cast<long>(l) * 64;
+    const float *sn = rope_sin + static_cast<long>(l) * 64;
+
+#pragma unroll 1
+    for (int j0 = 0; j0 < 64; j0 += 32) {
+      float a[32], bv[32];
+      tmem_ld32(tacc + j0, a);
+      tmem_ld32(tacc + j0 + 64, bv);
+      tmem_ld_wait();
+      if (!valid) continue;
+      apply_scales<FP8>(a, rs, bs + j0);
+      apply_scales<FP8>(bv, rs, bs + j0 + 64);
+      float ga[32], gb[32], c32[32], s32[32];
+      load32_f32_ldg(g + j0, ga);
+      load32_f32_ldg(g + j0 + 64, gb);
+      load32_f32_ldg(cs + j0, c32);
+      load32_f32_ldg(sn + j0, s32);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float x1 = a[i] * rstd * ga[i];
+        const float x2 = bv[i] * rstd * gb[i];
+        a[i] = x1 * c32[i] - x2 * s32[i];
+        bv[i] = x2 * c32[i] + x1 * s32[i];
+      }
+      store32_bf16(dst + j0, a);
+      store32_bf16(dst + j0 + 64, bv);
+    }
+#pragma unroll 1
+    for (int c = 128; c < 256; c += 32) {
+      float v[32];
+      tmem_ld32(tacc + c, v);
+      tmem_ld_wait();
+      if (!valid) continue;
+      apply_scales<FP8>(v, rs, bs + c);
+      float gg[32];
+      load32_f32_ldg(g + c, gg);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] *= rstd * gg[i];
+      store32_bf16(dst + c, v);
+    }
+  }
+};
+
+// ---------------------------------------------------------------- kernel
+// BN: accumulator columns per tile (256 or 128).  DUAL_B: the B tile is two
+// 128-row halves from two tensors (tmB rows, then tmB2 rows, same row index).
+// n_cols_tile: output columns one n-tile advances (BN, or 128 with DUAL_B).
+template <int BN, bool FP8, bool DUAL_B, class Epi>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmB2, int M, int n_tiles_n, int K,
+                   const Epi epi) {
+  using S = GemmShape<BN>;
+  constexpr int STAGES = S::STAGES;
+  constexpr int BK = FP8 ? 128 : 64;  // K elements per stage: one 128-byte row
+  constexpr int UK_BYTES = 32;        // K bytes per MMA instruction (16 bf16 / 32 e4m3)
+  constexpr uint32_t IDESC = FP8 ? idesc_e4m3(GEMM_BM, BN) : idesc_bf16(GEMM_BM, BN);
+  constexpr int B_ROWS_HALF = BN / 2;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = align1024(smem_raw);
+  uint8_t *sA = smem;
+  uint8_t *sB = smem + STAGES * S::A_BYTES;
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * S::STAGE_BYTES);
+  uint64_t *empty = full + STAGES;
+  uint64_t *tfull = empty + STAGES;
+  uint64_t *tempty = tfull + 2;
+  uint64_t *drain = tempty + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int m_tiles = (M + GEMM_BM - 1) / GEMM_BM;
+  const int n_tiles = m_tiles * n_tiles_n;
+  const int kblocks = (K + BK - 1) / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    if (DUAL_B) tma_prefetch_desc(&tmB2);
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, S::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      // ---------------- TMA producer
+      int s = 0;
+      uint32_t ph = 0;
+      long issued = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+        const int mt = t % m_tiles;
+        const int nt = t / m_tiles;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&empty[s], ph ^ 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], S::STAGE_BYTES);
+          tma_load_2d(sA + s * S::A_BYTES, &tmA, &full[s], kb * BK, mt * GEMM_BM);
+          if (DUAL_B) {
+            tma_load_2d(sB + s * S::B_BYTES, &tmB, &full[s], kb * BK, nt * B_ROWS_HALF);
+            tma_load_2d(sB + s * S::B_BYTES + B_ROWS_HALF * 128, &tmB2, &full[s], kb * BK,
+                        nt * B_ROWS_HALF);
+          } else {
+            tma_load_2d(sB + s * S::B_BYTES, &tmB, &full[s], kb * BK, nt * BN);
+          }
+          ++issued;
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        // Let the loads already issued land before the CTA's shared memory goes away.
+        for (long i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
+          mbar_wait(&full[i % STAGES], static_cast<uint32_t>((i / STAGES) & 1), nullptr,
+                    WAIT_LIMIT_NS / 4);
+      }
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      // ---------------- MMA issuer
+      int s = 0;
+      uint32_t ph = 0;
+      int local = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++local) {
+        const int buf = local & 1;
+        const uint32_t use = static_cast<uint32_t>(local >> 1);
+        if (!mbar_wait(&tempty[buf], (use & 1) ^ 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + buf * BN;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&full[s], ph, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(sA + s * S::A_BYTES);
+          const uint32_t b_base = smem_u32(sB + s * S::B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < 128 / UK_BYTES; ++kk) {
+            const uint64_t ad = sdesc_kmajor_sw128(a_base + kk * UK_BYTES);
+            const uint64_t bd = sdesc_kmajor_sw128(b_base + kk * UK_BYTES);
+            if (FP8)
+              umma_f8(d_tmem, ad, bd, IDESC, (kb | kk) != 0);
+            else
+              umma_bf16(d_tmem, ad, bd, IDESC, (kb | kk) != 0);
+          }
+          umma_commit(&empty[s]);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+        if (ok) umma_commit(&tfull[buf]);
+      }
+      // Every MMA issued above has finished once `drain` completes.
+      umma_commit(drain);
+      mbar_wait(drain, 0, nullptr, WAIT_LIMIT_NS / 4);
+    }
+  } else {
+    // ---------------- epilogue warps 0..3
+    const int r = warp * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    int local = 0;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++local) {
+      const int buf = local & 1;
+      const uint32_t use = static_cast<uint32_t>(local >> 1);
+      if (!mbar_wait_warp(&tfull[buf], use & 1, abort_flag)) break;
+      tc_fence_after();
+      const int mt = t % m_tiles;
+      const int nt = t / m_tiles;
+      epi(mt * GEMM_BM, nt * BN, tmem_base + lane_base + buf * BN, r);
+      tc_fence_before();
+      mbar_arrive(&tempty[buf]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 5) tmem_dealloc(tmem_base, S::TMEM_COLS);
+}
+
+}  // namespace ig4
