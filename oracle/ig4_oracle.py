@@ -206,9 +206,9 @@ def joint_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray) -> np.ndarray:
     text / image branches).  Returns [B, H, L, dh].
     """
     dh = q.shape[-1]
-    s = np.einsum("bhld,bhmd->bhlm", q, k) / np.sqrt(float(dh))
+    s = np.matmul(q, np.swapaxes(k, -1, -2)) / np.sqrt(float(dh))
     p = softmax(s, axis=-1)
-    return np.einsum("bhlm,bhmd->bhld", p, v)
+    return np.matmul(p, v)
 
 
 def split_heads(t: np.ndarray, H: int) -> np.ndarray:
@@ -347,8 +347,8 @@ def block_forward_rows(x, temb, pos, W, H, rows, theta=ROPE_THETA, sections=MROP
         q = split_heads((h[ls] @ w_q.T)[None], H)  # [1, H, n, dh]
         k = apply_mrope(rms_norm(k, eps, W["g_k"]), pos, theta, sections)
         q = apply_mrope(rms_norm(q, eps, W["g_q"]), pos[:, ls], theta, sections)
-        s = np.einsum("bhld,bhmd->bhlm", q, k) / np.sqrt(float(dh))
-        o = merge_heads(np.einsum("bhlm,bhmd->bhld", softmax(s, axis=-1), v))[0]  # [n, D]
+        s = np.matmul(q, np.swapaxes(k, -1, -2)) / np.sqrt(float(dh))
+        o = merge_heads(np.matmul(softmax(s, axis=-1), v))[0]  # [n, D]
         x1 = x[b, ls] + gate_msa[b][None, :] * (o @ W["w_o"].T)
         h2 = rms_norm(x1, eps) * (1.0 + scale_mlp[b][None, :]) + shift_mlp[b][None, :]
         y = x1 + gate_mlp[b][None, :] * (swiglu(h2, W["w_gate"], W["w_up"]) @ W["w_down"].T)
