@@ -192,7 +192,7 @@ def run_ours(args, rank, local_rank, world):
         build()
     if world > 1:
         dist.barrier()
-    import stream_diffusion_transformer_fwd_b200 as ig4
+    from stream_diffusion_transformer_fwd_b200 import ig4
     from synth import CONFIGS, make_block_activations, make_block_weights
 
     cfg = CONFIGS[args.config]

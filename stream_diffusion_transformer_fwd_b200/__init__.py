@@ -1,300 +1,6 @@
-"""Python binding of libig4 (include/ig4.h): an sm_100a implementation of the
-Ideogram 4 single-stream DiT block forward and the 34-block stack.
+"""B200 (sm_100a) implementation of the Ideogram 4 DiT block forward.
 
-Argument marshalling only: every step of the block runs in the library's CUDA
-kernels.  PyTorch supplies device memory and the current CUDA stream.  The
-functions carry the C entry points' names; each raises Ig4Error on a status
-other than IG4_OK.  Importing the package fails loudly if the shared library
-is missing (build it with ``python -m stream_diffusion_transformer_fwd_b200.build``).
+The C-ABI library (``libig4.so``, built from ``csrc/`` by ``build.py``) holds
+every kernel; ``stream_diffusion_transformer_fwd_b200.ig4`` is its Python
+binding and fails to import if the library is missing.
 """
-
-from __future__ import annotations
-
-import ctypes
-import os
-
-import torch
-
-_HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libig4.so")
-
-IG4_OK, IG4_ERR_INVALID_ARG, IG4_ERR_UNSUPPORTED, IG4_ERR_WORKSPACE, IG4_ERR_CUDA, \
-    IG4_ERR_TIMEOUT = range(6)
-IG4_F32, IG4_BF16, IG4_E4M3 = 0, 1, 2
-IG4_BLOCK_TRACE_EVENTS = 12
-
-_DTYPE_CODE = {torch.float32: IG4_F32, torch.bfloat16: IG4_BF16, torch.float8_e4m3fn: IG4_E4M3}
-_CODE_NAME = {IG4_F32: "f32", IG4_BF16: "bf16", IG4_E4M3: "e4m3"}
-_NAME_CODE = {v: k for k, v in _CODE_NAME.items()}
-
-if not os.path.exists(LIB_PATH):
-    raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m stream_diffusion_transformer_fwd_b200.build`"
-        " (there is no fallback implementation)")
-_lib = ctypes.CDLL(LIB_PATH)
-
-_vp = ctypes.c_void_p
-_i = ctypes.c_int
-_f = ctypes.c_float
-
-
-class Ig4Error(RuntimeError):
-    def __init__(self, status: int, where: str):
-        self.status = status
-        super().__init__(f"{where}: {_lib.ig4_status_string(status).decode()}")
-
-
-class Config(ctypes.Structure):
-    _fields_ = [("B", _i), ("T_text", _i), ("grid_t", _i), ("grid_h", _i), ("grid_w", _i),
-                ("D", _i), ("H", _i), ("head_dim", _i), ("I", _i), ("adaln_dim", _i),
-                ("rope_theta", ctypes.c_double), ("sections", _i * 3), ("eps", _f),
-                ("x_dtype", _i), ("w_dtype", _i)]
-
-
-class BlockWeights(ctypes.Structure):
-    _fields_ = [(n, _vp) for n in ("w_ada", "w_qkv", "w_o", "w_gate", "w_up", "w_down",
-                                   "s_ada", "s_qkv", "s_o", "s_gate", "s_up", "s_down",
-                                   "b_ada", "g_q", "g_k")]
-
-
-class StackWeights(ctypes.Structure):
-    _fields_ = [("n_blocks", _i), ("latent_ch", _i), ("blocks", ctypes.POINTER(BlockWeights)),
-                ("w_in", _vp), ("s_in", _vp), ("b_in", _vp),
-                ("w_f", _vp), ("s_f", _vp), ("b_f", _vp),
-                ("w_out", _vp), ("s_out", _vp), ("b_out", _vp)]
-
-
-def _sig(name, args, res=_i):
-    fn = getattr(_lib, name)
-    fn.argtypes = args
-    fn.restype = res
-    return fn
-
-
-_lib.ig4_status_string.argtypes = [_i]
-_lib.ig4_status_string.restype = ctypes.c_char_p
-_sig("ig4_abi_version", [])
-_sig("ig4_mrope_positions", [_i, _i, _i, _i, _vp, _i, _vp])
-_sig("ig4_rope_table", [_i, _vp, ctypes.c_double, ctypes.POINTER(_i), _vp, _vp, _vp])
-_sig("ig4_adaln_modulation", [_i, _i, _i, _vp, _vp, _i, _vp, _vp, _vp, _vp])
-_sig("ig4_norm_modulate", [_i, _i, _i, _vp, _i, _vp, _vp, _i, _f, _vp, _i, _vp, _vp])
-_sig("ig4_qkv_project", [_i, _i, _i, _i, _vp, _i, _vp, _vp, _i, _vp, _vp, _vp, _f, _vp, _vp,
-                         _vp, _vp, _vp, _i, _vp])
-_sig("ig4_joint_attention", [_i, _i, _i, _vp, _vp, _vp, _i, _vp, _vp])
-_sig("ig4_gated_residual_linear", [_i, _i, _i, _i, _vp, _i, _vp, _vp, _i, _vp, _vp, _i, _vp,
-                                   _vp, _i, _vp])
-_sig("ig4_swiglu", [_i, _i, _i, _vp, _i, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp])
-_sig("ig4_quantize_rows", [_i, _i, _vp, _vp, _vp, _vp])
-_sig("ig4_workspace_size", [ctypes.POINTER(Config)], ctypes.c_size_t)
-_sig("ig4_block_forward", [ctypes.POINTER(Config), ctypes.POINTER(BlockWeights), _vp, _vp, _vp,
-                           _vp, _vp, ctypes.c_size_t, _vp])
-_sig("ig4_block_forward_traced", [ctypes.POINTER(Config), ctypes.POINTER(BlockWeights), _vp, _vp,
-                                  _vp, _vp, _vp, ctypes.c_size_t, _vp, ctypes.POINTER(_vp), _i])
-_sig("ig4_stack_workspace_size", [ctypes.POINTER(Config), _i], ctypes.c_size_t)
-_sig("ig4_stack_forward", [ctypes.POINTER(Config), ctypes.POINTER(StackWeights), _vp, _vp, _vp,
-                           _vp, _vp, _vp, ctypes.c_size_t, _vp])
-_sig("ig4_last_device_error", [_vp])
-_sig("ig4_selftest_timeout", [_i, _vp])
-
-EXPORTED = ("ig4_status_string", "ig4_abi_version", "ig4_mrope_positions", "ig4_rope_table",
-            "ig4_adaln_modulation", "ig4_norm_modulate", "ig4_qkv_project",
-            "ig4_joint_attention", "ig4_gated_residual_linear", "ig4_swiglu",
-            "ig4_quantize_rows", "ig4_workspace_size", "ig4_block_forward",
-            "ig4_block_forward_traced", "ig4_stack_workspace_size", "ig4_stack_forward",
-            "ig4_last_device_error", "ig4_selftest_timeout")
-
-
-def library():
-    """The loaded ctypes library (for tests that call entry points directly)."""
-    return _lib
-
-
-# ------------------------------------------------------------------ helpers
-
-def _check(status: int, where: str):
-    if status != IG4_OK:
-        raise Ig4Error(status, where)
-
-
-def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
-
-
-def _stream(stream=None):
-    if stream is not None:
-        return ctypes.c_void_p(stream.cuda_stream)
-    if torch.cuda.is_available() and torch.cuda.is_initialized():
-        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    return ctypes.c_void_p(0)
-
-
-def dtype_code(t: torch.Tensor) -> int:
-    return _DTYPE_CODE[t.dtype]
-
-
-def make_config(B, T_text, grid_t, grid_h, grid_w, D=4608, H=18, head_dim=256, I=12288,
-                adaln_dim=512, rope_theta=5.0e6, sections=(24, 20, 20), eps=1e-6,
-                x_dtype="bf16", w_dtype="bf16") -> Config:
-    c = Config()
-    c.B, c.T_text, c.grid_t, c.grid_h, c.grid_w = B, T_text, grid_t, grid_h, grid_w
-    c.D, c.H, c.head_dim, c.I, c.adaln_dim = D, H, head_dim, I, adaln_dim
-    c.rope_theta = rope_theta
-    c.sections = (_i * 3)(*sections)
-    c.eps = eps
-    c.x_dtype = _NAME_CODE[x_dtype] if isinstance(x_dtype, str) else x_dtype
-    c.w_dtype = _NAME_CODE[w_dtype] if isinstance(w_dtype, str) else w_dtype
-    return c
-
-
-def config_from(cfg) -> Config:
-    """Config from any object with the ig4_config field names (e.g. synth.Config)."""
-    return make_config(cfg.B, cfg.T_text, cfg.grid_t, cfg.grid_h, cfg.grid_w, cfg.D, cfg.H,
-                       cfg.head_dim, cfg.I, cfg.adaln_dim, cfg.rope_theta, tuple(cfg.sections),
-                       cfg.eps, cfg.x_dtype, cfg.w_dtype)
-
-
-def block_weights(w: dict) -> BlockWeights:
-    """BlockWeights from a dict of device tensors (keys as in ig4_block_weights)."""
-    bw = BlockWeights()
-    for name, _ in BlockWeights._fields_:
-        t = w.get(name)
-        setattr(bw, name, None if t is None else t.data_ptr())
-    return bw
-
-
-# --------------------------------------------------------------- entry points
-
-def ig4_status_string(status: int) -> str:
-    return _lib.ig4_status_string(status).decode()
-
-
-def ig4_abi_version() -> int:
-    return _lib.ig4_abi_version()
-
-
-def ig4_mrope_positions(T_text, grid_t, grid_h, grid_w, out: torch.Tensor | None = None,
-                        device=None, stream=None) -> torch.Tensor:
-    """int32 [3, L] position table, on `device` (default: host)."""
-    L = T_text + grid_t * grid_h * grid_w
-    if out is None:
-        out = torch.empty((3, L), dtype=torch.int32,
-                          device=device if device is not None else "cpu")
-    on_dev = 1 if out.is_cuda else 0
-    _check(_lib.ig4_mrope_positions(T_text, grid_t, grid_h, grid_w, _ptr(out), on_dev,
-                                    _stream(stream) if on_dev else None), "ig4_mrope_positions")
-    return out
-
-
-def ig4_rope_table(pos, rope_theta, sections, cos_out, sin_out, stream=None):
-    L = pos.shape[1]
-    sec = (_i * 3)(*sections)
-    _check(_lib.ig4_rope_table(L, _ptr(pos), rope_theta, sec, _ptr(cos_out), _ptr(sin_out),
-                               _stream(stream)), "ig4_rope_table")
-
-
-def ig4_adaln_modulation(temb, w, w_scale, bias, mod_out, stream=None):
-    B, A = temb.shape
-    N = w.shape[0]
-    _check(_lib.ig4_adaln_modulation(B, A, N, _ptr(temb), _ptr(w), dtype_code(w), _ptr(w_scale),
-                                     _ptr(bias), _ptr(mod_out), _stream(stream)),
-           "ig4_adaln_modulation")
-
-
-def ig4_norm_modulate(B, L, D, x, shift, scale, mod_stride, eps, h_out, h_scale_out=None,
-                      stream=None):
-    _check(_lib.ig4_norm_modulate(B, L, D, _ptr(x), dtype_code(x), _ptr(shift), _ptr(scale),
-                                  mod_stride, eps, _ptr(h_out), dtype_code(h_out),
-                                  _ptr(h_scale_out), _stream(stream)), "ig4_norm_modulate")
-
-
-def ig4_qkv_project(B, L, D, H, h, h_scale, w_qkv, w_scale, g_q, g_k, eps, rope_cos, rope_sin,
-                    q_out, k_out, vt_out, vt_ld, stream=None):
-    _check(_lib.ig4_qkv_project(B, L, D, H, _ptr(h), dtype_code(h), _ptr(h_scale), _ptr(w_qkv),
-                                dtype_code(w_qkv), _ptr(w_scale), _ptr(g_q), _ptr(g_k), eps,
-                                _ptr(rope_cos), _ptr(rope_sin), _ptr(q_out), _ptr(k_out),
-                                _ptr(vt_out), vt_ld, _stream(stream)), "ig4_qkv_project")
-
-
-def ig4_joint_attention(B, H, L, q, k, vt, vt_ld, o_out, stream=None):
-    _check(_lib.ig4_joint_attention(B, H, L, _ptr(q), _ptr(k), _ptr(vt), vt_ld, _ptr(o_out),
-                                    _stream(stream)), "ig4_joint_attention")
-
-
-def ig4_gated_residual_linear(B, L, N, K, a, a_scale, w, w_scale, gate, gate_stride, x_res,
-                              x_out, stream=None):
-    _check(_lib.ig4_gated_residual_linear(B, L, N, K, _ptr(a), dtype_code(a), _ptr(a_scale),
-                                          _ptr(w), dtype_code(w), _ptr(w_scale), _ptr(gate),
-                                          gate_stride, _ptr(x_res), _ptr(x_out),
-                                          dtype_code(x_out), _stream(stream)),
-           "ig4_gated_residual_linear")
-
-
-def ig4_swiglu(M, I, K, h, h_scale, w_gate, w_up, s_gate, s_up, u_out, stream=None):
-    _check(_lib.ig4_swiglu(M, I, K, _ptr(h), dtype_code(h), _ptr(h_scale), _ptr(w_gate),
-                           _ptr(w_up), dtype_code(w_gate), _ptr(s_gate), _ptr(s_up), _ptr(u_out),
-                           _stream(stream)), "ig4_swiglu")
-
-
-def ig4_quantize_rows(M, K, x, q_out, scale_out, stream=None):
-    _check(_lib.ig4_quantize_rows(M, K, _ptr(x), _ptr(q_out), _ptr(scale_out), _stream(stream)),
-           "ig4_quantize_rows")
-
-
-def ig4_workspace_size(cfg: Config) -> int:
-    return int(_lib.ig4_workspace_size(ctypes.byref(cfg)))
-
-
-def ig4_block_forward(cfg: Config, weights: BlockWeights, x_in, x_out, pos, temb, workspace,
-                      events=None, stream=None):
-    """x_out = block(x_in).  `events`: optional list of IG4_BLOCK_TRACE_EVENTS
-    torch.cuda.Event(enable_timing=True) recorded around each kernel."""
-    ws_bytes = workspace.numel() * workspace.element_size()
-    if events is None:
-        st = _lib.ig4_block_forward(ctypes.byref(cfg), ctypes.byref(weights), _ptr(x_in),
-                                    _ptr(x_out), _ptr(pos), _ptr(temb), _ptr(workspace),
-                                    ws_bytes, _stream(stream))
-        _check(st, "ig4_block_forward")
-        return
-    for e in events:  # make sure each event owns a CUDA handle
-        e.record(stream) if stream is not None else e.record()
-    arr = (_vp * len(events))(*[e.cuda_event for e in events])
-    st = _lib.ig4_block_forward_traced(ctypes.byref(cfg), ctypes.byref(weights), _ptr(x_in),
-                                       _ptr(x_out), _ptr(pos), _ptr(temb), _ptr(workspace),
-                                       ws_bytes, _stream(stream), arr, len(events))
-    _check(st, "ig4_block_forward_traced")
-
-
-def ig4_stack_workspace_size(cfg: Config, latent_ch: int = 128) -> int:
-    return int(_lib.ig4_stack_workspace_size(ctypes.byref(cfg), latent_ch))
-
-
-def stack_weights(blocks: list, w_in, s_in, b_in, w_f, s_f, b_f, w_out, s_out, b_out,
-                  latent_ch=128) -> StackWeights:
-    arr = (BlockWeights * max(1, len(blocks)))(*blocks)
-    sw = StackWeights()
-    sw.n_blocks = len(blocks)
-    sw.latent_ch = latent_ch
-    sw.blocks = ctypes.cast(arr, ctypes.POINTER(BlockWeights))
-    sw._keep = arr  # keep the host array alive with the struct
-    for name, t in (("w_in", w_in), ("s_in", s_in), ("b_in", b_in), ("w_f", w_f), ("s_f", s_f),
-                    ("b_f", b_f), ("w_out", w_out), ("s_out", s_out), ("b_out", b_out)):
-        setattr(sw, name, None if t is None else t.data_ptr())
-    return sw
-
-
-def ig4_stack_forward(cfg: Config, sw: StackWeights, x_latent, text, out_latent, pos, temb,
-                      workspace, stream=None):
-    ws_bytes = workspace.numel() * workspace.element_size()
-    _check(_lib.ig4_stack_forward(ctypes.byref(cfg), ctypes.byref(sw), _ptr(x_latent),
-                                  _ptr(text), _ptr(out_latent), _ptr(pos), _ptr(temb),
-                                  _ptr(workspace), ws_bytes, _stream(stream)),
-           "ig4_stack_forward")
-
-
-def ig4_last_device_error(stream=None) -> int:
-    """Status of the device error word (synchronises the stream); does not raise."""
-    return _lib.ig4_last_device_error(_stream(stream))
-
-
-def ig4_selftest_timeout(wait_us: int, stream=None):
-    _check(_lib.ig4_selftest_timeout(wait_us, _stream(stream)), "ig4_selftest_timeout")

@@ -14,7 +14,7 @@ from tests._util import BF16_U, max_abs_over_rms, rel_l2, rms
 def lib():
     from stream_diffusion_transformer_fwd_b200.build import build
     build()
-    import stream_diffusion_transformer_fwd_b200 as ig4
+    from stream_diffusion_transformer_fwd_b200 import ig4
     return ig4
 
 

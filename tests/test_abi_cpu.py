@@ -19,7 +19,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def ig4():
     from stream_diffusion_transformer_fwd_b200.build import build
     build()
-    import stream_diffusion_transformer_fwd_b200 as m
+    from stream_diffusion_transformer_fwd_b200 import ig4 as m
     return m
 
 
