@@ -228,6 +228,33 @@ ig4_status ig4_block_forward_traced(const ig4_config *cfg, const ig4_block_weigh
                                     const float *temb, void *workspace, size_t ws_bytes,
                                     void *stream, void *const *events, int n_events);
 
+/* ------------------------------------------- block without a workspace ---
+ * ig4_block_forward for callers that cannot allocate device memory.  This
+ * entry point has no counterpart on the pages: it exists for callers such as
+ * inference runtimes that plan all device memory ahead and forbid allocation
+ * while they execute, real-time loops that cannot afford cudaMalloc's
+ * latency and implicit synchronisation, and hosts whose own caching allocator
+ * owns the GPU's memory.  Instead of a caller workspace it uses a scratch
+ * array of IG4_NOALLOC_SCRATCH_BYTES (64 MiB) that the library reserves as a
+ * static device variable: every GPU that loads the library holds those bytes
+ * until the process exits.  It allocates nothing and calls no allocating
+ * routine.  The caller still passes inputs and outputs as for
+ * ig4_block_forward (same layouts and errors).  Configurations whose
+ * ig4_workspace_size exceeds the scratch size return IG4_ERR_WORKSPACE
+ * without launching anything (e.g. the full-width block up to ~900 tokens,
+ * or the 1024-wide block up to ~4000 tokens, fit).
+ * The first call on a device looks up the scratch array's device address
+ * (a one-time set-up per device, done with that device current); make that
+ * first call before any stream capture.  All calls share the one array and
+ * it keeps the previous call's contents; no part of it needs to start at
+ * zero, because every byte a call reads there was written earlier in the
+ * same call.  Calls whose work overlaps on the GPU (different streams, or
+ * different host threads without ordering) race on the array: order them. */
+#define IG4_NOALLOC_SCRATCH_BYTES (64ull << 20)
+ig4_status ig4_block_forward_noalloc(const ig4_config *cfg, const ig4_block_weights *w,
+                                     const void *x_in, void *x_out, const int32_t *pos,
+                                     const float *temb, void *stream);
+
 /* ---------------------------------------------------------------- a-12 ---
  * Bytes of workspace ig4_stack_forward needs (0 if invalid). */
 size_t ig4_stack_workspace_size(const ig4_config *cfg, int latent_ch);

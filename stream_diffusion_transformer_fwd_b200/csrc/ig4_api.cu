@@ -801,6 +801,57 @@ ig4_status ig4_stack_forward(const ig4_config *cfg, const ig4_stack_weights *sw,
   return IG4_OK;
 }
 
+}  // extern "C"
+
+// ------------------------------------------------ block without a workspace
+// Scratch for ig4_block_forward_noalloc: a static device array, so the entry
+// point never allocates.  In host code `g_noalloc_scratch` names a host-side
+// stand-in, not device memory; its device address comes from
+// cudaGetSymbolAddress, looked up once per device.
+__device__ __align__(256) uint8_t g_noalloc_scratch[IG4_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+void *g_noalloc_ptr[MAX_DEVICES];
+std::mutex g_noalloc_mu;
+
+// Device address of the scratch array on the current device (set up on the
+// first call for that device).
+ig4_status noalloc_scratch(uint8_t **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return IG4_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return IG4_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = static_cast<uint8_t *>(g_noalloc_ptr[dev]);
+  return IG4_OK;
+}
+}  // namespace
+
+extern "C" {
+
+ig4_status ig4_block_forward_noalloc(const ig4_config *cfg, const ig4_block_weights *w,
+                                     const void *x_in, void *x_out, const int32_t *pos,
+                                     const float *temb, void *stream) {
+  IG4_TRY(check_config(cfg));
+  IG4_TRY(check_block_weights(cfg, w));
+  if (!x_in || !x_out || !pos || !temb) return IG4_ERR_INVALID_ARG;
+  if (!aligned16(x_in) || !aligned16(x_out) || !aligned16(temb)) return IG4_ERR_INVALID_ARG;
+  const long L = cfg->T_text + static_cast<long>(cfg->grid_t) * cfg->grid_h * cfg->grid_w;
+  const size_t xbytes = (cfg->x_dtype == IG4_F32 ? 4 : 2) * static_cast<size_t>(cfg->B) * L * cfg->D;
+  const uint8_t *xi = static_cast<const uint8_t *>(x_in);
+  const uint8_t *xo = static_cast<const uint8_t *>(x_out);
+  if (xi < xo + xbytes && xo < xi + xbytes) return IG4_ERR_INVALID_ARG;
+  if (block_ws_layout(cfg, nullptr).bytes > IG4_NOALLOC_SCRATCH_BYTES) return IG4_ERR_WORKSPACE;
+  uint8_t *scratch = nullptr;
+  IG4_TRY(noalloc_scratch(&scratch));
+  const BlockWs ws = block_ws_layout(cfg, scratch);
+  return block_forward_impl(cfg, w, x_in, x_out, pos, temb, ws, as_stream(stream), nullptr);
+}
+
 ig4_status ig4_last_device_error(void *stream) {
   if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return IG4_ERR_CUDA;
   unsigned int word = 0;

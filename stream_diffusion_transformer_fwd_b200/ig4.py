@@ -22,6 +22,7 @@ IG4_OK, IG4_ERR_INVALID_ARG, IG4_ERR_UNSUPPORTED, IG4_ERR_WORKSPACE, IG4_ERR_CUD
     IG4_ERR_TIMEOUT = range(6)
 IG4_F32, IG4_BF16, IG4_E4M3 = 0, 1, 2
 IG4_BLOCK_TRACE_EVENTS = 12
+IG4_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 _DTYPE_CODE = {torch.float32: IG4_F32, torch.bfloat16: IG4_BF16, torch.float8_e4m3fn: IG4_E4M3}
 _CODE_NAME = {IG4_F32: "f32", IG4_BF16: "bf16", IG4_E4M3: "e4m3"}
@@ -90,6 +91,8 @@ _sig("ig4_block_forward", [ctypes.POINTER(Config), ctypes.POINTER(BlockWeights),
                            _vp, _vp, ctypes.c_size_t, _vp])
 _sig("ig4_block_forward_traced", [ctypes.POINTER(Config), ctypes.POINTER(BlockWeights), _vp, _vp,
                                   _vp, _vp, _vp, ctypes.c_size_t, _vp, ctypes.POINTER(_vp), _i])
+_sig("ig4_block_forward_noalloc", [ctypes.POINTER(Config), ctypes.POINTER(BlockWeights), _vp,
+                                   _vp, _vp, _vp, _vp])
 _sig("ig4_stack_workspace_size", [ctypes.POINTER(Config), _i], ctypes.c_size_t)
 _sig("ig4_stack_forward", [ctypes.POINTER(Config), ctypes.POINTER(StackWeights), _vp, _vp, _vp,
                            _vp, _vp, _vp, ctypes.c_size_t, _vp])
@@ -100,7 +103,7 @@ EXPORTED = ("ig4_status_string", "ig4_abi_version", "ig4_mrope_positions", "ig4_
             "ig4_adaln_modulation", "ig4_norm_modulate", "ig4_qkv_project",
             "ig4_joint_attention", "ig4_gated_residual_linear", "ig4_swiglu",
             "ig4_quantize_rows", "ig4_workspace_size", "ig4_block_forward",
-            "ig4_block_forward_traced", "ig4_stack_workspace_size", "ig4_stack_forward",
+            "ig4_block_forward_traced", "ig4_block_forward_noalloc", "ig4_stack_workspace_size", "ig4_stack_forward",
             "ig4_last_device_error", "ig4_selftest_timeout")
 
 
@@ -262,6 +265,15 @@ def ig4_block_forward(cfg: Config, weights: BlockWeights, x_in, x_out, pos, temb
                                        _ptr(x_out), _ptr(pos), _ptr(temb), _ptr(workspace),
                                        ws_bytes, _stream(stream), arr, len(events))
     _check(st, "ig4_block_forward_traced")
+
+
+def ig4_block_forward_noalloc(cfg: Config, weights: BlockWeights, x_in, x_out, pos, temb,
+                              stream=None):
+    """x_out = block(x_in) with the library's static scratch instead of a workspace,
+    for callers that cannot allocate device memory (see include/ig4.h)."""
+    _check(_lib.ig4_block_forward_noalloc(ctypes.byref(cfg), ctypes.byref(weights), _ptr(x_in),
+                                          _ptr(x_out), _ptr(pos), _ptr(temb), _stream(stream)),
+           "ig4_block_forward_noalloc")
 
 
 def ig4_stack_workspace_size(cfg: Config, latent_ch: int = 128) -> int:
