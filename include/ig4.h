@@ -178,7 +178,7 @@ ig4_status ig4_joint_attention(int B, int H, int L, const void *q, const void *k
  * gate[b*gate_stride + n] * sum_k a[r][k] W[n][k] (scaled by a_scale[r] *
  * w_scale[n] in E4M3), b = r / L.  a [B*L][K] in a_dtype (BF16, or E4M3 +
  * a_scale when w_dtype is E4M3); x_res / x_out [B*L][N] in x_dtype and may be
- * the same buffer.  N % 256 == 0, K % 64 == 0 (bf16) / % 128 == 0 (E4M3). */
+ * the same buffer.  N % 128 == 0, K % 64 == 0 (bf16) / % 128 == 0 (E4M3). */
 ig4_status ig4_gated_residual_linear(int B, int L, int N, int K, const void *a, int a_dtype,
                                      const float *a_scale, const void *w, int w_dtype,
                                      const float *w_scale, const float *gate, int gate_stride,

@@ -28,11 +28,14 @@ constexpr int GEMM_THREADS = 192;
 
 template <int BN>
 struct GemmShape {
+  static_assert(BN == 256 || BN == 192 || BN == 128, "tile width");
   static constexpr int A_BYTES = GEMM_BM * 128;
   static constexpr int B_BYTES = BN * 128;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = (BN == 256) ? 4 : 6;
-  static constexpr int TMEM_COLS = 2 * BN;
+  // as many stages as fit in ~200 KB of shared memory
+  static constexpr int STAGES = (BN == 256) ? 4 : (BN == 192 ? 5 : 6);
+  // two accumulators of BN fp32 columns, rounded up to a power of two
+  static constexpr int TMEM_COLS = (2 * BN <= 256) ? 256 : 512;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 };
 
@@ -498,6 +501,187 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 5) tmem_dealloc(tmem_base, S::TMEM_COLS);
+}
+
+// ------------------------------------------------------ CTA-pair kernel
+// The same GEMM on a 2-CTA cluster: a pair tile is 256 rows x 256 columns;
+// each CTA loads its own 128 A rows and HALF of the 256 B rows (so with
+// DUAL_B the first CTA loads the gate rows and the second the up rows), the
+// leader issues tcgen05.mma.cta_group::2 with M = 256, and each CTA's
+// epilogue warps handle its own 128 accumulator rows exactly as above.  Per
+// 128-clock MMA each SM reads 8 KB of operands instead of 12 KB, and each SM
+// loads a third fewer bytes per flop.
+//
+// Barriers: full[s] in the leader (its producer posts the bytes of both
+// CTAs; both CTAs' loads complete on it); empty[s] and tfull[b] in both CTAs
+// (arrived by the leader's multicast commits); tempty[b] in the leader (one
+// arrival per epilogue warp of the pair).
+constexpr int PAIR_STAGES = 6;
+constexpr int PAIR_STAGE_BYTES = 2 * GEMM_BM * 128;  // A 16 KB + B half 16 KB
+constexpr int PAIR_SMEM_BYTES = PAIR_STAGES * PAIR_STAGE_BYTES + 1024 + 256;
+
+template <bool FP8, bool DUAL_B, class Epi>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmB2, int M, int n_tiles_n, int K,
+                     const Epi epi) {
+  constexpr int BN = 256;
+  constexpr int A_BYTES = GEMM_BM * 128;
+  constexpr int BH_BYTES = (BN / 2) * 128;
+  constexpr int BK = FP8 ? 128 : 64;
+  constexpr int UK_BYTES = 32;
+  constexpr uint32_t IDESC = FP8 ? idesc_e4m3(2 * GEMM_BM, BN) : idesc_bf16(2 * GEMM_BM, BN);
+  constexpr uint32_t TMEM_COLS = 512;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = align1024(smem_raw);
+  uint8_t *sA = smem;
+  uint8_t *sB = smem + PAIR_STAGES * A_BYTES;
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + PAIR_STAGES * PAIR_STAGE_BYTES);
+  uint64_t *empty = full + PAIR_STAGES;
+  uint64_t *tfull = empty + PAIR_STAGES;
+  uint64_t *tempty = tfull + 2;
+  uint64_t *drain = tempty + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1;
+  const int n_pairs = gridDim.x >> 1;
+  const int m_tiles = (M + 2 * GEMM_BM - 1) / (2 * GEMM_BM);
+  const int n_tiles = m_tiles * n_tiles_n;
+  const int kblocks = (K + BK - 1) / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < PAIR_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 2 * 4);  // one arrival per epilogue warp of the pair
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    if (DUAL_B) tma_prefetch_desc(&tmB2);
+  }
+  if (warp == 5) {
+    tmem_alloc_pair(tmem_slot, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      // ---------------- TMA producer (both CTAs)
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int t = pair; t < n_tiles && ok; t += n_pairs) {
+        const int mt = t % m_tiles;
+        const int nt = t / m_tiles;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait_cluster(&empty[s], ph ^ 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * PAIR_STAGE_BYTES);
+          const uint32_t bar = map_shared_to_rank(&full[s], 0);
+          tma_load_2d_pair(sA + s * A_BYTES, &tmA, bar, kb * BK,
+                           mt * 2 * GEMM_BM + static_cast<int>(rank) * GEMM_BM);
+          if (DUAL_B)
+            tma_load_2d_pair(sB + s * BH_BYTES, rank == 0 ? &tmB : &tmB2, bar, kb * BK,
+                             nt * (BN / 2));
+          else
+            tma_load_2d_pair(sB + s * BH_BYTES, &tmB, bar, kb * BK,
+                             nt * BN + static_cast<int>(rank) * (BN / 2));
+          if (++s == PAIR_STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+      }
+      if (!ok) sleep_ns(50000);  // let the loads already issued land
+    }
+  } else if (warp == 5) {
+    if (lane == 0 && rank == 0) {
+      // ---------------- MMA issuer (leader CTA)
+      int s = 0;
+      uint32_t ph = 0;
+      int local = 0;
+      bool ok = true;
+      for (int t = pair; t < n_tiles && ok; t += n_pairs, ++local) {
+        const int buf = local & 1;
+        const uint32_t use = static_cast<uint32_t>(local >> 1);
+        if (!mbar_wait_cluster(&tempty[buf], (use & 1) ^ 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + buf * BN;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait_cluster(&full[s], ph, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(sA + s * A_BYTES);
+          const uint32_t b_base = smem_u32(sB + s * BH_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < 128 / UK_BYTES; ++kk) {
+            const uint64_t ad = sdesc_kmajor_sw128(a_base + kk * UK_BYTES);
+            const uint64_t bd = sdesc_kmajor_sw128(b_base + kk * UK_BYTES);
+            if (FP8)
+              umma_f8_pair(d_tmem, ad, bd, IDESC, (kb | kk) != 0);
+            else
+              umma_bf16_pair(d_tmem, ad, bd, IDESC, (kb | kk) != 0);
+          }
+          umma_commit_pair_both(&empty[s]);
+          if (++s == PAIR_STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+        if (ok) umma_commit_pair_both(&tfull[buf]);
+      }
+      umma_commit_pair_both(drain);
+      mbar_wait_cluster(drain, 0, nullptr, WAIT_LIMIT_NS / 4);
+    }
+  } else {
+    // ---------------- epilogue warps 0..3 (both CTAs, own 128 rows)
+    const int r = warp * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t tempty_leader0 = map_shared_to_rank(&tempty[0], 0);
+    const uint32_t tempty_leader1 = map_shared_to_rank(&tempty[1], 0);
+    int local = 0;
+    for (int t = pair; t < n_tiles; t += n_pairs, ++local) {
+      const int buf = local & 1;
+      const uint32_t use = static_cast<uint32_t>(local >> 1);
+      const bool ok = mbar_wait_cluster(&tfull[buf], use & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const int mt = t % m_tiles;
+      const int nt = t / m_tiles;
+      epi(mt * 2 * GEMM_BM + static_cast<int>(rank) * GEMM_BM, nt * BN,
+          tmem_base + lane_base + buf * BN, r);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(buf ? tempty_leader1 : tempty_leader0);
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  if (warp == 5) tmem_dealloc_pair(tmem_base, TMEM_COLS);
 }
 
 }  // namespace ig4
