@@ -313,7 +313,9 @@ ig4_status launch_attention(int B, int H, int L, const void *q, const void *k, c
   const long BH = static_cast<long>(B) * H;
   IG4_TRY(map_3d_bf16(&mq, q, 256, L, BH, 256, static_cast<long>(L) * 256, 64, ATT_BM));
   IG4_TRY(map_3d_bf16(&mk, k, 256, L, BH, 256, static_cast<long>(L) * 256, 64, ATT_BN));
-  IG4_TRY(map_3d_bf16(&mv, vt, L, 256, BH, vt_ld, 256L * vt_ld, ATT_BN, 256));
+  // V^T boxes are 64 keys (128 bytes, the swizzle span) x 256 head dims; a
+  // 128-key tile takes two of them.
+  IG4_TRY(map_3d_bf16(&mv, vt, L, 256, BH, vt_ld, 256L * vt_ld, 64, 256));
   IG4_TRY(allow_smem(attention_kernel, ATT_SMEM_BYTES));
   dim3 grid((L + ATT_BM - 1) / ATT_BM, H, B);
   attention_kernel<<<grid, ATT_THREADS, ATT_SMEM_BYTES, st>>>(

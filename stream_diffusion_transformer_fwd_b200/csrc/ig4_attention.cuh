@@ -1,19 +1,38 @@
 // ig4_attention.cuh - fused flash-style joint attention, head_dim 256, sm_100a.
 //
-// One CTA computes o for 128 query rows of one (sample, head):
-//   S_j = Q K_j^T (tcgen05, fp32 in TMEM, two 64-column buffers),
-//   online softmax in registers (one thread per query row, log2 domain),
-//   P_j (bf16) written to shared memory in the MMA operand layout,
-//   O += P_j V_j (tcgen05, fp32 in TMEM, 256 columns).
-// V arrives transposed ([256, keys], keys contiguous) so that every operand
-// is K-major with the 128-byte swizzle.  The running maximum used for the
-// exponentials is only moved when a row's maximum grows by more than 2^8
-// (in exp2 units), so O in TMEM is rescaled rarely; since the same maximum
-// is used for the numerator and the denominator the result is unchanged.
+// One CTA computes o for 128 query rows of one (sample, head), walking the
+// keys in tiles of 128:
+//   S_j = Q K_j^T     16 tcgen05.mma (M=128, N=128, K=16) with A = Q read from
+//                     TMEM and B = K_j from shared memory; fp32 scores in TMEM;
+//   softmax           one thread per query row, exp2 domain, in registers;
+//   P_j               bf16 into shared memory in the MMA operand layout;
+//   O += P_j V_j      8 tcgen05.mma (M=128, N=256, K=16), O (fp32) in TMEM.
+// 128-key tiles keep every MMA at N >= 128, the width at which an MMA runs
+// at the full tensor rate (N = 64 instructions take ~1.5x their ideal time).
+// Q sits in TMEM as the A operand of the scores, so the scores read only K
+// from shared memory.
 //
-// Warp roles (192 threads): warps 0-3 softmax + output, warp 4 TMA loads
-// (Q once, K_j and V_j through a 2-stage ring), warp 5 TMEM allocation and
-// the MMA issue order S_0, S_1, PV_0, S_2, PV_1, ...
+// TMEM (512 columns): Q as bf16 pairs [0,128), one S buffer [128,256), O
+// [256,512).  S_{j+1} is issued as soon as the softmax has read S_j out of
+// TMEM (not when P_j is ready), so the scores of the next tile are computed
+// while the exponentials of this one run.
+//
+// Shared memory: one ring of three 64 KB slots filled by TMA in the order the
+// MMAs consume them - Q, K_0, K_1, V_0, K_2, V_1, K_3, V_2, ... - plus one
+// 32 KB P buffer.  V arrives transposed ([256, keys], keys contiguous), so
+// every operand is K-major with the 128-byte swizzle.
+//
+// The running maximum used for the exponentials only moves when a row's
+// maximum grows by more than 8 (a factor 2^8), so O is rescaled rarely;
+// numerator and denominator use the same maximum, so the result is unchanged.
+//
+// Warp roles (192 threads): warps 0-3 softmax + output (warp w owns TMEM
+// lanes / query rows 32w..32w+31), warp 4 TMA producer, warp 5 TMEM
+// allocation and MMA issue: S_0, S_1, PV_0, S_2, PV_1, ...
+//
+// Barrier parity: every barrier a role waits on completes at most one phase
+// ahead of that wait, so try_wait.parity never mistakes a later phase for the
+// awaited one.  Every wait is bounded.
 #pragma once
 
 #include "ig4_ptx.cuh"
@@ -21,23 +40,46 @@
 namespace ig4 {
 
 constexpr int ATT_BM = 128;
-constexpr int ATT_BN = 64;
+constexpr int ATT_BN = 128;   // keys per tile
 constexpr int ATT_DH = 256;
 constexpr int ATT_THREADS = 192;
-constexpr int ATT_Q_BYTES = ATT_BM * ATT_DH * 2;      // 64 KB: 4 chunks of [128 x 128 B]
-constexpr int ATT_K_BYTES = ATT_BN * ATT_DH * 2;      // 32 KB: 4 chunks of [64 x 128 B]
-constexpr int ATT_V_BYTES = ATT_DH * ATT_BN * 2;      // 32 KB: [256 x 128 B]
-constexpr int ATT_P_BYTES = ATT_BM * ATT_BN * 2;      // 16 KB: [128 x 128 B]
-constexpr int ATT_OFF_K = ATT_Q_BYTES;
-constexpr int ATT_OFF_V = ATT_OFF_K + 2 * ATT_K_BYTES;
-constexpr int ATT_OFF_P = ATT_OFF_V + 2 * ATT_V_BYTES;
+constexpr int ATT_SLOTS = 3;
+constexpr int ATT_SLOT_BYTES = 65536;                  // Q, K_j (4 chunks [128 x 128 B]) or
+                                                       // V_j^T (2 chunks [256 x 128 B])
+constexpr int ATT_P_BYTES = ATT_BM * ATT_BN * 2;       // 32 KB: 2 chunks [128 x 128 B]
+constexpr int ATT_OFF_P = ATT_SLOTS * ATT_SLOT_BYTES;
 constexpr int ATT_OFF_BAR = ATT_OFF_P + ATT_P_BYTES;
 constexpr int ATT_SMEM_BYTES = ATT_OFF_BAR + 256 + 1024;
 constexpr uint32_t ATT_TMEM_COLS = 512;
+constexpr uint32_t ATT_TMEM_Q = 0;
+constexpr uint32_t ATT_TMEM_S = 128;
 constexpr uint32_t ATT_TMEM_O = 256;
 // log2(e) / sqrt(256)
 constexpr float ATT_SCALE_LOG2 = 0.09016844005556021f;
 constexpr float ATT_RESCALE_THRESHOLD = 8.0f;
+
+// The ring's load / consumption order: item 0 is Q; then K_0, K_1 (if any);
+// then, for each tile j, V_j followed by K_{j+2} (if that tile exists).
+// kind(): 0 = Q, 1 = K, 2 = V, with the tile index in *tile.
+struct AttRing {
+  int nkv;
+  __device__ __forceinline__ int items() const { return 1 + 2 * nkv; }
+  __device__ __forceinline__ int kind(int i, int *tile) const {
+    if (i == 0) { *tile = 0; return 0; }
+    if (i == 1) { *tile = 0; return 1; }
+    if (nkv == 1) { *tile = 0; return 2; }  // items: Q, K_0, V_0
+    if (i == 2) { *tile = 1; return 1; }
+    // items from 3 on: V_0, K_2, V_1, K_3, ..., V_{nkv-3}, K_{nkv-1}, V_{nkv-2}, V_{nkv-1}
+    const int k = i - 3;
+    const int pairs = nkv - 2;  // (V_j, K_{j+2}) for j < nkv - 2
+    if (k < 2 * pairs) {
+      *tile = (k & 1) ? (k >> 1) + 2 : (k >> 1);
+      return (k & 1) ? 1 : 2;
+    }
+    *tile = (nkv - 2) + (k - 2 * pairs);
+    return 2;
+  }
+};
 
 __global__ void __launch_bounds__(ATT_THREADS, 1)
     attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -46,21 +88,17 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t *sQ = smem;
-  uint8_t *sK = smem + ATT_OFF_K;
-  uint8_t *sV = smem + ATT_OFF_V;
   uint8_t *sP = smem + ATT_OFF_P;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + ATT_OFF_BAR);
-  uint64_t *q_full = bars + 0;
-  uint64_t *k_full = bars + 1;   // [2]
-  uint64_t *k_empty = bars + 3;  // [2]
-  uint64_t *v_full = bars + 5;   // [2]
-  uint64_t *v_empty = bars + 7;  // [2]
-  uint64_t *s_full = bars + 9;   // [2]
-  uint64_t *p_full = bars + 11;
-  uint64_t *pv_done = bars + 12;
-  uint64_t *drain = bars + 13;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 14);
+  uint64_t *full = bars + 0;     // [ATT_SLOTS]
+  uint64_t *empty = bars + 3;    // [ATT_SLOTS]
+  uint64_t *s_full = bars + 6;   // S_j in TMEM
+  uint64_t *s_free = bars + 7;   // S_j read out of TMEM (one arrival per softmax warp)
+  uint64_t *p_full = bars + 8;   // P_j in shared memory (one arrival per softmax warp)
+  uint64_t *pv_done = bars + 9;  // PV_j (and every earlier MMA) complete
+  uint64_t *q_tmem = bars + 10;  // Q copied into TMEM (one arrival per softmax warp)
+  uint64_t *drain = bars + 11;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 12);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -70,18 +108,18 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   const int b = blockIdx.z;
   const int bh = b * H + h;
   const int nkv = (L + ATT_BN - 1) / ATT_BN;
+  const AttRing ring{nkv};
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&k_full[s], 1);
-      mbar_init(&k_empty[s], 1);
-      mbar_init(&v_full[s], 1);
-      mbar_init(&v_empty[s], 1);
-      mbar_init(&s_full[s], 1);
+    for (int s = 0; s < ATT_SLOTS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
     }
-    mbar_init(p_full, 128);
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 4);
+    mbar_init(p_full, 4);
     mbar_init(pv_done, 1);
+    mbar_init(q_tmem, 4);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -103,30 +141,32 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   if (warp == 4) {
     if (lane == 0) {
       // ------------------------------------------------ TMA producer
-      long issued_k = 0, issued_v = 0;
+      const int n = ring.items();
+      int i = 0;
       bool ok = true;
-      mbar_arrive_expect_tx(q_full, ATT_Q_BYTES);
-      for (int c = 0; c < 4; ++c) tma_load_3d(sQ + c * (ATT_BM * 128), &tmQ, q_full, c * 64, q0, bh);
-      for (int j = 0; j < nkv && ok; ++j) {
-        const int s = j & 1;
-        const uint32_t ph = static_cast<uint32_t>(j >> 1) & 1;
-        if (!mbar_wait(&k_empty[s], ph ^ 1, abort_flag)) { ok = false; break; }
-        mbar_arrive_expect_tx(&k_full[s], ATT_K_BYTES);
-        for (int c = 0; c < 4; ++c)
-          tma_load_3d(sK + s * ATT_K_BYTES + c * (ATT_BN * 128), &tmK, &k_full[s], c * 64,
-                      j * ATT_BN, bh);
-        ++issued_k;
-        if (!mbar_wait(&v_empty[s], ph ^ 1, abort_flag)) { ok = false; break; }
-        mbar_arrive_expect_tx(&v_full[s], ATT_V_BYTES);
-        tma_load_3d(sV + s * ATT_V_BYTES, &tmV, &v_full[s], j * ATT_BN, 0, bh);
-        ++issued_v;
+      for (; i < n; ++i) {
+        const int slot = i % ATT_SLOTS;
+        const uint32_t ph = static_cast<uint32_t>(i / ATT_SLOTS) & 1;
+        if (!mbar_wait(&empty[slot], ph ^ 1, abort_flag)) { ok = false; break; }
+        mbar_arrive_expect_tx(&full[slot], ATT_SLOT_BYTES);
+        uint8_t *dst = smem + slot * ATT_SLOT_BYTES;
+        int t = 0;
+        const int kind = ring.kind(i, &t);
+        if (kind == 0) {
+          for (int c = 0; c < 4; ++c) tma_load_3d(dst + c * 16384, &tmQ, &full[slot], c * 64, q0, bh);
+        } else if (kind == 1) {
+          for (int c = 0; c < 4; ++c)
+            tma_load_3d(dst + c * 16384, &tmK, &full[slot], c * 64, t * ATT_BN, bh);
+        } else {
+          for (int c = 0; c < 2; ++c)
+            tma_load_3d(dst + c * 32768, &tmV, &full[slot], t * ATT_BN + c * 64, 0, bh);
+        }
       }
       if (!ok) {
-        mbar_wait(q_full, 0, nullptr, WAIT_LIMIT_NS / 4);
-        for (long i = (issued_k > 2 ? issued_k - 2 : 0); i < issued_k; ++i)
-          mbar_wait(&k_full[i & 1], static_cast<uint32_t>(i >> 1) & 1, nullptr, WAIT_LIMIT_NS / 4);
-        for (long i = (issued_v > 2 ? issued_v - 2 : 0); i < issued_v; ++i)
-          mbar_wait(&v_full[i & 1], static_cast<uint32_t>(i >> 1) & 1, nullptr, WAIT_LIMIT_NS / 4);
+        // let the loads already issued land before the shared memory goes away
+        for (int k = (i > ATT_SLOTS ? i - ATT_SLOTS : 0); k < i; ++k)
+          mbar_wait(&full[k % ATT_SLOTS], static_cast<uint32_t>(k / ATT_SLOTS) & 1, nullptr,
+                    WAIT_LIMIT_NS / 4);
       }
     }
   } else if (warp == 5) {
@@ -134,43 +174,53 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       // ------------------------------------------------ MMA issuer
       constexpr uint32_t IDESC_S = idesc_bf16(ATT_BM, ATT_BN);
       constexpr uint32_t IDESC_PV = idesc_bf16(ATT_BM, ATT_DH);
-      const uint32_t q_base = smem_u32(sQ);
       const uint32_t p_base = smem_u32(sP);
-      bool ok = mbar_wait(q_full, 0, abort_flag);
-      auto issue_s = [&](int j) -> bool {
-        const int s = j & 1;
-        const uint32_t ph = static_cast<uint32_t>(j >> 1) & 1;
-        if (!mbar_wait(&k_full[s], ph, abort_flag)) return false;
+      int item = 1;  // ring item consumed next (item 0, Q, is read by the softmax warps)
+      bool ok = mbar_wait(q_tmem, 0, abort_flag);
+      if (ok) mbar_arrive(&empty[0]);  // Q's slot is free once Q is in TMEM
+      auto take = [&](uint32_t *base) -> bool {
+        const int slot = item % ATT_SLOTS;
+        if (!mbar_wait(&full[slot], static_cast<uint32_t>(item / ATT_SLOTS) & 1, abort_flag))
+          return false;
         tc_fence_after();
-        const uint32_t k_base = smem_u32(sK + s * ATT_K_BYTES);
-#pragma unroll
-        for (int kk = 0; kk < ATT_DH / 16; ++kk) {
-          const uint64_t ad = sdesc_kmajor_sw128(q_base + (kk >> 2) * (ATT_BM * 128) + (kk & 3) * 32);
-          const uint64_t bd = sdesc_kmajor_sw128(k_base + (kk >> 2) * (ATT_BN * 128) + (kk & 3) * 32);
-          umma_bf16(tmem + s * ATT_BN, ad, bd, IDESC_S, kk > 0);
-        }
-        umma_commit(&k_empty[s]);
-        umma_commit(&s_full[s]);
+        *base = smem_u32(smem + slot * ATT_SLOT_BYTES);
         return true;
       };
-      if (ok) ok = issue_s(0);
-      if (ok && nkv > 1) ok = issue_s(1);
+      auto give = [&]() {
+        umma_commit(&empty[item % ATT_SLOTS]);
+        ++item;
+      };
+      auto issue_s = [&]() -> bool {  // S_j into the S buffer, K_j from the ring
+        uint32_t k_base;
+        if (!take(&k_base)) return false;
+#pragma unroll
+        for (int kk = 0; kk < ATT_DH / 16; ++kk) {
+          const uint64_t bd = sdesc_kmajor_sw128(k_base + (kk >> 2) * 16384 + (kk & 3) * 32);
+          umma_bf16_ts(tmem + ATT_TMEM_S, tmem + ATT_TMEM_Q + kk * 8, bd, IDESC_S, kk > 0);
+        }
+        give();
+        umma_commit(s_full);
+        return true;
+      };
+      if (ok) ok = issue_s();  // S_0
       for (int j = 0; j < nkv && ok; ++j) {
-        const int s = j & 1;
-        const uint32_t ph = static_cast<uint32_t>(j >> 1) & 1;
+        // S_{j+1} as soon as S_j has been read out of TMEM
+        if (j + 1 < nkv) {
+          if (!mbar_wait(s_free, static_cast<uint32_t>(j) & 1, abort_flag)) break;
+          if (!(ok = issue_s())) break;
+        }
+        // PV_j once P_j is in shared memory
         if (!mbar_wait(p_full, static_cast<uint32_t>(j) & 1, abort_flag)) break;
-        if (!mbar_wait(&v_full[s], ph, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t v_base = smem_u32(sV + s * ATT_V_BYTES);
+        uint32_t v_base;
+        if (!(ok = take(&v_base))) break;
 #pragma unroll
         for (int kk = 0; kk < ATT_BN / 16; ++kk) {
-          const uint64_t ad = sdesc_kmajor_sw128(p_base + kk * 32);
-          const uint64_t bd = sdesc_kmajor_sw128(v_base + kk * 32);
+          const uint64_t ad = sdesc_kmajor_sw128(p_base + (kk >> 2) * 16384 + (kk & 3) * 32);
+          const uint64_t bd = sdesc_kmajor_sw128(v_base + (kk >> 2) * 32768 + (kk & 3) * 32);
           umma_bf16(tmem + ATT_TMEM_O, ad, bd, IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&v_empty[s]);
+        give();
         umma_commit(pv_done);
-        if (j + 2 < nkv) ok = issue_s(j + 2);
       }
       umma_commit(drain);
       mbar_wait(drain, 0, nullptr, WAIT_LIMIT_NS / 4);
@@ -181,38 +231,74 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     float m_used = -INFINITY;
     float l_sum = 0.0f;
-    bool ok = true;
-    uint8_t *prow = sP + r * 128;
-    for (int j = 0; j < nkv; ++j) {
-      const int s = j & 1;
-      const uint32_t ph = static_cast<uint32_t>(j >> 1) & 1;
-      if (!mbar_wait_warp(&s_full[s], ph, abort_flag)) { ok = false; break; }
+    bool ok = mbar_wait_warp(&full[0], 0, abort_flag);  // Q (ring item 0)
+    if (ok) {
+      // Q row r: four 64-column chunks of 128 bytes in the 128-byte-swizzled
+      // TMA layout -> TMEM columns [ATT_TMEM_Q + 32c, +32), bf16 pairs.
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        const uint8_t *qrow = smem + c * 16384 + r * 128;
+        uint32_t w[32];
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          const uint4 v = *reinterpret_cast<const uint4 *>(qrow + ((g ^ (r & 7)) << 4));
+          w[4 * g + 0] = v.x;
+          w[4 * g + 1] = v.y;
+          w[4 * g + 2] = v.z;
+          w[4 * g + 3] = v.w;
+        }
+        tmem_st32_u(tmem + lane_base + ATT_TMEM_Q + c * 32, w);
+      }
+      tmem_st_wait();
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(q_tmem);
+
+    for (int j = 0; j < nkv && ok; ++j) {
+      if (!mbar_wait_warp(s_full, static_cast<uint32_t>(j) & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      float t[64];
-      {
-        float a[32], c[32];
-        tmem_ld32(tmem + lane_base + s * ATT_BN, a);
-        tmem_ld32(tmem + lane_base + s * ATT_BN + 32, c);
+      float t[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float a[32];
+        tmem_ld32(tmem + lane_base + ATT_TMEM_S + c * 32, a);
         tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          t[i] = a[i] * ATT_SCALE_LOG2;
-          t[32 + i] = c[i] * ATT_SCALE_LOG2;
-        }
+        for (int i = 0; i < 32; ++i) t[32 * c + i] = a[i];
       }
+      // S_j is in registers: the S buffer may take S_{j+1}.
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free);
+
       const int kbase = j * ATT_BN;
       if (kbase + ATT_BN > L) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i)
+        for (int i = 0; i < 128; ++i)
           if (kbase + i >= L) t[i] = -INFINITY;
       }
-      float mx = t[0];
+      float m16[16];
 #pragma unroll
-      for (int i = 1; i < 64; ++i) mx = fmaxf(mx, t[i]);
+      for (int q = 0; q < 16; ++q) {
+        const float a0 = fmaxf(t[8 * q + 0], t[8 * q + 1]);
+        const float a1 = fmaxf(t[8 * q + 2], t[8 * q + 3]);
+        const float a2 = fmaxf(t[8 * q + 4], t[8 * q + 5]);
+        const float a3 = fmaxf(t[8 * q + 6], t[8 * q + 7]);
+        m16[q] = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) m16[q] = fmaxf(m16[q], m16[q + 8]);
+      const float mx = fmaxf(fmaxf(fmaxf(m16[0], m16[1]), fmaxf(m16[2], m16[3])),
+                             fmaxf(fmaxf(m16[4], m16[5]), fmaxf(m16[6], m16[7]))) *
+                       ATT_SCALE_LOG2;
 
       if (j > 0) {
-        // PV_{j-1} must be done: it reads P (single buffer) and writes O.
-        if (!mbar_wait_warp(pv_done, static_cast<uint32_t>(j - 1) & 1, abort_flag)) { ok = false; break; }
+        // PV_{j-1} must be done: it reads the P buffer and writes O.
+        if (!mbar_wait_warp(pv_done, static_cast<uint32_t>(j - 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         const bool need = mx > m_used + ATT_RESCALE_THRESHOLD;
         if (__any_sync(0xffffffffu, need)) {
@@ -234,28 +320,33 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         m_used = mx;
       }
 
-      float rowsum = 0.0f;
+      const float neg_m = -m_used;
+      float sums[16];
 #pragma unroll
-      for (int g = 0; g < 8; ++g) {
+      for (int g = 0; g < 16; ++g) {
         float p[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          p[e] = exp2_approx(t[8 * g + e] - m_used);
-          rowsum += p[e];
-        }
+        for (int e = 0; e < 8; ++e) p[e] = exp2_approx(fmaf(t[8 * g + e], ATT_SCALE_LOG2, neg_m));
+        sums[g] = ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
         uint4 w;
         w.x = pack_bf16x2(p[0], p[1]);
         w.y = pack_bf16x2(p[2], p[3]);
         w.z = pack_bf16x2(p[4], p[5]);
         w.w = pack_bf16x2(p[6], p[7]);
-        *reinterpret_cast<uint4 *>(prow + ((g ^ (r & 7)) << 4)) = w;
+        // key chunk g/8 (64 keys), 16-byte piece g%8 of row r, swizzled
+        *reinterpret_cast<uint4 *>(sP + (g >> 3) * 16384 + r * 128 + (((g & 7) ^ (r & 7)) << 4)) = w;
       }
-      l_sum += rowsum;
+#pragma unroll
+      for (int g = 0; g < 8; ++g) sums[g] += sums[g + 8];
+      l_sum += ((sums[0] + sums[1]) + (sums[2] + sums[3])) + ((sums[4] + sums[5]) + (sums[6] + sums[7]));
+      // this thread's P writes -> async proxy; then one arrival per warp
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(p_full);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
     }
-    if (ok && mbar_wait_warp(pv_done, static_cast<uint32_t>(nkv - 1) & 1, abort_flag)) {
+    const int jl = nkv - 1;
+    if (ok && mbar_wait_warp(pv_done, static_cast<uint32_t>(jl) & 1, abort_flag)) {
       tc_fence_after();
       const int lq = q0 + r;
       const bool valid = lq < L;
