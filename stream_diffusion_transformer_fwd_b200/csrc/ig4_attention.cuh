@@ -25,6 +25,9 @@
 // The running maximum used for the exponentials only moves when a row's
 // maximum grows by more than 8 (a factor 2^8), so O is rescaled rarely;
 // numerator and denominator use the same maximum, so the result is unchanged.
+// The softmax computes a tile's exponentials (into packed bf16 registers)
+// before it waits for the previous PV product, and only the store of P into
+// the single P buffer (and the rare O rescale) waits for it.
 //
 // Warp roles (192 threads): warps 0-3 softmax + output (warp w owns TMEM
 // lanes / query rows 32w..32w+31), warp 4 TMA producer, warp 5 TMEM
@@ -293,6 +296,41 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                              fmaxf(fmaxf(m16[4], m16[5]), fmaxf(m16[6], m16[7]))) *
                        ATT_SCALE_LOG2;
 
+      // Running maximum for this tile (moved only when it grows by more than
+      // the threshold) and the factor that rescales what came before.
+      float m_new = m_used;
+      float f = 1.0f;
+      bool need = false;
+      if (j == 0) {
+        m_new = mx;
+      } else if (mx > m_used + ATT_RESCALE_THRESHOLD) {
+        need = true;
+        m_new = mx;
+        f = exp2_approx(m_used - mx);
+      }
+      const bool any_need = __any_sync(0xffffffffu, need);
+
+      // Exponentials into packed bf16 registers first: they need neither
+      // PV_{j-1} nor the P buffer, so they overlap the tensor core's work.
+      const float neg_m = -m_new;
+      uint32_t pk[64];
+      float sums[16];
+#pragma unroll
+      for (int g = 0; g < 16; ++g) {
+        float p[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) p[e] = exp2_approx(fmaf(t[8 * g + e], ATT_SCALE_LOG2, neg_m));
+        sums[g] = ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
+        pk[4 * g + 0] = pack_bf16x2(p[0], p[1]);
+        pk[4 * g + 1] = pack_bf16x2(p[2], p[3]);
+        pk[4 * g + 2] = pack_bf16x2(p[4], p[5]);
+        pk[4 * g + 3] = pack_bf16x2(p[6], p[7]);
+      }
+#pragma unroll
+      for (int g = 0; g < 8; ++g) sums[g] += sums[g + 8];
+      const float rowsum =
+          ((sums[0] + sums[1]) + (sums[2] + sums[3])) + ((sums[4] + sums[5]) + (sums[6] + sums[7]));
+
       if (j > 0) {
         // PV_{j-1} must be done: it reads the P buffer and writes O.
         if (!mbar_wait_warp(pv_done, static_cast<uint32_t>(j - 1) & 1, abort_flag)) {
@@ -300,11 +338,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           break;
         }
         tc_fence_after();
-        const bool need = mx > m_used + ATT_RESCALE_THRESHOLD;
-        if (__any_sync(0xffffffffu, need)) {
-          const float f = need ? exp2_approx(m_used - mx) : 1.0f;
-          if (need) m_used = mx;
-          l_sum *= f;
+        if (any_need) {
 #pragma unroll 1
           for (int c = 0; c < ATT_DH; c += 32) {
             float o[32];
@@ -316,29 +350,16 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           }
           tmem_st_wait();
         }
-      } else {
-        m_used = mx;
       }
+      l_sum = l_sum * f + rowsum;
+      m_used = m_new;
 
-      const float neg_m = -m_used;
-      float sums[16];
 #pragma unroll
       for (int g = 0; g < 16; ++g) {
-        float p[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) p[e] = exp2_approx(fmaf(t[8 * g + e], ATT_SCALE_LOG2, neg_m));
-        sums[g] = ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
-        uint4 w;
-        w.x = pack_bf16x2(p[0], p[1]);
-        w.y = pack_bf16x2(p[2], p[3]);
-        w.z = pack_bf16x2(p[4], p[5]);
-        w.w = pack_bf16x2(p[6], p[7]);
         // key chunk g/8 (64 keys), 16-byte piece g%8 of row r, swizzled
-        *reinterpret_cast<uint4 *>(sP + (g >> 3) * 16384 + r * 128 + (((g & 7) ^ (r & 7)) << 4)) = w;
+        *reinterpret_cast<uint4 *>(sP + (g >> 3) * 16384 + r * 128 + (((g & 7) ^ (r & 7)) << 4)) =
+            make_uint4(pk[4 * g + 0], pk[4 * g + 1], pk[4 * g + 2], pk[4 * g + 3]);
       }
-#pragma unroll
-      for (int g = 0; g < 8; ++g) sums[g] += sums[g + 8];
-      l_sum += ((sums[0] + sums[1]) + (sums[2] + sums[3])) + ((sums[4] + sums[5]) + (sums[6] + sums[7]));
       // this thread's P writes -> async proxy; then one arrival per warp
       fence_proxy_async_smem();
       tc_fence_before();
