@@ -178,6 +178,61 @@ class ClockSampler:
 
 # ----------------------------------------------------------------- our arm
 
+def e2e_pipelined(host_in, out_like, step_fn, steps, warmup):
+    """End-to-end time of `steps` calls through the C ABI, each with its own
+    host->device copy of the inputs (pinned host memory) and device->host copy
+    of the result.  Two device buffer sets let the copies of neighbouring
+    steps overlap the compute of the current one (separate copy streams); the
+    timed region runs from before the first input copy to after the last
+    result copy.  Returns (ms, h2d bytes per step, d2h bytes per step)."""
+    import torch
+
+    comp = torch.cuda.current_stream()
+    h2d_st = torch.cuda.Stream()
+    d2h_st = torch.cuda.Stream()
+    hin = [[t.pin_memory() for t in host_in] for _ in range(2)]
+    din = [[torch.empty_like(t, device=out_like.device) for t in host_in] for _ in range(2)]
+    dout = [torch.empty_like(out_like) for _ in range(2)]
+    hout = [torch.empty(out_like.shape, dtype=out_like.dtype).pin_memory() for _ in range(2)]
+    ev_h2d = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_d2h = [torch.cuda.Event() for _ in range(2)]
+
+    def run(n):
+        for i in range(n):
+            b = i % 2
+            with torch.cuda.stream(h2d_st):
+                if i >= 2:
+                    h2d_st.wait_event(ev_comp[b])  # step i-2 has finished reading din[b]
+                for d, h in zip(din[b], hin[b]):
+                    d.copy_(h, non_blocking=True)
+                ev_h2d[b].record(h2d_st)
+            comp.wait_event(ev_h2d[b])
+            if i >= 2:
+                comp.wait_event(ev_d2h[b])  # step i-2's result has left dout[b]
+            step_fn(din[b], dout[b])
+            ev_comp[b].record(comp)
+            with torch.cuda.stream(d2h_st):
+                d2h_st.wait_event(ev_comp[b])
+                hout[b].copy_(dout[b], non_blocking=True)
+                ev_d2h[b].record(d2h_st)
+        for b in range(min(n, 2)):
+            comp.wait_event(ev_d2h[b])
+
+    run(warmup)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(comp)
+    h2d_st.wait_stream(comp)
+    run(steps)
+    e1.record(comp)
+    torch.cuda.synchronize()
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = out_like.numel() * out_like.element_size()
+    return e0.elapsed_time(e1), h2d, d2h
+
+
 def run_ours(args, rank, local_rank, world):
     import torch
     import torch.distributed as dist
@@ -196,6 +251,8 @@ def run_ours(args, rank, local_rank, world):
     from synth import CONFIGS, make_block_activations, make_block_weights
 
     cfg = CONFIGS[args.config]
+    if cfg.n_blocks > 1:
+        return run_stack(args, cfg, ig4, rank, world, dev)
     fp8 = cfg.w_dtype == "e4m3"
     names = KERNEL_NAMES_FP8 if fp8 else KERNEL_NAMES
     acts = make_block_activations(cfg, seed=rank)
@@ -243,35 +300,17 @@ def run_ours(args, rank, local_rank, world):
             per_kernel_ms[j] += evs[i][j].elapsed_time(evs[i][j + 1])
     per_kernel_ms = [t / K for t in per_kernel_ms]
 
-    # ---- end-to-end region: pinned host buffers, H2D inputs and D2H result each step
-    x_h = acts["x"].pin_memory()
-    temb_h = acts["temb"].pin_memory()
-    pos_h = ig4.ig4_mrope_positions(cfg.T_text, cfg.grid_t, cfg.grid_h, cfg.grid_w).pin_memory()
-    y_h = torch.empty_like(x_h).pin_memory()
-    x_d, temb_d, pos_d = torch.empty_like(x), torch.empty_like(temb), torch.empty_like(pos)
-    for _ in range(max(1, W // 2)):
-        x_d.copy_(x_h, non_blocking=True)
-        ig4.ig4_block_forward(c, bw, x_d, y, pos_d.copy_(pos_h, non_blocking=True),
-                              temb_d.copy_(temb_h, non_blocking=True), ws)
-        y_h.copy_(y, non_blocking=True)
-    torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
+    # ---- end-to-end region: every step copies its inputs from pinned host
+    # memory and reads its result back, pipelined over two buffer sets
+    pos_h = ig4.ig4_mrope_positions(cfg.T_text, cfg.grid_t, cfg.grid_h, cfg.grid_w)
+    host_in = [acts["x"], acts["temb"], pos_h]
+
+    def step_fn(dev_in, out):
+        ig4.ig4_block_forward(c, bw, dev_in[0], out, dev_in[2], dev_in[1], ws)
+
     if world > 1:
         dist.barrier()
-    torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(K):
-        x_d.copy_(x_h, non_blocking=True)
-        temb_d.copy_(temb_h, non_blocking=True)
-        pos_d.copy_(pos_h, non_blocking=True)
-        ig4.ig4_block_forward(c, bw, x_d, y, pos_d, temb_d, ws)
-        y_h.copy_(y, non_blocking=True)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    ms_e2e = e0.elapsed_time(e1)
-    h2d = x_h.numel() * x_h.element_size() + temb_h.numel() * 4 + pos_h.numel() * 4
-    d2h = y_h.numel() * y_h.element_size()
+    ms_e2e, h2d, d2h = e2e_pipelined(host_in, y, step_fn, K, max(1, W // 2))
 
     if world > 1:
         t = torch.tensor([ms_total, ms_e2e], dtype=torch.float64, device=dev)
@@ -360,6 +399,113 @@ def run_ours(args, rank, local_rank, world):
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e / K, 4)},
         "gpu_launches": n_launch * K,
         "cpu_baseline": cpu_base,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def stack_work(cfg):
+    """Algorithmic FLOPs of one stack call: the blocks, the latent in/out
+    projections and the final AdaLN."""
+    blk, _ = block_work(cfg)
+    N, C, D, A = cfg.n_img, cfg.latent_ch, cfg.D, cfg.adaln_dim
+    return cfg.n_blocks * blk + 2.0 * 2 * cfg.B * N * C * D + 4.0 * cfg.B * A * D
+
+
+def run_stack(args, cfg, ig4, rank, world, dev):
+    """One denoiser step of the 34-block stack per bench step."""
+    import torch
+    import torch.distributed as dist
+
+    from synth import make_block_weights_device, make_stack_inputs
+
+    fp8 = cfg.w_dtype == "e4m3"
+    st = make_stack_inputs(cfg, seed=rank)
+    sd = {k: (None if v is None else v.to(dev)) for k, v in st.items()}
+    blocks = [make_block_weights_device(cfg, rank, i, dev) for i in range(cfg.n_blocks)]
+    bws = [ig4.block_weights(b) for b in blocks]
+    sw = ig4.stack_weights(bws, sd["w_in"], sd["s_in"], sd["b_in"], sd["w_f"], sd["s_f"], sd["b_f"],
+                           sd["w_out"], sd["s_out"], sd["b_out"], cfg.latent_ch)
+    c = ig4.config_from(cfg)
+    pos = ig4.ig4_mrope_positions(cfg.T_text, cfg.grid_t, cfg.grid_h, cfg.grid_w, device=dev)
+    ws = torch.empty(ig4.ig4_stack_workspace_size(c, cfg.latent_ch), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(sd["x_latent"])
+    stream = torch.cuda.current_stream()
+    K, W = args.steps, args.warmup
+
+    def call(lat, text, temb, pos_, o):
+        ig4.ig4_stack_forward(c, sw, lat, text, o, pos_, temb, ws)
+
+    for _ in range(W):
+        call(sd["x_latent"], sd["text"], sd["temb"], pos, out)
+    torch.cuda.synchronize()
+    assert ig4.ig4_last_device_error() == ig4.IG4_OK
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(K):
+        call(sd["x_latent"], sd["text"], sd["temb"], pos, out)
+    end.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    err = ig4.ig4_last_device_error()
+    ms_total = start.elapsed_time(end)
+
+    host_in = [st["x_latent"], st["text"], st["temb"], pos.cpu()]
+
+    def step_fn(dev_in, o):
+        call(dev_in[0], dev_in[1], dev_in[2], dev_in[3], o)
+
+    if world > 1:
+        dist.barrier()
+    ms_e2e, h2d, d2h = e2e_pipelined(host_in, out, step_fn, K, 1)
+    if world > 1:
+        t = torch.tensor([ms_total, ms_e2e], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total, ms_e2e = t.tolist()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    flops = stack_work(cfg)
+    blk, per = block_work(cfg)
+    value = world * flops * K / (ms_total * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    held_max = bool(clocks) and clocks["sm_mhz"] >= 0.95 * clocks["sm_max_mhz"]
+    tkey = "bf16_tflops" if held_max else "bf16_tflops_sustained"
+    bf16_peak = peaks.get(tkey, FALLBACK_PEAKS[tkey])
+    # mixed bound: the GEMMs at the FP8 rate (2x bf16), attention at the bf16 rate
+    gemm_f = cfg.n_blocks * (blk - per["attention"] - per["adaln"])
+    attn_f = cfg.n_blocks * per["attention"]
+    t_min = gemm_f / ((2.0 if fp8 else 1.0) * bf16_peak * 1e12) + attn_f / (bf16_peak * 1e12)
+    mixed_peak = flops / t_min / 1e12
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": K, "warmup": W, "ms_per_step": round(ms_total / K, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8-e4m3 weights, bf16 activations" if fp8 else "bf16",
+        "data": "synthetic (seeded; block weights drawn on the GPU with a seeded generator)",
+        "config": {"workload": (f"{cfg.name}: {cfg.n_blocks}-block stack, B={cfg.B}, "
+                                f"{cfg.T_text} text + {cfg.grid_h}x{cfg.grid_w} image tokens, "
+                                f"latent {cfg.latent_ch} ch in/out, D={cfg.D}, w={cfg.w_dtype}"),
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2 (weights of 34 blocks per step)",
+                   "gflop_per_step": round(flops / 1e9, 1)},
+        "roofline": {"bound": "tensor", "achieved": round(value / world, 1),
+                     "peak": round(mixed_peak, 1), "unit": "TFLOP/s",
+                     "frac": round(value / world / mixed_peak, 4), "traffic": None,
+                     "kernel": "whole step (GEMMs at 2x and attention at 1x the " + tkey + ")",
+                     "peak_source": f"{tkey} ({peak_src}) x nominal fp8/bf16 ratio for the GEMMs"},
+        "clocks": clocks, "device_error": ig4.ig4_status_string(err),
+        "e2e": {"value": round(world * flops * K / (ms_e2e * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(ms_e2e / K, 3)},
+        "gpu_launches": K * (cfg.n_blocks * (11 if fp8 else 9) + (7 if fp8 else 5)),
+        "cpu_baseline": None,
     }
     print(json.dumps(line), flush=True)
     return 0

@@ -12,6 +12,7 @@ of a parity error.
 from .configs import CONFIGS, Config, get_config  # noqa: F401
 from .block_inputs import (  # noqa: F401
     make_block_weights,
+    make_block_weights_device,
     make_block_activations,
     make_stack_inputs,
     quantize_e4m3_per_channel,

@@ -97,6 +97,40 @@ def make_block_activations(cfg: Config, seed: int = 0) -> dict:
     return {"x": x, "temb": temb}
 
 
+def make_block_weights_device(cfg: Config, seed: int, block: int, device) -> dict:
+    """Weights of one block drawn on `device` with a seeded torch generator.
+
+    Same shapes, distributions and storage formats as make_block_weights
+    (E4M3 codes with per-output-channel scales for FP8), but not the same
+    values: meant for timing full-size stacks, whose 9.3e9 parameters would
+    take minutes to draw on the host.  Parity tests use make_block_weights.
+    """
+    D, I, A, dh = cfg.D, cfg.I, cfg.adaln_dim, cfg.head_dim
+    gen = torch.Generator(device=device)
+
+    def draw(name, n_out, n_in, std):
+        gen.manual_seed(zlib.crc32(f"{seed}/{block}/{name}".encode()))
+        w = torch.randn((n_out, n_in), generator=gen, device=device, dtype=torch.float32) * std
+        if cfg.w_dtype == "bf16":
+            return w.to(torch.bfloat16), None
+        amax = w.abs().amax(dim=1)
+        scale = torch.where(amax > 0, amax / E4M3_MAX, torch.ones_like(amax))
+        q = (w / scale[:, None]).clamp_(-E4M3_MAX, E4M3_MAX).to(torch.float8_e4m3fn)
+        return q, scale
+
+    out = {}
+    out["w_ada"], out["s_ada"] = draw("w_ada", 6 * D, A, 0.02)
+    out["b_ada"] = torch.zeros(6 * D, device=device)
+    out["w_qkv"], out["s_qkv"] = draw("w_qkv", 3 * D, D, 1.0 / np.sqrt(D))
+    out["w_o"], out["s_o"] = draw("w_o", D, D, 1.0 / np.sqrt(D))
+    out["w_gate"], out["s_gate"] = draw("w_gate", I, D, 1.0 / np.sqrt(D))
+    out["w_up"], out["s_up"] = draw("w_up", I, D, 1.0 / np.sqrt(D))
+    out["w_down"], out["s_down"] = draw("w_down", D, I, 1.0 / np.sqrt(I))
+    out["g_q"] = torch.ones(dh, device=device)
+    out["g_k"] = torch.ones(dh, device=device)
+    return out
+
+
 def make_stack_inputs(cfg: Config, seed: int = 0, stress: bool = False) -> dict:
     """Stack-level inputs: latents [B, N, C] and text [B, T, D] (x_dtype), temb fp32,
     in-proj w_in [D, C] / b_in, final AdaLN w_f [2D, A] / b_f, out-proj w_out [C, D] /
