@@ -2,40 +2,42 @@
 //
 // One CTA computes o for 128 query rows of one (sample, head), walking the
 // keys in tiles of 128:
-//   S_j = Q K_j^T     16 tcgen05.mma (M=128, N=128, K=16) with A = Q read from
-//                     TMEM and B = K_j from shared memory; fp32 scores in TMEM;
+//   S_j = Q K_j^T     16 tcgen05.mma (M=128, N=128, K=16), Q and K_j from
+//                     shared memory, fp32 scores into TMEM;
 //   softmax           one thread per query row, exp2 domain, in registers;
-//   P_j               bf16 into shared memory in the MMA operand layout;
-//   O += P_j V_j      8 tcgen05.mma (M=128, N=256, K=16), O (fp32) in TMEM.
-// 128-key tiles keep every MMA at N >= 128, the width at which an MMA runs
-// at the full tensor rate (N = 64 instructions take ~1.5x their ideal time).
-// Q sits in TMEM as the A operand of the scores, so the scores read only K
-// from shared memory.
+//   P_j               bf16, written into TMEM (tcgen05.st), two buffers;
+//   O += P_j V_j      8 tcgen05.mma (M=128, N=256, K=16) with A = P_j read
+//                     from TMEM and B = V_j from shared memory; O (fp32) in TMEM.
+// 128-key tiles keep every MMA at N >= 128, the width at which an MMA runs at
+// the full tensor rate.
 //
-// TMEM (512 columns): Q as bf16 pairs [0,128), one S buffer [128,256), O
-// [256,512).  S_{j+1} is issued as soon as the softmax has read S_j out of
-// TMEM (not when P_j is ready), so the scores of the next tile are computed
-// while the exponentials of this one run.
+// TMEM (512 columns): S [0,128), P_0 [128,192), P_1 [192,256) (bf16 pairs),
+// O [256,512).  With two P buffers the softmax of tile j never waits for
+// PV_{j-1}: it only needs PV_{j-2} (long done) before it overwrites P_{j%2},
+// and PV_{j-1} only when it has to rescale O.
 //
-// Shared memory: one ring of three 64 KB slots filled by TMA in the order the
-// MMAs consume them - Q, K_0, K_1, V_0, K_2, V_1, K_3, V_2, ... - plus one
-// 32 KB P buffer.  V arrives transposed ([256, keys], keys contiguous), so
-// every operand is K-major with the 128-byte swizzle.
+// Shared memory: Q (64 KB, loaded once) and a ring of five 32 KB slots that
+// TMA fills with half tiles in the order the MMAs consume them - K_0, K_1,
+// V_0, K_2, V_1, K_3, V_2, ... - each split in two halves (K: head dims
+// [0,128) and [128,256); V: keys [0,64) and [64,128)), so a slot is released
+// as soon as the MMAs of its half have run.  V arrives transposed ([256,
+// keys], keys contiguous), so every shared-memory operand is K-major with the
+// 128-byte swizzle.
 //
 // The running maximum used for the exponentials only moves when a row's
 // maximum grows by more than 8 (a factor 2^8), so O is rescaled rarely;
 // numerator and denominator use the same maximum, so the result is unchanged.
-// The softmax computes a tile's exponentials (into packed bf16 registers)
-// before it waits for the previous PV product, and only the store of P into
-// the single P buffer (and the rare O rescale) waits for it.
 //
-// Warp roles (192 threads): warps 0-3 softmax + output (warp w owns TMEM
+// Warp roles (224 threads): warps 0-3 softmax + output (warp w owns TMEM
 // lanes / query rows 32w..32w+31), warp 4 TMA producer, warp 5 TMEM
-// allocation and MMA issue: S_0, S_1, PV_0, S_2, PV_1, ...
+// allocation and the S MMAs, warp 6 the PV MMAs.  The two MMA threads wait
+// on different events (scores read out vs. probabilities written), so one
+// keeps the tensor pipe fed while the other waits.
 //
 // Barrier parity: every barrier a role waits on completes at most one phase
 // ahead of that wait, so try_wait.parity never mistakes a later phase for the
-// awaited one.  Every wait is bounded.
+// awaited one (this is why P-ready and PV-done exist once per P buffer).
+// Every wait is bounded.
 #pragma once
 
 #include "ig4_ptx.cuh"
@@ -45,35 +47,34 @@ namespace ig4 {
 constexpr int ATT_BM = 128;
 constexpr int ATT_BN = 128;   // keys per tile
 constexpr int ATT_DH = 256;
-constexpr int ATT_THREADS = 192;
-constexpr int ATT_SLOTS = 3;
-constexpr int ATT_SLOT_BYTES = 65536;                  // Q, K_j (4 chunks [128 x 128 B]) or
-                                                       // V_j^T (2 chunks [256 x 128 B])
-constexpr int ATT_P_BYTES = ATT_BM * ATT_BN * 2;       // 32 KB: 2 chunks [128 x 128 B]
-constexpr int ATT_OFF_P = ATT_SLOTS * ATT_SLOT_BYTES;
-constexpr int ATT_OFF_BAR = ATT_OFF_P + ATT_P_BYTES;
+constexpr int ATT_THREADS = 224;
+constexpr int ATT_SLOTS = 5;
+constexpr int ATT_SLOT_BYTES = 32768;  // K half: 2 chunks [128 keys x 128 B]; V half: [256 x 128 B]
+constexpr int ATT_Q_BYTES = 65536;     // 4 chunks [128 rows x 128 B]
+constexpr int ATT_OFF_RING = ATT_Q_BYTES;
+constexpr int ATT_OFF_BAR = ATT_OFF_RING + ATT_SLOTS * ATT_SLOT_BYTES;
 constexpr int ATT_SMEM_BYTES = ATT_OFF_BAR + 256 + 1024;
 constexpr uint32_t ATT_TMEM_COLS = 512;
-constexpr uint32_t ATT_TMEM_Q = 0;
-constexpr uint32_t ATT_TMEM_S = 128;
+constexpr uint32_t ATT_TMEM_S = 0;
+constexpr uint32_t ATT_TMEM_P = 128;  // + 64 * buffer
 constexpr uint32_t ATT_TMEM_O = 256;
 // log2(e) / sqrt(256)
 constexpr float ATT_SCALE_LOG2 = 0.09016844005556021f;
 constexpr float ATT_RESCALE_THRESHOLD = 8.0f;
 
-// The ring's load / consumption order: item 0 is Q; then K_0, K_1 (if any);
-// then, for each tile j, V_j followed by K_{j+2} (if that tile exists).
-// kind(): 0 = Q, 1 = K, 2 = V, with the tile index in *tile.
+// The order in which the ring receives whole tiles ("items"): K_0; K_1 (if
+// any); then, for each tile j, V_j followed by K_{j+2} (if that tile
+// exists).  Each item travels as two 32 KB halves.
 struct AttRing {
   int nkv;
-  __device__ __forceinline__ int items() const { return 1 + 2 * nkv; }
-  __device__ __forceinline__ int kind(int i, int *tile) const {
-    if (i == 0) { *tile = 0; return 0; }
-    if (i == 1) { *tile = 0; return 1; }
-    if (nkv == 1) { *tile = 0; return 2; }  // items: Q, K_0, V_0
-    if (i == 2) { *tile = 1; return 1; }
-    // items from 3 on: V_0, K_2, V_1, K_3, ..., V_{nkv-3}, K_{nkv-1}, V_{nkv-2}, V_{nkv-1}
-    const int k = i - 3;
+  __device__ __forceinline__ int items() const { return 2 * nkv; }
+  // kind of item u: 1 = K, 2 = V, with the tile index in *tile
+  __device__ __forceinline__ int kind(int u, int *tile) const {
+    if (u == 0) { *tile = 0; return 1; }
+    if (nkv == 1) { *tile = 0; return 2; }  // items: K_0, V_0
+    if (u == 1) { *tile = 1; return 1; }
+    // items from 2 on: V_0, K_2, V_1, K_3, ..., V_{nkv-3}, K_{nkv-1}, V_{nkv-2}, V_{nkv-1}
+    const int k = u - 2;
     const int pairs = nkv - 2;  // (V_j, K_{j+2}) for j < nkv - 2
     if (k < 2 * pairs) {
       *tile = (k & 1) ? (k >> 1) + 2 : (k >> 1);
@@ -82,6 +83,9 @@ struct AttRing {
     *tile = (nkv - 2) + (k - 2 * pairs);
     return 2;
   }
+  // the item that carries K_t, and the one that carries V_t
+  __device__ __forceinline__ int item_k(int t) const { return t < 2 ? t : 2 * t - 1; }
+  __device__ __forceinline__ int item_v(int t) const { return min(2 * t + 2, 2 * nkv - 1); }
 };
 
 __global__ void __launch_bounds__(ATT_THREADS, 1)
@@ -91,17 +95,18 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t *sP = smem + ATT_OFF_P;
+  uint8_t *ring = smem + ATT_OFF_RING;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + ATT_OFF_BAR);
-  uint64_t *full = bars + 0;     // [ATT_SLOTS]
-  uint64_t *empty = bars + 3;    // [ATT_SLOTS]
-  uint64_t *s_full = bars + 6;   // S_j in TMEM
-  uint64_t *s_free = bars + 7;   // S_j read out of TMEM (one arrival per softmax warp)
-  uint64_t *p_full = bars + 8;   // P_j in shared memory (one arrival per softmax warp)
-  uint64_t *pv_done = bars + 9;  // PV_j (and every earlier MMA) complete
-  uint64_t *q_tmem = bars + 10;  // Q copied into TMEM (one arrival per softmax warp)
-  uint64_t *drain = bars + 11;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 12);
+  uint64_t *full = bars + 0;      // [ATT_SLOTS]
+  uint64_t *empty = bars + 5;     // [ATT_SLOTS]
+  uint64_t *q_full = bars + 10;   // Q landed
+  uint64_t *s_full = bars + 11;   // S_j in TMEM
+  uint64_t *s_free = bars + 12;   // S_j read out of TMEM (one arrival per softmax warp)
+  uint64_t *p_full = bars + 13;   // [2] P_j in TMEM buffer j%2 (one arrival per softmax warp)
+  uint64_t *pv_done = bars + 15;  // [2] PV_j complete (buffer j%2)
+  uint64_t *drain_s = bars + 17;
+  uint64_t *drain_pv = bars + 18;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 20);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -111,19 +116,22 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   const int b = blockIdx.z;
   const int bh = b * H + h;
   const int nkv = (L + ATT_BN - 1) / ATT_BN;
-  const AttRing ring{nkv};
+  const AttRing ring_order{nkv};
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < ATT_SLOTS; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
+    mbar_init(q_full, 1);
     mbar_init(s_full, 1);
     mbar_init(s_free, 4);
-    mbar_init(p_full, 4);
-    mbar_init(pv_done, 1);
-    mbar_init(q_tmem, 4);
-    mbar_init(drain, 1);
+    mbar_init(&p_full[0], 4);
+    mbar_init(&p_full[1], 4);
+    mbar_init(&pv_done[0], 1);
+    mbar_init(&pv_done[1], 1);
+    mbar_init(drain_s, 1);
+    mbar_init(drain_pv, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -144,7 +152,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   if (warp == 4) {
     if (lane == 0) {
       // ------------------------------------------------ TMA producer
-      const int n = ring.items();
+      mbar_arrive_expect_tx(q_full, ATT_Q_BYTES);
+      for (int c = 0; c < 4; ++c) tma_load_3d(smem + c * 16384, &tmQ, q_full, c * 64, q0, bh);
+      const int n = 2 * ring_order.items();  // half items
       int i = 0;
       bool ok = true;
       for (; i < n; ++i) {
@@ -152,21 +162,19 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         const uint32_t ph = static_cast<uint32_t>(i / ATT_SLOTS) & 1;
         if (!mbar_wait(&empty[slot], ph ^ 1, abort_flag)) { ok = false; break; }
         mbar_arrive_expect_tx(&full[slot], ATT_SLOT_BYTES);
-        uint8_t *dst = smem + slot * ATT_SLOT_BYTES;
+        uint8_t *dst = ring + slot * ATT_SLOT_BYTES;
+        const int half = i & 1;
         int t = 0;
-        const int kind = ring.kind(i, &t);
-        if (kind == 0) {
-          for (int c = 0; c < 4; ++c) tma_load_3d(dst + c * 16384, &tmQ, &full[slot], c * 64, q0, bh);
-        } else if (kind == 1) {
-          for (int c = 0; c < 4; ++c)
-            tma_load_3d(dst + c * 16384, &tmK, &full[slot], c * 64, t * ATT_BN, bh);
-        } else {
+        if (ring_order.kind(i >> 1, &t) == 1) {
           for (int c = 0; c < 2; ++c)
-            tma_load_3d(dst + c * 32768, &tmV, &full[slot], t * ATT_BN + c * 64, 0, bh);
+            tma_load_3d(dst + c * 16384, &tmK, &full[slot], (2 * half + c) * 64, t * ATT_BN, bh);
+        } else {
+          tma_load_3d(dst, &tmV, &full[slot], t * ATT_BN + half * 64, 0, bh);
         }
       }
       if (!ok) {
         // let the loads already issued land before the shared memory goes away
+        mbar_wait(q_full, 0, nullptr, WAIT_LIMIT_NS / 4);
         for (int k = (i > ATT_SLOTS ? i - ATT_SLOTS : 0); k < i; ++k)
           mbar_wait(&full[k % ATT_SLOTS], static_cast<uint32_t>(k / ATT_SLOTS) & 1, nullptr,
                     WAIT_LIMIT_NS / 4);
@@ -174,59 +182,69 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     }
   } else if (warp == 5) {
     if (lane == 0) {
-      // ------------------------------------------------ MMA issuer
+      // ------------------------------------------------ S issuer: S_t = Q K_t^T
       constexpr uint32_t IDESC_S = idesc_bf16(ATT_BM, ATT_BN);
-      constexpr uint32_t IDESC_PV = idesc_bf16(ATT_BM, ATT_DH);
-      const uint32_t p_base = smem_u32(sP);
-      int item = 1;  // ring item consumed next (item 0, Q, is read by the softmax warps)
-      bool ok = mbar_wait(q_tmem, 0, abort_flag);
-      if (ok) mbar_arrive(&empty[0]);  // Q's slot is free once Q is in TMEM
-      auto take = [&](uint32_t *base) -> bool {
-        const int slot = item % ATT_SLOTS;
-        if (!mbar_wait(&full[slot], static_cast<uint32_t>(item / ATT_SLOTS) & 1, abort_flag))
-          return false;
-        tc_fence_after();
-        *base = smem_u32(smem + slot * ATT_SLOT_BYTES);
-        return true;
-      };
-      auto give = [&]() {
-        umma_commit(&empty[item % ATT_SLOTS]);
-        ++item;
-      };
-      auto issue_s = [&]() -> bool {  // S_j into the S buffer, K_j from the ring
-        uint32_t k_base;
-        if (!take(&k_base)) return false;
+      const uint32_t q_base = smem_u32(smem);
+      bool ok = mbar_wait(q_full, 0, abort_flag);
+      for (int t = 0; t < nkv && ok; ++t) {
+        // the S buffer is free once the softmax has read S_{t-1}
+        if (t > 0 && !mbar_wait(s_free, static_cast<uint32_t>(t - 1) & 1, abort_flag)) break;
+        const int u = ring_order.item_k(t);
+        for (int half = 0; half < 2 && ok; ++half) {
+          const int i = 2 * u + half;
+          const int slot = i % ATT_SLOTS;
+          if (!mbar_wait(&full[slot], static_cast<uint32_t>(i / ATT_SLOTS) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t k_base = smem_u32(ring + slot * ATT_SLOT_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < ATT_DH / 16; ++kk) {
-          const uint64_t bd = sdesc_kmajor_sw128(k_base + (kk >> 2) * 16384 + (kk & 3) * 32);
-          umma_bf16_ts(tmem + ATT_TMEM_S, tmem + ATT_TMEM_Q + kk * 8, bd, IDESC_S, kk > 0);
+          for (int kq = 0; kq < 8; ++kq) {
+            const int kk = half * 8 + kq;  // K step of 16 head dims
+            const uint64_t ad = sdesc_kmajor_sw128(q_base + (kk >> 2) * 16384 + (kk & 3) * 32);
+            const uint64_t bd = sdesc_kmajor_sw128(k_base + (kq >> 2) * 16384 + (kq & 3) * 32);
+            umma_bf16(tmem + ATT_TMEM_S, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&empty[slot]);
         }
-        give();
-        umma_commit(s_full);
-        return true;
-      };
-      if (ok) ok = issue_s();  // S_0
-      for (int j = 0; j < nkv && ok; ++j) {
-        // S_{j+1} as soon as S_j has been read out of TMEM
-        if (j + 1 < nkv) {
-          if (!mbar_wait(s_free, static_cast<uint32_t>(j) & 1, abort_flag)) break;
-          if (!(ok = issue_s())) break;
-        }
-        // PV_j once P_j is in shared memory
-        if (!mbar_wait(p_full, static_cast<uint32_t>(j) & 1, abort_flag)) break;
-        uint32_t v_base;
-        if (!(ok = take(&v_base))) break;
-#pragma unroll
-        for (int kk = 0; kk < ATT_BN / 16; ++kk) {
-          const uint64_t ad = sdesc_kmajor_sw128(p_base + (kk >> 2) * 16384 + (kk & 3) * 32);
-          const uint64_t bd = sdesc_kmajor_sw128(v_base + (kk >> 2) * 32768 + (kk & 3) * 32);
-          umma_bf16(tmem + ATT_TMEM_O, ad, bd, IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        give();
-        umma_commit(pv_done);
+        if (ok) umma_commit(s_full);
       }
-      umma_commit(drain);
-      mbar_wait(drain, 0, nullptr, WAIT_LIMIT_NS / 4);
+      umma_commit(drain_s);
+      mbar_wait(drain_s, 0, nullptr, WAIT_LIMIT_NS / 4);
+    }
+  } else if (warp == 6) {
+    if (lane == 0) {
+      // ------------------------------------------------ PV issuer: O += P_j V_j
+      constexpr uint32_t IDESC_PV = idesc_bf16(ATT_BM, ATT_DH);
+      bool ok = true;
+      for (int j = 0; j < nkv && ok; ++j) {
+        const int pb = j & 1;
+        if (!mbar_wait(&p_full[pb], static_cast<uint32_t>(j >> 1) & 1, abort_flag)) break;
+        tc_fence_after();
+        const int u = ring_order.item_v(j);
+        for (int half = 0; half < 2 && ok; ++half) {
+          const int i = 2 * u + half;
+          const int slot = i % ATT_SLOTS;
+          if (!mbar_wait(&full[slot], static_cast<uint32_t>(i / ATT_SLOTS) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t v_base = smem_u32(ring + slot * ATT_SLOT_BYTES);
+#pragma unroll
+          for (int kq = 0; kq < 4; ++kq) {
+            const int kk = half * 4 + kq;  // K step of 16 keys
+            const uint64_t bd = sdesc_kmajor_sw128(v_base + kq * 32);
+            umma_bf16_ts(tmem + ATT_TMEM_O, tmem + ATT_TMEM_P + 64 * pb + kk * 8, bd, IDESC_PV,
+                         (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty[slot]);
+        }
+        if (ok) umma_commit(&pv_done[pb]);
+      }
+      umma_commit(drain_pv);
+      mbar_wait(drain_pv, 0, nullptr, WAIT_LIMIT_NS / 4);
     }
   } else {
     // -------------------------------------------- softmax warps 0..3
@@ -234,29 +252,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     float m_used = -INFINITY;
     float l_sum = 0.0f;
-    bool ok = mbar_wait_warp(&full[0], 0, abort_flag);  // Q (ring item 0)
-    if (ok) {
-      // Q row r: four 64-column chunks of 128 bytes in the 128-byte-swizzled
-      // TMA layout -> TMEM columns [ATT_TMEM_Q + 32c, +32), bf16 pairs.
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        const uint8_t *qrow = smem + c * 16384 + r * 128;
-        uint32_t w[32];
-#pragma unroll
-        for (int g = 0; g < 8; ++g) {
-          const uint4 v = *reinterpret_cast<const uint4 *>(qrow + ((g ^ (r & 7)) << 4));
-          w[4 * g + 0] = v.x;
-          w[4 * g + 1] = v.y;
-          w[4 * g + 2] = v.z;
-          w[4 * g + 3] = v.w;
-        }
-        tmem_st32_u(tmem + lane_base + ATT_TMEM_Q + c * 32, w);
-      }
-      tmem_st_wait();
-    }
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(q_tmem);
+    bool ok = true;
+    const uint64_t scale2 = f2_pack(ATT_SCALE_LOG2, ATT_SCALE_LOG2);
 
     for (int j = 0; j < nkv && ok; ++j) {
       if (!mbar_wait_warp(s_full, static_cast<uint32_t>(j) & 1, abort_flag)) { ok = false; break; }
@@ -281,20 +278,15 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         for (int i = 0; i < 128; ++i)
           if (kbase + i >= L) t[i] = -INFINITY;
       }
-      float m16[16];
+      float m4[4] = {t[0], t[1], t[2], t[3]};
 #pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        const float a0 = fmaxf(t[8 * q + 0], t[8 * q + 1]);
-        const float a1 = fmaxf(t[8 * q + 2], t[8 * q + 3]);
-        const float a2 = fmaxf(t[8 * q + 4], t[8 * q + 5]);
-        const float a3 = fmaxf(t[8 * q + 6], t[8 * q + 7]);
-        m16[q] = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+      for (int i = 4; i < 128; i += 8) {
+        m4[0] = fmax3(m4[0], t[i + 0], t[i + 1]);
+        m4[1] = fmax3(m4[1], t[i + 2], t[i + 3]);
+        m4[2] = fmax3(m4[2], t[i + 4], t[i + 5]);
+        m4[3] = fmax3(m4[3], t[i + 6], t[i + 7]);
       }
-#pragma unroll
-      for (int q = 0; q < 8; ++q) m16[q] = fmaxf(m16[q], m16[q + 8]);
-      const float mx = fmaxf(fmaxf(fmaxf(m16[0], m16[1]), fmaxf(m16[2], m16[3])),
-                             fmaxf(fmaxf(m16[4], m16[5]), fmaxf(m16[6], m16[7]))) *
-                       ATT_SCALE_LOG2;
+      const float mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * ATT_SCALE_LOG2;
 
       // Running maximum for this tile (moved only when it grows by more than
       // the threshold) and the factor that rescales what came before.
@@ -310,64 +302,67 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       }
       const bool any_need = __any_sync(0xffffffffu, need);
 
-      // Exponentials into packed bf16 registers first: they need neither
-      // PV_{j-1} nor the P buffer, so they overlap the tensor core's work.
-      const float neg_m = -m_new;
+      // p = 2^(s * scale - m), packed to bf16 pairs; row sum in fp32 pairs
+      const uint64_t negm2 = f2_pack(-m_new, -m_new);
       uint32_t pk[64];
-      float sums[16];
+      uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
-      for (int g = 0; g < 16; ++g) {
-        float p[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) p[e] = exp2_approx(fmaf(t[8 * g + e], ATT_SCALE_LOG2, neg_m));
-        sums[g] = ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
-        pk[4 * g + 0] = pack_bf16x2(p[0], p[1]);
-        pk[4 * g + 1] = pack_bf16x2(p[2], p[3]);
-        pk[4 * g + 2] = pack_bf16x2(p[4], p[5]);
-        pk[4 * g + 3] = pack_bf16x2(p[6], p[7]);
+      for (int i = 0; i < 64; ++i) {
+        const uint64_t x2 = ffma2(f2_pack(t[2 * i], t[2 * i + 1]), scale2, negm2);
+        const float p0 = exp2_approx(f2_lo(x2));
+        const float p1 = exp2_approx(f2_hi(x2));
+        const uint64_t p2 = f2_pack(p0, p1);
+        acc[i & 3] = fadd2(acc[i & 3], p2);
+        pk[i] = pack_bf16x2(p0, p1);
       }
-#pragma unroll
-      for (int g = 0; g < 8; ++g) sums[g] += sums[g + 8];
-      const float rowsum =
-          ((sums[0] + sums[1]) + (sums[2] + sums[3])) + ((sums[4] + sums[5]) + (sums[6] + sums[7]));
+      const uint64_t s2 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
+      const float rowsum = f2_lo(s2) + f2_hi(s2);
 
-      if (j > 0) {
-        // PV_{j-1} must be done: it reads the P buffer and writes O.
-        if (!mbar_wait_warp(pv_done, static_cast<uint32_t>(j - 1) & 1, abort_flag)) {
+      const int pb = j & 1;
+      if (j >= 2) {
+        // PV_{j-2} read this P buffer
+        if (!mbar_wait_warp(&pv_done[pb], static_cast<uint32_t>((j >> 1) - 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+      }
+      if (any_need) {
+        // PV_{j-1} must be done: it writes O
+        if (!mbar_wait_warp(&pv_done[pb ^ 1], static_cast<uint32_t>((j - 1) >> 1) & 1,
+                            abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        if (any_need) {
 #pragma unroll 1
-          for (int c = 0; c < ATT_DH; c += 32) {
-            float o[32];
-            tmem_ld32(tmem + lane_base + ATT_TMEM_O + c, o);
-            tmem_ld_wait();
+        for (int c = 0; c < ATT_DH; c += 32) {
+          float o[32];
+          tmem_ld32(tmem + lane_base + ATT_TMEM_O + c, o);
+          tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] *= f;
-            tmem_st32(tmem + lane_base + ATT_TMEM_O + c, o);
-          }
-          tmem_st_wait();
+          for (int i = 0; i < 32; ++i) o[i] *= f;
+          tmem_st32(tmem + lane_base + ATT_TMEM_O + c, o);
         }
       }
+      tc_fence_after();
+      {
+        uint32_t w[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) w[i] = pk[i];
+        tmem_st32_u(tmem + lane_base + ATT_TMEM_P + 64 * pb, w);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) w[i] = pk[32 + i];
+        tmem_st32_u(tmem + lane_base + ATT_TMEM_P + 64 * pb + 32, w);
+      }
+      tmem_st_wait();
       l_sum = l_sum * f + rowsum;
       m_used = m_new;
-
-#pragma unroll
-      for (int g = 0; g < 16; ++g) {
-        // key chunk g/8 (64 keys), 16-byte piece g%8 of row r, swizzled
-        *reinterpret_cast<uint4 *>(sP + (g >> 3) * 16384 + r * 128 + (((g & 7) ^ (r & 7)) << 4)) =
-            make_uint4(pk[4 * g + 0], pk[4 * g + 1], pk[4 * g + 2], pk[4 * g + 3]);
-      }
-      // this thread's P writes -> async proxy; then one arrival per warp
-      fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[pb]);
     }
     const int jl = nkv - 1;
-    if (ok && mbar_wait_warp(pv_done, static_cast<uint32_t>(jl) & 1, abort_flag)) {
+    if (ok && mbar_wait_warp(&pv_done[jl & 1], static_cast<uint32_t>(jl >> 1) & 1, abort_flag)) {
       tc_fence_after();
       const int lq = q0 + r;
       const bool valid = lq < L;
