@@ -129,10 +129,10 @@ ig4_status map_3d_bf16(CUtensorMap *m, const void *base, long d0, long d1, long 
 
 // -------------------------------------------------------------- GEMMs
 
-// 256-wide tiles over more than one 128-row block run on CTA pairs (M = 256
-// per pair tile, B rows split between the two CTAs); the B tensor map's box
-// is then 128 rows instead of 256.
-inline bool use_pair(int BN, int M) { return BN == 256 && M > GEMM_BM; }
+// 256- and 192-wide tiles over more than one 128-row block run on CTA pairs
+// (M = 256 per pair tile, B rows split between the two CTAs); the B tensor
+// map's box is then BN / 2 rows.
+inline bool use_pair(int BN, int M) { return (BN == 256 || BN == 192) && M > GEMM_BM; }
 inline int b_box_rows(int BN, int M) { return use_pair(BN, M) ? BN / 2 : BN; }
 
 template <int BN, bool FP8, bool DUAL_B, class Epi>
@@ -140,9 +140,10 @@ ig4_status launch_gemm(const CUtensorMap &A, const CUtensorMap &B, const CUtenso
                        int n_tiles_n, int K, const Epi &epi, cudaStream_t st) {
   DeviceInfo *di = nullptr;
   IG4_TRY(device_info(&di));
-  if constexpr (BN == 256) {
+  if constexpr (BN == 256 || BN == 192) {
     if (use_pair(BN, M)) {
-      auto kern = gemm_pair_kernel<FP8, DUAL_B, Epi>;
+      auto kern = gemm_pair_kernel<BN, FP8, DUAL_B, Epi>;
+      constexpr int PAIR_SMEM_BYTES = PairShape<BN>::SMEM_BYTES;
       IG4_TRY(allow_smem(kern, PAIR_SMEM_BYTES));
       const long tiles = static_cast<long>((M + 2 * GEMM_BM - 1) / (2 * GEMM_BM)) * n_tiles_n;
       const int pairs = static_cast<int>(std::min<long>(tiles, di->sms / 2));
@@ -324,20 +325,29 @@ ig4_status launch_attention(int B, int H, int L, const void *q, const void *k, c
 }
 
 // Tile width for an output of N columns: the candidate (256, 192, 128 that
-// divides N) with the best product of wave efficiency on the SMs (tiles /
-// (waves * SMs)) and per-tile MMA efficiency (narrower tiles read more shared
-// memory per flop; measured on the 4608 x 4608 x 4608 out-projection, 192-wide
-// tiles ran 10% slower per tile than 256-wide ones).
+// divides N) with the best product of wave efficiency (tiles / (waves *
+// workers), where a worker is a CTA pair for 256 and 192 over more than 128
+// rows and a single CTA otherwise) and per-tile MMA efficiency (single-CTA
+// 192- and 128-wide tiles read more shared memory per flop; measured on the
+// 4608 x 4608 x 4608 out-projection, single-CTA 192-wide tiles ran 10% slower
+// per tile than 256-wide ones; on the 4608 x 4608 out- and down-projections
+// 192-wide pair tiles ran at 0.79 of the 256-wide pair rate per flop, so they
+// only win where 256-wide tiles leave most of a wave of pairs idle).
 int choose_bn(int M, int N, int sms) {
   const int cand[3] = {256, 192, 128};
-  const double mma_eff[3] = {1.0, 0.88, 0.8};
+  const double mma_eff_single[3] = {1.0, 0.88, 0.8};
+  const double mma_eff_pair[3] = {1.0, 0.8, 0.0};
   int best = 0;
   double best_score = -1.0;
   for (int i = 0; i < 3; ++i) {
     if (N % cand[i]) continue;
-    const long tiles = static_cast<long>((M + GEMM_BM - 1) / GEMM_BM) * (N / cand[i]);
-    const long waves = (tiles + sms - 1) / sms;
-    const double score = mma_eff[i] * static_cast<double>(tiles) / static_cast<double>(waves * sms);
+    const bool pair = use_pair(cand[i], M);
+    const int bm = pair ? 2 * GEMM_BM : GEMM_BM;
+    const int workers = pair ? sms / 2 : sms;
+    const long tiles = static_cast<long>((M + bm - 1) / bm) * (N / cand[i]);
+    const long waves = (tiles + workers - 1) / workers;
+    const double eff = pair ? mma_eff_pair[i] : mma_eff_single[i];
+    const double score = eff * static_cast<double>(tiles) / static_cast<double>(waves * workers);
     if (score > best_score + 1e-9) {
       best_score = score;
       best = cand[i];

@@ -504,8 +504,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 }
 
 // ------------------------------------------------------ CTA-pair kernel
-// The same GEMM on a 2-CTA cluster: a pair tile is 256 rows x 256 columns;
-// each CTA loads its own 128 A rows and HALF of the 256 B rows (so with
+// The same GEMM on a 2-CTA cluster: a pair tile is 256 rows x BN columns
+// (BN = 256, or 192 where 256-wide tiles leave the last wave of pairs mostly
+// idle); each CTA loads its own 128 A rows and HALF of the BN B rows (so with
 // DUAL_B the first CTA loads the gate rows and the second the up rows), the
 // leader issues tcgen05.mma.cta_group::2 with M = 256, and each CTA's
 // epilogue warps handle its own 128 accumulator rows exactly as above.  Per
@@ -516,18 +517,27 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 // CTAs; both CTAs' loads complete on it); empty[s] and tfull[b] in both CTAs
 // (arrived by the leader's multicast commits); tempty[b] in the leader (one
 // arrival per epilogue warp of the pair).
-constexpr int PAIR_STAGES = 6;
-constexpr int PAIR_STAGE_BYTES = 2 * GEMM_BM * 128;  // A 16 KB + B half 16 KB
-constexpr int PAIR_SMEM_BYTES = PAIR_STAGES * PAIR_STAGE_BYTES + 1024 + 256;
+template <int BN>
+struct PairShape {
+  static_assert(BN == 256 || BN == 192, "pair tile width");
+  static constexpr int A_BYTES = GEMM_BM * 128;          // 16 KB
+  static constexpr int BH_BYTES = (BN / 2) * 128;        // 16 KB or 12 KB (a multiple of 1 KB)
+  static constexpr int STAGE_BYTES = A_BYTES + BH_BYTES;
+  static constexpr int STAGES = BN == 256 ? 6 : 7;       // ~200 KB of shared memory
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+};
 
-template <bool FP8, bool DUAL_B, class Epi>
+template <int BN, bool FP8, bool DUAL_B, class Epi>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmB2, int M, int n_tiles_n, int K,
                      const Epi epi) {
-  constexpr int BN = 256;
-  constexpr int A_BYTES = GEMM_BM * 128;
-  constexpr int BH_BYTES = (BN / 2) * 128;
+  static_assert(!DUAL_B || BN == 256, "SwiGLU pairs split 128 gate / 128 up rows");
+  using P = PairShape<BN>;
+  constexpr int PAIR_STAGES = P::STAGES;
+  constexpr int PAIR_STAGE_BYTES = P::STAGE_BYTES;
+  constexpr int A_BYTES = P::A_BYTES;
+  constexpr int BH_BYTES = P::BH_BYTES;
   constexpr int BK = FP8 ? 128 : 64;
   constexpr int UK_BYTES = 32;
   constexpr uint32_t IDESC = FP8 ? idesc_e4m3(2 * GEMM_BM, BN) : idesc_bf16(2 * GEMM_BM, BN);

@@ -136,10 +136,13 @@ def test_quantize_rows(ig4, M, K):
     (1, 1000, 768, 4608, "bf16", "bf16"),   # many tiles, long K
     (2, 150, 512, 1024, "f32", "e4m3"),
     (1, 300, 1024, 2816, "bf16", "e4m3"),
-    (1, 200, 384, 512, "f32", "bf16"),      # 192-wide tiles
+    (1, 200, 384, 512, "f32", "bf16"),      # 128-wide single-CTA tiles
     (1, 200, 640, 512, "f32", "bf16"),      # 128-wide tiles
-    (1, 4608, 4608, 256, "f32", "bf16"),    # the block's out-projection shape (192-wide)
-    (2, 100, 384, 512, "f32", "e4m3"),      # 192-wide tiles, E4M3
+    (1, 4608, 4608, 256, "f32", "bf16"),    # the block's out-projection shape (256-wide pair tiles)
+    (1, 1100, 4608, 256, "bf16", "bf16"),   # 192-wide pair tiles, ragged last pair tile
+    (1, 1152, 4608, 256, "f32", "e4m3"),    # 192-wide pair tiles, E4M3 (512px shape)
+    (1, 4864, 4608, 512, "bf16", "bf16"),   # 256-wide pair tiles (2048x352 shape)
+    (2, 100, 384, 512, "f32", "e4m3"),      # E4M3, batch boundary inside a tile
 ])
 def test_gated_residual_linear(ig4, B, L, N, K, xdt, wdt):
     M = B * L
