@@ -1,7 +1,9 @@
 """CPU oracle for the Ideogram 4 DiT block (TEST INFRASTRUCTURE ONLY).
 
 A plain, slow, float64 numpy statement of what one Ideogram4TransformerBlock
-forward and the 34-block stack compute.  Only ``tests/``,
+forward and the 34-block stack compute (``ig4_oracle``), and of one sampler
+step with asymmetric classifier-free guidance and its schedule
+(``ig4_sampler``).  Only ``tests/``,
 ``__graft_entry__.smoke()`` and the CPU legs of ``bench.py`` may import it; the
 product path (``stream_diffusion_transformer_fwd_b200``) never does, and this
 package imports nothing from the product.  It shares no code, table or
