@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -28,6 +29,27 @@ constexpr int ABI_VERSION = 1;
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// Inverse of the standard normal CDF Phi(x) = erfc(-x / sqrt 2) / 2 for
+// 0 < p < 1, by bisection (Phi is monotone; 200 halvings reach the spacing of
+// doubles), +-infinity at p = 1 and p = 0.  The upper half uses the symmetry
+// Phi^-1(p) = -Phi^-1(1 - p), so the bisection always works in the lower
+// tail, where erfc keeps full relative precision.
+inline double normal_quantile(double p) {
+  if (p <= 0.0) return -INFINITY;
+  if (p >= 1.0) return INFINITY;
+  if (p > 0.5) return -normal_quantile(1.0 - p);
+  double lo = -40.0, hi = 0.0;
+  for (int it = 0; it < 200; ++it) {
+    const double mid = 0.5 * (lo + hi);
+    if (mid == lo || mid == hi) break;
+    if (0.5 * std::erfc(-mid / std::sqrt(2.0)) < p)
+      lo = mid;
+    else
+      hi = mid;
+  }
+  return 0.5 * (lo + hi);
+}
 
 ig4_status last_launch_status() {
   return cudaGetLastError() == cudaSuccess ? IG4_OK : IG4_ERR_CUDA;
@@ -884,6 +906,114 @@ ig4_status ig4_stack_forward(const ig4_config *cfg, const ig4_stack_weights *sw,
   IG4_TRY(launch_linear_store(B * N, C, D, ws.hf, false, nullptr, w_out, nullptr, sw->b_out,
                               out_latent, IG4_BF16, C, 0, 0, 0, st));
   return IG4_OK;
+}
+
+// ---------------------------------------------------------------- sampler
+
+ig4_status ig4_flow_schedule(int num_steps, double mu_base, double std_dev, int height_px,
+                             int width_px, double *t_out) {
+  if (num_steps < 1 || num_steps > 100000 || !(std_dev > 0.0) || !std::isfinite(mu_base) ||
+      !std::isfinite(std_dev) || height_px < 1 || width_px < 1 || !t_out)
+    return IG4_ERR_INVALID_ARG;
+  const double mu =
+      mu_base + 0.5 * std::log(static_cast<double>(height_px) * static_cast<double>(width_px) /
+                               (512.0 * 512.0));
+  t_out[0] = 1.0;
+  t_out[num_steps] = 0.0;
+  for (int i = 1; i < num_steps; ++i) {
+    // the (1 - i/N) quantile: Phi^-1(1 - q) = -Phi^-1(q), q = i/N
+    const double x = -normal_quantile(static_cast<double>(i) / num_steps);
+    t_out[i] = 1.0 / (1.0 + std::exp(-(mu + std_dev * x)));
+  }
+  return IG4_OK;
+}
+
+ig4_status ig4_guidance_schedule(int num_steps, int n_polish, float gw_main, float gw_polish,
+                                 float *gw_out) {
+  if (num_steps < 1 || n_polish < 0 || n_polish > num_steps || !gw_out ||
+      !std::isfinite(gw_main) || !std::isfinite(gw_polish))
+    return IG4_ERR_INVALID_ARG;
+  for (int i = 0; i < num_steps; ++i) gw_out[i] = i < num_steps - n_polish ? gw_main : gw_polish;
+  return IG4_OK;
+}
+
+ig4_status ig4_cfg_euler(long long n, const void *v_cond, const void *v_uncond, float gw, float dt,
+                         const float *z_in, float *z_out, void *z16_out, void *stream) {
+  if (n < 0 || n % 8 || !z_in || (!z_out && !z16_out) || (!v_cond) != (!v_uncond) ||
+      (v_cond && !z_out))
+    return IG4_ERR_INVALID_ARG;
+  const void *ptrs[] = {v_cond, v_uncond, z_in, z_out, z16_out};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return IG4_ERR_INVALID_ARG;
+  if (!std::isfinite(gw) || !std::isfinite(dt)) return IG4_ERR_INVALID_ARG;
+  if (n == 0) return IG4_OK;
+  DeviceInfo *di = nullptr;
+  IG4_TRY(device_info(&di));
+  const long n8 = n / 8;
+  const int grid = static_cast<int>(std::min<long>((n8 + 255) / 256, 8L * di->sms));
+  cfg_euler_kernel<<<grid, 256, 0, as_stream(stream)>>>(
+      static_cast<const uint4 *>(v_cond), static_cast<const uint4 *>(v_uncond), gw, dt,
+      reinterpret_cast<const float4 *>(z_in), reinterpret_cast<float4 *>(z_out),
+      static_cast<uint4 *>(z16_out), n8);
+  return last_launch_status();
+}
+
+namespace {
+struct DenoiseWs {
+  void *z16, *v_c, *v_u;
+  uint8_t *stack;
+  size_t bytes;
+};
+
+DenoiseWs denoise_ws_layout(const ig4_config *c, int C, uint8_t *base) {
+  DenoiseWs w{};
+  const size_t lat = round_up(2ull * c->B * c->grid_t * c->grid_h * c->grid_w * C, 256);
+  w.z16 = base;
+  w.v_c = base ? base + lat : nullptr;
+  w.v_u = base ? base + 2 * lat : nullptr;
+  w.stack = base ? base + 3 * lat : nullptr;
+  w.bytes = 3 * lat + stack_ws_layout(c, C, nullptr).bytes;
+  return w;
+}
+}  // namespace
+
+size_t ig4_denoise_workspace_size(const ig4_config *cfg, int latent_ch) {
+  if (ig4_stack_workspace_size(cfg, latent_ch) == 0) return 0;
+  return denoise_ws_layout(cfg, latent_ch, nullptr).bytes;
+}
+
+ig4_status ig4_denoise_step(const ig4_config *cfg, const ig4_stack_weights *cond,
+                            const ig4_stack_weights *uncond, float *z, const void *text,
+                            const int32_t *pos_cond, const int32_t *pos_uncond,
+                            const float *temb_cond, const float *temb_uncond, float t_cur,
+                            float t_next, float gw, void *workspace, size_t ws_bytes,
+                            void *stream) {
+  IG4_TRY(check_config(cfg));
+  if (!cond || !uncond || !z || !pos_cond || !pos_uncond || !temb_cond || !temb_uncond ||
+      !workspace)
+    return IG4_ERR_INVALID_ARG;
+  if (cfg->x_dtype != IG4_BF16) return IG4_ERR_UNSUPPORTED;
+  const int C = cond->latent_ch;
+  if (uncond->latent_ch != C || C < 128 || C % 128) return IG4_ERR_INVALID_ARG;
+  if (!std::isfinite(t_cur) || !std::isfinite(t_next) || !std::isfinite(gw))
+    return IG4_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return IG4_ERR_WORKSPACE;
+  const DenoiseWs ws = denoise_ws_layout(cfg, C, static_cast<uint8_t *>(workspace));
+  if (ws_bytes < ws.bytes) return IG4_ERR_WORKSPACE;
+  const size_t stack_bytes = ws_bytes - (ws.stack - static_cast<uint8_t *>(workspace));
+  const long long n = static_cast<long long>(cfg->B) * cfg->grid_t * cfg->grid_h * cfg->grid_w * C;
+  // the stacks read the latent in bf16
+  IG4_TRY(ig4_cfg_euler(n, nullptr, nullptr, 0.0f, 0.0f, z, nullptr, ws.z16, stream));
+  // conditional transformer over [text | image]
+  IG4_TRY(ig4_stack_forward(cfg, cond, ws.z16, text, ws.v_c, pos_cond, temb_cond, ws.stack,
+                            stack_bytes, stream));
+  // separate unconditional transformer over the image tokens alone
+  ig4_config cu = *cfg;
+  cu.T_text = 0;
+  IG4_TRY(ig4_stack_forward(&cu, uncond, ws.z16, nullptr, ws.v_u, pos_uncond, temb_uncond,
+                            ws.stack, stack_bytes, stream));
+  // v = v_u + gw (v_c - v_u); z += (t_cur - t_next) v
+  return ig4_cfg_euler(n, ws.v_c, ws.v_u, gw, t_cur - t_next, z, z, nullptr, stream);
 }
 
 }  // extern "C"

@@ -323,6 +323,42 @@ __global__ void copy_rows_kernel(const uint4 *__restrict__ src, uint4 *__restric
   }
 }
 
+// ------------------------------------------------ sampler: guided Euler step
+// z_out = z_in + dt * (v_u + gw * (v_c - v_u)) over n elements, 8 per thread
+// (one 16-byte load of each bf16 velocity, two of the fp32 latent); also
+// writes the bf16 copy of z_out the next stack call reads, if z16 != nullptr.
+// With v_c = v_u = nullptr it only converts z_in to bf16 (dt is ignored).
+__global__ void cfg_euler_kernel(const uint4 *__restrict__ v_c, const uint4 *__restrict__ v_u,
+                                 float gw, float dt, const float4 *z_in, float4 *z_out,
+                                 uint4 *__restrict__ z16, long n8) {
+  for (long i = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<long>(gridDim.x) * blockDim.x) {
+    const float4 za = z_in[2 * i];
+    const float4 zb = z_in[2 * i + 1];
+    float z[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
+    if (v_c != nullptr) {
+      const uint4 c = v_c[i];
+      const uint4 u = v_u[i];
+      const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+      const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 cf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&cw[q]));
+        const float2 uf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&uw[q]));
+        const float g0 = fmaf(gw, cf.x - uf.x, uf.x);
+        const float g1 = fmaf(gw, cf.y - uf.y, uf.y);
+        z[2 * q] = fmaf(dt, g0, z[2 * q]);
+        z[2 * q + 1] = fmaf(dt, g1, z[2 * q + 1]);
+      }
+      z_out[2 * i] = make_float4(z[0], z[1], z[2], z[3]);
+      z_out[2 * i + 1] = make_float4(z[4], z[5], z[6], z[7]);
+    }
+    if (z16 != nullptr)
+      z16[i] = make_uint4(pack_bf16x2(z[0], z[1]), pack_bf16x2(z[2], z[3]),
+                          pack_bf16x2(z[4], z[5]), pack_bf16x2(z[6], z[7]));
+  }
+}
+
 // ---------------------------------------------------- timeout self-test
 // Waits on an mbarrier that nothing completes; the bounded wait gives up at
 // limit_ns, flags the device error word and the kernel returns.

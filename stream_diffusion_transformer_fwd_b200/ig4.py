@@ -96,6 +96,14 @@ _sig("ig4_block_forward_noalloc", [ctypes.POINTER(Config), ctypes.POINTER(BlockW
 _sig("ig4_stack_workspace_size", [ctypes.POINTER(Config), _i], ctypes.c_size_t)
 _sig("ig4_stack_forward", [ctypes.POINTER(Config), ctypes.POINTER(StackWeights), _vp, _vp, _vp,
                            _vp, _vp, _vp, ctypes.c_size_t, _vp])
+_sig("ig4_flow_schedule", [_i, ctypes.c_double, ctypes.c_double, _i, _i,
+                           ctypes.POINTER(ctypes.c_double)])
+_sig("ig4_guidance_schedule", [_i, _i, _f, _f, ctypes.POINTER(_f)])
+_sig("ig4_cfg_euler", [ctypes.c_longlong, _vp, _vp, _f, _f, _vp, _vp, _vp, _vp])
+_sig("ig4_denoise_workspace_size", [ctypes.POINTER(Config), _i], ctypes.c_size_t)
+_sig("ig4_denoise_step", [ctypes.POINTER(Config), ctypes.POINTER(StackWeights),
+                          ctypes.POINTER(StackWeights), _vp, _vp, _vp, _vp, _vp, _vp, _f, _f, _f,
+                          _vp, ctypes.c_size_t, _vp])
 _sig("ig4_last_device_error", [_vp])
 _sig("ig4_selftest_timeout", [_i, _vp])
 
@@ -103,8 +111,10 @@ EXPORTED = ("ig4_status_string", "ig4_abi_version", "ig4_mrope_positions", "ig4_
             "ig4_adaln_modulation", "ig4_norm_modulate", "ig4_qkv_project",
             "ig4_joint_attention", "ig4_gated_residual_linear", "ig4_swiglu",
             "ig4_quantize_rows", "ig4_workspace_size", "ig4_block_forward",
-            "ig4_block_forward_traced", "ig4_block_forward_noalloc", "ig4_stack_workspace_size", "ig4_stack_forward",
-            "ig4_last_device_error", "ig4_selftest_timeout")
+            "ig4_block_forward_traced", "ig4_block_forward_noalloc", "ig4_stack_workspace_size",
+            "ig4_stack_forward", "ig4_flow_schedule", "ig4_guidance_schedule", "ig4_cfg_euler",
+            "ig4_denoise_workspace_size", "ig4_denoise_step", "ig4_last_device_error",
+            "ig4_selftest_timeout")
 
 
 def library():
@@ -301,6 +311,44 @@ def ig4_stack_forward(cfg: Config, sw: StackWeights, x_latent, text, out_latent,
                                   _ptr(text), _ptr(out_latent), _ptr(pos), _ptr(temb),
                                   _ptr(workspace), ws_bytes, _stream(stream)),
            "ig4_stack_forward")
+
+
+def ig4_flow_schedule(num_steps: int, mu_base: float, std: float, height_px: int,
+                      width_px: int) -> list:
+    """The num_steps + 1 sampler times t_0 = 1 > ... > t_N = 0 (host)."""
+    out = (ctypes.c_double * (num_steps + 1))() if num_steps >= 0 else None
+    _check(_lib.ig4_flow_schedule(num_steps, mu_base, std, height_px, width_px, out),
+           "ig4_flow_schedule")
+    return list(out)
+
+
+def ig4_guidance_schedule(num_steps: int, n_polish: int, gw_main: float = 7.0,
+                          gw_polish: float = 3.0) -> list:
+    """Guidance weight of each step (host)."""
+    out = (_f * max(1, num_steps))()
+    _check(_lib.ig4_guidance_schedule(num_steps, n_polish, gw_main, gw_polish, out),
+           "ig4_guidance_schedule")
+    return list(out)[:num_steps]
+
+
+def ig4_cfg_euler(v_cond, v_uncond, gw: float, dt: float, z_in, z_out=None, z16_out=None,
+                  stream=None):
+    _check(_lib.ig4_cfg_euler(z_in.numel(), _ptr(v_cond), _ptr(v_uncond), gw, dt, _ptr(z_in),
+                              _ptr(z_out), _ptr(z16_out), _stream(stream)), "ig4_cfg_euler")
+
+
+def ig4_denoise_workspace_size(cfg: Config, latent_ch: int = 128) -> int:
+    return int(_lib.ig4_denoise_workspace_size(ctypes.byref(cfg), latent_ch))
+
+
+def ig4_denoise_step(cfg: Config, cond: StackWeights, uncond: StackWeights, z, text, pos_cond,
+                     pos_uncond, temb_cond, temb_uncond, t_cur: float, t_next: float, gw: float,
+                     workspace, stream=None):
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(_lib.ig4_denoise_step(ctypes.byref(cfg), ctypes.byref(cond), ctypes.byref(uncond),
+                                 _ptr(z), _ptr(text), _ptr(pos_cond), _ptr(pos_uncond),
+                                 _ptr(temb_cond), _ptr(temb_uncond), t_cur, t_next, gw,
+                                 _ptr(workspace), ws_bytes, _stream(stream)), "ig4_denoise_step")
 
 
 def ig4_last_device_error(stream=None) -> int:
