@@ -39,6 +39,23 @@ struct GemmShape {
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 };
 
+// Tile t of a persistent GEMM -> (m tile, n tile).  Tiles are taken in
+// groups of group_m m tiles: within a group the m tile runs fastest, then
+// the n tile.  group_m >= m_tiles is plain m-fastest order, right when A fits
+// in L2 (every wave re-reads A from L2 and streams B once); a group of 8
+// makes the tiles that run at the same time share ~8 A slabs and ~10 B slabs
+// when A is too large to stay resident.  A bijection for any sizes.
+__device__ __forceinline__ void tile_coords(int t, int m_tiles, int n_tiles_n, int group_m,
+                                            int *mt, int *nt) {
+  const int gsize = min(group_m, m_tiles);
+  const int group = gsize * n_tiles_n;
+  const int first_m = (t / group) * gsize;
+  const int gm = min(m_tiles - first_m, gsize);
+  const int local = t - (t / group) * group;
+  *mt = first_m + local % gm;
+  *nt = local / gm;
+}
+
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
   const uintptr_t a = reinterpret_cast<uintptr_t>(p);
   return reinterpret_cast<uint8_t *>((a + 1023) & ~static_cast<uintptr_t>(1023));
@@ -346,7 +363,7 @@ template <int BN, bool FP8, bool DUAL_B, class Epi>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmB2, int M, int n_tiles_n, int K,
-                   const Epi epi) {
+                   int group_m, const Epi epi) {
   using S = GemmShape<BN>;
   constexpr int STAGES = S::STAGES;
   constexpr int BK = FP8 ? 128 : 64;  // K elements per stage: one 128-byte row
@@ -407,8 +424,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       long issued = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-        const int mt = t % m_tiles;
-        const int nt = t / m_tiles;
+        int mt, nt;
+        tile_coords(t, m_tiles, n_tiles_n, group_m, &mt, &nt);
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1, abort_flag)) {
             ok = false;
@@ -489,8 +506,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const uint32_t use = static_cast<uint32_t>(local >> 1);
       if (!mbar_wait_warp(&tfull[buf], use & 1, abort_flag)) break;
       tc_fence_after();
-      const int mt = t % m_tiles;
-      const int nt = t / m_tiles;
+      int mt, nt;
+      tile_coords(t, m_tiles, n_tiles_n, group_m, &mt, &nt);
       epi(mt * GEMM_BM, nt * BN, tmem_base + lane_base + buf * BN, r);
       tc_fence_before();
       mbar_arrive(&tempty[buf]);
@@ -531,7 +548,7 @@ template <int BN, bool FP8, bool DUAL_B, class Epi>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmB2, int M, int n_tiles_n, int K,
-                     const Epi epi) {
+                     int group_m, const Epi epi) {
   static_assert(!DUAL_B || BN == 256, "SwiGLU pairs split 128 gate / 128 up rows");
   using P = PairShape<BN>;
   constexpr int PAIR_STAGES = P::STAGES;
@@ -598,8 +615,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       uint32_t ph = 0;
       bool ok = true;
       for (int t = pair; t < n_tiles && ok; t += n_pairs) {
-        const int mt = t % m_tiles;
-        const int nt = t / m_tiles;
+        int mt, nt;
+        tile_coords(t, m_tiles, n_tiles_n, group_m, &mt, &nt);
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait_cluster(&empty[s], ph ^ 1, abort_flag)) {
             ok = false;
@@ -677,8 +694,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const bool ok = mbar_wait_cluster(&tfull[buf], use & 1, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      const int mt = t % m_tiles;
-      const int nt = t / m_tiles;
+      int mt, nt;
+      tile_coords(t, m_tiles, n_tiles_n, group_m, &mt, &nt);
       epi(mt * 2 * GEMM_BM + static_cast<int>(rank) * GEMM_BM, nt * BN,
           tmem_base + lane_base + buf * BN, r);
       tc_fence_before();

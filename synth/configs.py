@@ -66,6 +66,10 @@ CONFIGS = {
     # one denoiser step of the 34-block stack, FP8 weights, batch 2 at 1024 px
     "stack_1024px_fp8": Config("stack_1024px_fp8", B=2, T_text=512, grid_t=1, grid_h=64,
                                grid_w=64, w_dtype="e4m3", n_blocks=34),
+    # one sampler step at 1024 px: the conditional 34-block stack over 512 text +
+    # 64x64 image tokens and the separate image-only unconditional stack, FP8
+    "step_1024px_fp8": Config("step_1024px_fp8", B=1, T_text=512, grid_t=1, grid_h=64,
+                              grid_w=64, w_dtype="e4m3", n_blocks=34),
 }
 
 
