@@ -42,4 +42,7 @@ from .ig4_oracle import (  # noqa: F401
     split_heads,
     stack_forward,
     swiglu,
+    text_cond_projection,
+    TEXT_RAW_LAYERS,
+    TEXT_RAW_WIDTH,
 )

@@ -391,6 +391,33 @@ def stack_forward(x_latent, text, temb, pos, block_weights, n_blocks, w_in, b_in
 
 
 # ---------------------------------------------------------------------------
+# text conditioning projection (the step before the stack)
+# ---------------------------------------------------------------------------
+
+TEXT_RAW_LAYERS = 13     # hidden states of 13 text-encoder layers, concatenated
+TEXT_RAW_WIDTH = 4096    # per layer: 13 * 4096 = 53248 fp32 features per token
+
+
+def text_cond_projection(raw, g_norm, w_proj, b_proj, eps: float = EPS) -> np.ndarray:
+    """Projected text conditioning the stack consumes as its text prefix.
+
+    "Ideogram 4 快速开始" (SimpleTuner quickstart), section "Text embed cache":
+    the text encoder output concatenates the hidden states of 13 layers
+    (13 * 4096 = 53248 fp32 values per token); the transformer's frozen
+    llm_cond_norm and llm_cond_proj layers project these raw features to the
+    conditioning tensor the transformer consumes (a bf16 cache of ~4.5 MiB for
+    a 512-token caption, i.e. 4608 values per token).
+    Readings: llm_cond_norm is one RMSNorm over the whole concatenated
+    feature with a learned weight (eps 1e-6); llm_cond_proj is a linear layer
+    53248 -> D with a bias.
+
+    raw: [..., K_raw]; g_norm: [K_raw]; w_proj: [D, K_raw]; b_proj: [D].
+    """
+    h = rms_norm(np.asarray(raw, dtype=np.float64), eps, np.asarray(g_norm, dtype=np.float64))
+    return h @ np.asarray(w_proj, dtype=np.float64).T + np.asarray(b_proj, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
 # algorithmic work (closed forms used by the measurement code)
 # ---------------------------------------------------------------------------
 
