@@ -271,6 +271,29 @@ ig4_status ig4_stack_forward(const ig4_config *cfg, const ig4_stack_weights *sw,
                              const int32_t *pos, const float *temb, void *workspace,
                              size_t ws_bytes, void *stream);
 
+/* -------------------------------------------------- text conditioning ---
+ * The step before the stack ("Ideogram 4 快速开始" (SimpleTuner quickstart),
+ * section "Text embed cache"): the text encoder output concatenates the
+ * hidden states of 13 layers, 13 * 4096 = 53248 fp32 features per token, and
+ * the transformer's frozen llm_cond_norm and llm_cond_proj layers project
+ * them to the conditioning the stack reads as its text prefix (4608 values
+ * per token, bf16).  Readings: llm_cond_norm is one RMSNorm with a learned
+ * weight over the whole concatenated feature; llm_cond_proj a linear layer
+ * with bias:  text_out = (raw * rsqrt(mean(raw^2) + eps) * g_norm) W^T + b.
+ *
+ * raw fp32 [M][K_raw] (M = tokens of all samples), g_norm fp32 [K_raw],
+ * w_proj [D][K_raw] (bf16, or E4M3 codes with the per-output-channel fp32
+ * w_scale [D]; with E4M3 the normed features are quantised to E4M3 with a
+ * per-token scale, as in the block's FP8 path), b_proj fp32 [D], text_out
+ * bf16 [M][D]; all device, 16-byte aligned.  K_raw and D multiples of 128.
+ * Workspace (256-byte aligned) of ig4_text_cond_workspace_size bytes holds
+ * the normed features.  Errors: IG4_ERR_INVALID_ARG, IG4_ERR_WORKSPACE. */
+size_t ig4_text_cond_workspace_size(int M, int K_raw, int w_dtype);
+ig4_status ig4_text_cond_project(int M, int K_raw, int D, const float *raw, const float *g_norm,
+                                 float eps, const void *w_proj, const float *w_scale, int w_dtype,
+                                 const float *b_proj, void *text_out, void *workspace,
+                                 size_t ws_bytes, void *stream);
+
 /* ------------------------------------------------------------ sampler ---
  * One step of the sampler around the stack ("Ideogram 4.0" survey page,
  * section 训练方法: the DiT predicts a flow-matching velocity and inference

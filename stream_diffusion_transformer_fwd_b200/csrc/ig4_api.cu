@@ -488,6 +488,37 @@ ig4_status launch_linear_store(int M, int N, int K, const void *a, bool f8, cons
   return launch_gemm<128, false, false>(ma, mb, mb, M, N / 128, K, e, st);
 }
 
+// Plain linear layer into bf16 with a bias, tile width chosen for the shape
+// (the text conditioning projection: K = 53248, N = 4608, M = tokens).
+template <int BN, bool FP8>
+ig4_status launch_store_bf16_bn(int M, int N, int K, const void *a, const float *a_scale,
+                                const void *w, const float *w_scale, const float *bias, void *out,
+                                cudaStream_t st) {
+  CUtensorMap ma, mb;
+  IG4_TRY(gemm_maps(&ma, &mb, a, w, FP8 ? 1 : 2, M, N, K, b_box_rows(BN, M)));
+  EpiStore<BN, FP8, __nv_bfloat16> e{static_cast<__nv_bfloat16 *>(out), N, M, N, bias,
+                                     FP8 ? a_scale : nullptr, FP8 ? w_scale : nullptr, 0, 0, 0};
+  return launch_gemm<BN, FP8, false>(ma, mb, mb, M, N / BN, K, e, st);
+}
+
+template <bool FP8>
+ig4_status launch_store_bf16(int M, int N, int K, const void *a, const float *a_scale,
+                             const void *w, const float *w_scale, const float *bias, void *out,
+                             cudaStream_t st) {
+  DeviceInfo *di = nullptr;
+  IG4_TRY(device_info(&di));
+  switch (choose_bn(M, N, di->sms)) {
+    case 256:
+      return launch_store_bf16_bn<256, FP8>(M, N, K, a, a_scale, w, w_scale, bias, out, st);
+    case 192:
+      return launch_store_bf16_bn<192, FP8>(M, N, K, a, a_scale, w, w_scale, bias, out, st);
+    case 128:
+      return launch_store_bf16_bn<128, FP8>(M, N, K, a, a_scale, w, w_scale, bias, out, st);
+    default:
+      return IG4_ERR_UNSUPPORTED;
+  }
+}
+
 // ------------------------------------------------------- workspace layout
 
 struct BlockWs {
@@ -916,6 +947,47 @@ ig4_status ig4_stack_forward(const ig4_config *cfg, const ig4_stack_weights *sw,
   IG4_TRY(launch_linear_store(B * N, C, D, ws.hf, false, nullptr, w_out, nullptr, sw->b_out,
                               out_latent, IG4_BF16, C, 0, 0, 0, st));
   return IG4_OK;
+}
+
+// --------------------------------------------------- text conditioning
+
+size_t ig4_text_cond_workspace_size(int M, int K_raw, int w_dtype) {
+  if (M < 1 || K_raw < 128 || K_raw % 128 || !valid_dtype_w(w_dtype)) return 0;
+  const size_t es = is_fp8(w_dtype) ? 1 : 2;
+  return round_up(es * M * static_cast<size_t>(K_raw), 256) +
+         round_up(sizeof(float) * static_cast<size_t>(M), 256);
+}
+
+ig4_status ig4_text_cond_project(int M, int K_raw, int D, const float *raw, const float *g_norm,
+                                 float eps, const void *w_proj, const float *w_scale, int w_dtype,
+                                 const float *b_proj, void *text_out, void *workspace,
+                                 size_t ws_bytes, void *stream) {
+  if (M < 1 || K_raw < 128 || K_raw % 128 || D < 128 || D % 128 || !(eps > 0.0f))
+    return IG4_ERR_INVALID_ARG;
+  if (!valid_dtype_w(w_dtype)) return IG4_ERR_INVALID_ARG;
+  const bool f8 = is_fp8(w_dtype);
+  if (!raw || !g_norm || !w_proj || !b_proj || !text_out || !workspace || (f8 && !w_scale))
+    return IG4_ERR_INVALID_ARG;
+  const void *ptrs[] = {raw, g_norm, w_proj, b_proj, text_out};
+  for (const void *p : ptrs)
+    if (!aligned16(p)) return IG4_ERR_INVALID_ARG;
+  if (f8 && !aligned16(w_scale)) return IG4_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return IG4_ERR_WORKSPACE;
+  if (ws_bytes < ig4_text_cond_workspace_size(M, K_raw, w_dtype)) return IG4_ERR_WORKSPACE;
+  cudaStream_t st = as_stream(stream);
+  uint8_t *h = static_cast<uint8_t *>(workspace);
+  float *h_scale = reinterpret_cast<float *>(
+      h + round_up((f8 ? 1 : 2) * static_cast<size_t>(M) * K_raw, 256));
+  // llm_cond_norm: RMSNorm over the concatenated features, into bf16 / E4M3
+  if (f8)
+    wide_rmsnorm_kernel<true><<<M, WIDE_NORM_THREADS, 0, st>>>(raw, g_norm, K_raw, eps, h, h_scale);
+  else
+    wide_rmsnorm_kernel<false><<<M, WIDE_NORM_THREADS, 0, st>>>(raw, g_norm, K_raw, eps, h,
+                                                                nullptr);
+  IG4_TRY(last_launch_status());
+  // llm_cond_proj: K_raw -> D with bias, bf16 out
+  if (f8) return launch_store_bf16<true>(M, D, K_raw, h, h_scale, w_proj, w_scale, b_proj, text_out, st);
+  return launch_store_bf16<false>(M, D, K_raw, h, nullptr, w_proj, nullptr, b_proj, text_out, st);
 }
 
 // ---------------------------------------------------------------- sampler

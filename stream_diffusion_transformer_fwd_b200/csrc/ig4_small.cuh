@@ -323,6 +323,82 @@ __global__ void copy_rows_kernel(const uint4 *__restrict__ src, uint4 *__restric
   }
 }
 
+// ------------------------------------- text conditioning: wide RMSNorm rows
+// h = x * rsqrt(mean(x^2) + eps) * g over rows of K fp32 features (the 53248
+// concatenated text-encoder features per token), one CTA per row.  Pass 1
+// sums the squares (and, for E4M3 output, the max of |x g|) over 16-byte
+// loads; pass 2 reads the row again (from L2) and writes bf16, or E4M3 codes
+// with the per-row scale max|h| / 448.  K is a multiple of 8.
+constexpr int WIDE_NORM_THREADS = 512;
+
+template <bool OUT_FP8>
+__global__ void __launch_bounds__(WIDE_NORM_THREADS)
+    wide_rmsnorm_kernel(const float *__restrict__ x, const float *__restrict__ g, int K, float eps,
+                        void *__restrict__ out, float *__restrict__ out_scale) {
+  __shared__ float red[2][WIDE_NORM_THREADS / 32];
+  const long row = blockIdx.x;
+  const float4 *xr = reinterpret_cast<const float4 *>(x + row * K);
+  const float4 *g4 = reinterpret_cast<const float4 *>(g);
+  const int n8 = K / 8;
+  float ss = 0.0f, amax = 0.0f;
+  for (int i = threadIdx.x; i < n8; i += WIDE_NORM_THREADS) {
+    const float4 a = __ldg(xr + 2 * i);
+    const float4 b = __ldg(xr + 2 * i + 1);
+    ss += a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w + b.x * b.x + b.y * b.y + b.z * b.z +
+          b.w * b.w;
+    if (OUT_FP8) {
+      const float4 ga = __ldg(g4 + 2 * i);
+      const float4 gb = __ldg(g4 + 2 * i + 1);
+      amax = fmaxf(amax, fmaxf(fmaxf(fabsf(a.x * ga.x), fabsf(a.y * ga.y)),
+                               fmaxf(fabsf(a.z * ga.z), fabsf(a.w * ga.w))));
+      amax = fmaxf(amax, fmaxf(fmaxf(fabsf(b.x * gb.x), fabsf(b.y * gb.y)),
+                               fmaxf(fabsf(b.z * gb.z), fabsf(b.w * gb.w))));
+    }
+  }
+  ss = warp_sum(ss);
+  amax = warp_max(amax);
+  const int warp = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) {
+    red[0][warp] = ss;
+    red[1][warp] = amax;
+  }
+  __syncthreads();
+  ss = 0.0f;
+  amax = 0.0f;
+#pragma unroll
+  for (int w = 0; w < WIDE_NORM_THREADS / 32; ++w) {
+    ss += red[0][w];
+    amax = fmaxf(amax, red[1][w]);
+  }
+  const float rstd = rsqrtf(ss / static_cast<float>(K) + eps);
+  float mul = rstd;
+  if (OUT_FP8) {
+    const float qs = amax > 0.0f ? amax * rstd / 448.0f : 1.0f;
+    mul = rstd / qs;
+    if (threadIdx.x == 0) out_scale[row] = qs;
+  }
+  for (int i = threadIdx.x; i < n8; i += WIDE_NORM_THREADS) {
+    const float4 a = __ldg(xr + 2 * i);
+    const float4 b = __ldg(xr + 2 * i + 1);
+    const float4 ga = __ldg(g4 + 2 * i);
+    const float4 gb = __ldg(g4 + 2 * i + 1);
+    const float v[8] = {a.x * mul * ga.x, a.y * mul * ga.y, a.z * mul * ga.z, a.w * mul * ga.w,
+                        b.x * mul * gb.x, b.y * mul * gb.y, b.z * mul * gb.z, b.w * mul * gb.w};
+    if (OUT_FP8) {
+      uint2 w;
+      w.x = static_cast<uint32_t>(pack_e4m3x2(v[0], v[1])) |
+            (static_cast<uint32_t>(pack_e4m3x2(v[2], v[3])) << 16);
+      w.y = static_cast<uint32_t>(pack_e4m3x2(v[4], v[5])) |
+            (static_cast<uint32_t>(pack_e4m3x2(v[6], v[7])) << 16);
+      reinterpret_cast<uint2 *>(static_cast<uint8_t *>(out) + row * K)[i] = w;
+    } else {
+      reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(out) + row * K)[i] =
+          make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                     pack_bf16x2(v[6], v[7]));
+    }
+  }
+}
+
 // ------------------------------------------------ sampler: guided Euler step
 // z_out = z_in + dt * (v_u + gw * (v_c - v_u)) over n elements, 8 per thread
 // (one 16-byte load of each bf16 velocity, two of the fp32 latent); also

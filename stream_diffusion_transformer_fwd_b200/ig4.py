@@ -96,6 +96,9 @@ _sig("ig4_block_forward_noalloc", [ctypes.POINTER(Config), ctypes.POINTER(BlockW
 _sig("ig4_stack_workspace_size", [ctypes.POINTER(Config), _i], ctypes.c_size_t)
 _sig("ig4_stack_forward", [ctypes.POINTER(Config), ctypes.POINTER(StackWeights), _vp, _vp, _vp,
                            _vp, _vp, _vp, ctypes.c_size_t, _vp])
+_sig("ig4_text_cond_workspace_size", [_i, _i, _i], ctypes.c_size_t)
+_sig("ig4_text_cond_project", [_i, _i, _i, _vp, _vp, _f, _vp, _vp, _i, _vp, _vp, _vp,
+                               ctypes.c_size_t, _vp])
 _sig("ig4_flow_schedule", [_i, ctypes.c_double, ctypes.c_double, _i, _i,
                            ctypes.POINTER(ctypes.c_double)])
 _sig("ig4_guidance_schedule", [_i, _i, _f, _f, ctypes.POINTER(_f)])
@@ -112,7 +115,8 @@ EXPORTED = ("ig4_status_string", "ig4_abi_version", "ig4_mrope_positions", "ig4_
             "ig4_joint_attention", "ig4_gated_residual_linear", "ig4_swiglu",
             "ig4_quantize_rows", "ig4_workspace_size", "ig4_block_forward",
             "ig4_block_forward_traced", "ig4_block_forward_noalloc", "ig4_stack_workspace_size",
-            "ig4_stack_forward", "ig4_flow_schedule", "ig4_guidance_schedule", "ig4_cfg_euler",
+            "ig4_stack_forward", "ig4_text_cond_workspace_size", "ig4_text_cond_project",
+            "ig4_flow_schedule", "ig4_guidance_schedule", "ig4_cfg_euler",
             "ig4_denoise_workspace_size", "ig4_denoise_step", "ig4_last_device_error",
             "ig4_selftest_timeout")
 
@@ -311,6 +315,23 @@ def ig4_stack_forward(cfg: Config, sw: StackWeights, x_latent, text, out_latent,
                                   _ptr(text), _ptr(out_latent), _ptr(pos), _ptr(temb),
                                   _ptr(workspace), ws_bytes, _stream(stream)),
            "ig4_stack_forward")
+
+
+def ig4_text_cond_workspace_size(M: int, K_raw: int, w_dtype: str = "bf16") -> int:
+    return int(_lib.ig4_text_cond_workspace_size(M, K_raw, _NAME_CODE[w_dtype]))
+
+
+def ig4_text_cond_project(raw, g_norm, eps: float, w_proj, w_scale, b_proj, text_out, workspace,
+                          stream=None):
+    """text_out = RMSNorm(raw) * g_norm @ w_proj^T + b_proj (raw fp32 [M, K_raw])."""
+    K_raw = raw.shape[-1]
+    M = raw.numel() // K_raw
+    D = w_proj.shape[0]
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(_lib.ig4_text_cond_project(M, K_raw, D, _ptr(raw), _ptr(g_norm), eps, _ptr(w_proj),
+                                      _ptr(w_scale), dtype_code(w_proj), _ptr(b_proj),
+                                      _ptr(text_out), _ptr(workspace), ws_bytes,
+                                      _stream(stream)), "ig4_text_cond_project")
 
 
 def ig4_flow_schedule(num_steps: int, mu_base: float, std: float, height_px: int,

@@ -15,6 +15,7 @@ from .block_inputs import (  # noqa: F401
     make_block_weights_device,
     make_block_activations,
     make_stack_inputs,
+    make_text_cond_inputs,
     quantize_e4m3_per_channel,
     tensor_rng,
 )

@@ -149,3 +149,19 @@ def make_stack_inputs(cfg: Config, seed: int = 0, stress: bool = False) -> dict:
     out["w_out"], out["s_out"] = _linear(seed, 0, "w_out", C, D, cfg.w_dtype)
     out["b_out"] = _bias(seed, 0, "b_out", C, stress)
     return out
+
+
+def make_text_cond_inputs(M: int, K_raw: int, D: int, w_dtype: str = "bf16", seed: int = 0,
+                          stress: bool = False) -> dict:
+    """Inputs of the text conditioning projection: raw fp32 [M, K_raw] ~ N(0, 1)
+    (concatenated text-encoder features), g_norm fp32 [K_raw] (1, or 1 + N(0, 0.2^2)
+    with stress), w_proj [D, K_raw] ~ N(0, 1/K_raw) (+ scale for E4M3), b_proj
+    fp32 [D] (0, or N(0, 0.1^2) with stress)."""
+    out = {"raw": torch.from_numpy(_normal(seed, 0, "text_raw", (M, K_raw)))}
+    if stress:
+        out["g_norm"] = torch.from_numpy(1.0 + _normal(seed, 0, "g_text", (K_raw,), 0.2))
+    else:
+        out["g_norm"] = torch.ones(K_raw, dtype=torch.float32)
+    out["w_proj"], out["s_proj"] = _linear(seed, 0, "w_text_proj", D, K_raw, w_dtype)
+    out["b_proj"] = _bias(seed, 0, "b_text_proj", D, stress)
+    return out
