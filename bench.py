@@ -260,6 +260,8 @@ def run_ours(args, rank, local_rank, world):
     from synth import CONFIGS, make_block_activations, make_block_weights
 
     cfg = CONFIGS[args.config]
+    if cfg.name.startswith("textcond_"):
+        return run_textcond(args, cfg, ig4, rank, world, dev)
     if cfg.name.startswith("step_"):
         return run_step(args, cfg, ig4, rank, world, dev)
     if cfg.n_blocks > 1:
@@ -523,7 +525,8 @@ def run_stack(args, cfg, ig4, rank, world, dev):
         "e2e": {"value": round(world * flops * K / (ms_e2e * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(ms_e2e / K, 3)},
-        "gpu_launches": K * (cfg.n_blocks * (11 if fp8 else 9) + (7 if fp8 else 5)),
+        # per block 11 (FP8) or 9 launches, the rotary table only in the first block
+        "gpu_launches": K * (cfg.n_blocks * (10 if fp8 else 8) + 1 + (7 if fp8 else 5)),
         "cpu_baseline": None,
     }
     print(json.dumps(line), flush=True)
@@ -623,7 +626,7 @@ def run_step(args, cfg, ig4, rank, world, dev):
     t_min = gemm_f / ((2.0 if fp8 else 1.0) * bf16_peak * 1e12) + attn_f / (bf16_peak * 1e12)
     mixed_peak = flops / t_min / 1e12
     value = world * flops * K / (ms_total * 1e-3) / 1e12
-    per_stack = cfg.n_blocks * (11 if fp8 else 9)
+    per_stack = cfg.n_blocks * (10 if fp8 else 8) + 1
     launches = 2 * per_stack + (7 if fp8 else 5) + (6 if fp8 else 4) + 2
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
@@ -653,6 +656,88 @@ def run_step(args, cfg, ig4, rank, world, dev):
     }
     print(json.dumps(line), flush=True)
     del keep_c, keep_u
+    return 0
+
+
+def run_textcond(args, cfg, ig4, rank, world, dev):
+    """The text conditioning projection (llm_cond_norm + llm_cond_proj) of one
+    caption of cfg.T_text tokens per bench step."""
+    import torch
+    import torch.distributed as dist
+
+    from synth import make_text_cond_inputs
+
+    K_raw, D = 13 * 4096, cfg.D
+    M = cfg.B * cfg.T_text
+    inp = make_text_cond_inputs(M, K_raw, D, cfg.w_dtype, seed=rank)
+    d = {k: (None if v is None else v.to(dev)) for k, v in inp.items()}
+    out = torch.empty(M, D, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(ig4.ig4_text_cond_workspace_size(M, K_raw, cfg.w_dtype), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream()
+    K, W = args.steps, args.warmup
+
+    def call(raw, o):
+        ig4.ig4_text_cond_project(raw, d["g_norm"], cfg.eps, d["w_proj"], d["s_proj"], d["b_proj"],
+                                  o, ws)
+
+    for _ in range(W):
+        call(d["raw"], out)
+    torch.cuda.synchronize()
+    assert ig4.ig4_last_device_error() == ig4.IG4_OK
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(K):
+        call(d["raw"], out)
+    end.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    err = ig4.ig4_last_device_error()
+    ms_total = start.elapsed_time(end)
+    ms_e2e, h2d, d2h = e2e_pipelined([inp["raw"]], out, lambda din, o: call(din[0], o), K, 1)
+    if world > 1:
+        tt = torch.tensor([ms_total, ms_e2e], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_total, ms_e2e = tt.tolist()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    fp8 = cfg.w_dtype == "e4m3"
+    flops = 2.0 * M * K_raw * D
+    value = world * flops * K / (ms_total * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    held_max = bool(clocks) and clocks["sm_mhz"] >= 0.95 * clocks["sm_max_mhz"]
+    tkey = "bf16_tflops" if held_max else "bf16_tflops_sustained"
+    peak = (2.0 if fp8 else 1.0) * peaks.get(tkey, FALLBACK_PEAKS[tkey])
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": K, "warmup": W, "ms_per_step": round(ms_total / K, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8-e4m3 weights and features" if fp8 else "bf16",
+        "data": "synthetic (seeded N(0,1) raw features, N(0,1/fan_in) weights)",
+        "config": {"workload": (f"{cfg.name}: text conditioning projection, {M} tokens x "
+                                f"{K_raw} raw features -> {D}, w={cfg.w_dtype}"),
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2",
+                   "gflop_per_step": round(flops / 1e9, 1)},
+        "roofline": {"bound": "tensor", "achieved": round(value / world, 1), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(value / world / peak, 4), "traffic": None,
+                     "kernel": "norm + projection GEMM (GEMM flops only)",
+                     "peak_source": f"{'2 x ' if fp8 else ''}{tkey} ({peak_src})"},
+        "clocks": clocks, "device_error": ig4.ig4_status_string(err),
+        "e2e": {"value": round(world * flops * K / (ms_e2e * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(ms_e2e / K, 4)},
+        "gpu_launches": 2 * K,
+        "cpu_baseline": None,
+    }
+    print(json.dumps(line), flush=True)
     return 0
 
 

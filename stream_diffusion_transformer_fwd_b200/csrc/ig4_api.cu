@@ -259,13 +259,25 @@ template <typename XT, bool FP8>
 ig4_status launch_norm_t(int rows, int L, int D, const void *x, const float *shift,
                          const float *scale, int mod_stride, float eps, void *h, float *hs,
                          int remap_n, int remap_L, int remap_off, cudaStream_t st) {
-  const int grid = (rows + NORM_THREADS / 32 - 1) / (NORM_THREADS / 32);
+  DeviceInfo *di = nullptr;
+  IG4_TRY(device_info(&di));
+  // rows of one sample, and samples; one chunk of rows per CTA, about one CTA per SM
+  const int nb = remap_n > 0 ? remap_n : L;
+  const int B = rows / nb;
+  if (B < 1 || B * nb != rows) return IG4_ERR_INVALID_ARG;
+  const long per_cta = (static_cast<long>(rows) + di->sms - 1) / di->sms;
+  const int rows_per_cta =
+      static_cast<int>(std::max<long>(NORM_WARPS, (per_cta + NORM_WARPS - 1) / NORM_WARPS * NORM_WARPS));
+  const dim3 grid((nb + rows_per_cta - 1) / rows_per_cta, B);
+  const size_t smem = 2ull * D * sizeof(float);
+  if (smem > 48 * 1024) return IG4_ERR_UNSUPPORTED;
   const int nv = (D / 8 + 31) / 32;
   const XT *xp = static_cast<const XT *>(x);
 #define IG4_NORM_CASE(NV)                                                                        \
   if (nv <= NV) {                                                                                \
-    norm_modulate_kernel<XT, FP8, NV><<<grid, NORM_THREADS, 0, st>>>(                            \
-        xp, shift, scale, mod_stride, rows, L, D, eps, h, hs, remap_n, remap_L, remap_off);      \
+    norm_modulate_kernel<XT, FP8, NV><<<grid, NORM_THREADS, smem, st>>>(                         \
+        xp, shift, scale, mod_stride, L, D, eps, h, hs, remap_n, remap_L, remap_off,            \
+        rows_per_cta);                                                                           \
     return last_launch_status();                                                                 \
   }
   IG4_NORM_CASE(2)
@@ -597,9 +609,12 @@ struct Tracer {
 };
 
 // The block on already validated arguments.
+// rope_ready: ws.cos / ws.sin already hold the table of these positions (the
+// stack computes it for its first block only; every block shares it).
 ig4_status block_forward_impl(const ig4_config *c, const ig4_block_weights *w, const void *x_in,
                               void *x_out, const int32_t *pos, const float *temb,
-                              const BlockWs &ws, cudaStream_t st, Tracer *tr) {
+                              const BlockWs &ws, cudaStream_t st, Tracer *tr,
+                              bool rope_ready = false) {
   const int L = c->T_text + c->grid_t * c->grid_h * c->grid_w;
   const int M = c->B * L;
   const int D = c->D, I = c->I, H = c->H;
@@ -613,7 +628,8 @@ ig4_status block_forward_impl(const ig4_config *c, const ig4_block_weights *w, c
   IG4_TRY(launch_adaln(c->B, c->adaln_dim, 6 * D, temb, w->w_ada, c->w_dtype, w->s_ada, w->b_ada,
                        ws.mod, st));
   IG4_TRY(t.mark());
-  IG4_TRY(launch_rope_table(L, pos, c->rope_theta, c->sections, ws.cos, ws.sin, st));
+  if (!rope_ready)
+    IG4_TRY(launch_rope_table(L, pos, c->rope_theta, c->sections, ws.cos, ws.sin, st));
   IG4_TRY(t.mark());
   IG4_TRY(launch_norm(M, L, D, x_in, c->x_dtype, ws.mod + 0 * D, ws.mod + 1 * D, ms, c->eps, ws.h,
                       hdt, ws.h_scale, 0, 0, 0, st));
@@ -936,7 +952,8 @@ ig4_status ig4_stack_forward(const ig4_config *cfg, const ig4_stack_weights *sw,
   void *cur = ws.s0;
   void *nxt = ws.s1;
   for (int i = 0; i < sw->n_blocks; ++i) {
-    IG4_TRY(block_forward_impl(cfg, &sw->blocks[i], cur, nxt, pos, temb, ws.blk, st, nullptr));
+    IG4_TRY(block_forward_impl(cfg, &sw->blocks[i], cur, nxt, pos, temb, ws.blk, st, nullptr,
+                               i > 0));
     std::swap(cur, nxt);
   }
   // Final layer on the image tokens: RMSNorm + (shift, scale), then D -> C.

@@ -10,10 +10,13 @@ namespace ig4 {
 
 // ------------------------------------------------------------ AdaLN GEMV
 // mod[b][n] = sum_k SiLU(temb[b][k]) W[n][k] (* s[n]) + bias[n].
-// One warp per output row n (4 rows per warp in flight), B <= 8 samples share
-// each weight read; SiLU(temb) sits in shared memory.
+// One warp per group of 4 output rows: the warp first issues the loads of all
+// 4 weight rows (up to 4 16-byte vectors per lane and row, A * esize <= 2048
+// bytes), then reduces them, so 16 loads per lane are in flight at once.
+// B <= 8 samples share each weight read; SiLU(temb) sits in shared memory.
 constexpr int ADALN_THREADS = 256;
 constexpr int ADALN_ROWS_PER_WARP = 4;
+constexpr int ADALN_MAXV = 4;
 
 template <bool FP8>
 __global__ void __launch_bounds__(ADALN_THREADS)
@@ -30,6 +33,18 @@ __global__ void __launch_bounds__(ADALN_THREADS)
   const int esize = FP8 ? 1 : 2;
   const int vec_per_row = A * esize / 16;
   const int elems_per_vec = 16 / esize;
+  uint4 q[ADALN_ROWS_PER_WARP][ADALN_MAXV];
+#pragma unroll
+  for (int rr = 0; rr < ADALN_ROWS_PER_WARP; ++rr) {
+    const int n = n_base + rr;
+    const uint4 *row = reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(w) +
+                                                       static_cast<long>(n) * A * esize);
+#pragma unroll
+    for (int j = 0; j < ADALN_MAXV; ++j) {
+      const int v = lane + 32 * j;
+      if (n < N && v < vec_per_row) q[rr][j] = __ldg(row + v);
+    }
+  }
 #pragma unroll
   for (int rr = 0; rr < ADALN_ROWS_PER_WARP; ++rr) {
     const int n = n_base + rr;
@@ -37,17 +52,17 @@ __global__ void __launch_bounds__(ADALN_THREADS)
     float acc[8];
 #pragma unroll
     for (int b = 0; b < 8; ++b) acc[b] = 0.0f;
-    const uint4 *row = reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(w) +
-                                                       static_cast<long>(n) * A * esize);
-    for (int v = lane; v < vec_per_row; v += 32) {
-      const uint4 q = __ldg(row + v);
+#pragma unroll
+    for (int j = 0; j < ADALN_MAXV; ++j) {
+      const int v = lane + 32 * j;
+      if (v >= vec_per_row) break;
       float wv[16];
       if (FP8) {
-        const uint8_t *c = reinterpret_cast<const uint8_t *>(&q);
+        const uint8_t *c = reinterpret_cast<const uint8_t *>(&q[rr][j]);
 #pragma unroll
         for (int e = 0; e < 16; ++e) wv[e] = e4m3_to_f(c[e]);
       } else {
-        const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+        const uint32_t u[4] = {q[rr][j].x, q[rr][j].y, q[rr][j].z, q[rr][j].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           wv[2 * e] = __uint_as_float(u[e] << 16);
@@ -83,109 +98,170 @@ __global__ void __launch_bounds__(ADALN_THREADS)
 
 // ------------------------------------------------------ RMSNorm + modulate
 // h[r] = x[r] rsqrt(mean(x[r]^2) + eps) (1 + scale[b]) + shift[b].
-// One warp per row; the row stays in registers (NV 8-element vectors per
-// lane, D <= 256 * NV).  Optional row remap: input row = (r / remap_n) *
-// remap_L + remap_off + r % remap_n (the stack's final norm reads only the
-// image tokens).  FP8 output: per-row scale max|h| / 448 and E4M3 codes.
+// Grid (row chunks, samples): a CTA stages (1 + scale[b]) and shift[b] of its
+// sample in shared memory once, then its warps walk the chunk's rows, one
+// row per warp at a time with the row in registers (NV 8-element vectors per
+// lane, D <= 256 * NV); for bf16 input the next row's loads are issued before
+// the current row is normalised, so HBM latency overlaps the arithmetic.
+// Optional row remap: input row = (r / remap_n) * remap_L + remap_off +
+// r % remap_n (the stack's final norm reads only the image tokens).  FP8
+// output: per-row scale max|h| / 448 and E4M3 codes.
 constexpr int NORM_THREADS = 256;
+constexpr int NORM_WARPS = NORM_THREADS / 32;
+
+template <typename XT, int NV>
+struct NormRow;
+
+template <int NV>
+struct NormRow<__nv_bfloat16, NV> {
+  uint4 q[NV];
+  __device__ __forceinline__ void load(const __nv_bfloat16 *xr, int lane, int nvec) {
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int vi = lane + 32 * i;
+      if (vi < nvec) q[i] = __ldg(reinterpret_cast<const uint4 *>(xr) + vi);
+    }
+  }
+  __device__ __forceinline__ void unpack(int i, float (&v)[8]) const {
+    const uint32_t u[4] = {q[i].x, q[i].y, q[i].z, q[i].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v[2 * e] = __uint_as_float(u[e] << 16);
+      v[2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
+    }
+  }
+};
+
+template <int NV>
+struct NormRow<float, NV> {
+  float4 q[NV][2];
+  __device__ __forceinline__ void load(const float *xr, int lane, int nvec) {
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int vi = lane + 32 * i;
+      if (vi < nvec) {
+        q[i][0] = __ldg(reinterpret_cast<const float4 *>(xr) + 2 * vi);
+        q[i][1] = __ldg(reinterpret_cast<const float4 *>(xr) + 2 * vi + 1);
+      }
+    }
+  }
+  __device__ __forceinline__ void unpack(int i, float (&v)[8]) const {
+    v[0] = q[i][0].x; v[1] = q[i][0].y; v[2] = q[i][0].z; v[3] = q[i][0].w;
+    v[4] = q[i][1].x; v[5] = q[i][1].y; v[6] = q[i][1].z; v[7] = q[i][1].w;
+  }
+};
 
 template <typename XT, bool OUT_FP8, int NV>
-__global__ void __launch_bounds__(NORM_THREADS)
+__global__ void __launch_bounds__(NORM_THREADS, 1)
     norm_modulate_kernel(const XT *__restrict__ x, const float *__restrict__ shift,
-                         const float *__restrict__ scale, int mod_stride, int rows, int L, int D,
-                         float eps, void *__restrict__ h_out, float *__restrict__ h_scale,
-                         int remap_n, int remap_L, int remap_off) {
+                         const float *__restrict__ scale, int mod_stride, int L, int D, float eps,
+                         void *__restrict__ h_out, float *__restrict__ h_scale, int remap_n,
+                         int remap_L, int remap_off, int rows_per_cta) {
+  extern __shared__ float4 smod[];  // [D/4] (1 + scale), then [D/4] shift
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int r = blockIdx.x * (NORM_THREADS / 32) + warp;
-  if (r >= rows) return;
-  long in_row = r;
-  int b;
-  if (remap_n > 0) {
-    b = r / remap_n;
-    in_row = static_cast<long>(b) * remap_L + remap_off + r % remap_n;
-  } else {
-    b = r / L;
-  }
-  const XT *xr = x + in_row * D;
+  const int nb = remap_n > 0 ? remap_n : L;  // rows per sample
+  const int b = blockIdx.y;
+  const int r_begin = blockIdx.x * rows_per_cta;
+  const int r_end = min(r_begin + rows_per_cta, nb);
+  if (r_begin >= nb) return;
   const int nvec = D / 8;
-  float v[NV][8];
-  float ss = 0.0f;
-#pragma unroll
-  for (int i = 0; i < NV; ++i) {
+  const float4 *sc4 = reinterpret_cast<const float4 *>(scale + static_cast<long>(b) * mod_stride);
+  const float4 *sh4 = reinterpret_cast<const float4 *>(shift + static_cast<long>(b) * mod_stride);
+  for (int i = threadIdx.x; i < D / 4; i += NORM_THREADS) {
+    float4 s = __ldg(sc4 + i);
+    s.x += 1.0f;
+    s.y += 1.0f;
+    s.z += 1.0f;
+    s.w += 1.0f;
+    smod[i] = s;
+    smod[D / 4 + i] = __ldg(sh4 + i);
+  }
+  __syncthreads();
+  auto in_row = [&](int rr) -> long {
+    return remap_n > 0 ? static_cast<long>(b) * remap_L + remap_off + rr
+                       : static_cast<long>(b) * L + rr;
+  };
+  constexpr bool PREFETCH = sizeof(XT) == 2;
+  NormRow<XT, NV> cur, nxt;
+  // h of vector i of the current row (the row stays packed in registers;
+  // the unpacked values are recomputed per pass to keep register use low)
+  auto modulated = [&](int i, float rstd, float (&h)[8]) {
     const int vi = lane + 32 * i;
-    if (vi < nvec) {
-      if constexpr (sizeof(XT) == 4) {
-        const float4 a = __ldg(reinterpret_cast<const float4 *>(xr) + 2 * vi);
-        const float4 c = __ldg(reinterpret_cast<const float4 *>(xr) + 2 * vi + 1);
-        v[i][0] = a.x; v[i][1] = a.y; v[i][2] = a.z; v[i][3] = a.w;
-        v[i][4] = c.x; v[i][5] = c.y; v[i][6] = c.z; v[i][7] = c.w;
-      } else {
-        const uint4 q = __ldg(reinterpret_cast<const uint4 *>(xr) + vi);
-        const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+    cur.unpack(i, h);
+    const float4 s0 = smod[2 * vi], s1 = smod[2 * vi + 1];
+    const float4 t0 = smod[D / 4 + 2 * vi], t1 = smod[D / 4 + 2 * vi + 1];
+    const float scv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+    const float shv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          v[i][2 * e] = __uint_as_float(u[e] << 16);
-          v[i][2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
+    for (int e = 0; e < 8; ++e) h[e] = fmaf(h[e] * rstd, scv[e], shv[e]);
+  };
+  int rr = r_begin + warp;
+  if (rr < r_end) cur.load(x + in_row(rr) * D, lane, nvec);
+  for (; rr < r_end; rr += NORM_WARPS) {
+    const int rn = rr + NORM_WARPS;
+    if (PREFETCH && rn < r_end) nxt.load(x + in_row(rn) * D, lane, nvec);
+    float ss = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      if (lane + 32 * i < nvec) {
+        float v[8];
+        cur.unpack(i, v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ss = fmaf(v[e], v[e], ss);
+      }
+    }
+    ss = warp_sum(ss);
+    const float rstd = rsqrtf(ss / static_cast<float>(D) + eps);
+    const long r = static_cast<long>(b) * nb + rr;  // output row
+    if constexpr (OUT_FP8) {
+      float amax = 0.0f;
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        if (lane + 32 * i < nvec) {
+          float h[8];
+          modulated(i, rstd, h);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(h[e]));
         }
       }
+      amax = warp_max(amax);
+      const float qs = amax > 0.0f ? amax / 448.0f : 1.0f;
+      const float inv = 1.0f / qs;
+      uint8_t *hr = static_cast<uint8_t *>(h_out) + r * D;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) ss = fmaf(v[i][e], v[i][e], ss);
-    }
-  }
-  ss = warp_sum(ss);
-  const float rstd = rsqrtf(ss / static_cast<float>(D) + eps);
-  const float *sh = shift + static_cast<long>(b) * mod_stride;
-  const float *sc = scale + static_cast<long>(b) * mod_stride;
-  float amax = 0.0f;
+      for (int i = 0; i < NV; ++i) {
+        const int vi = lane + 32 * i;
+        if (vi < nvec) {
+          float h[8];
+          modulated(i, rstd, h);
+          uint2 w;
+          w.x = static_cast<uint32_t>(pack_e4m3x2(h[0] * inv, h[1] * inv)) |
+                (static_cast<uint32_t>(pack_e4m3x2(h[2] * inv, h[3] * inv)) << 16);
+          w.y = static_cast<uint32_t>(pack_e4m3x2(h[4] * inv, h[5] * inv)) |
+                (static_cast<uint32_t>(pack_e4m3x2(h[6] * inv, h[7] * inv)) << 16);
+          reinterpret_cast<uint2 *>(hr)[vi] = w;
+        }
+      }
+      if (lane == 0) h_scale[r] = qs;
+    } else {
+      __nv_bfloat16 *hr = static_cast<__nv_bfloat16 *>(h_out) + r * D;
 #pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    const int vi = lane + 32 * i;
-    if (vi < nvec) {
-      const float4 s0 = __ldg(reinterpret_cast<const float4 *>(sc) + 2 * vi);
-      const float4 s1 = __ldg(reinterpret_cast<const float4 *>(sc) + 2 * vi + 1);
-      const float4 t0 = __ldg(reinterpret_cast<const float4 *>(sh) + 2 * vi);
-      const float4 t1 = __ldg(reinterpret_cast<const float4 *>(sh) + 2 * vi + 1);
-      const float scv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-      const float shv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        v[i][e] = fmaf(v[i][e] * rstd, 1.0f + scv[e], shv[e]);
-        amax = fmaxf(amax, fabsf(v[i][e]));
+      for (int i = 0; i < NV; ++i) {
+        const int vi = lane + 32 * i;
+        if (vi < nvec) {
+          float h[8];
+          modulated(i, rstd, h);
+          reinterpret_cast<uint4 *>(hr)[vi] =
+              make_uint4(pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]),
+                         pack_bf16x2(h[4], h[5]), pack_bf16x2(h[6], h[7]));
+        }
       }
     }
-  }
-  if constexpr (OUT_FP8) {
-    amax = warp_max(amax);
-    const float qs = amax > 0.0f ? amax / 448.0f : 1.0f;
-    const float inv = 1.0f / qs;
-    uint8_t *hr = static_cast<uint8_t *>(h_out) + static_cast<long>(r) * D;
-#pragma unroll
-    for (int i = 0; i < NV; ++i) {
-      const int vi = lane + 32 * i;
-      if (vi < nvec) {
-        uint2 w;
-        w.x = static_cast<uint32_t>(pack_e4m3x2(v[i][0] * inv, v[i][1] * inv)) |
-              (static_cast<uint32_t>(pack_e4m3x2(v[i][2] * inv, v[i][3] * inv)) << 16);
-        w.y = static_cast<uint32_t>(pack_e4m3x2(v[i][4] * inv, v[i][5] * inv)) |
-              (static_cast<uint32_t>(pack_e4m3x2(v[i][6] * inv, v[i][7] * inv)) << 16);
-        reinterpret_cast<uint2 *>(hr)[vi] = w;
-      }
-    }
-    if (lane == 0) h_scale[r] = qs;
-  } else {
-    __nv_bfloat16 *hr = static_cast<__nv_bfloat16 *>(h_out) + static_cast<long>(r) * D;
-#pragma unroll
-    for (int i = 0; i < NV; ++i) {
-      const int vi = lane + 32 * i;
-      if (vi < nvec) {
-        uint4 w;
-        w.x = pack_bf16x2(v[i][0], v[i][1]);
-        w.y = pack_bf16x2(v[i][2], v[i][3]);
-        w.z = pack_bf16x2(v[i][4], v[i][5]);
-        w.w = pack_bf16x2(v[i][6], v[i][7]);
-        reinterpret_cast<uint4 *>(hr)[vi] = w;
-      }
+    if (PREFETCH) {
+      cur = nxt;
+    } else if (rn < r_end) {
+      cur.load(x + in_row(rn) * D, lane, nvec);
     }
   }
 }
