@@ -28,6 +28,8 @@ from .ig4_oracle import (  # noqa: F401
     block_forward,
     block_forward_rows,
     dequant_e4m3,
+    dequant_nvfp4,
+    e2m1_decode_table,
     e4m3_decode_table,
     joint_attention,
     merge_heads,

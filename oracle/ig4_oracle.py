@@ -390,6 +390,47 @@ def stack_forward(x_latent, text, temb, pos, block_weights, n_blocks, w_in, b_in
     return s_f[:, T:, :] @ np.asarray(w_out, dtype=np.float64).T + np.asarray(b_out, dtype=np.float64)
 
 
+def e2m1_decode_table() -> np.ndarray:
+    """Value of each of the 16 FP4 E2M1 codes, float64.
+
+    E2M1 (the float4_e2m1fn format the SGLang / ComfyUI NVFP4 weights use):
+    bit 3 sign, bits 2..1 exponent with bias 1, bit 0 mantissa; exponent 0 is
+    subnormal (value = mantissa * 0.5); no infinities or NaNs.
+    """
+    out = np.empty(16, dtype=np.float64)
+    for code in range(16):
+        sign = -1.0 if code & 8 else 1.0
+        e = (code >> 1) & 3
+        m = code & 1
+        mag = m * 0.5 if e == 0 else (1.0 + 0.5 * m) * 2.0 ** (e - 1)
+        out[code] = sign * mag
+    return out
+
+
+def dequant_nvfp4(packed, sf, s) -> np.ndarray:
+    """NVFP4 weight -> float64: W[n, k] = s[n] * decode_e4m3(sf[n, k // 16]) *
+    decode_e2m1(code[n, k]), code[n, 2i] in the low nibble of packed[n, i].
+
+    Source: "不用再充会员！Ideogram 4.0 NF4 免费本地部署" (the ComfyUI / ROCm
+    deployment article), section "2.2 NVFP4 Mixed": 4-bit floating-point
+    weights sharing an FP8 E4M3 scale per block of 64 (the page calls the
+    element format E2M3, which does not fit in 4 bits; the float4_e2m1fn type
+    it names elsewhere is E2M1, used here), FFN linears in NVFP4 and the
+    attention projections kept in FP8.  Stored here per 16-element sub-block,
+    the block the tensor cores apply, each 64-block's scale repeated; plus a
+    per-output-channel fp32 scale (reading: without it the block scales of
+    N(0, 1/4608) weights fall into E4M3's subnormal range).
+    """
+    packed = np.asarray(packed, dtype=np.uint8)
+    N = packed.shape[0]
+    codes = np.empty((N, 2 * packed.shape[1]), dtype=np.uint8)
+    codes[:, 0::2] = packed & 15
+    codes[:, 1::2] = packed >> 4
+    vals = e2m1_decode_table()[codes]
+    sbv = e4m3_decode_table()[np.asarray(sf, dtype=np.uint8)]
+    return np.asarray(s, dtype=np.float64)[:, None] * np.repeat(sbv, 16, axis=1) * vals
+
+
 # ---------------------------------------------------------------------------
 # text conditioning projection (the step before the stack)
 # ---------------------------------------------------------------------------

@@ -165,3 +165,61 @@ def make_text_cond_inputs(M: int, K_raw: int, D: int, w_dtype: str = "bf16", see
     out["w_proj"], out["s_proj"] = _linear(seed, 0, "w_text_proj", D, K_raw, w_dtype)
     out["b_proj"] = _bias(seed, 0, "b_text_proj", D, stress)
     return out
+
+
+# ----------------------------------------------------------------- NVFP4
+# E2M1 ("fp4"): sign, 2 exponent bits (bias 1), 1 mantissa bit; magnitudes of
+# codes 0..7: 0, 0.5, 1, 1.5, 2, 3, 4, 6.
+_E2M1_MAG = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0], dtype=np.float64)
+
+
+def _e2m1_encode(v: np.ndarray) -> np.ndarray:
+    """Nearest E2M1 code of each value (ties to the even code), saturating at
+    +-6; returns uint8 codes 0..15 (bit 3 = sign)."""
+    a = np.minimum(np.abs(v.astype(np.float64)), 6.0)
+    # distance to each magnitude; ties resolved toward the even code index
+    d = np.abs(a[..., None] - _E2M1_MAG)
+    best = np.argmin(d + 1e-12 * (np.arange(8) % 2), axis=-1).astype(np.uint8)
+    sign = ((v < 0) & (best > 0)).astype(np.uint8) << 3
+    return best | sign
+
+
+def _e4m3_round(v: np.ndarray) -> torch.Tensor:
+    """fp32 -> E4M3 (round to nearest even, saturating to +-448)."""
+    t = torch.from_numpy(np.ascontiguousarray(v, dtype=np.float32))
+    return t.clamp_(-E4M3_MAX, E4M3_MAX).to(torch.float8_e4m3fn)
+
+
+def quantize_nvfp4(w: np.ndarray, block: int = 64):
+    """fp32 [N, K] -> (codes uint8 [N, K/2], element 2i in the low nibble;
+    block scales E4M3 [N, K/16], each `block`-element block's scale repeated
+    over its 16-element sub-blocks; per-row fp32 scale [N]).
+
+    W[n, k] ~= s[n] * sb[n, k // 16] * e2m1(code[n, k]); s[n] = max|W[n]| /
+    (6 * 448) puts the largest block scale at 448, sb = RNE_E4M3(block amax /
+    (6 s[n])), codes = RNE_E2M1(W / (s sb))."""
+    w = np.asarray(w, dtype=np.float32)
+    N, K = w.shape
+    assert K % block == 0 and block % 16 == 0
+    amax = np.abs(w).max(axis=1)
+    s = np.where(amax > 0, amax / (6.0 * E4M3_MAX), 1.0).astype(np.float32)
+    bam = np.abs(w.reshape(N, K // block, block)).max(axis=2)
+    sb = _e4m3_round(bam / (6.0 * s[:, None]))
+    sbf = sb.to(torch.float32).numpy().astype(np.float64)
+    denom = np.repeat(s[:, None].astype(np.float64) * sbf, block, axis=1)
+    q = np.where(denom > 0, w / np.where(denom > 0, denom, 1.0), 0.0)
+    codes = _e2m1_encode(q)
+    packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+    sb16 = np.repeat(sb.view(torch.uint8).numpy(), block // 16, axis=1)
+    return (torch.from_numpy(packed), torch.from_numpy(np.ascontiguousarray(sb16)).view(torch.float8_e4m3fn),
+            torch.from_numpy(s))
+
+
+def make_nvfp4_linear(seed: int, block: int, name: str, n_out: int, n_in: int, std=None,
+                      block_elems: int = 64) -> dict:
+    """A linear layer's weight [n_out, n_in] ~ N(0, 1/n_in) in NVFP4 (see
+    quantize_nvfp4); keys codes, sf (E4M3 [n_out, n_in/16]), s (fp32 [n_out])."""
+    std = (1.0 / np.sqrt(n_in)) if std is None else std
+    w = _normal(seed, block, name, (n_out, n_in), std)
+    codes, sf, s = quantize_nvfp4(w, block_elems)
+    return {"codes": codes, "sf": sf, "s": s}
