@@ -260,6 +260,8 @@ def run_ours(args, rank, local_rank, world):
     from synth import CONFIGS, make_block_activations, make_block_weights
 
     cfg = CONFIGS[args.config]
+    if cfg.name.startswith("ffn_"):
+        return run_ffn_nvfp4(args, cfg, ig4, rank, world, dev)
     if cfg.name.startswith("textcond_"):
         return run_textcond(args, cfg, ig4, rank, world, dev)
     if cfg.name.startswith("step_"):
@@ -656,6 +658,119 @@ def run_step(args, cfg, ig4, rank, world, dev):
     }
     print(json.dumps(line), flush=True)
     del keep_c, keep_u
+    return 0
+
+
+def run_ffn_nvfp4(args, cfg, ig4, rank, world, dev):
+    """The block's FFN linears as NVFP4 GEMMs per bench step: gate and up
+    (M tokens x 2I rows x D) and down (M x D x I), block-scaled FP4 operands."""
+    import torch
+    import torch.distributed as dist
+
+    from synth.block_inputs import make_nvfp4_linear, quantize_nvfp4, _normal
+
+    M, D, I = cfg.M, cfg.D, cfg.I
+
+    def operand(codes, sf, s):
+        packed = torch.empty(ig4.ig4_nvfp4_scale_bytes(codes.shape[0], 2 * codes.shape[1]),
+                             dtype=torch.uint8, device=dev)
+        ig4.ig4_nvfp4_pack_scales(sf.view(torch.uint8).to(dev), packed)
+        return codes.to(dev), packed, s.to(dev)
+
+    w_gu = make_nvfp4_linear(rank, 0, "w_gate_up", 2 * I, D)
+    w_dn = make_nvfp4_linear(rank, 0, "w_down", D, I)
+    h = quantize_nvfp4(_normal(rank, 0, "h2", (M, D)), 16)
+    u = quantize_nvfp4(_normal(rank, 0, "u", (M, I)), 16)
+    W1 = operand(w_gu["codes"], w_gu["sf"], w_gu["s"])
+    W2 = operand(w_dn["codes"], w_dn["sf"], w_dn["s"])
+    A1 = operand(*h)
+    A2 = operand(*u)
+    o1 = torch.empty(M, 2 * I, dtype=torch.bfloat16, device=dev)
+    o2 = torch.empty(M, D, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+    K, W = args.steps, args.warmup
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+
+    def call(i=None):
+        if i is not None:
+            ev[i][0].record(stream)
+        ig4.ig4_nvfp4_linear(A1[0], A1[1], A1[2], W1[0], W1[1], W1[2], None, o1)
+        if i is not None:
+            ev[i][1].record(stream)
+        ig4.ig4_nvfp4_linear(A2[0], A2[1], A2[2], W2[0], W2[1], W2[2], None, o2)
+        if i is not None:
+            ev[i][2].record(stream)
+
+    for _ in range(W):
+        call()
+    torch.cuda.synchronize()
+    assert ig4.ig4_last_device_error() == ig4.IG4_OK
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(K):
+        call()
+    end.record(stream)
+    torch.cuda.synchronize()
+    ms_total = start.elapsed_time(end)
+    for i in range(K):
+        call(i)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    err = ig4.ig4_last_device_error()
+    ms_gu = sum(ev[i][0].elapsed_time(ev[i][1]) for i in range(K)) / K
+    ms_dn = sum(ev[i][1].elapsed_time(ev[i][2]) for i in range(K)) / K
+    host_in = [A1[0].cpu(), A2[0].cpu()]
+
+    def step_fn(din, o):
+        ig4.ig4_nvfp4_linear(din[0], A1[1], A1[2], W1[0], W1[1], W1[2], None, o1)
+        ig4.ig4_nvfp4_linear(din[1], A2[1], A2[2], W2[0], W2[1], W2[2], None, o)
+
+    ms_e2e, h2d, d2h = e2e_pipelined(host_in, o2, step_fn, K, 1)
+    if world > 1:
+        tt = torch.tensor([ms_total, ms_e2e], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_total, ms_e2e = tt.tolist()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    f_gu = 2.0 * M * D * 2 * I
+    f_dn = 2.0 * M * I * D
+    flops = f_gu + f_dn
+    value = world * flops * K / (ms_total * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    held_max = bool(clocks) and clocks["sm_mhz"] >= 0.95 * clocks["sm_max_mhz"]
+    tkey = "bf16_tflops" if held_max else "bf16_tflops_sustained"
+    peak = 4.0 * peaks.get(tkey, FALLBACK_PEAKS[tkey])
+    ach = f_gu / (ms_gu * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": K, "warmup": W, "ms_per_step": round(ms_total / K, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1 + ue4m3 block scales)",
+        "data": "synthetic (seeded N(0,1) activations and N(0,1/fan_in) weights, quantised)",
+        "config": {"workload": (f"{cfg.name}: FFN linears of the {cfg.L}-token block in NVFP4: "
+                                f"gate/up {M}x{2 * I}x{D} and down {M}x{D}x{I}"),
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2", "gflop_per_step": round(flops / 1e9, 1)},
+        "roofline": {"bound": "tensor", "achieved": round(ach, 1), "peak": round(peak, 1),
+                     "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": None,
+                     "kernel": "gemm_nvf4_kernel (gate/up)",
+                     "peak_source": f"4 x {tkey} ({peak_src}): nominal fp4/bf16 dense ratio"},
+        "kernel_ms": {"gate_up": round(ms_gu, 4), "down": round(ms_dn, 4)},
+        "kernel_tflops": {"gate_up": round(ach, 1), "down": round(f_dn / (ms_dn * 1e-3) / 1e12, 1)},
+        "clocks": clocks, "device_error": ig4.ig4_status_string(err),
+        "e2e": {"value": round(world * flops * K / (ms_e2e * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(ms_e2e / K, 4)},
+        "gpu_launches": 2 * K,
+        "cpu_baseline": None,
+    }
+    print(json.dumps(line), flush=True)
     return 0
 
 

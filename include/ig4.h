@@ -271,6 +271,37 @@ ig4_status ig4_stack_forward(const ig4_config *cfg, const ig4_stack_weights *sw,
                              const int32_t *pos, const float *temb, void *workspace,
                              size_t ws_bytes, void *stream);
 
+/* -------------------------------------------------------------- NVFP4 ---
+ * Block-scaled 4-bit linear layers ("不用再充会员！Ideogram 4.0 NF4 免费本地部署"
+ * deployment article, section "2.2 NVFP4 Mixed": FFN linears stored as
+ * 4-bit floats sharing an E4M3 scale per block; "SGLang cookbook: Ideogram
+ * 4": NVFP4 runs on B200 / Blackwell).  Operands are E2M1 codes (sign, 2
+ * exponent bits with bias 1, 1 mantissa bit), two per byte with element 2i
+ * in the low nibble, rows K-contiguous; each row has one UE4M3 scale per 16
+ * K-elements (a 64-element block format repeats its scale over the four
+ * 16-element sub-blocks) and one fp32 scale:
+ *   out[m][n] = a_scale[m] * w_scale[n] * sum_k A(m,k) W(n,k) (+ bias[n]),
+ *   A(m,k) = e4m3(a_sf[m][k/16]) * e2m1(a_code[m][k]), W likewise.
+ *
+ * ig4_nvfp4_scale_bytes: bytes of a packed scale array for `rows` rows of K
+ * elements (rows rounded up to 128; 0 if K is not a multiple of 64).
+ * ig4_nvfp4_pack_scales: row-major UE4M3 scales [rows][K/16] (device) ->
+ * the packed order the tensor cores read (per 128 rows and 64 K-elements a
+ * 512-byte block; byte 16 (r % 32) + 4 ((r % 128) / 32) + (k / 16) % 4);
+ * padding rows get zero scales.
+ * ig4_nvfp4_linear: M >= 1, N a multiple of 128, K a multiple of 256;
+ * a_codes [M][K/2], w_codes [N][K/2] bytes; a_sf, w_sf packed scales;
+ * a_scale [M], w_scale [N], bias [N] (or NULL) fp32; out [M][N] fp32 or bf16
+ * (out_dtype).  All device pointers 16-byte aligned; stream-ordered.
+ * Errors: IG4_ERR_INVALID_ARG. */
+size_t ig4_nvfp4_scale_bytes(int rows, int K);
+ig4_status ig4_nvfp4_pack_scales(int rows, int K, const void *sf_rows, void *sf_packed,
+                                 void *stream);
+ig4_status ig4_nvfp4_linear(int M, int N, int K, const void *a_codes, const void *a_sf,
+                            const float *a_scale, const void *w_codes, const void *w_sf,
+                            const float *w_scale, const float *bias, void *out, int out_dtype,
+                            void *stream);
+
 /* -------------------------------------------------- text conditioning ---
  * The step before the stack ("Ideogram 4 快速开始" (SimpleTuner quickstart),
  * section "Text embed cache"): the text encoder output concatenates the

@@ -531,6 +531,37 @@ ig4_status launch_store_bf16(int M, int N, int K, const void *a, const float *a_
   }
 }
 
+// NVFP4 linear layer on 128- or 256-wide tiles.
+template <int BN>
+ig4_status launch_nvf4(int M, int N, int K, const void *a_codes, const void *a_sf,
+                       const float *a_scale, const void *w_codes, const void *w_sf,
+                       const float *w_scale, const float *bias, void *out, int out_dtype, int sms,
+                       cudaStream_t st) {
+  CUtensorMap ma, mb;
+  IG4_TRY(map_2d(&ma, a_codes, 1, M, K / 2, K / 2, GEMM_BM, 128));
+  IG4_TRY(map_2d(&mb, w_codes, 1, N, K / 2, K / 2, BN, 128));
+  const int n_tiles_n = N / BN;
+  const long tiles = static_cast<long>((M + GEMM_BM - 1) / GEMM_BM) * n_tiles_n;
+  const int grid = static_cast<int>(std::min<long>(tiles, sms));
+  const int group_m = gemm_group_m(M, K / 2, 1);
+  const uint8_t *sa = static_cast<const uint8_t *>(a_sf);
+  const uint8_t *sw = static_cast<const uint8_t *>(w_sf);
+  constexpr int SMEM = Nvf4Shape<BN>::SMEM_BYTES;
+  if (out_dtype == IG4_F32) {
+    EpiStore<BN, true, float> e{static_cast<float *>(out), N, M, N, bias, a_scale, w_scale, 0, 0, 0};
+    auto kern = gemm_nvf4_kernel<BN, decltype(e)>;
+    IG4_TRY(allow_smem(kern, SMEM));
+    kern<<<grid, GEMM_THREADS, SMEM, st>>>(ma, mb, sa, sw, M, n_tiles_n, K, group_m, e);
+  } else {
+    EpiStore<BN, true, __nv_bfloat16> e{static_cast<__nv_bfloat16 *>(out), N, M, N, bias, a_scale,
+                                        w_scale, 0, 0, 0};
+    auto kern = gemm_nvf4_kernel<BN, decltype(e)>;
+    IG4_TRY(allow_smem(kern, SMEM));
+    kern<<<grid, GEMM_THREADS, SMEM, st>>>(ma, mb, sa, sw, M, n_tiles_n, K, group_m, e);
+  }
+  return last_launch_status();
+}
+
 // ------------------------------------------------------- workspace layout
 
 struct BlockWs {
@@ -964,6 +995,48 @@ ig4_status ig4_stack_forward(const ig4_config *cfg, const ig4_stack_weights *sw,
   IG4_TRY(launch_linear_store(B * N, C, D, ws.hf, false, nullptr, w_out, nullptr, sw->b_out,
                               out_latent, IG4_BF16, C, 0, 0, 0, st));
   return IG4_OK;
+}
+
+// ----------------------------------------------------------------- NVFP4
+
+
+size_t ig4_nvfp4_scale_bytes(int rows, int K) {
+  if (rows < 1 || K < 64 || K % 64) return 0;
+  return static_cast<size_t>((rows + 127) / 128) * (K / 64) * 512;
+}
+
+ig4_status ig4_nvfp4_pack_scales(int rows, int K, const void *sf_rows, void *sf_packed,
+                                 void *stream) {
+  if (rows < 1 || K < 64 || K % 64 || !sf_rows || !sf_packed) return IG4_ERR_INVALID_ARG;
+  const long total = static_cast<long>(ig4_nvfp4_scale_bytes(rows, K));
+  DeviceInfo *di = nullptr;
+  IG4_TRY(device_info(&di));
+  const int grid = static_cast<int>(std::min<long>((total + 255) / 256, 8L * di->sms));
+  nvf4_pack_scales_kernel<<<grid, 256, 0, as_stream(stream)>>>(
+      static_cast<const uint8_t *>(sf_rows), static_cast<uint8_t *>(sf_packed), rows, K, total);
+  return last_launch_status();
+}
+
+ig4_status ig4_nvfp4_linear(int M, int N, int K, const void *a_codes, const void *a_sf,
+                            const float *a_scale, const void *w_codes, const void *w_sf,
+                            const float *w_scale, const float *bias, void *out, int out_dtype,
+                            void *stream) {
+  if (M < 1 || N < 128 || N % 128 || K < 256 || K % 256) return IG4_ERR_INVALID_ARG;
+  if (out_dtype != IG4_F32 && out_dtype != IG4_BF16) return IG4_ERR_INVALID_ARG;
+  const void *ptrs[] = {a_codes, a_sf, a_scale, w_codes, w_sf, w_scale, out};
+  for (const void *p : ptrs)
+    if (!p || !aligned16(p)) return IG4_ERR_INVALID_ARG;
+  if (bias && !aligned16(bias)) return IG4_ERR_INVALID_ARG;
+  DeviceInfo *di = nullptr;
+  IG4_TRY(device_info(&di));
+  // 256-wide tiles (one accumulator, fewer operand bytes per flop) once there
+  // are at least two waves of them, else 128-wide tiles
+  const long tiles256 = static_cast<long>((M + GEMM_BM - 1) / GEMM_BM) * (N / 256);
+  if (N % 256 == 0 && tiles256 >= 2L * di->sms)
+    return launch_nvf4<256>(M, N, K, a_codes, a_sf, a_scale, w_codes, w_sf, w_scale, bias, out,
+                            out_dtype, di->sms, as_stream(stream));
+  return launch_nvf4<128>(M, N, K, a_codes, a_sf, a_scale, w_codes, w_sf, w_scale, bias, out,
+                          out_dtype, di->sms, as_stream(stream));
 }
 
 // --------------------------------------------------- text conditioning

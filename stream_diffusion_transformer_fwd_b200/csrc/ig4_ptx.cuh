@@ -97,6 +97,17 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }
 
+// Plain bulk copy global -> shared of `bytes` (multiple of 16, both
+// addresses 16-byte aligned), completing on `bar`'s transaction count.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes,
+                                          uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *m, uint64_t *bar, int c0,
                                             int c1) {
   asm volatile(
@@ -198,6 +209,30 @@ __device__ __forceinline__ void umma_f8(uint32_t d_tmem, uint64_t a_desc, uint64
       : "memory");
 }
 
+// Block-scaled FP4 MMA (NVFP4): A and B E2M1, one UE4M3 scale per 16
+// K-elements of each operand row, read from TMEM at sfa_tmem / sfb_tmem
+// (four columns each: column c holds the four scales of rows c*32 + lane);
+// K = 64 per instruction.
+__device__ __forceinline__ void umma_nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], "
+      "p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Copy a 512-byte scale-factor block (32 rows of 16 bytes in shared memory)
+// into TMEM lanes 0..31, four 32-bit columns, replicated to the other three
+// lane quarters (tcgen05.cp 32x128b.warpx4).
+__device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t s_desc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(s_desc)
+               : "memory");
+}
+
 // Arrive once on `bar` when every tcgen05 operation this thread issued so far
 // has completed.
 __device__ __forceinline__ void umma_commit(uint64_t *bar) {
@@ -268,6 +303,25 @@ __device__ __forceinline__ uint64_t sdesc_kmajor_sw128(uint32_t saddr) {
   d |= static_cast<uint64_t>(1u) << 46;
   d |= static_cast<uint64_t>(2u) << 61;
   return d;
+}
+
+// Shared-memory descriptor of an unswizzled K-major operand made of 8-row x
+// 16-byte core matrices stacked every `sbo` bytes (the 512-byte scale-factor
+// blocks: 4 core matrices, sbo = 128).
+__device__ __forceinline__ uint64_t sdesc_kmajor_none(uint32_t saddr, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(1u) << 16;  // leading offset (one core matrix wide: unused)
+  d |= static_cast<uint64_t>(sbo >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  return d;  // layout type 0: no swizzle
+}
+
+// Instruction descriptor of a block-scaled FP4 MMA: A, B E2M1 (format 1),
+// UE4M3 scales (bit 23 = 0), K-major, dense K = 64, fp32 accumulation.
+__host__ __device__ constexpr uint32_t idesc_nvf4(int M, int N) {
+  return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 // Instruction descriptor of a dense MMA with fp32 accumulation, both operands

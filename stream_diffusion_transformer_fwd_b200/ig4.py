@@ -96,6 +96,9 @@ _sig("ig4_block_forward_noalloc", [ctypes.POINTER(Config), ctypes.POINTER(BlockW
 _sig("ig4_stack_workspace_size", [ctypes.POINTER(Config), _i], ctypes.c_size_t)
 _sig("ig4_stack_forward", [ctypes.POINTER(Config), ctypes.POINTER(StackWeights), _vp, _vp, _vp,
                            _vp, _vp, _vp, ctypes.c_size_t, _vp])
+_sig("ig4_nvfp4_scale_bytes", [_i, _i], ctypes.c_size_t)
+_sig("ig4_nvfp4_pack_scales", [_i, _i, _vp, _vp, _vp])
+_sig("ig4_nvfp4_linear", [_i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp])
 _sig("ig4_text_cond_workspace_size", [_i, _i, _i], ctypes.c_size_t)
 _sig("ig4_text_cond_project", [_i, _i, _i, _vp, _vp, _f, _vp, _vp, _i, _vp, _vp, _vp,
                                ctypes.c_size_t, _vp])
@@ -115,7 +118,8 @@ EXPORTED = ("ig4_status_string", "ig4_abi_version", "ig4_mrope_positions", "ig4_
             "ig4_joint_attention", "ig4_gated_residual_linear", "ig4_swiglu",
             "ig4_quantize_rows", "ig4_workspace_size", "ig4_block_forward",
             "ig4_block_forward_traced", "ig4_block_forward_noalloc", "ig4_stack_workspace_size",
-            "ig4_stack_forward", "ig4_text_cond_workspace_size", "ig4_text_cond_project",
+            "ig4_stack_forward", "ig4_nvfp4_scale_bytes", "ig4_nvfp4_pack_scales",
+            "ig4_nvfp4_linear", "ig4_text_cond_workspace_size", "ig4_text_cond_project",
             "ig4_flow_schedule", "ig4_guidance_schedule", "ig4_cfg_euler",
             "ig4_denoise_workspace_size", "ig4_denoise_step", "ig4_last_device_error",
             "ig4_selftest_timeout")
@@ -315,6 +319,26 @@ def ig4_stack_forward(cfg: Config, sw: StackWeights, x_latent, text, out_latent,
                                   _ptr(text), _ptr(out_latent), _ptr(pos), _ptr(temb),
                                   _ptr(workspace), ws_bytes, _stream(stream)),
            "ig4_stack_forward")
+
+
+def ig4_nvfp4_scale_bytes(rows: int, K: int) -> int:
+    return int(_lib.ig4_nvfp4_scale_bytes(rows, K))
+
+
+def ig4_nvfp4_pack_scales(sf_rows, sf_packed, stream=None):
+    """Row-major UE4M3 scales [rows, K/16] (uint8 or float8_e4m3fn) -> packed order."""
+    rows, k16 = sf_rows.shape
+    _check(_lib.ig4_nvfp4_pack_scales(rows, 16 * k16, _ptr(sf_rows), _ptr(sf_packed),
+                                      _stream(stream)), "ig4_nvfp4_pack_scales")
+
+
+def ig4_nvfp4_linear(a_codes, a_sf, a_scale, w_codes, w_sf, w_scale, bias, out, stream=None):
+    """out = a_scale[:, None] * w_scale[None] * (A W^T) (+ bias); codes [rows, K/2] uint8."""
+    M, K = a_codes.shape[0], 2 * a_codes.shape[1]
+    N = w_codes.shape[0]
+    _check(_lib.ig4_nvfp4_linear(M, N, K, _ptr(a_codes), _ptr(a_sf), _ptr(a_scale), _ptr(w_codes),
+                                 _ptr(w_sf), _ptr(w_scale), _ptr(bias), _ptr(out),
+                                 dtype_code(out), _stream(stream)), "ig4_nvfp4_linear")
 
 
 def ig4_text_cond_workspace_size(M: int, K_raw: int, w_dtype: str = "bf16") -> int:

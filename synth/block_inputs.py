@@ -173,15 +173,18 @@ def make_text_cond_inputs(M: int, K_raw: int, D: int, w_dtype: str = "bf16", see
 _E2M1_MAG = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0], dtype=np.float64)
 
 
+_E2M1_MID = 0.5 * (_E2M1_MAG[1:] + _E2M1_MAG[:-1])  # decision points between codes
+
+
 def _e2m1_encode(v: np.ndarray) -> np.ndarray:
     """Nearest E2M1 code of each value (ties to the even code), saturating at
     +-6; returns uint8 codes 0..15 (bit 3 = sign)."""
     a = np.minimum(np.abs(v.astype(np.float64)), 6.0)
-    # distance to each magnitude; ties resolved toward the even code index
-    d = np.abs(a[..., None] - _E2M1_MAG)
-    best = np.argmin(d + 1e-12 * (np.arange(8) % 2), axis=-1).astype(np.uint8)
-    sign = ((v < 0) & (best > 0)).astype(np.uint8) << 3
-    return best | sign
+    idx = np.searchsorted(_E2M1_MID, a, side="left")  # midpoints strictly below a
+    tie = (idx < 7) & (a == _E2M1_MID[np.minimum(idx, 6)])
+    idx = np.where(tie & (idx % 2 == 1), idx + 1, idx).astype(np.uint8)
+    sign = ((v < 0) & (idx > 0)).astype(np.uint8) << 3
+    return idx | sign
 
 
 def _e4m3_round(v: np.ndarray) -> torch.Tensor:

@@ -70,6 +70,10 @@ CONFIGS = {
     # 64x64 image tokens and the separate image-only unconditional stack, FP8
     "step_1024px_fp8": Config("step_1024px_fp8", B=1, T_text=512, grid_t=1, grid_h=64,
                               grid_w=64, w_dtype="e4m3", n_blocks=34),
+    # the block's FFN linears with NVFP4 weights (the NVFP4 Mixed scheme keeps
+    # the attention projections in FP8): gate/up and down at 1024 px
+    "ffn_1024px_nvfp4": Config("ffn_1024px_nvfp4", B=1, T_text=512, grid_t=1, grid_h=64,
+                               grid_w=64, w_dtype="nvfp4"),
     # the text conditioning projection of a 2048-token caption (13 x 4096 = 53248
     # raw features per token -> 4608), FP8 weights as released
     "textcond_2048_fp8": Config("textcond_2048_fp8", B=1, T_text=2048, grid_t=1, grid_h=0,
