@@ -12,6 +12,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "ig4.h"
 #include "ig4_attention.cuh"
@@ -29,6 +30,25 @@ constexpr int ABI_VERSION = 1;
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while the previous kernel on the stream drains; every kernel launched this
+// way waits (griddepcontrol.wait, pdl_wait()) before touching global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args &&...args) {
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = grid;
+  lc.blockDim = block;
+  lc.dynamicSmemBytes = smem;
+  lc.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  return cudaLaunchKernelEx(&lc, kern, std::forward<Args>(args)...);
+}
 
 // Inverse of the standard normal CDF Phi(x) = erfc(-x / sqrt 2) / 2 for
 // 0 < p < 1, by bisection (Phi is monotone; 200 halvings reach the spacing of
@@ -184,13 +204,15 @@ ig4_status launch_gemm(const CUtensorMap &A, const CUtensorMap &B, const CUtenso
       lc.blockDim = dim3(GEMM_THREADS);
       lc.dynamicSmemBytes = PAIR_SMEM_BYTES;
       lc.stream = st;
-      cudaLaunchAttribute attr[1];
+      cudaLaunchAttribute attr[2];
       attr[0].id = cudaLaunchAttributeClusterDimension;
       attr[0].val.clusterDim.x = 2;
       attr[0].val.clusterDim.y = 1;
       attr[0].val.clusterDim.z = 1;
+      attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[1].val.programmaticStreamSerializationAllowed = 1;
       lc.attrs = attr;
-      lc.numAttrs = 1;
+      lc.numAttrs = 2;
       if (cudaLaunchKernelEx(&lc, kern, A, B, B2, M, n_tiles_n, K, group_m, epi) != cudaSuccess)
         return IG4_ERR_CUDA;
       return last_launch_status();
@@ -201,7 +223,9 @@ ig4_status launch_gemm(const CUtensorMap &A, const CUtensorMap &B, const CUtenso
   IG4_TRY(allow_smem(kern, SMEM));
   const long tiles = static_cast<long>((M + GEMM_BM - 1) / GEMM_BM) * n_tiles_n;
   const int grid = static_cast<int>(std::min<long>(tiles, di->sms));
-  kern<<<grid, GEMM_THREADS, SMEM, st>>>(A, B, B2, M, n_tiles_n, K, group_m, epi);
+  if (launch_pdl(kern, dim3(grid), dim3(GEMM_THREADS), SMEM, st, A, B, B2, M, n_tiles_n, K,
+                 group_m, epi) != cudaSuccess)
+    return IG4_ERR_CUDA;
   return last_launch_status();
 }
 
@@ -248,10 +272,13 @@ ig4_status launch_adaln(int B, int A, int N, const float *temb, const void *w, i
   const int rows_per_cta = (ADALN_THREADS / 32) * ADALN_ROWS_PER_WARP;
   const int grid = (N + rows_per_cta - 1) / rows_per_cta;
   const int smem = B * A * 4;
-  if (is_fp8(w_dtype))
-    adaln_kernel<true><<<grid, ADALN_THREADS, smem, st>>>(temb, w, w_scale, bias, mod, B, A, N);
-  else
-    adaln_kernel<false><<<grid, ADALN_THREADS, smem, st>>>(temb, w, w_scale, bias, mod, B, A, N);
+  const cudaError_t e =
+      is_fp8(w_dtype)
+          ? launch_pdl(adaln_kernel<true>, dim3(grid), dim3(ADALN_THREADS), smem, st, temb, w,
+                       w_scale, bias, mod, B, A, N)
+          : launch_pdl(adaln_kernel<false>, dim3(grid), dim3(ADALN_THREADS), smem, st, temb, w,
+                       w_scale, bias, mod, B, A, N);
+  if (e != cudaSuccess) return IG4_ERR_CUDA;
   return last_launch_status();
 }
 
@@ -275,9 +302,10 @@ ig4_status launch_norm_t(int rows, int L, int D, const void *x, const float *shi
   const XT *xp = static_cast<const XT *>(x);
 #define IG4_NORM_CASE(NV)                                                                        \
   if (nv <= NV) {                                                                                \
-    norm_modulate_kernel<XT, FP8, NV><<<grid, NORM_THREADS, smem, st>>>(                         \
-        xp, shift, scale, mod_stride, L, D, eps, h, hs, remap_n, remap_L, remap_off,            \
-        rows_per_cta);                                                                           \
+    if (launch_pdl(norm_modulate_kernel<XT, FP8, NV>, grid, dim3(NORM_THREADS), smem, st, xp,   \
+                   shift, scale, mod_stride, L, D, eps, h, hs, remap_n, remap_L, remap_off,     \
+                   rows_per_cta) != cudaSuccess)                                                 \
+      return IG4_ERR_CUDA;                                                                       \
     return last_launch_status();                                                                 \
   }
   IG4_NORM_CASE(2)
@@ -308,7 +336,9 @@ ig4_status launch_norm(int rows, int L, int D, const void *x, int x_dtype, const
 ig4_status launch_rope_table(int L, const int32_t *pos, double theta, const int sec[3], float *c,
                              float *s, cudaStream_t st) {
   const int n = L * 64;
-  rope_table_kernel<<<(n + 255) / 256, 256, 0, st>>>(pos, L, theta, sec[0], sec[1], c, s);
+  if (launch_pdl(rope_table_kernel, dim3((n + 255) / 256), dim3(256), 0, st, pos, L, theta, sec[0],
+                 sec[1], c, s) != cudaSuccess)
+    return IG4_ERR_CUDA;
   return last_launch_status();
 }
 
@@ -318,7 +348,9 @@ ig4_status launch_quantize(int M, int K, const void *x, void *q, float *scale, c
   uint8_t *qp = static_cast<uint8_t *>(q);
 #define IG4_Q_CASE(NV)                                                                   \
   if (nv <= NV) {                                                                        \
-    quantize_rows_kernel<NV><<<M, QUANT_THREADS, 0, st>>>(xp, qp, scale, K);             \
+    if (launch_pdl(quantize_rows_kernel<NV>, dim3(M), dim3(QUANT_THREADS), 0, st, xp, qp,  \
+                   scale, K) != cudaSuccess)                                             \
+      return IG4_ERR_CUDA;                                                               \
     return last_launch_status();                                                         \
   }
   IG4_Q_CASE(1)
@@ -363,8 +395,9 @@ ig4_status launch_attention(int B, int H, int L, const void *q, const void *k, c
   IG4_TRY(map_3d_bf16(&mv, vt, L, 256, BH, vt_ld, 256L * vt_ld, 64, 256));
   IG4_TRY(allow_smem(attention_kernel, ATT_SMEM_BYTES));
   dim3 grid((L + ATT_BM - 1) / ATT_BM, H, B);
-  attention_kernel<<<grid, ATT_THREADS, ATT_SMEM_BYTES, st>>>(
-      mq, mk, mv, static_cast<__nv_bfloat16 *>(o), L, H);
+  if (launch_pdl(attention_kernel, grid, dim3(ATT_THREADS), ATT_SMEM_BYTES, st, mq, mk, mv,
+                 static_cast<__nv_bfloat16 *>(o), L, H) != cudaSuccess)
+    return IG4_ERR_CUDA;
   return last_launch_status();
 }
 
@@ -468,8 +501,10 @@ ig4_status launch_swiglu(int M, int I, int K, const void *h, bool f8, const floa
 ig4_status launch_dequant(int N, int K, const void *q, const float *s, void *out, cudaStream_t st) {
   const long total16 = static_cast<long>(N) * K / 16;
   const int grid = static_cast<int>(std::min<long>((total16 + 255) / 256, 148L * 16));
-  dequant_e4m3_rows_kernel<<<grid, 256, 0, st>>>(static_cast<const uint8_t *>(q), s,
-                                                 static_cast<__nv_bfloat16 *>(out), K, total16);
+  if (launch_pdl(dequant_e4m3_rows_kernel, dim3(grid), dim3(256), 0, st,
+                 static_cast<const uint8_t *>(q), s, static_cast<__nv_bfloat16 *>(out), K,
+                 total16) != cudaSuccess)
+    return IG4_ERR_CUDA;
   return last_launch_status();
 }
 
@@ -551,13 +586,17 @@ ig4_status launch_nvf4(int M, int N, int K, const void *a_codes, const void *a_s
     EpiStore<BN, true, float> e{static_cast<float *>(out), N, M, N, bias, a_scale, w_scale, 0, 0, 0};
     auto kern = gemm_nvf4_kernel<BN, decltype(e)>;
     IG4_TRY(allow_smem(kern, SMEM));
-    kern<<<grid, GEMM_THREADS, SMEM, st>>>(ma, mb, sa, sw, M, n_tiles_n, K, group_m, e);
+    if (launch_pdl(kern, dim3(grid), dim3(GEMM_THREADS), SMEM, st, ma, mb, sa, sw, M, n_tiles_n, K,
+                   group_m, e) != cudaSuccess)
+      return IG4_ERR_CUDA;
   } else {
     EpiStore<BN, true, __nv_bfloat16> e{static_cast<__nv_bfloat16 *>(out), N, M, N, bias, a_scale,
                                         w_scale, 0, 0, 0};
     auto kern = gemm_nvf4_kernel<BN, decltype(e)>;
     IG4_TRY(allow_smem(kern, SMEM));
-    kern<<<grid, GEMM_THREADS, SMEM, st>>>(ma, mb, sa, sw, M, n_tiles_n, K, group_m, e);
+    if (launch_pdl(kern, dim3(grid), dim3(GEMM_THREADS), SMEM, st, ma, mb, sa, sw, M, n_tiles_n, K,
+                   group_m, e) != cudaSuccess)
+      return IG4_ERR_CUDA;
   }
   return last_launch_status();
 }
@@ -963,8 +1002,10 @@ ig4_status ig4_stack_forward(const ig4_config *cfg, const ig4_stack_weights *sw,
     const int vpr = D * 2 / 16;
     const long total = static_cast<long>(B) * T * vpr;
     const int grid = static_cast<int>(std::min<long>((total + 255) / 256, 148L * 8));
-    copy_rows_kernel<<<grid, 256, 0, st>>>(static_cast<const uint4 *>(text),
-                                           static_cast<uint4 *>(ws.s0), T, L, 0, vpr, total);
+    if (launch_pdl(copy_rows_kernel, dim3(grid), dim3(256), 0, st,
+                   static_cast<const uint4 *>(text), static_cast<uint4 *>(ws.s0), T, L, 0, vpr,
+                   total) != cudaSuccess)
+      return IG4_ERR_CUDA;
     IG4_TRY(last_launch_status());
   }
   // The latent in/out projections are 0.01% of the step's work: they run in
@@ -1069,11 +1110,12 @@ ig4_status ig4_text_cond_project(int M, int K_raw, int D, const float *raw, cons
   float *h_scale = reinterpret_cast<float *>(
       h + round_up((f8 ? 1 : 2) * static_cast<size_t>(M) * K_raw, 256));
   // llm_cond_norm: RMSNorm over the concatenated features, into bf16 / E4M3
-  if (f8)
-    wide_rmsnorm_kernel<true><<<M, WIDE_NORM_THREADS, 0, st>>>(raw, g_norm, K_raw, eps, h, h_scale);
-  else
-    wide_rmsnorm_kernel<false><<<M, WIDE_NORM_THREADS, 0, st>>>(raw, g_norm, K_raw, eps, h,
-                                                                nullptr);
+  const cudaError_t e =
+      f8 ? launch_pdl(wide_rmsnorm_kernel<true>, dim3(M), dim3(WIDE_NORM_THREADS), 0, st, raw,
+                      g_norm, K_raw, eps, static_cast<void *>(h), h_scale)
+         : launch_pdl(wide_rmsnorm_kernel<false>, dim3(M), dim3(WIDE_NORM_THREADS), 0, st, raw,
+                      g_norm, K_raw, eps, static_cast<void *>(h), static_cast<float *>(nullptr));
+  if (e != cudaSuccess) return IG4_ERR_CUDA;
   IG4_TRY(last_launch_status());
   // llm_cond_proj: K_raw -> D with bias, bf16 out
   if (f8) return launch_store_bf16<true>(M, D, K_raw, h, h_scale, w_proj, w_scale, b_proj, text_out, st);
@@ -1123,10 +1165,11 @@ ig4_status ig4_cfg_euler(long long n, const void *v_cond, const void *v_uncond, 
   IG4_TRY(device_info(&di));
   const long n8 = n / 8;
   const int grid = static_cast<int>(std::min<long>((n8 + 255) / 256, 8L * di->sms));
-  cfg_euler_kernel<<<grid, 256, 0, as_stream(stream)>>>(
-      static_cast<const uint4 *>(v_cond), static_cast<const uint4 *>(v_uncond), gw, dt,
-      reinterpret_cast<const float4 *>(z_in), reinterpret_cast<float4 *>(z_out),
-      static_cast<uint4 *>(z16_out), n8);
+  if (launch_pdl(cfg_euler_kernel, dim3(grid), dim3(256), 0, as_stream(stream),
+                 static_cast<const uint4 *>(v_cond), static_cast<const uint4 *>(v_uncond), gw, dt,
+                 reinterpret_cast<const float4 *>(z_in), reinterpret_cast<float4 *>(z_out),
+                 static_cast<uint4 *>(z16_out), n8) != cudaSuccess)
+    return IG4_ERR_CUDA;
   return last_launch_status();
 }
 

@@ -30,6 +30,19 @@ __device__ __forceinline__ unsigned long long globaltimer_ns() {
   return t;
 }
 
+// ------------------------------------------- programmatic dependent launch
+// Kernels are launched with programmatic stream serialization: a kernel may
+// start (barrier set-up, TMEM allocation, descriptor prefetch) while the one
+// before it on the stream drains, and waits here before its first global
+// memory access until that kernel has finished and its writes are visible.
+// Without the launch attribute both instructions do nothing.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the next kernel on the stream be scheduled once every CTA of this one
+// has issued this (its CTAs still wait in pdl_wait for this kernel's end).
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {

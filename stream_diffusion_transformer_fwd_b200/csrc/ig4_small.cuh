@@ -23,6 +23,8 @@ __global__ void __launch_bounds__(ADALN_THREADS)
     adaln_kernel(const float *__restrict__ temb, const void *__restrict__ w,
                  const float *__restrict__ w_scale, const float *__restrict__ bias,
                  float *__restrict__ mod, int B, int A, int N) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ float s_act[];  // [B][A]
   for (int i = threadIdx.x; i < B * A; i += blockDim.x) s_act[i] = silu_f(temb[i]);
   __syncthreads();
@@ -157,6 +159,8 @@ __global__ void __launch_bounds__(NORM_THREADS, 1)
                          const float *__restrict__ scale, int mod_stride, int L, int D, float eps,
                          void *__restrict__ h_out, float *__restrict__ h_scale, int remap_n,
                          int remap_L, int remap_off, int rows_per_cta) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ float4 smod[];  // [D/4] (1 + scale), then [D/4] shift
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -271,6 +275,8 @@ __global__ void __launch_bounds__(NORM_THREADS, 1)
 __global__ void rope_table_kernel(const int32_t *__restrict__ pos, int L, double theta, int sec0,
                                   int sec1, float *__restrict__ cos_out,
                                   float *__restrict__ sin_out) {
+  pdl_wait();
+  pdl_trigger();
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= L * 64) return;
   const int l = idx >> 6;
@@ -293,6 +299,8 @@ template <int NV>
 __global__ void __launch_bounds__(QUANT_THREADS)
     quantize_rows_kernel(const __nv_bfloat16 *__restrict__ x, uint8_t *__restrict__ q,
                          float *__restrict__ scale, int K) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float red[QUANT_THREADS / 32];
   const long r = blockIdx.x;
   const int nvec = K / 8;
@@ -342,6 +350,8 @@ __global__ void __launch_bounds__(QUANT_THREADS)
 // out[n][k] = decode(q[n][k]) * s[n], 16 codes per thread step.
 __global__ void dequant_e4m3_rows_kernel(const uint8_t *__restrict__ q, const float *__restrict__ s,
                                          __nv_bfloat16 *__restrict__ out, int K, long total16) {
+  pdl_wait();
+  pdl_trigger();
   for (long idx = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; idx < total16;
        idx += static_cast<long>(gridDim.x) * blockDim.x) {
     const long e0 = idx * 16;
@@ -389,6 +399,8 @@ __global__ void mrope_positions_kernel(int T, int gt, int gh, int gw, int32_t *_
 // dst[(b*L + off + i)] = src[(b*n + i)] for rows of `width` bytes (16-byte vectors).
 __global__ void copy_rows_kernel(const uint4 *__restrict__ src, uint4 *__restrict__ dst, int n,
                                  int L, int off, int vec_per_row, long total_vec) {
+  pdl_wait();
+  pdl_trigger();
   for (long idx = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; idx < total_vec;
        idx += static_cast<long>(gridDim.x) * blockDim.x) {
     const long row = idx / vec_per_row;
@@ -411,6 +423,8 @@ template <bool OUT_FP8>
 __global__ void __launch_bounds__(WIDE_NORM_THREADS)
     wide_rmsnorm_kernel(const float *__restrict__ x, const float *__restrict__ g, int K, float eps,
                         void *__restrict__ out, float *__restrict__ out_scale) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float red[2][WIDE_NORM_THREADS / 32];
   const long row = blockIdx.x;
   const float4 *xr = reinterpret_cast<const float4 *>(x + row * K);
@@ -483,6 +497,8 @@ __global__ void __launch_bounds__(WIDE_NORM_THREADS)
 __global__ void cfg_euler_kernel(const uint4 *__restrict__ v_c, const uint4 *__restrict__ v_u,
                                  float gw, float dt, const float4 *z_in, float4 *z_out,
                                  uint4 *__restrict__ z16, long n8) {
+  pdl_wait();
+  pdl_trigger();
   for (long i = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; i < n8;
        i += static_cast<long>(gridDim.x) * blockDim.x) {
     const float4 za = z_in[2 * i];
