@@ -322,6 +322,18 @@ def run_ours(args, rank, local_rank, world):
             per_kernel_ms[j] += evs[i][j].elapsed_time(evs[i][j + 1])
     per_kernel_ms = [t / K for t in per_kernel_ms]
 
+    # ---- the kernel with the largest share, timed alone: K more calls with
+    # events only around it (the other kernels keep overlapping their launch
+    # with the kernel before them, as in the timed region)
+    dom_j = max(range(n_launch), key=lambda j: per_kernel_ms[j])
+    ev_dom = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    for i in range(K):
+        evl = [None] * n_ev
+        evl[dom_j], evl[dom_j + 1] = ev_dom[i][0], ev_dom[i][1]
+        ig4.ig4_block_forward(c, bw, x, y, pos, temb, ws, events=evl)
+    torch.cuda.synchronize()
+    dom_ms_alone = sum(ev_dom[i][0].elapsed_time(ev_dom[i][1]) for i in range(K)) / K
+
     # ---- end-to-end region: every step copies its inputs from pinned host
     # memory and reads its result back, pipelined over two buffer sets
     pos_h = ig4.ig4_mrope_positions(cfg.T_text, cfg.grid_t, cfg.grid_h, cfg.grid_w)
@@ -352,9 +364,9 @@ def run_ours(args, rank, local_rank, world):
     tkey = "bf16_tflops" if held_max else "bf16_tflops_sustained"
     tensor_peak = peaks.get(tkey, FALLBACK_PEAKS[tkey])
     tnote = f"bf16 {'burst' if held_max else 'sustained'} ({peak_src})"
-    dom = max(range(n_launch), key=lambda j: per_kernel_ms[j])
+    dom = dom_j
     dom_name = names[dom]
-    dom_ms = per_kernel_ms[dom]
+    dom_ms = dom_ms_alone
     if dom_name in per_kernel_flops and dom_name != "adaln":
         achieved = per_kernel_flops[dom_name] / (dom_ms * 1e-3) / 1e12
         if fp8 and dom_name != "attention":
@@ -420,7 +432,8 @@ def run_ours(args, rank, local_rank, world):
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e / K, 4)},
         "gpu_launches": n_launch * K,
-        "kernel_ms_basis": "CUDA events between the kernels of K further traced calls",
+        "kernel_ms_basis": ("CUDA events between the kernels of K further traced calls; the "
+                            "roofline kernel from K more calls with events around it only"),
         "cpu_baseline": cpu_base,
     }
     print(json.dumps(line), flush=True)

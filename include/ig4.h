@@ -221,7 +221,10 @@ ig4_status ig4_block_forward(const ig4_config *cfg, const ig4_block_weights *w,
  * tracing) or IG4_BLOCK_TRACE_EVENTS.  Launch order: 0 AdaLN, 1 rotary table,
  * 2 norm1, 3 QKV+norm+rope, 4 attention, 5 out-proj+residual, 6 norm2,
  * 7 gate/up+SwiGLU, 8 down+residual; the E4M3 path adds 9 quantise(o) and
- * 10 quantise(u), recorded in launch order (quantise(o) before out-proj). */
+ * 10 quantise(u), recorded in launch order (quantise(o) before out-proj).
+ * An entry may be NULL: that boundary is not recorded (e.g. only the two
+ * events around one kernel, so the other kernels keep overlapping their
+ * launches with the kernel before them). */
 #define IG4_BLOCK_TRACE_EVENTS 12
 ig4_status ig4_block_forward_traced(const ig4_config *cfg, const ig4_block_weights *w,
                                     const void *x_in, void *x_out, const int32_t *pos,

@@ -672,9 +672,10 @@ struct Tracer {
   cudaStream_t st;
   ig4_status mark() {
     if (!ev || next >= n) return IG4_OK;
-    return cudaEventRecord(reinterpret_cast<cudaEvent_t>(ev[next++]), st) == cudaSuccess
-               ? IG4_OK
-               : IG4_ERR_CUDA;
+    void *e = ev[next++];
+    if (!e) return IG4_OK;  // this boundary is not recorded
+    return cudaEventRecord(reinterpret_cast<cudaEvent_t>(e), st) == cudaSuccess ? IG4_OK
+                                                                                 : IG4_ERR_CUDA;
   }
 };
 

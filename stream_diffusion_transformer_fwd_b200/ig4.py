@@ -268,7 +268,8 @@ def ig4_workspace_size(cfg: Config) -> int:
 def ig4_block_forward(cfg: Config, weights: BlockWeights, x_in, x_out, pos, temb, workspace,
                       events=None, stream=None):
     """x_out = block(x_in).  `events`: optional list of IG4_BLOCK_TRACE_EVENTS
-    torch.cuda.Event(enable_timing=True) recorded around each kernel."""
+    torch.cuda.Event(enable_timing=True) (or None: that boundary is not recorded)
+    recorded around each kernel."""
     ws_bytes = workspace.numel() * workspace.element_size()
     if events is None:
         st = _lib.ig4_block_forward(ctypes.byref(cfg), ctypes.byref(weights), _ptr(x_in),
@@ -277,8 +278,9 @@ def ig4_block_forward(cfg: Config, weights: BlockWeights, x_in, x_out, pos, temb
         _check(st, "ig4_block_forward")
         return
     for e in events:  # make sure each event owns a CUDA handle
-        e.record(stream) if stream is not None else e.record()
-    arr = (_vp * len(events))(*[e.cuda_event for e in events])
+        if e is not None:
+            e.record(stream) if stream is not None else e.record()
+    arr = (_vp * len(events))(*[None if e is None else e.cuda_event for e in events])
     st = _lib.ig4_block_forward_traced(ctypes.byref(cfg), ctypes.byref(weights), _ptr(x_in),
                                        _ptr(x_out), _ptr(pos), _ptr(temb), _ptr(workspace),
                                        ws_bytes, _stream(stream), arr, len(events))
