@@ -566,6 +566,69 @@ ig4_status launch_store_bf16(int M, int N, int K, const void *a, const float *a_
   }
 }
 
+// Packed NVFP4 scale blocks as a 3D tensor of 4-byte words: [row blocks of
+// 128][K/64 chunks][128 words]; a box takes 4 chunks (one stage) of
+// `blocks` row blocks.
+ig4_status map_sf_3d(CUtensorMap *m, const void *base, long rows, long K, int blocks) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return IG4_ERR_CUDA;
+  const long rb = (rows + 127) / 128;
+  cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(K / 64), static_cast<cuuint64_t>(rb)};
+  cuuint64_t strides[2] = {512, static_cast<cuuint64_t>(K / 64) * 512};
+  cuuint32_t box[3] = {128, 4, static_cast<cuuint32_t>(blocks)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void *>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? IG4_OK : IG4_ERR_CUDA;
+}
+
+// NVFP4 linear layer on CTA pairs (256 x 256 tiles).
+ig4_status launch_nvf4_pair(int M, int N, int K, const void *a_codes, const void *a_sf,
+                            const float *a_scale, const void *w_codes, const void *w_sf,
+                            const float *w_scale, const float *bias, void *out, int out_dtype,
+                            int sms, cudaStream_t st) {
+  CUtensorMap ma, mb, msa, msb;
+  IG4_TRY(map_2d(&ma, a_codes, 1, M, K / 2, K / 2, GEMM_BM, 128));
+  IG4_TRY(map_2d(&mb, w_codes, 1, N, K / 2, K / 2, 128, 128));
+  IG4_TRY(map_sf_3d(&msa, a_sf, M, K, 1));
+  IG4_TRY(map_sf_3d(&msb, w_sf, N, K, 2));
+  const int n_tiles_n = N / 256;
+  const long tiles = static_cast<long>((M + 2 * GEMM_BM - 1) / (2 * GEMM_BM)) * n_tiles_n;
+  const int pairs = static_cast<int>(std::min<long>(tiles, sms / 2));
+  const int group_m = gemm_group_m(M, K / 2, 1);
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(2 * pairs);
+  lc.blockDim = dim3(GEMM_THREADS);
+  lc.dynamicSmemBytes = NVF4P_SMEM_BYTES;
+  lc.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 2;
+  cudaError_t e;
+  if (out_dtype == IG4_F32) {
+    EpiStore<256, true, float> ep{static_cast<float *>(out), N, M, N, bias, a_scale, w_scale, 0, 0, 0};
+    auto kern = gemm_nvf4_pair_kernel<decltype(ep)>;
+    IG4_TRY(allow_smem(kern, NVF4P_SMEM_BYTES));
+    e = cudaLaunchKernelEx(&lc, kern, ma, mb, msa, msb, M, n_tiles_n, K, group_m, ep);
+  } else {
+    EpiStore<256, true, __nv_bfloat16> ep{static_cast<__nv_bfloat16 *>(out), N, M, N, bias,
+                                          a_scale, w_scale, 0, 0, 0};
+    auto kern = gemm_nvf4_pair_kernel<decltype(ep)>;
+    IG4_TRY(allow_smem(kern, NVF4P_SMEM_BYTES));
+    e = cudaLaunchKernelEx(&lc, kern, ma, mb, msa, msb, M, n_tiles_n, K, group_m, ep);
+  }
+  if (e != cudaSuccess) return IG4_ERR_CUDA;
+  return last_launch_status();
+}
+
 // NVFP4 linear layer on 128- or 256-wide tiles.
 template <int BN>
 ig4_status launch_nvf4(int M, int N, int K, const void *a_codes, const void *a_sf,
@@ -1071,8 +1134,12 @@ ig4_status ig4_nvfp4_linear(int M, int N, int K, const void *a_codes, const void
   if (bias && !aligned16(bias)) return IG4_ERR_INVALID_ARG;
   DeviceInfo *di = nullptr;
   IG4_TRY(device_info(&di));
-  // 256-wide tiles (one accumulator, fewer operand bytes per flop) once there
-  // are at least two waves of them, else 128-wide tiles
+  // CTA pairs with 256 x 256 tiles (half the B bytes per CTA) for more than one
+  // 128-row block; else single CTAs with 256-wide tiles (one accumulator) once
+  // there are two waves of them, or 128-wide tiles
+  if (N % 256 == 0 && M > GEMM_BM)
+    return launch_nvf4_pair(M, N, K, a_codes, a_sf, a_scale, w_codes, w_sf, w_scale, bias, out,
+                            out_dtype, di->sms, as_stream(stream));
   const long tiles256 = static_cast<long>((M + GEMM_BM - 1) / GEMM_BM) * (N / 256);
   if (N % 256 == 0 && tiles256 >= 2L * di->sms)
     return launch_nvf4<256>(M, N, K, a_codes, a_sf, a_scale, w_codes, w_sf, w_scale, bias, out,

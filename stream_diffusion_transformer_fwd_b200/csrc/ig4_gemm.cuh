@@ -722,6 +722,183 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   if (warp == 5) tmem_dealloc(tmem_base, NVF4_TMEM_COLS);
 }
 
+// NVFP4 on CTA pairs: a pair tile is 256 rows x 256 columns (tcgen05.mma
+// cta_group::2, M = 256): each CTA loads its 128 A rows, half of the B rows,
+// its A scale blocks and the scale blocks of all 256 B rows (both CTAs' MMAs
+// read the B scales of every column); all loads complete on the leader's
+// barrier.  Per stage and CTA: 32 KB of codes + 6 KB of scales per 512 MMA
+// clocks at the FP4 rate, the same bytes per clock as the FP8 pair kernel.
+// One TMEM accumulator (256 columns) plus a 48-column scale region per stage.
+constexpr int NVF4P_STAGES = 5;
+constexpr int NVF4P_A_BYTES = GEMM_BM * 128;
+constexpr int NVF4P_BH_BYTES = 128 * 128;
+constexpr int NVF4P_SFA_BYTES = 2048;
+constexpr int NVF4P_SFB_BYTES = 4096;
+constexpr int NVF4P_STAGE_BYTES = NVF4P_A_BYTES + NVF4P_BH_BYTES + NVF4P_SFA_BYTES + NVF4P_SFB_BYTES;
+constexpr int NVF4P_SMEM_BYTES = NVF4P_STAGES * NVF4P_STAGE_BYTES + 1024 + 256;
+constexpr uint32_t NVF4P_SF_COLS = 48;
+static_assert(256 + NVF4P_STAGES * NVF4P_SF_COLS <= 512, "TMEM");
+
+template <class Epi>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                          const __grid_constant__ CUtensorMap tmSFA,
+                          const __grid_constant__ CUtensorMap tmSFB, int M, int n_tiles_n, int K,
+                          int group_m, const Epi epi) {
+  constexpr int BN = 256;
+  constexpr uint32_t IDESC = idesc_nvf4(2 * GEMM_BM, BN);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = align1024(smem_raw);
+  uint8_t *sA = smem;
+  uint8_t *sB = sA + NVF4P_STAGES * NVF4P_A_BYTES;
+  uint8_t *sSFA = sB + NVF4P_STAGES * NVF4P_BH_BYTES;
+  uint8_t *sSFB = sSFA + NVF4P_STAGES * NVF4P_SFA_BYTES;
+  uint64_t *full = reinterpret_cast<uint64_t *>(sSFB + NVF4P_STAGES * NVF4P_SFB_BYTES);
+  uint64_t *empty = full + NVF4P_STAGES;
+  uint64_t *tfull = empty + NVF4P_STAGES;
+  uint64_t *tempty = tfull + 1;
+  uint64_t *drain = tempty + 1;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1;
+  const int n_pairs = gridDim.x >> 1;
+  const int m_tiles = (M + 2 * GEMM_BM - 1) / (2 * GEMM_BM);
+  const int n_tiles = m_tiles * n_tiles_n;
+  const int kblocks = K / 256;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NVF4P_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(tfull, 1);
+    mbar_init(tempty, 2 * 4);  // one arrival per epilogue warp of the pair
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmSFA);
+    tma_prefetch_desc(&tmSFB);
+  }
+  if (warp == 5) {
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();
+  pdl_trigger();
+
+  if (warp == 4) {
+    if (lane == 0) {
+      // ---------------- loads (both CTAs), completing on the leader's barrier
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int t = pair; t < n_tiles && ok; t += n_pairs) {
+        int mt, nt;
+        tile_coords(t, m_tiles, n_tiles_n, group_m, &mt, &nt);
+        const int mrow = mt * 2 * GEMM_BM + static_cast<int>(rank) * GEMM_BM;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait_cluster(&empty[s], ph ^ 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * NVF4P_STAGE_BYTES);
+          const uint32_t bar = map_shared_to_rank(&full[s], 0);
+          tma_load_2d_pair(sA + s * NVF4P_A_BYTES, &tmA, bar, kb * 128, mrow);
+          tma_load_2d_pair(sB + s * NVF4P_BH_BYTES, &tmB, bar, kb * 128,
+                           nt * BN + static_cast<int>(rank) * (BN / 2));
+          // scale blocks: [128 words of 4 B] x [4 K chunks] x [row blocks]
+          tma_load_3d_pair(sSFA + s * NVF4P_SFA_BYTES, &tmSFA, bar, 0, 4 * kb, mrow / 128);
+          tma_load_3d_pair(sSFB + s * NVF4P_SFB_BYTES, &tmSFB, bar, 0, 4 * kb, nt * 2);
+          if (++s == NVF4P_STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+      }
+      if (!ok) sleep_ns(50000);  // let the loads already issued land
+    }
+  } else if (warp == 5) {
+    if (lane == 0 && rank == 0) {
+      // ---------------- MMA issuer (leader CTA)
+      int s = 0;
+      uint32_t ph = 0;
+      int local = 0;
+      bool ok = true;
+      for (int t = pair; t < n_tiles && ok; t += n_pairs, ++local) {
+        if (!mbar_wait_cluster(tempty, (static_cast<uint32_t>(local) & 1) ^ 1, abort_flag)) break;
+        tc_fence_after();
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait_cluster(&full[s], ph, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sf = tmem_base + 256 + NVF4P_SF_COLS * s;
+          const uint32_t sfa_s = smem_u32(sSFA + s * NVF4P_SFA_BYTES);
+          const uint32_t sfb_s = smem_u32(sSFB + s * NVF4P_SFB_BYTES);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            tmem_cp_sf_pair(sf + 4 * j, sdesc_kmajor_none(sfa_s + 512 * j, 128));
+            tmem_cp_sf_pair(sf + 16 + 8 * j, sdesc_kmajor_none(sfb_s + 512 * j, 128));
+            tmem_cp_sf_pair(sf + 16 + 8 * j + 4, sdesc_kmajor_none(sfb_s + 2048 + 512 * j, 128));
+          }
+          const uint32_t a_base = smem_u32(sA + s * NVF4P_A_BYTES);
+          const uint32_t b_base = smem_u32(sB + s * NVF4P_BH_BYTES);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint64_t ad = sdesc_kmajor_sw128(a_base + 32 * j);
+            const uint64_t bd = sdesc_kmajor_sw128(b_base + 32 * j);
+            umma_nvf4_pair(tmem_base, ad, bd, IDESC, sf + 4 * j, sf + 16 + 8 * j, (kb | j) != 0);
+          }
+          umma_commit_pair_both(&empty[s]);
+          if (++s == NVF4P_STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+        if (ok) umma_commit_pair_both(tfull);
+      }
+      umma_commit_pair_both(drain);
+      mbar_wait_cluster(drain, 0, nullptr, WAIT_LIMIT_NS / 4);
+    }
+  } else {
+    // ---------------- epilogue warps 0..3 (both CTAs, own 128 rows)
+    const int r = warp * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t tempty_leader = map_shared_to_rank(tempty, 0);
+    int local = 0;
+    for (int t = pair; t < n_tiles; t += n_pairs, ++local) {
+      const bool ok = mbar_wait_cluster(tfull, static_cast<uint32_t>(local) & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      int mt, nt;
+      tile_coords(t, m_tiles, n_tiles_n, group_m, &mt, &nt);
+      epi(mt * 2 * GEMM_BM + static_cast<int>(rank) * GEMM_BM, nt * BN, tmem_base + lane_base, r);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty_leader);
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  if (warp == 5) tmem_dealloc_pair(tmem_base, 512);
+}
+
 // Scale factors [rows][K/16] (row-major UE4M3 bytes) -> the tensor cores'
 // block order (see gemm_nvf4_kernel); rows padded to a multiple of 128 with
 // zero scales.  One thread per output byte.

@@ -441,6 +441,29 @@ __device__ __forceinline__ void umma_f8_pair(uint32_t d_tmem, uint64_t a_desc, u
       : "memory");
 }
 
+// Block-scaled FP4 MMA on a CTA pair (M = 256): each CTA supplies its 128 A
+// rows and half of B from its own shared memory, and its scale factors from
+// its own TMEM at the given column addresses (A: its 128 rows; B: all N rows).
+__device__ __forceinline__ void umma_nvf4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t sfa_tmem,
+                                               uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], "
+      "p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// tcgen05.cp 32x128b.warpx4 for a CTA pair: issued by the leader, it copies
+// the 512-byte block at the same shared-memory offset of each CTA into that
+// CTA's TMEM.
+__device__ __forceinline__ void tmem_cp_sf_pair(uint32_t taddr, uint64_t s_desc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(s_desc)
+               : "memory");
+}
+
 // Arrive (release, cluster scope) on the mbarrier at a shared::cluster address.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster)

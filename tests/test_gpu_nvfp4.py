@@ -40,8 +40,9 @@ def _packed(ig4, sf):
                                              (300, 384, 1024, torch.float32),
                                              (1000, 1024, 4608, torch.bfloat16),
                                              (77, 256, 12288, torch.float32),
-                                             (4608, 4608, 512, torch.float32),    # 256-wide tiles
-                                             (4600, 4608, 768, torch.bfloat16)])  # ragged M
+                                             (128, 75776, 256, torch.float32),    # 256-wide tiles
+                                             (4608, 4608, 512, torch.float32),    # CTA pairs
+                                             (4600, 4608, 768, torch.bfloat16)])  # pairs, ragged M
 def test_nvfp4_linear(ig4, M, N, K, out_dtype):
     a_codes, a_sf, a_s, a_ref = _operand(1, "a", M, K, 16, 1.0)        # activations: 16-blocks
     w_codes, w_sf, w_s, w_ref = _operand(2, "w", N, K, 64, 1.0 / np.sqrt(K))  # weights: 64-blocks
