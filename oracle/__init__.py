@@ -27,13 +27,18 @@ from .ig4_oracle import (  # noqa: F401
     block_flops,
     block_forward,
     block_forward_rows,
+    bf16_round,
     dequant_e4m3,
     dequant_nvfp4,
     e2m1_decode_table,
     e4m3_decode_table,
+    e2m1_encode,
+    e4m3_encode,
     joint_attention,
     merge_heads,
     modulate,
+    nvfp4_activation_values,
+    quantize_nvfp4_activations,
     mrope_angles,
     mrope_axis_of_pair,
     mrope_positions,

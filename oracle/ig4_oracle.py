@@ -273,7 +273,7 @@ BLOCK_WEIGHT_NAMES = ("w_ada", "b_ada", "w_qkv", "g_q", "g_k", "w_o", "w_gate", 
 
 
 def block_forward(x, temb, pos, W, H, theta=ROPE_THETA, sections=MROPE_SECTION, eps=EPS,
-                  return_intermediates=False):
+                  return_intermediates=False, ffn_nvfp4=False):
     """One Ideogram4TransformerBlock forward, float64.
 
     x: [B, L, D] residual stream ([text | image] tokens); temb: [B, adaln_dim];
@@ -290,6 +290,11 @@ def block_forward(x, temb, pos, W, H, theta=ROPE_THETA, sections=MROPE_SECTION, 
       7 x1 = x + gate_msa * (o W_o^T);
       8 h2 = RMSNorm(x1) (1 + scale_mlp) + shift_mlp;
         y = x1 + gate_mlp * (silu(h2 W_g^T) * (h2 W_u^T)) W_d^T.
+    ffn_nvfp4: the FFN linears consume NVFP4 activations, as the NVFP4-mixed
+    checkpoint runs them (deployment article, section "2.2 NVFP4 Mixed":
+    FFN linears in NVFP4, attention projections and the time embedding in
+    FP8): h2 and u are replaced by nvfp4_activation_values of themselves;
+    the weights in W are the dequantised ones.
     """
     x = np.asarray(x, dtype=np.float64)
     B, L, D = x.shape
@@ -310,8 +315,8 @@ def block_forward(x, temb, pos, W, H, theta=ROPE_THETA, sections=MROPE_SECTION, 
     x1 = x + gate_msa[:, None, :] * (o @ W["w_o"].T)
 
     h2 = modulate(x1, shift_mlp, scale_mlp, eps)
-    u = swiglu(h2, W["w_gate"], W["w_up"])
-    y = x1 + gate_mlp[:, None, :] * (u @ W["w_down"].T)
+    u = swiglu(nvfp4_activation_values(h2) if ffn_nvfp4 else h2, W["w_gate"], W["w_up"])
+    y = x1 + gate_mlp[:, None, :] * ((nvfp4_activation_values(u) if ffn_nvfp4 else u) @ W["w_down"].T)
     if not return_intermediates:
         return y
     mod = np.concatenate([shift_msa, scale_msa, gate_msa, shift_mlp, scale_mlp, gate_mlp], axis=1)
@@ -319,7 +324,7 @@ def block_forward(x, temb, pos, W, H, theta=ROPE_THETA, sections=MROPE_SECTION, 
 
 
 def block_forward_rows(x, temb, pos, W, H, rows, theta=ROPE_THETA, sections=MROPE_SECTION,
-                       eps=EPS):
+                       eps=EPS, ffn_nvfp4=False):
     """The same block, evaluated only for the output tokens in `rows`.
 
     rows: integer array of flat token indices into B*L.  Every step except
@@ -351,7 +356,11 @@ def block_forward_rows(x, temb, pos, W, H, rows, theta=ROPE_THETA, sections=MROP
         o = merge_heads(np.matmul(softmax(s, axis=-1), v))[0]  # [n, D]
         x1 = x[b, ls] + gate_msa[b][None, :] * (o @ W["w_o"].T)
         h2 = rms_norm(x1, eps) * (1.0 + scale_mlp[b][None, :]) + shift_mlp[b][None, :]
-        y = x1 + gate_mlp[b][None, :] * (swiglu(h2, W["w_gate"], W["w_up"]) @ W["w_down"].T)
+        if ffn_nvfp4:
+            u = swiglu(nvfp4_activation_values(h2), W["w_gate"], W["w_up"])
+            y = x1 + gate_mlp[b][None, :] * (nvfp4_activation_values(u) @ W["w_down"].T)
+        else:
+            y = x1 + gate_mlp[b][None, :] * (swiglu(h2, W["w_gate"], W["w_up"]) @ W["w_down"].T)
         for n, r in enumerate(sel):
             out[np.nonzero(rows == r)[0]] = y[n]
     return out
@@ -429,6 +438,100 @@ def dequant_nvfp4(packed, sf, s) -> np.ndarray:
     vals = e2m1_decode_table()[codes]
     sbv = e4m3_decode_table()[np.asarray(sf, dtype=np.uint8)]
     return np.asarray(s, dtype=np.float64)[:, None] * np.repeat(sbv, 16, axis=1) * vals
+
+
+def bf16_round(x) -> np.ndarray:
+    """Nearest bfloat16 value of each element (round to nearest, ties to an
+    even last mantissa bit), returned as float64.  bfloat16 is float32 with
+    the low 16 significand bits dropped; float64 inputs go through float32
+    first (the precision the block's activations are computed in)."""
+    f = np.ascontiguousarray(np.asarray(x, dtype=np.float64).astype(np.float32))
+    bits = f.view(np.uint32).astype(np.uint64)
+    low = bits & 0xFFFF
+    keep = bits >> 16
+    up = (low > 0x8000) | ((low == 0x8000) & ((keep & 1) == 1))
+    out = ((keep + up.astype(np.uint64)) << 16).astype(np.uint32)
+    return out.view(np.float32).astype(np.float64)
+
+
+def _nearest_code(a: np.ndarray, grid: np.ndarray) -> np.ndarray:
+    """Index of the value of the ascending `grid` nearest to each a >= 0,
+    ties to the even index, saturating at the last entry."""
+    a = np.minimum(a, grid[-1])
+    hi = np.clip(np.searchsorted(grid, a, side="left"), 0, len(grid) - 1)
+    lo = np.maximum(hi - 1, 0)
+    d_lo = a - grid[lo]
+    d_hi = grid[hi] - a
+    tie_pick = np.where(lo % 2 == 0, lo, hi)
+    return np.where(d_lo < d_hi, lo, np.where(d_hi < d_lo, hi, tie_pick))
+
+
+def e4m3_encode(v) -> np.ndarray:
+    """FP8 E4M3 code of each value: round to nearest (ties to the even code),
+    saturating at +-448; sign bit set for negative values."""
+    v = np.asarray(v, dtype=np.float64)
+    grid = e4m3_decode_table()[:127]           # codes 0x00..0x7E, ascending
+    code = _nearest_code(np.abs(v), grid).astype(np.uint8)
+    return code | ((v < 0).astype(np.uint8) << 7)
+
+
+def e2m1_encode(v) -> np.ndarray:
+    """FP4 E2M1 code (0..15) of each value: nearest of {0, .5, 1, 1.5, 2, 3,
+    4, 6}, ties to the even code, saturating at +-6; sign bit (bit 3) set for
+    negative values that do not round to zero."""
+    v = np.asarray(v, dtype=np.float64)
+    grid = e2m1_decode_table()[:8]
+    code = _nearest_code(np.abs(v), grid).astype(np.uint8)
+    return code | (((v < 0) & (code > 0)).astype(np.uint8) << 3)
+
+
+NVFP4_BLOCK = 16           # elements per block scale (the tensor cores' block)
+E2M1_MAX = 6.0
+E4M3_MAX = 448.0
+
+
+def quantize_nvfp4_activations(x):
+    """Activation rows -> NVFP4: (codes uint8 [M, K] in 0..15, block-scale
+    E4M3 codes uint8 [M, K/16], row scales float32 [M]).
+
+    The recipe (the weights' NVFP4 layout of the deployment article, section
+    "2.2 NVFP4 Mixed", applied to the activations the FFN linears consume,
+    with 16-element blocks):
+      s[m]      = amax_k |x[m, k]| / (6 * 448), or 1 for an all-zero row;
+      sc[m, b]  = RNE_E4M3(amax over block b of |x[m, :]| / (6 * s[m]));
+      code[m,k] = RNE_E2M1(x[m, k] * (1 / (s[m] * sc[m, k / 16]))), or 0 where
+                  that product is 0.
+    Every step is a float32 operation (the precision the quantising kernel
+    takes the same decisions in): each product and quotient is rounded to
+    float32 before the next step.
+    """
+    x = np.asarray(x, dtype=np.float32)
+    M, K = x.shape
+    assert K % NVFP4_BLOCK == 0
+    ax = np.abs(x)
+    amax = ax.max(axis=1)
+    s = np.where(amax > 0, amax / np.float32(E2M1_MAX * E4M3_MAX), np.float32(1)).astype(np.float32)
+    bam = ax.reshape(M, K // NVFP4_BLOCK, NVFP4_BLOCK).max(axis=2)
+    t = (np.float32(E2M1_MAX) * s).astype(np.float32)
+    bs = (bam / t[:, None]).astype(np.float32)
+    sc = e4m3_encode(bs)
+    scv = e4m3_decode_table()[sc].astype(np.float32)
+    d = (s[:, None] * scv).astype(np.float32)
+    inv = np.where(d > 0, np.float32(1) / np.where(d > 0, d, np.float32(1)), np.float32(0)).astype(np.float32)
+    q = (x * np.repeat(inv, NVFP4_BLOCK, axis=1)).astype(np.float32)
+    return e2m1_encode(q), sc, s
+
+
+def nvfp4_activation_values(x) -> np.ndarray:
+    """float64 values of the NVFP4 quantisation of bf16 activations:
+    s[m] * decode_E4M3(sc[m, k / 16]) * decode_E2M1(code[m, k]), taken of the
+    bf16 rounding of x (the precision the block stores activations in)."""
+    xb = bf16_round(x)
+    shape = xb.shape
+    rows = xb.reshape(-1, shape[-1])
+    codes, sc, s = quantize_nvfp4_activations(rows)
+    vals = e2m1_decode_table()[codes] * np.repeat(e4m3_decode_table()[sc], NVFP4_BLOCK, axis=1)
+    return (s.astype(np.float64)[:, None] * vals).reshape(shape)
 
 
 # ---------------------------------------------------------------------------
