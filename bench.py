@@ -34,6 +34,10 @@ KERNEL_NAMES = ["adaln", "rope_table", "norm1", "qkv_norm_rope", "attention", "o
                 "norm2", "gate_up_swiglu", "down_residual"]
 KERNEL_NAMES_FP8 = ["adaln", "rope_table", "norm1", "qkv_norm_rope", "attention", "quantize_o",
                     "out_proj_residual", "norm2", "gate_up_swiglu", "quantize_u", "down_residual"]
+# NVFP4 Mixed: norm2 and the NVFP4 quantiser of h2 share one trace interval
+KERNEL_NAMES_NVFP4 = ["adaln", "rope_table", "norm1", "qkv_norm_rope", "attention", "quantize_o",
+                      "out_proj_residual", "norm2_quantize", "gate_up_swiglu", "quantize_u",
+                      "down_residual"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 REFERENCE_ROWS = 32
 # The source files that define each kernel's device code (a recorded DRAM
@@ -83,8 +87,8 @@ def kernel_bytes(cfg, name):
     """Algorithmic HBM bytes of the memory-bound kernels (one launch)."""
     M, D, L = cfg.M, cfg.D, cfg.L
     xs = 4 if cfg.x_dtype == "f32" else 2
-    ws = 1 if cfg.w_dtype == "e4m3" else 2
-    hs = 1 if cfg.w_dtype == "e4m3" else 2
+    ws = 1 if cfg.w_dtype in ("e4m3", "nvfp4_mixed") else 2
+    hs = 1 if cfg.w_dtype in ("e4m3", "nvfp4_mixed") else 2
     if name == "adaln":
         return 6 * D * cfg.adaln_dim * ws + 6 * D * 4 * (1 + cfg.B)
     if name in ("norm1", "norm2"):
@@ -94,7 +98,11 @@ def kernel_bytes(cfg, name):
     if name == "quantize_o":
         return M * D * 3
     if name == "quantize_u":
-        return M * cfg.I * 3
+        # NVFP4: bf16 in, codes (1/2 B) and scales (1/16 B) out; FP8: bf16 in, byte out
+        return M * cfg.I * (2.5625 if cfg.w_dtype == "nvfp4_mixed" else 3)
+    if name == "norm2_quantize":
+        # x in, bf16 h2 out and back in, NVFP4 codes and scales out
+        return M * D * (xs + 4.5625)
     return None
 
 
@@ -268,11 +276,14 @@ def run_ours(args, rank, local_rank, world):
         return run_step(args, cfg, ig4, rank, world, dev)
     if cfg.n_blocks > 1:
         return run_stack(args, cfg, ig4, rank, world, dev)
-    fp8 = cfg.w_dtype == "e4m3"
-    names = KERNEL_NAMES_FP8 if fp8 else KERNEL_NAMES
+    nv4 = cfg.w_dtype == "nvfp4_mixed"
+    fp8 = cfg.w_dtype == "e4m3" or nv4
+    names = KERNEL_NAMES_NVFP4 if nv4 else (KERNEL_NAMES_FP8 if fp8 else KERNEL_NAMES)
     acts = make_block_activations(cfg, seed=rank)
     wts = make_block_weights(cfg, seed=rank)
     wd = {k: (None if v is None else v.to(dev)) for k, v in wts.items()}
+    if nv4:
+        wd = ig4.nvfp4_pack_block_scales(wd)
     bw = ig4.block_weights(wd)
     c = ig4.config_from(cfg)
     x = acts["x"].to(dev)
@@ -369,7 +380,10 @@ def run_ours(args, rank, local_rank, world):
     dom_ms = dom_ms_alone
     if dom_name in per_kernel_flops and dom_name != "adaln":
         achieved = per_kernel_flops[dom_name] / (dom_ms * 1e-3) / 1e12
-        if fp8 and dom_name != "attention":
+        if nv4 and dom_name in ("gate_up_swiglu", "down_residual"):
+            peak = 4.0 * tensor_peak
+            peak_note = f"4 x {tnote}: nominal fp4/bf16 dense ratio"
+        elif fp8 and dom_name != "attention":
             peak = 2.0 * tensor_peak
             peak_note = f"2 x {tnote}: nominal fp8/bf16 dense ratio"
         else:
@@ -409,7 +423,9 @@ def run_ours(args, rank, local_rank, world):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "fp8-e4m3 weights, bf16 activations" if fp8 else "bf16",
+        "dtype": ("NVFP4 Mixed: nvfp4 (e2m1 + ue4m3 block scales) FFN weights and activations, "
+                  "fp8-e4m3 AdaLN/attention weights, bf16 attention" if nv4 else
+                  "fp8-e4m3 weights, bf16 activations" if fp8 else "bf16"),
         "data": "synthetic (seeded N(0,1) activations, N(0,1/fan_in) weights, random init)",
         "config": {
             "workload": (f"{cfg.name} Ideogram4 block: B={cfg.B}, {cfg.T_text} text + "
@@ -418,7 +434,7 @@ def run_ours(args, rank, local_rank, world):
                          f"x={cfg.x_dtype}"),
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "l2": "inputs larger than L2 (block weights alone are "
-                  f"{(8 * cfg.D * cfg.D + 6 * cfg.D * cfg.I) * (1 if fp8 else 2) / 1e6:.0f} MB per step)",
+                  f"{(8 * cfg.D * cfg.D + 6 * cfg.D * cfg.I * (0.5625 if nv4 else 1)) * (1 if fp8 else 2) / 1e6:.0f} MB per step)",
             "gflop_per_step": round(flops / 1e9, 1),
         },
         "pct_of_peak": round(100.0 * value / world / tensor_peak, 2),
@@ -431,7 +447,7 @@ def run_ours(args, rank, local_rank, world):
         "device_error": ig4.ig4_status_string(err),
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e / K, 4)},
-        "gpu_launches": n_launch * K,
+        "gpu_launches": (n_launch + (1 if nv4 else 0)) * K,  # NVFP4: norm2 + quantiser share a slot
         "kernel_ms_basis": ("CUDA events between the kernels of K further traced calls; the "
                             "roofline kernel from K more calls with events around it only"),
         "cpu_baseline": cpu_base,
@@ -892,7 +908,8 @@ def cpu_baseline(cfg, acts, wts):
     temb = to_f64(acts["temb"])
     pos = O.mrope_positions(cfg.T_text, cfg.grid_t, cfg.grid_h, cfg.grid_w)
     t0 = time.perf_counter()
-    O.block_forward(x, temb, pos, W, cfg.H, cfg.rope_theta, cfg.sections, cfg.eps)
+    O.block_forward(x, temb, pos, W, cfg.H, cfg.rope_theta, cfg.sections, cfg.eps,
+                    ffn_nvfp4=cfg.w_dtype == "nvfp4_mixed")
     dt = time.perf_counter() - t0
     flops, _ = block_work(cfg)
     return {"value": round(flops / dt / 1e12, 4), "unit": "TFLOP/s", "cores": _cores(),
@@ -928,7 +945,8 @@ def run_reference(args, rank, world):
     for i in range(args.warmup + args.steps):
         rows = rng.choice(L, size=S, replace=False)  # rows of sample 0
         t0 = time.perf_counter()
-        O.block_forward_rows(x, temb, pos, W, cfg.H, rows, cfg.rope_theta, cfg.sections, cfg.eps)
+        O.block_forward_rows(x, temb, pos, W, cfg.H, rows, cfg.rope_theta, cfg.sections, cfg.eps,
+                             ffn_nvfp4=cfg.w_dtype == "nvfp4_mixed")
         if i >= args.warmup:
             times.append(time.perf_counter() - t0)
     total = sum(times)

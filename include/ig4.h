@@ -59,13 +59,20 @@ typedef enum ig4_status {
 typedef enum ig4_dtype {
   IG4_F32 = 0,
   IG4_BF16 = 1,
-  IG4_E4M3 = 2   /* FP8 E4M3 "fn" (max 448), with an fp32 scale array */
+  IG4_E4M3 = 2,  /* FP8 E4M3 "fn" (max 448), with an fp32 scale array */
+  /* block / stack weights only ("2.2 NVFP4 Mixed" of the deployment article
+   * cited at the NVFP4 section below): the FFN linears w_gate, w_up, w_down
+   * in NVFP4 (E2M1 codes [N][K/2], packed E4M3 block scales sf_*, fp32
+   * channel scales s_*), every other linear in E4M3 with its s_* scale.
+   * The FFN then consumes NVFP4 activations (ig4_nvfp4_quantize of the
+   * bf16 h2 and u).  Needs I % 256 == 0 and B*L > 128. */
+  IG4_NVFP4_MIXED = 3
 } ig4_dtype;
 
 /* Shape and precision of one block call.  L = T_text + grid_t*grid_h*grid_w.
  * Supported: head_dim == 256, D == H*256, D % 256 == 0, I % 128 == 0,
  * adaln_dim % 8 == 0 and <= 1024, B*L >= 1, x_dtype F32 or BF16,
- * w_dtype BF16 or E4M3. */
+ * w_dtype BF16, E4M3 or NVFP4_MIXED (then also I % 256 == 0, B*L > 128). */
 typedef struct ig4_config {
   int B, T_text, grid_t, grid_h, grid_w;
   int D, H, head_dim, I, adaln_dim;
@@ -73,18 +80,22 @@ typedef struct ig4_config {
   int sections[3];     /* (24, 20, 20): must sum to 64 */
   float eps;           /* RMSNorm epsilon, 1e-6 */
   int x_dtype;         /* residual stream storage: IG4_F32 or IG4_BF16 */
-  int w_dtype;         /* linear weights: IG4_BF16, or IG4_E4M3 with s_* scales */
+  int w_dtype;         /* linear weights: IG4_BF16, IG4_E4M3 with s_* scales, or
+                          IG4_NVFP4_MIXED */
 } ig4_config;
 
 /* One block's weights (device pointers).  w_* are [out, in] row-major in
  * w_dtype: w_ada [6D, adaln_dim], w_qkv [3D, D] (rows: q | k | v, head-major,
  * column n = head*256 + d), w_o [D, D], w_gate [I, D], w_up [I, D],
- * w_down [D, I].  s_* are fp32 per-output-channel scales [out] (E4M3 only,
- * else ignored).  b_ada fp32 [6D], g_q / g_k fp32 [head_dim]. */
+ * w_down [D, I].  s_* are fp32 per-output-channel scales [out] (E4M3 and
+ * NVFP4_MIXED, else ignored).  b_ada fp32 [6D], g_q / g_k fp32 [head_dim].
+ * sf_gate / sf_up / sf_down: packed NVFP4 block scales of the FFN weights
+ * (ig4_nvfp4_pack_scales), IG4_NVFP4_MIXED only, else ignored (zero them). */
 typedef struct ig4_block_weights {
   const void *w_ada, *w_qkv, *w_o, *w_gate, *w_up, *w_down;
   const float *s_ada, *s_qkv, *s_o, *s_gate, *s_up, *s_down;
   const float *b_ada, *g_q, *g_k;
+  const void *sf_gate, *sf_up, *sf_down;
 } ig4_block_weights;
 
 /* Stack weights: a host array of n_blocks block weight structs, the latent
@@ -296,7 +307,15 @@ ig4_status ig4_stack_forward(const ig4_config *cfg, const ig4_stack_weights *sw,
  * a_codes [M][K/2], w_codes [N][K/2] bytes; a_sf, w_sf packed scales;
  * a_scale [M], w_scale [N], bias [N] (or NULL) fp32; out [M][N] fp32 or bf16
  * (out_dtype).  All device pointers 16-byte aligned; stream-ordered.
- * Errors: IG4_ERR_INVALID_ARG. */
+ * Errors: IG4_ERR_INVALID_ARG.
+ * ig4_nvfp4_quantize: activations x bf16 [M][K] (device, K a multiple of
+ * 64) -> codes [M][K/2], packed scales (ig4_nvfp4_scale_bytes(M, K) bytes;
+ * padding rows are not written) and row_scale fp32 [M], by the recipe
+ *   row_scale[m] = max_k |x[m][k]| / (6 * 448)  (1 for an all-zero row),
+ *   sf[m][b]     = RNE_E4M3(max over block b |x[m][.]| / (6 row_scale[m])),
+ *   code[m][k]   = RNE_E2M1(x[m][k] * (1 / (row_scale[m] sf[m][k/16]))),
+ * each step a float32 operation, E2M1 saturating at 6 (a block whose scale
+ * rounds to 0 gets zero codes).  Errors: IG4_ERR_INVALID_ARG. */
 size_t ig4_nvfp4_scale_bytes(int rows, int K);
 ig4_status ig4_nvfp4_pack_scales(int rows, int K, const void *sf_rows, void *sf_packed,
                                  void *stream);
@@ -304,6 +323,8 @@ ig4_status ig4_nvfp4_linear(int M, int N, int K, const void *a_codes, const void
                             const float *a_scale, const void *w_codes, const void *w_sf,
                             const float *w_scale, const float *bias, void *out, int out_dtype,
                             void *stream);
+ig4_status ig4_nvfp4_quantize(int M, int K, const void *x, void *codes, void *sf_packed,
+                              float *row_scale, void *stream);
 
 /* -------------------------------------------------- text conditioning ---
  * The step before the stack ("Ideogram 4 快速开始" (SimpleTuner quickstart),

@@ -17,13 +17,14 @@
 #include "ig4.h"
 #include "ig4_attention.cuh"
 #include "ig4_gemm.cuh"
+#include "ig4_nvf4.cuh"
 #include "ig4_small.cuh"
 
 using namespace ig4;
 
 namespace {
 
-constexpr int ABI_VERSION = 1;
+constexpr int ABI_VERSION = 2;
 
 // ------------------------------------------------------------------ utils
 
@@ -238,7 +239,9 @@ ig4_status gemm_maps(CUtensorMap *ma, CUtensorMap *mb, const void *a, const void
   return IG4_OK;
 }
 
-bool is_fp8(int dt) { return dt == IG4_E4M3; }
+// E4M3 linears (all of them, or all but the NVFP4 FFN of the mixed format)
+bool is_fp8(int dt) { return dt == IG4_E4M3 || dt == IG4_NVFP4_MIXED; }
+bool is_nvf4_mixed(int dt) { return dt == IG4_NVFP4_MIXED; }
 
 // ------------------------------------------------------------ validation
 
@@ -257,8 +260,12 @@ ig4_status check_config(const ig4_config *c) {
       c->sections[0] + c->sections[1] + c->sections[2] != 64)
     return IG4_ERR_INVALID_ARG;
   if (!(c->rope_theta > 0.0) || !(c->eps > 0.0f)) return IG4_ERR_INVALID_ARG;
-  if (!valid_dtype_x(c->x_dtype) || !valid_dtype_w(c->w_dtype)) return IG4_ERR_INVALID_ARG;
+  if (!valid_dtype_x(c->x_dtype) || !(valid_dtype_w(c->w_dtype) || is_nvf4_mixed(c->w_dtype)))
+    return IG4_ERR_INVALID_ARG;
   if (c->head_dim != 256 || c->D != 256 * c->H) return IG4_ERR_UNSUPPORTED;
+  // the NVFP4 FFN runs on CTA pairs with K-steps of 256
+  if (is_nvf4_mixed(c->w_dtype) && (c->I % 256 != 0 || static_cast<long>(c->B) * L <= 128))
+    return IG4_ERR_UNSUPPORTED;
   if (c->D > 6144) return IG4_ERR_UNSUPPORTED;
   if (c->I % 128 != 0) return IG4_ERR_UNSUPPORTED;
   if (c->adaln_dim % 16 != 0 || c->adaln_dim > 1024 || c->B > 8) return IG4_ERR_UNSUPPORTED;
@@ -584,19 +591,16 @@ ig4_status map_sf_3d(CUtensorMap *m, const void *base, long rows, long K, int bl
   return r == CUDA_SUCCESS ? IG4_OK : IG4_ERR_CUDA;
 }
 
-// NVFP4 linear layer on CTA pairs (256 x 256 tiles).
-ig4_status launch_nvf4_pair(int M, int N, int K, const void *a_codes, const void *a_sf,
-                            const float *a_scale, const void *w_codes, const void *w_sf,
-                            const float *w_scale, const float *bias, void *out, int out_dtype,
-                            int sms, cudaStream_t st) {
-  CUtensorMap ma, mb, msa, msb;
-  IG4_TRY(map_2d(&ma, a_codes, 1, M, K / 2, K / 2, GEMM_BM, 128));
-  IG4_TRY(map_2d(&mb, w_codes, 1, N, K / 2, K / 2, 128, 128));
-  IG4_TRY(map_sf_3d(&msa, a_sf, M, K, 1));
-  IG4_TRY(map_sf_3d(&msb, w_sf, N, K, 2));
-  const int n_tiles_n = N / 256;
+// NVFP4 GEMM on CTA pairs (256 x 256 tiles), maps built by the caller.
+template <bool DUAL_B, class Epi>
+ig4_status launch_nvf4_pair_maps(const CUtensorMap &ma, const CUtensorMap &mb,
+                                 const CUtensorMap &mb2, const CUtensorMap &msa,
+                                 const CUtensorMap &msb, const CUtensorMap &msb2, int M,
+                                 int n_tiles_n, int K, const Epi &ep, cudaStream_t st) {
+  DeviceInfo *di = nullptr;
+  IG4_TRY(device_info(&di));
   const long tiles = static_cast<long>((M + 2 * GEMM_BM - 1) / (2 * GEMM_BM)) * n_tiles_n;
-  const int pairs = static_cast<int>(std::min<long>(tiles, sms / 2));
+  const int pairs = static_cast<int>(std::min<long>(tiles, di->sms / 2));
   const int group_m = gemm_group_m(M, K / 2, 1);
   cudaLaunchConfig_t lc = {};
   lc.gridDim = dim3(2 * pairs);
@@ -612,20 +616,90 @@ ig4_status launch_nvf4_pair(int M, int N, int K, const void *a_codes, const void
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = attr;
   lc.numAttrs = 2;
-  cudaError_t e;
+  auto kern = gemm_nvf4_pair_kernel<DUAL_B, Epi>;
+  IG4_TRY(allow_smem(kern, NVF4P_SMEM_BYTES));
+  if (cudaLaunchKernelEx(&lc, kern, ma, mb, mb2, msa, msb, msb2, M, n_tiles_n, K, group_m, ep) !=
+      cudaSuccess)
+    return IG4_ERR_CUDA;
+  return last_launch_status();
+}
+
+// A operand maps of an NVFP4 GEMM: codes [M][K/2] and packed scales.
+ig4_status nvf4_a_maps(CUtensorMap *ma, CUtensorMap *msa, const void *codes, const void *sf,
+                       int M, int K) {
+  IG4_TRY(map_2d(ma, codes, 1, M, K / 2, K / 2, GEMM_BM, 128));
+  return map_sf_3d(msa, sf, M, K, 1);
+}
+
+// NVFP4 linear layer on CTA pairs: out = a_scale w_scale (A W^T) (+ bias).
+ig4_status launch_nvf4_pair(int M, int N, int K, const void *a_codes, const void *a_sf,
+                            const float *a_scale, const void *w_codes, const void *w_sf,
+                            const float *w_scale, const float *bias, void *out, int out_dtype,
+                            cudaStream_t st) {
+  CUtensorMap ma, mb, msa, msb;
+  IG4_TRY(nvf4_a_maps(&ma, &msa, a_codes, a_sf, M, K));
+  IG4_TRY(map_2d(&mb, w_codes, 1, N, K / 2, K / 2, 128, 128));
+  IG4_TRY(map_sf_3d(&msb, w_sf, N, K, 2));
   if (out_dtype == IG4_F32) {
     EpiStore<256, true, float> ep{static_cast<float *>(out), N, M, N, bias, a_scale, w_scale, 0, 0, 0};
-    auto kern = gemm_nvf4_pair_kernel<decltype(ep)>;
-    IG4_TRY(allow_smem(kern, NVF4P_SMEM_BYTES));
-    e = cudaLaunchKernelEx(&lc, kern, ma, mb, msa, msb, M, n_tiles_n, K, group_m, ep);
-  } else {
-    EpiStore<256, true, __nv_bfloat16> ep{static_cast<__nv_bfloat16 *>(out), N, M, N, bias,
-                                          a_scale, w_scale, 0, 0, 0};
-    auto kern = gemm_nvf4_pair_kernel<decltype(ep)>;
-    IG4_TRY(allow_smem(kern, NVF4P_SMEM_BYTES));
-    e = cudaLaunchKernelEx(&lc, kern, ma, mb, msa, msb, M, n_tiles_n, K, group_m, ep);
+    return launch_nvf4_pair_maps<false>(ma, mb, mb, msa, msb, msb, M, N / 256, K, ep, st);
   }
-  if (e != cudaSuccess) return IG4_ERR_CUDA;
+  EpiStore<256, true, __nv_bfloat16> ep{static_cast<__nv_bfloat16 *>(out), N, M, N, bias,
+                                        a_scale, w_scale, 0, 0, 0};
+  return launch_nvf4_pair_maps<false>(ma, mb, mb, msa, msb, msb, M, N / 256, K, ep, st);
+}
+
+// NVFP4 gate/up + SwiGLU: u = silu(a_scale s_g (h W_g^T)) * (a_scale s_u (h W_u^T)), bf16.
+ig4_status launch_nvf4_swiglu(int M, int I, int K, const void *h_codes, const void *h_sf,
+                              const float *h_scale, const void *wg, const void *sfg,
+                              const float *sg, const void *wu, const void *sfu, const float *su,
+                              void *u, cudaStream_t st) {
+  CUtensorMap ma, msa, mg, mu, msg, msu;
+  IG4_TRY(nvf4_a_maps(&ma, &msa, h_codes, h_sf, M, K));
+  IG4_TRY(map_2d(&mg, wg, 1, I, K / 2, K / 2, 128, 128));
+  IG4_TRY(map_2d(&mu, wu, 1, I, K / 2, K / 2, 128, 128));
+  IG4_TRY(map_sf_3d(&msg, sfg, I, K, 1));
+  IG4_TRY(map_sf_3d(&msu, sfu, I, K, 1));
+  EpiSwiGLU<true> ep{static_cast<__nv_bfloat16 *>(u), I, M, h_scale, sg, su};
+  return launch_nvf4_pair_maps<true>(ma, mg, mu, msa, msg, msu, M, I / 128, K, ep, st);
+}
+
+// NVFP4 down-projection + gated residual: x_out = x_res + gate * (a_scale w_scale (u W^T)).
+template <typename XT>
+ig4_status launch_nvf4_resid_t(int B, int L, int N, int K, const void *a_codes, const void *a_sf,
+                               const float *a_scale, const void *w, const void *w_sf,
+                               const float *w_scale, const float *gate, int gate_stride,
+                               const void *x_res, void *x_out, cudaStream_t st) {
+  const int M = B * L;
+  CUtensorMap ma, msa, mb, msb;
+  IG4_TRY(nvf4_a_maps(&ma, &msa, a_codes, a_sf, M, K));
+  IG4_TRY(map_2d(&mb, w, 1, N, K / 2, K / 2, 128, 128));
+  IG4_TRY(map_sf_3d(&msb, w_sf, N, K, 2));
+  EpiResidGate<256, true, XT> ep{static_cast<const XT *>(x_res), static_cast<XT *>(x_out), gate,
+                                 gate_stride, L, M, N, a_scale, w_scale};
+  return launch_nvf4_pair_maps<false>(ma, mb, mb, msa, msb, msb, M, N / 256, K, ep, st);
+}
+
+ig4_status launch_nvf4_resid(int B, int L, int N, int K, const void *a_codes, const void *a_sf,
+                             const float *a_scale, const void *w, const void *w_sf,
+                             const float *w_scale, const float *gate, int gate_stride,
+                             const void *x_res, void *x_out, int x_dtype, cudaStream_t st) {
+  if (x_dtype == IG4_F32)
+    return launch_nvf4_resid_t<float>(B, L, N, K, a_codes, a_sf, a_scale, w, w_sf, w_scale, gate,
+                                      gate_stride, x_res, x_out, st);
+  return launch_nvf4_resid_t<__nv_bfloat16>(B, L, N, K, a_codes, a_sf, a_scale, w, w_sf, w_scale,
+                                            gate, gate_stride, x_res, x_out, st);
+}
+
+// bf16 rows -> NVFP4 codes, packed scales and row scales (one warp per row).
+ig4_status launch_nvf4_quantize(int M, int K, const void *x, void *codes, void *sf,
+                                float *row_scale, cudaStream_t st) {
+  const int rows_per_cta = NVF4Q_THREADS / 32;
+  if (launch_pdl(nvf4_quantize_kernel, dim3((M + rows_per_cta - 1) / rows_per_cta),
+                 dim3(NVF4Q_THREADS), 0, st, static_cast<const __nv_bfloat16 *>(x), M, K,
+                 static_cast<uint8_t *>(codes), static_cast<uint8_t *>(sf), row_scale) !=
+      cudaSuccess)
+    return IG4_ERR_CUDA;
   return last_launch_status();
 }
 
@@ -677,6 +751,7 @@ struct BlockWs {
   void *u;        // bf16 [M][I]
   void *uq;       // e4m3 [M][I]
   float *u_scale;
+  void *h_sf, *u_sf;  // packed NVFP4 scales of h2 and u (NVFP4-mixed FFN)
   int vt_ld;
   size_t bytes;
 };
@@ -688,6 +763,7 @@ BlockWs block_ws_layout(const ig4_config *c, uint8_t *base) {
   const long M = c->B * L;
   const long D = c->D, I = c->I, H = c->H;
   const bool f8 = is_fp8(c->w_dtype);
+  const bool nv4 = is_nvf4_mixed(c->w_dtype);
   w.vt_ld = static_cast<int>(round_up(L, 8));
   size_t off = 0;
   auto take = [&](size_t n) -> uint8_t * {
@@ -698,7 +774,7 @@ BlockWs block_ws_layout(const ig4_config *c, uint8_t *base) {
   w.mod = reinterpret_cast<float *>(take(sizeof(float) * c->B * 6 * D));
   w.cos = reinterpret_cast<float *>(take(sizeof(float) * L * 64));
   w.sin = reinterpret_cast<float *>(take(sizeof(float) * L * 64));
-  w.h = take((f8 ? 1 : 2) * M * D);
+  w.h = take((f8 && !nv4 ? 1 : 2) * M * D);  // NVFP4 FFN: h2 in bf16 before quantising
   w.h_scale = reinterpret_cast<float *>(take(f8 ? sizeof(float) * M : 0));
   w.q = take(2 * c->B * H * L * 256);
   w.k = take(2 * c->B * H * L * 256);
@@ -709,6 +785,10 @@ BlockWs block_ws_layout(const ig4_config *c, uint8_t *base) {
   w.u = take(2 * M * I);
   w.uq = take(f8 ? M * I : 0);
   w.u_scale = reinterpret_cast<float *>(take(f8 ? sizeof(float) * M : 0));
+  // NVFP4 FFN: h2 codes reuse oq (M D / 2 bytes), u codes reuse uq
+  const long rb = (M + 127) / 128;
+  w.h_sf = take(nv4 ? rb * (D / 64) * 512 : 0);
+  w.u_sf = take(nv4 ? rb * (I / 64) * 512 : 0);
   w.bytes = off;
   return w;
 }
@@ -722,6 +802,11 @@ ig4_status check_block_weights(const ig4_config *c, const ig4_block_weights *w) 
   if (is_fp8(c->w_dtype)) {
     const void *s[] = {w->s_ada, w->s_qkv, w->s_o, w->s_gate, w->s_up, w->s_down};
     for (const void *p : s)
+      if (!p || !aligned16(p)) return IG4_ERR_INVALID_ARG;
+  }
+  if (is_nvf4_mixed(c->w_dtype)) {
+    const void *sf[] = {w->sf_gate, w->sf_up, w->sf_down};
+    for (const void *p : sf)
       if (!p || !aligned16(p)) return IG4_ERR_INVALID_ARG;
   }
   return IG4_OK;
@@ -780,6 +865,23 @@ ig4_status block_forward_impl(const ig4_config *c, const ig4_block_weights *w, c
   IG4_TRY(launch_resid(c->B, L, D, D, f8 ? ws.oq : ws.o, f8, ws.o_scale, w->w_o, w->s_o,
                        ws.mod + 2 * D, ms, x_in, x_out, c->x_dtype, st));
   IG4_TRY(t.mark());
+  if (is_nvf4_mixed(c->w_dtype)) {
+    // FFN in NVFP4: h2 (bf16) and u (bf16) are quantised to NVFP4 for the
+    // block-scaled FP4 GEMMs; the h2 quantiser shares the norm's trace slot
+    IG4_TRY(launch_norm(M, L, D, x_out, c->x_dtype, ws.mod + 3 * D, ws.mod + 4 * D, ms, c->eps,
+                        ws.h, IG4_BF16, nullptr, 0, 0, 0, st));
+    IG4_TRY(launch_nvf4_quantize(M, D, ws.h, ws.oq, ws.h_sf, ws.h_scale, st));
+    IG4_TRY(t.mark());
+    IG4_TRY(launch_nvf4_swiglu(M, I, D, ws.oq, ws.h_sf, ws.h_scale, w->w_gate, w->sf_gate,
+                               w->s_gate, w->w_up, w->sf_up, w->s_up, ws.u, st));
+    IG4_TRY(t.mark());
+    IG4_TRY(launch_nvf4_quantize(M, I, ws.u, ws.uq, ws.u_sf, ws.u_scale, st));
+    IG4_TRY(t.mark());
+    IG4_TRY(launch_nvf4_resid(c->B, L, D, I, ws.uq, ws.u_sf, ws.u_scale, w->w_down, w->sf_down,
+                              w->s_down, ws.mod + 5 * D, ms, x_out, x_out, c->x_dtype, st));
+    IG4_TRY(t.mark());
+    return IG4_OK;
+  }
   IG4_TRY(launch_norm(M, L, D, x_out, c->x_dtype, ws.mod + 3 * D, ws.mod + 4 * D, ms, c->eps,
                       ws.h, hdt, ws.h_scale, 0, 0, 0, st));
   IG4_TRY(t.mark());
@@ -1139,13 +1241,22 @@ ig4_status ig4_nvfp4_linear(int M, int N, int K, const void *a_codes, const void
   // there are two waves of them, or 128-wide tiles
   if (N % 256 == 0 && M > GEMM_BM)
     return launch_nvf4_pair(M, N, K, a_codes, a_sf, a_scale, w_codes, w_sf, w_scale, bias, out,
-                            out_dtype, di->sms, as_stream(stream));
+                            out_dtype, as_stream(stream));
   const long tiles256 = static_cast<long>((M + GEMM_BM - 1) / GEMM_BM) * (N / 256);
   if (N % 256 == 0 && tiles256 >= 2L * di->sms)
     return launch_nvf4<256>(M, N, K, a_codes, a_sf, a_scale, w_codes, w_sf, w_scale, bias, out,
                             out_dtype, di->sms, as_stream(stream));
   return launch_nvf4<128>(M, N, K, a_codes, a_sf, a_scale, w_codes, w_sf, w_scale, bias, out,
                           out_dtype, di->sms, as_stream(stream));
+}
+
+ig4_status ig4_nvfp4_quantize(int M, int K, const void *x, void *codes, void *sf_packed,
+                              float *row_scale, void *stream) {
+  if (M < 1 || K < 64 || K % 64) return IG4_ERR_INVALID_ARG;
+  const void *ptrs[] = {x, codes, sf_packed, row_scale};
+  for (const void *p : ptrs)
+    if (!p || !aligned16(p)) return IG4_ERR_INVALID_ARG;
+  return launch_nvf4_quantize(M, K, x, codes, sf_packed, row_scale, as_stream(stream));
 }
 
 // --------------------------------------------------- text conditioning

@@ -729,6 +729,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 // barrier.  Per stage and CTA: 32 KB of codes + 6 KB of scales per 512 MMA
 // clocks at the FP4 rate, the same bytes per clock as the FP8 pair kernel.
 // One TMEM accumulator (256 columns) plus a 48-column scale region per stage.
+// DUAL_B (SwiGLU gate/up): B rows of the tile's first 128 columns come from
+// tmB (gate) and of the last 128 from tmB2 (up), both at rows nt * 128, with
+// their scale blocks from tmSFB / tmSFB2 (one 128-row block each); otherwise
+// B rows nt * 256 + [0, 256) come from tmB and their two scale blocks from
+// tmSFB.
 constexpr int NVF4P_STAGES = 5;
 constexpr int NVF4P_A_BYTES = GEMM_BM * 128;
 constexpr int NVF4P_BH_BYTES = 128 * 128;
@@ -739,11 +744,13 @@ constexpr int NVF4P_SMEM_BYTES = NVF4P_STAGES * NVF4P_STAGE_BYTES + 1024 + 256;
 constexpr uint32_t NVF4P_SF_COLS = 48;
 static_assert(256 + NVF4P_STAGES * NVF4P_SF_COLS <= 512, "TMEM");
 
-template <class Epi>
+template <bool DUAL_B, class Epi>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                          const __grid_constant__ CUtensorMap tmB2,
                           const __grid_constant__ CUtensorMap tmSFA,
-                          const __grid_constant__ CUtensorMap tmSFB, int M, int n_tiles_n, int K,
+                          const __grid_constant__ CUtensorMap tmSFB,
+                          const __grid_constant__ CUtensorMap tmSFB2, int M, int n_tiles_n, int K,
                           int group_m, const Epi epi) {
   constexpr int BN = 256;
   constexpr uint32_t IDESC = idesc_nvf4(2 * GEMM_BM, BN);
@@ -786,6 +793,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     tma_prefetch_desc(&tmB);
     tma_prefetch_desc(&tmSFA);
     tma_prefetch_desc(&tmSFB);
+    if (DUAL_B) {
+      tma_prefetch_desc(&tmB2);
+      tma_prefetch_desc(&tmSFB2);
+    }
   }
   if (warp == 5) {
     tmem_alloc_pair(tmem_slot, 512);
@@ -816,11 +827,18 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * NVF4P_STAGE_BYTES);
           const uint32_t bar = map_shared_to_rank(&full[s], 0);
           tma_load_2d_pair(sA + s * NVF4P_A_BYTES, &tmA, bar, kb * 128, mrow);
-          tma_load_2d_pair(sB + s * NVF4P_BH_BYTES, &tmB, bar, kb * 128,
-                           nt * BN + static_cast<int>(rank) * (BN / 2));
           // scale blocks: [128 words of 4 B] x [4 K chunks] x [row blocks]
           tma_load_3d_pair(sSFA + s * NVF4P_SFA_BYTES, &tmSFA, bar, 0, 4 * kb, mrow / 128);
-          tma_load_3d_pair(sSFB + s * NVF4P_SFB_BYTES, &tmSFB, bar, 0, 4 * kb, nt * 2);
+          if constexpr (DUAL_B) {
+            tma_load_2d_pair(sB + s * NVF4P_BH_BYTES, rank ? &tmB2 : &tmB, bar, kb * 128, nt * 128);
+            tma_load_3d_pair(sSFB + s * NVF4P_SFB_BYTES, &tmSFB, bar, 0, 4 * kb, nt);
+            tma_load_3d_pair(sSFB + s * NVF4P_SFB_BYTES + NVF4P_SFB_BYTES / 2, &tmSFB2, bar, 0,
+                             4 * kb, nt);
+          } else {
+            tma_load_2d_pair(sB + s * NVF4P_BH_BYTES, &tmB, bar, kb * 128,
+                             nt * BN + static_cast<int>(rank) * (BN / 2));
+            tma_load_3d_pair(sSFB + s * NVF4P_SFB_BYTES, &tmSFB, bar, 0, 4 * kb, nt * 2);
+          }
           if (++s == NVF4P_STAGES) {
             s = 0;
             ph ^= 1;

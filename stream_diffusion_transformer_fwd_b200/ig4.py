@@ -20,12 +20,12 @@ LIB_PATH = os.path.join(_HERE, "libig4.so")
 
 IG4_OK, IG4_ERR_INVALID_ARG, IG4_ERR_UNSUPPORTED, IG4_ERR_WORKSPACE, IG4_ERR_CUDA, \
     IG4_ERR_TIMEOUT = range(6)
-IG4_F32, IG4_BF16, IG4_E4M3 = 0, 1, 2
+IG4_F32, IG4_BF16, IG4_E4M3, IG4_NVFP4_MIXED = 0, 1, 2, 3
 IG4_BLOCK_TRACE_EVENTS = 12
 IG4_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 _DTYPE_CODE = {torch.float32: IG4_F32, torch.bfloat16: IG4_BF16, torch.float8_e4m3fn: IG4_E4M3}
-_CODE_NAME = {IG4_F32: "f32", IG4_BF16: "bf16", IG4_E4M3: "e4m3"}
+_CODE_NAME = {IG4_F32: "f32", IG4_BF16: "bf16", IG4_E4M3: "e4m3", IG4_NVFP4_MIXED: "nvfp4_mixed"}
 _NAME_CODE = {v: k for k, v in _CODE_NAME.items()}
 
 if not os.path.exists(LIB_PATH):
@@ -55,7 +55,7 @@ class Config(ctypes.Structure):
 class BlockWeights(ctypes.Structure):
     _fields_ = [(n, _vp) for n in ("w_ada", "w_qkv", "w_o", "w_gate", "w_up", "w_down",
                                    "s_ada", "s_qkv", "s_o", "s_gate", "s_up", "s_down",
-                                   "b_ada", "g_q", "g_k")]
+                                   "b_ada", "g_q", "g_k", "sf_gate", "sf_up", "sf_down")]
 
 
 class StackWeights(ctypes.Structure):
@@ -99,6 +99,7 @@ _sig("ig4_stack_forward", [ctypes.POINTER(Config), ctypes.POINTER(StackWeights),
 _sig("ig4_nvfp4_scale_bytes", [_i, _i], ctypes.c_size_t)
 _sig("ig4_nvfp4_pack_scales", [_i, _i, _vp, _vp, _vp])
 _sig("ig4_nvfp4_linear", [_i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp])
+_sig("ig4_nvfp4_quantize", [_i, _i, _vp, _vp, _vp, _vp, _vp])
 _sig("ig4_text_cond_workspace_size", [_i, _i, _i], ctypes.c_size_t)
 _sig("ig4_text_cond_project", [_i, _i, _i, _vp, _vp, _f, _vp, _vp, _i, _vp, _vp, _vp,
                                ctypes.c_size_t, _vp])
@@ -119,7 +120,7 @@ EXPORTED = ("ig4_status_string", "ig4_abi_version", "ig4_mrope_positions", "ig4_
             "ig4_quantize_rows", "ig4_workspace_size", "ig4_block_forward",
             "ig4_block_forward_traced", "ig4_block_forward_noalloc", "ig4_stack_workspace_size",
             "ig4_stack_forward", "ig4_nvfp4_scale_bytes", "ig4_nvfp4_pack_scales",
-            "ig4_nvfp4_linear", "ig4_text_cond_workspace_size", "ig4_text_cond_project",
+            "ig4_nvfp4_linear", "ig4_nvfp4_quantize", "ig4_text_cond_workspace_size", "ig4_text_cond_project",
             "ig4_flow_schedule", "ig4_guidance_schedule", "ig4_cfg_euler",
             "ig4_denoise_workspace_size", "ig4_denoise_step", "ig4_last_device_error",
             "ig4_selftest_timeout")
@@ -172,6 +173,20 @@ def config_from(cfg) -> Config:
     return make_config(cfg.B, cfg.T_text, cfg.grid_t, cfg.grid_h, cfg.grid_w, cfg.D, cfg.H,
                        cfg.head_dim, cfg.I, cfg.adaln_dim, cfg.rope_theta, tuple(cfg.sections),
                        cfg.eps, cfg.x_dtype, cfg.w_dtype)
+
+
+def nvfp4_pack_block_scales(w: dict, stream=None) -> dict:
+    """For NVFP4-mixed block weights on the device: adds sf_gate / sf_up /
+    sf_down, the packed block scales (ig4_nvfp4_pack_scales) of the row-major
+    scales sfr_gate / sfr_up / sfr_down."""
+    out = dict(w)
+    for name in ("gate", "up", "down"):
+        rows = w["sfr_" + name]
+        packed = torch.empty(ig4_nvfp4_scale_bytes(rows.shape[0], 16 * rows.shape[1]),
+                             dtype=torch.uint8, device=rows.device)
+        ig4_nvfp4_pack_scales(rows, packed, stream)
+        out["sf_" + name] = packed
+    return out
 
 
 def block_weights(w: dict) -> BlockWeights:
@@ -341,6 +356,14 @@ def ig4_nvfp4_linear(a_codes, a_sf, a_scale, w_codes, w_sf, w_scale, bias, out, 
     _check(_lib.ig4_nvfp4_linear(M, N, K, _ptr(a_codes), _ptr(a_sf), _ptr(a_scale), _ptr(w_codes),
                                  _ptr(w_sf), _ptr(w_scale), _ptr(bias), _ptr(out),
                                  dtype_code(out), _stream(stream)), "ig4_nvfp4_linear")
+
+
+def ig4_nvfp4_quantize(x, codes, sf_packed, row_scale, stream=None):
+    """bf16 activations x [M, K] -> NVFP4 codes [M, K/2] uint8, packed block
+    scales (ig4_nvfp4_scale_bytes(M, K) bytes) and fp32 row scales [M]."""
+    M, K = x.shape
+    _check(_lib.ig4_nvfp4_quantize(M, K, _ptr(x), _ptr(codes), _ptr(sf_packed), _ptr(row_scale),
+                                   _stream(stream)), "ig4_nvfp4_quantize")
 
 
 def ig4_text_cond_workspace_size(M: int, K_raw: int, w_dtype: str = "bf16") -> int:

@@ -64,19 +64,29 @@ def _bias(seed, block, name, n, stress):
 def make_block_weights(cfg: Config, seed: int = 0, block: int = 0, stress: bool = False,
                        zero_adaln: bool = False) -> dict:
     """Weights of one block: w_* [out, in] (bf16 or E4M3 codes), s_* fp32 scales
-    (E4M3 only, else None), b_ada fp32 [6D], g_q / g_k fp32 [head_dim]."""
+    (E4M3 only, else None), b_ada fp32 [6D], g_q / g_k fp32 [head_dim].  With
+    w_dtype "nvfp4_mixed" the FFN weights are NVFP4 (see make_nvfp4_linear:
+    w_* codes, sfr_* row-major block scales, s_* channel scales)."""
     D, I, A, dh = cfg.D, cfg.I, cfg.adaln_dim, cfg.head_dim
     wd = cfg.w_dtype
+    wa = "e4m3" if wd == "nvfp4_mixed" else wd  # AdaLN and attention projections
     out = {}
-    out["w_ada"], out["s_ada"] = _linear(seed, block, "w_ada", 6 * D, A, wd, std=0.02)
+    out["w_ada"], out["s_ada"] = _linear(seed, block, "w_ada", 6 * D, A, wa, std=0.02)
     if zero_adaln:
         out["w_ada"] = torch.zeros_like(out["w_ada"])
     out["b_ada"] = torch.zeros(6 * D) if zero_adaln else _bias(seed, block, "b_ada", 6 * D, stress)
-    out["w_qkv"], out["s_qkv"] = _linear(seed, block, "w_qkv", 3 * D, D, wd)
-    out["w_o"], out["s_o"] = _linear(seed, block, "w_o", D, D, wd)
-    out["w_gate"], out["s_gate"] = _linear(seed, block, "w_gate", I, D, wd)
-    out["w_up"], out["s_up"] = _linear(seed, block, "w_up", I, D, wd)
-    out["w_down"], out["s_down"] = _linear(seed, block, "w_down", D, I, wd)
+    out["w_qkv"], out["s_qkv"] = _linear(seed, block, "w_qkv", 3 * D, D, wa)
+    out["w_o"], out["s_o"] = _linear(seed, block, "w_o", D, D, wa)
+    if wd == "nvfp4_mixed":
+        # FFN linears in NVFP4 (E2M1 codes, row-major E4M3 block scales sfr_*,
+        # channel scales s_*); every other linear in E4M3
+        for name, n_out, n_in in (("gate", I, D), ("up", I, D), ("down", D, I)):
+            q = make_nvfp4_linear(seed, block, "w_" + name, n_out, n_in)
+            out["w_" + name], out["sfr_" + name], out["s_" + name] = q["codes"], q["sf"], q["s"]
+    else:
+        out["w_gate"], out["s_gate"] = _linear(seed, block, "w_gate", I, D, wd)
+        out["w_up"], out["s_up"] = _linear(seed, block, "w_up", I, D, wd)
+        out["w_down"], out["s_down"] = _linear(seed, block, "w_down", D, I, wd)
     if stress:
         out["g_q"] = torch.from_numpy(1.0 + _normal(seed, block, "g_q", (dh,), 0.2))
         out["g_k"] = torch.from_numpy(1.0 + _normal(seed, block, "g_k", (dh,), 0.2))

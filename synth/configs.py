@@ -29,7 +29,7 @@ class Config:
     sections: tuple = (24, 20, 20)
     eps: float = 1e-6
     x_dtype: str = "bf16"     # residual stream storage: "f32" or "bf16"
-    w_dtype: str = "bf16"     # linear weight storage: "bf16" or "e4m3"
+    w_dtype: str = "bf16"     # linear weight storage: "bf16", "e4m3" or "nvfp4_mixed"
     n_blocks: int = 1         # > 1 only for the stack workload
     latent_ch: int = 128
 
@@ -74,6 +74,13 @@ CONFIGS = {
     # the attention projections in FP8): gate/up and down at 1024 px
     "ffn_1024px_nvfp4": Config("ffn_1024px_nvfp4", B=1, T_text=512, grid_t=1, grid_h=64,
                                grid_w=64, w_dtype="nvfp4"),
+    # the whole block with the NVFP4 Mixed weights: FFN linears in NVFP4, the
+    # AdaLN and attention projections in FP8 (1024 px, and a small case with
+    # 64 text + 12x12 image tokens at D = 1024)
+    "1024px_nvfp4": Config("1024px_nvfp4", B=1, T_text=512, grid_t=1, grid_h=64, grid_w=64,
+                           w_dtype="nvfp4_mixed"),
+    "small_nvfp4": Config("small_nvfp4", B=1, T_text=64, grid_t=1, grid_h=12, grid_w=12, D=1024,
+                          H=4, I=2816, w_dtype="nvfp4_mixed"),
     # the text conditioning projection of a 2048-token caption (13 x 4096 = 53248
     # raw features per token -> 4608), FP8 weights as released
     "textcond_2048_fp8": Config("textcond_2048_fp8", B=1, T_text=2048, grid_t=1, grid_h=0,

@@ -39,7 +39,7 @@ def test_header_symbols_are_exported(ig4):
 
 
 def test_status_strings_and_version(ig4):
-    assert ig4.ig4_abi_version() == 1
+    assert ig4.ig4_abi_version() == 2
     for code, name in enumerate(["IG4_OK", "IG4_ERR_INVALID_ARG", "IG4_ERR_UNSUPPORTED",
                                  "IG4_ERR_WORKSPACE", "IG4_ERR_CUDA", "IG4_ERR_TIMEOUT"]):
         assert ig4.ig4_status_string(code) == name
@@ -162,3 +162,16 @@ def test_op_validation_returns_before_launch(ig4):
     assert lib.ig4_selftest_timeout(0, None) == ig4.IG4_ERR_INVALID_ARG
     assert lib.ig4_adaln_modulation(9, 512, 8, p, p, 1, None, None, p, None) == \
         ig4.IG4_ERR_INVALID_ARG
+
+
+def test_nvfp4_mixed_config_rules(ig4):
+    """NVFP4 Mixed block configs: accepted with I % 256 == 0 and more than 128
+    tokens; the workspace adds a bf16 h2 buffer and the packed scales."""
+    def ws(T, gh, I, wd):
+        return ig4.ig4_workspace_size(ig4.make_config(1, T, 1, gh, gh, D=1024, H=4, I=I,
+                                                      w_dtype=wd))
+    assert ws(64, 12, 2816, "nvfp4_mixed") > ws(64, 12, 2816, "e4m3") > 0
+    assert ws(16, 8, 2816, "nvfp4_mixed") == 0      # 80 tokens
+    assert ws(16, 8, 2816, "e4m3") > 0
+    assert ws(64, 12, 2944, "nvfp4_mixed") == 0     # I = 23 x 128
+    assert ws(64, 12, 2944, "e4m3") > 0

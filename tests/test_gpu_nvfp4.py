@@ -69,3 +69,108 @@ def test_nvfp4_argument_errors(ig4):
     with pytest.raises(ig4.Ig4Error) as e:  # K = 200 is not a multiple of 256
         ig4.ig4_nvfp4_linear(z[:400].view(4, 100), z, f, z[:12800].view(128, 100), z, f, None, out)
     assert e.value.status == ig4.IG4_ERR_INVALID_ARG
+
+
+# ------------------------------------------------- activation quantiser
+
+def _unpack_codes(packed: np.ndarray) -> np.ndarray:
+    out = np.empty((packed.shape[0], 2 * packed.shape[1]), dtype=np.uint8)
+    out[:, 0::2] = packed & 15
+    out[:, 1::2] = packed >> 4
+    return np.where(out == 8, 0, out)  # -0 and +0 are the same value
+
+
+def _unpack_scales(packed: np.ndarray, M: int, K: int) -> np.ndarray:
+    """Row-major [M][K/16] scale codes from the packed order the header
+    documents: a 512-byte block per 128 rows and 64 K-elements (row blocks
+    outer), byte 16 (r % 32) + 4 ((r % 128) / 32) + (k / 16) % 4."""
+    r = np.arange(M)[:, None]
+    b = np.arange(K // 16)[None, :]
+    off = ((r // 128) * (K // 64) + b // 4) * 512 + 16 * (r % 32) + 4 * ((r % 128) // 32) + b % 4
+    return packed[off]
+
+
+def test_nvfp4_quantize_bit_exact(ig4):
+    rng = np.random.default_rng(11)
+    M, K = 300, 1088  # ragged rows; K a multiple of 64 but not of 128
+    x = rng.standard_normal((M, K)) * np.exp(rng.uniform(-6, 6, (M, 1)))
+    x[5] = 0.0                      # all-zero row: row scale 1, zero codes
+    x[7, 64:80] = 0.0               # all-zero block
+    x[9, :16] *= 1e-7               # block whose scale underflows E4M3 to 0
+    x[11, 3] = 1e4 * np.abs(x[11]).max()  # one outlier carries the row scale
+    xb = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16)
+    codes = torch.empty(M, K // 2, dtype=torch.uint8, device="cuda")
+    sf = torch.zeros(ig4.ig4_nvfp4_scale_bytes(M, K), dtype=torch.uint8, device="cuda")
+    rs = torch.empty(M, dtype=torch.float32, device="cuda")
+    ig4.ig4_nvfp4_quantize(xb.cuda(), codes, sf, rs)
+    torch.cuda.synchronize()
+    assert ig4.ig4_last_device_error() == ig4.IG4_OK
+    ref_codes, ref_sc, ref_s = O.quantize_nvfp4_activations(xb.float().numpy())
+    assert np.array_equal(rs.cpu().numpy(), ref_s)
+    assert np.array_equal(_unpack_scales(sf.cpu().numpy(), M, K), ref_sc)
+    assert np.array_equal(_unpack_codes(codes.cpu().numpy()), np.where(ref_codes == 8, 0, ref_codes))
+    assert ref_s[5] == 1.0 and np.all(ref_sc[9, 0] == 0)
+
+
+def test_nvfp4_quantize_argument_errors(ig4):
+    x = torch.zeros(4, 96, dtype=torch.bfloat16, device="cuda")
+    z = torch.zeros(4096, dtype=torch.uint8, device="cuda")
+    f = torch.zeros(4, dtype=torch.float32, device="cuda")
+    with pytest.raises(ig4.Ig4Error) as e:  # K = 96 is not a multiple of 64
+        ig4.ig4_nvfp4_quantize(x, z, z, f)
+    assert e.value.status == ig4.IG4_ERR_INVALID_ARG
+
+
+# ------------------------------------- the block with NVFP4 Mixed weights
+
+def _nvfp4_block(ig4, seed, zero_attn_gate):
+    from synth import get_config, make_block_activations, make_block_weights
+    from oracle.inputs import block_weights_f64, to_f64
+    from tests.gpu_common import run_block, to_dev
+
+    cfg = get_config("small_nvfp4")
+    D = cfg.D
+    acts = make_block_activations(cfg, seed=seed)
+    wts = make_block_weights(cfg, seed=seed, stress=True)
+    if zero_attn_gate:  # gate_msa = 0: x1 = x exactly on both sides
+        wts["w_ada"].view(torch.uint8)[2 * D:3 * D] = 0
+        wts["b_ada"][2 * D:3 * D] = 0.0
+    wd = ig4.nvfp4_pack_block_scales(to_dev(wts))
+    y = run_block(ig4, cfg, wd, acts["x"].cuda(), acts["temb"].cuda())
+    pos = O.mrope_positions(cfg.T_text, cfg.grid_t, cfg.grid_h, cfg.grid_w)
+    x = to_f64(acts["x"])
+    y_ref = O.block_forward(x, to_f64(acts["temb"]), pos, block_weights_f64(wts), cfg.H,
+                            cfg.rope_theta, cfg.sections, cfg.eps, ffn_nvfp4=True)
+    return y.float().cpu().double().numpy(), y_ref, x
+
+
+def test_block_nvfp4_mixed_ffn_exact_quantisation(ig4):
+    """With the attention gate at zero, x1 = x on both sides and the FFN sees
+    the same h2: the GPU's NVFP4 decisions are the oracle's, up to the rare
+    element whose bf16 rounding differs, so delta = y - x agrees closely."""
+    from tests.gpu_common import delta_tolerance
+    y, y_ref, x = _nvfp4_block(ig4, 21, True)
+    d, d_ref = y - x, y_ref - x
+    e_y, e_d = rel_l2(y, y_ref), rel_l2(d, d_ref)
+    tol_d = delta_tolerance(2e-2, y_ref, d_ref, True)
+    print(f"nvfp4-mixed block, zero attention gate: relL2(y)={e_y:.3e} relL2(delta)={e_d:.3e} "
+          f"(tol {tol_d:.3e})")
+    assert e_y <= 1e-2 and e_d <= tol_d
+
+
+def test_block_nvfp4_mixed_full(ig4):
+    """Both branches on.  The oracle leaves the FP8 activations of the
+    attention projections unquantised (as for the FP8 block); that error
+    reaches h2, where NVFP4's decisions turn it into whole grid steps on the
+    elements and blocks near a rounding boundary, so delta takes a looser
+    bound than in the test above; y keeps the FP8 block's 3e-2."""
+    y, y_ref, x = _nvfp4_block(ig4, 22, False)
+    e_y, e_d = rel_l2(y, y_ref), rel_l2(y - x, y_ref - x)
+    print(f"nvfp4-mixed block: relL2(y)={e_y:.3e} relL2(delta)={e_d:.3e}")
+    assert e_y <= 3e-2 and e_d <= 0.15
+
+
+def test_block_nvfp4_mixed_needs_more_than_128_tokens(ig4):
+    from synth import get_config
+    cfg = get_config("small_nvfp4").with_(T_text=16, grid_h=8, grid_w=8)  # 80 tokens
+    assert ig4.ig4_workspace_size(ig4.config_from(cfg)) == 0
