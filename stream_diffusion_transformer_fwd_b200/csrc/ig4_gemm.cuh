@@ -168,15 +168,21 @@ struct EpiStore {
   const float *bias;
   const float *a_scale, *b_scale;
   int remap_n, remap_L, remap_off;
+  static constexpr int COLS = BN;
 
   __device__ __forceinline__ void operator()(int m0, int n0, uint32_t tacc, int r) const {
+    part(m0, n0, tacc, r, 0, BN);
+  }
+
+  // columns [lo, hi) of the tile (multiples of 32)
+  __device__ __forceinline__ void part(int m0, int n0, uint32_t tacc, int r, int lo, int hi) const {
     const int row = m0 + r;
     const bool valid = row < M;
     long orow = row;
     if (remap_n > 0) orow = static_cast<long>(row / remap_n) * remap_L + remap_off + row % remap_n;
     const float rs = (FP8 && valid) ? __ldg(a_scale + row) : 1.0f;
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
+    for (int c = lo; c < hi; c += 32) {
       float v[32];
       tmem_ld32(tacc + c, v);
       tmem_ld_wait();
@@ -203,15 +209,21 @@ struct EpiResidGate {
   int gate_stride;
   int L, M, N;
   const float *a_scale, *b_scale;
+  static constexpr int COLS = BN;
 
   __device__ __forceinline__ void operator()(int m0, int n0, uint32_t tacc, int r) const {
+    part(m0, n0, tacc, r, 0, BN);
+  }
+
+  // columns [lo, hi) of the tile (multiples of 32)
+  __device__ __forceinline__ void part(int m0, int n0, uint32_t tacc, int r, int lo, int hi) const {
     const int row = m0 + r;
     const bool valid = row < M;
     const int b = valid ? row / L : 0;
     const float rs = (FP8 && valid) ? __ldg(a_scale + row) : 1.0f;
     const float *grow = gate + static_cast<long>(b) * gate_stride + n0;
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
+    for (int c = lo; c < hi; c += 32) {
       float v[32];
       tmem_ld32(tacc + c, v);
       tmem_ld_wait();
@@ -236,14 +248,21 @@ struct EpiSwiGLU {
   __nv_bfloat16 *u;
   int I, M;
   const float *a_scale, *s_gate, *s_up;
+  static constexpr int COLS = 128;  // output columns per tile
 
   __device__ __forceinline__ void operator()(int m0, int n0, uint32_t tacc, int r) const {
+    part(m0, n0, tacc, r, 0, 128);
+  }
+
+  // output columns [lo, hi) of the tile: accumulator columns [lo, hi) (gate)
+  // and [128 + lo, 128 + hi) (up)
+  __device__ __forceinline__ void part(int m0, int n0, uint32_t tacc, int r, int lo, int hi) const {
     const int row = m0 + r;
     const bool valid = row < M;
     const float rs = (FP8 && valid) ? __ldg(a_scale + row) : 1.0f;
     const int n = n0 / 2;  // tile index * 128
 #pragma unroll 1
-    for (int c = 0; c < 128; c += 32) {
+    for (int c = lo; c < hi; c += 32) {
       float g[32], up[32];
       tmem_ld32(tacc + c, g);
       tmem_ld32(tacc + 128 + c, up);
@@ -728,7 +747,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 // read the B scales of every column); all loads complete on the leader's
 // barrier.  Per stage and CTA: 32 KB of codes + 6 KB of scales per 512 MMA
 // clocks at the FP4 rate, the same bytes per clock as the FP8 pair kernel.
-// One TMEM accumulator (256 columns) plus a 48-column scale region per stage.
+// TMEM: two 256-column accumulators that overlap in 64 columns, acc 0 at
+// [0, 256) and acc 1 at [192, 448), and one 48-column scale region at 448
+// (the scale blocks of k-block g are copied in after the MMAs of k-block
+// g - 1 were issued; tcgen05.cp and tcgen05.mma from one thread run in
+// issue order).  The epilogue of a tile drains the overlapped columns
+// first and releases them (ovl), so the next tile's MMAs start while it
+// converts the remaining 192 columns.
 // DUAL_B (SwiGLU gate/up): B rows of the tile's first 128 columns come from
 // tmB (gate) and of the last 128 from tmB2 (up), both at rows nt * 128, with
 // their scale blocks from tmSFB / tmSFB2 (one 128-row block each); otherwise
@@ -741,8 +766,9 @@ constexpr int NVF4P_SFA_BYTES = 2048;
 constexpr int NVF4P_SFB_BYTES = 4096;
 constexpr int NVF4P_STAGE_BYTES = NVF4P_A_BYTES + NVF4P_BH_BYTES + NVF4P_SFA_BYTES + NVF4P_SFB_BYTES;
 constexpr int NVF4P_SMEM_BYTES = NVF4P_STAGES * NVF4P_STAGE_BYTES + 1024 + 256;
-constexpr uint32_t NVF4P_SF_COLS = 48;
-static_assert(256 + NVF4P_STAGES * NVF4P_SF_COLS <= 512, "TMEM");
+constexpr uint32_t NVF4P_ACC1_COL = 192;
+constexpr uint32_t NVF4P_SF_COL = 448;
+static_assert(NVF4P_ACC1_COL + 256 <= NVF4P_SF_COL && NVF4P_SF_COL + 48 <= 512, "TMEM");
 
 template <bool DUAL_B, class Epi>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
@@ -762,9 +788,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   uint8_t *sSFB = sSFA + NVF4P_STAGES * NVF4P_SFA_BYTES;
   uint64_t *full = reinterpret_cast<uint64_t *>(sSFB + NVF4P_STAGES * NVF4P_SFB_BYTES);
   uint64_t *empty = full + NVF4P_STAGES;
-  uint64_t *tfull = empty + NVF4P_STAGES;
-  uint64_t *tempty = tfull + 1;
-  uint64_t *drain = tempty + 1;
+  uint64_t *tfull = empty + NVF4P_STAGES;  // [2]: accumulator ready
+  uint64_t *tempty = tfull + 2;            // [2]: accumulator drained
+  uint64_t *ovl = tempty + 2;              // overlapped columns drained
+  uint64_t *drain = ovl + 1;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -782,8 +809,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(tfull, 1);
-    mbar_init(tempty, 2 * 4);  // one arrival per epilogue warp of the pair
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 2 * 4);  // one arrival per epilogue warp of the pair
+    }
+    mbar_init(ovl, 2 * 4);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -852,18 +882,23 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       // ---------------- MMA issuer (leader CTA)
       int s = 0;
       uint32_t ph = 0;
-      int local = 0;
       bool ok = true;
-      for (int t = pair; t < n_tiles && ok; t += n_pairs, ++local) {
-        if (!mbar_wait_cluster(tempty, (static_cast<uint32_t>(local) & 1) ^ 1, abort_flag)) break;
+      const uint32_t sf = tmem_base + NVF4P_SF_COL;
+      for (int t = pair, i = 0; t < n_tiles && ok; t += n_pairs, ++i) {
+        const int acc = i & 1;
+        // this accumulator's own columns: drained by the epilogue of tile i - 2;
+        // the overlapped ones: by the epilogue of tile i - 1
+        if (!mbar_wait_cluster(&tempty[acc], static_cast<uint32_t>((i >> 1) & 1) ^ 1, abort_flag))
+          break;
+        if (i > 0 && !mbar_wait_cluster(ovl, static_cast<uint32_t>((i - 1) & 1), abort_flag)) break;
         tc_fence_after();
+        const uint32_t d = tmem_base + (acc ? NVF4P_ACC1_COL : 0);
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait_cluster(&full[s], ph, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sf = tmem_base + 256 + NVF4P_SF_COLS * s;
           const uint32_t sfa_s = smem_u32(sSFA + s * NVF4P_SFA_BYTES);
           const uint32_t sfb_s = smem_u32(sSFB + s * NVF4P_SFB_BYTES);
 #pragma unroll
@@ -878,7 +913,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           for (int j = 0; j < 4; ++j) {
             const uint64_t ad = sdesc_kmajor_sw128(a_base + 32 * j);
             const uint64_t bd = sdesc_kmajor_sw128(b_base + 32 * j);
-            umma_nvf4_pair(tmem_base, ad, bd, IDESC, sf + 4 * j, sf + 16 + 8 * j, (kb | j) != 0);
+            umma_nvf4_pair(d, ad, bd, IDESC, sf + 4 * j, sf + 16 + 8 * j, (kb | j) != 0);
           }
           umma_commit_pair_both(&empty[s]);
           if (++s == NVF4P_STAGES) {
@@ -886,7 +921,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             ph ^= 1;
           }
         }
-        if (ok) umma_commit_pair_both(tfull);
+        if (ok) umma_commit_pair_both(&tfull[acc]);
       }
       umma_commit_pair_both(drain);
       mbar_wait_cluster(drain, 0, nullptr, WAIT_LIMIT_NS / 4);
@@ -895,18 +930,27 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     // ---------------- epilogue warps 0..3 (both CTAs, own 128 rows)
     const int r = warp * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tempty_leader = map_shared_to_rank(tempty, 0);
-    int local = 0;
-    for (int t = pair; t < n_tiles; t += n_pairs, ++local) {
-      const bool ok = mbar_wait_cluster(tfull, static_cast<uint32_t>(local) & 1, abort_flag);
+    const uint32_t ovl_leader = map_shared_to_rank(ovl, 0);
+    constexpr int C = Epi::COLS;  // 64 accumulator columns overlap: the top 64 of
+    constexpr int OV = C - 64;    // acc 0's epilogue columns, the bottom 64 of acc 1's
+    for (int t = pair, i = 0; t < n_tiles; t += n_pairs, ++i) {
+      const int acc = i & 1;
+      const bool ok =
+          mbar_wait_cluster(&tfull[acc], static_cast<uint32_t>((i >> 1) & 1), abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       int mt, nt;
       tile_coords(t, m_tiles, n_tiles_n, group_m, &mt, &nt);
-      epi(mt * 2 * GEMM_BM + static_cast<int>(rank) * GEMM_BM, nt * BN, tmem_base + lane_base, r);
+      const int m0 = mt * 2 * GEMM_BM + static_cast<int>(rank) * GEMM_BM;
+      const uint32_t tacc = tmem_base + (acc ? NVF4P_ACC1_COL : 0) + lane_base;
+      epi.part(m0, nt * BN, tacc, r, acc ? 0 : OV, acc ? 64 : C);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(tempty_leader);
+      if (lane == 0) mbar_arrive_cluster(ovl_leader);
+      epi.part(m0, nt * BN, tacc, r, acc ? 64 : 0, acc ? C : OV);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(map_shared_to_rank(&tempty[acc], 0));
     }
   }
 
