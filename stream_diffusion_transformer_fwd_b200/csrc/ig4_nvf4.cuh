@@ -76,6 +76,7 @@ __global__ void __launch_bounds__(NVF4Q_THREADS)
   const uint4 *xr = reinterpret_cast<const uint4 *>(x + static_cast<long>(row) * K);
   const int nblk = K / 16;
   float amax = 0.0f;
+#pragma unroll 4
   for (int b = lane; b < nblk; b += 32) {
     float f[16];
     unpack_bf16x16(__ldg(xr + 2 * b), __ldg(xr + 2 * b + 1), f);
@@ -86,6 +87,7 @@ __global__ void __launch_bounds__(NVF4Q_THREADS)
   const float s = amax > 0.0f ? amax / 2688.0f : 1.0f;
   const float t = 6.0f * s;
   uint2 *cr = reinterpret_cast<uint2 *>(codes + static_cast<long>(row) * (K / 2));
+#pragma unroll 2
   for (int b = lane; b < nblk; b += 32) {
     float f[16];
     unpack_bf16x16(__ldg(xr + 2 * b), __ldg(xr + 2 * b + 1), f);
