@@ -21,6 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libig4.so")
 IG4_OK, IG4_ERR_INVALID_ARG, IG4_ERR_UNSUPPORTED, IG4_ERR_WORKSPACE, IG4_ERR_CUDA, \
     IG4_ERR_TIMEOUT = range(6)
 IG4_F32, IG4_BF16, IG4_E4M3, IG4_NVFP4_MIXED = 0, 1, 2, 3
+IG4_ABI_VERSION = 2  # the include/ig4.h revision this binding marshals for
 IG4_BLOCK_TRACE_EVENTS = 12
 IG4_NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -75,6 +76,9 @@ def _sig(name, args, res=_i):
 _lib.ig4_status_string.argtypes = [_i]
 _lib.ig4_status_string.restype = ctypes.c_char_p
 _sig("ig4_abi_version", [])
+if _lib.ig4_abi_version() != IG4_ABI_VERSION:
+    raise ImportError(f"{LIB_PATH} has ABI revision {_lib.ig4_abi_version()}, this binding expects "
+                      f"{IG4_ABI_VERSION}: rebuild it")
 _sig("ig4_mrope_positions", [_i, _i, _i, _i, _vp, _i, _vp])
 _sig("ig4_rope_table", [_i, _vp, ctypes.c_double, ctypes.POINTER(_i), _vp, _vp, _vp])
 _sig("ig4_adaln_modulation", [_i, _i, _i, _vp, _vp, _i, _vp, _vp, _vp, _vp])
