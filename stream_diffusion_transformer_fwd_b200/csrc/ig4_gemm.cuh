@@ -541,444 +541,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   if (warp == 5) tmem_dealloc(tmem_base, S::TMEM_COLS);
 }
 
-// ------------------------------------------------------ NVFP4 kernel
-// C = (A * SFA) (B * SFB)^T on block-scaled FP4 tensor-core MMAs
-// (tcgen05.mma kind::mxf4nvf4, block16): A [M][K] and B [N][K] are E2M1 codes,
-// two per byte (K contiguous), each row carrying one UE4M3 scale per 16
-// K-elements.  Tiles 128 x 128, 256 K-elements (128 bytes per row) per stage:
-// TMA brings the A and B code tiles (128-byte swizzle) and a 1D bulk copy
-// each 2 KB scale block of A and of B, stored in global memory already in the
-// order the tensor cores read them (per 128 rows and 64 K-elements, 512 bytes:
-// byte 16 * (r % 32) + 4 * (r / 32) + (k / 16) % 4).  The MMA thread copies a
-// stage's scales into TMEM (tcgen05.cp 32x128b.warpx4, a TMEM region per
-// stage) and issues four K = 64 MMAs.  The epilogue applies the per-row scale
-// of A and the per-column scale of B in fp32 (EpiStore with FP8 = true).
-// Two tile widths: 128 (two TMEM accumulators, six stages) and 256 (one
-// accumulator, four stages; B brings 2 scale blocks per K chunk): TMEM holds
-// the accumulators plus a 16 + 4 * (BN / 128)... scale region per stage.
-template <int BN>
-struct Nvf4Shape {
-  static constexpr int ACC = BN == 128 ? 2 : 1;               // accumulator buffers
-  static constexpr int STAGES = BN == 128 ? 6 : 4;
-  static constexpr int A_BYTES = GEMM_BM * 128;                // 16 KB of codes
-  static constexpr int B_BYTES = BN * 128;
-  static constexpr int SFA_BYTES = 2048;                       // 4 blocks of 512 B
-  static constexpr int SFB_BYTES = 2048 * (BN / 128);
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
-  static constexpr uint32_t SF_COLS = 16 + 16 * (BN / 128);   // TMEM scale columns per stage
-  static constexpr uint32_t TMEM_SF = ACC * BN;
-  static_assert(TMEM_SF + STAGES * SF_COLS <= 512, "TMEM");
-};
-constexpr int NVF4_BN = 128;
-constexpr uint32_t NVF4_TMEM_COLS = 512;
-
-template <int BN, class Epi>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
-    gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const uint8_t *__restrict__ sfa, const uint8_t *__restrict__ sfb, int M,
-                     int n_tiles_n, int K, int group_m, const Epi epi) {
-  using S = Nvf4Shape<BN>;
-  constexpr int NVF4_STAGES = S::STAGES;
-  constexpr uint32_t IDESC = idesc_nvf4(GEMM_BM, BN);
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = align1024(smem_raw);
-  uint8_t *sA = smem;
-  uint8_t *sB = sA + NVF4_STAGES * S::A_BYTES;
-  uint8_t *sSFA = sB + NVF4_STAGES * S::B_BYTES;
-  uint8_t *sSFB = sSFA + NVF4_STAGES * S::SFA_BYTES;
-  uint64_t *full = reinterpret_cast<uint64_t *>(sSFB + NVF4_STAGES * S::SFB_BYTES);
-  uint64_t *empty = full + NVF4_STAGES;
-  uint64_t *tfull = empty + NVF4_STAGES;
-  uint64_t *tempty = tfull + 2;
-  uint64_t *drain = tempty + 2;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int m_tiles = (M + GEMM_BM - 1) / GEMM_BM;
-  const int n_tiles = m_tiles * n_tiles_n;
-  const int kblocks = K / 256;
-  const long sf_row_block = static_cast<long>(K / 64) * 512;  // bytes per 128 rows
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < NVF4_STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 128);
-    }
-    mbar_init(drain, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 4 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
-  }
-  if (warp == 5) {
-    tmem_alloc(tmem_slot, NVF4_TMEM_COLS);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-  pdl_wait();
-  pdl_trigger();
-
-  if (warp == 4) {
-    if (lane == 0) {
-      // ---------------- loads: code tiles by TMA, scale blocks by bulk copy
-      int s = 0;
-      uint32_t ph = 0;
-      long issued = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-        int mt, nt;
-        tile_coords(t, m_tiles, n_tiles_n, group_m, &mt, &nt);
-        for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(&empty[s], ph ^ 1, abort_flag)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&full[s], S::STAGE_BYTES);
-          tma_load_2d(sA + s * S::A_BYTES, &tmA, &full[s], kb * 128, mt * GEMM_BM);
-          tma_load_2d(sB + s * S::B_BYTES, &tmB, &full[s], kb * 128, nt * BN);
-          bulk_load(sSFA + s * S::SFA_BYTES, sfa + mt * sf_row_block + kb * 2048, 2048, &full[s]);
-#pragma unroll
-          for (int q = 0; q < BN / 128; ++q)
-            bulk_load(sSFB + s * S::SFB_BYTES + 2048 * q,
-                      sfb + (nt * (BN / 128) + q) * sf_row_block + kb * 2048, 2048, &full[s]);
-          ++issued;
-          if (++s == NVF4_STAGES) {
-            s = 0;
-            ph ^= 1;
-          }
-        }
-      }
-      if (!ok) {
-        for (long i = (issued > NVF4_STAGES ? issued - NVF4_STAGES : 0); i < issued; ++i)
-          mbar_wait(&full[i % NVF4_STAGES], static_cast<uint32_t>((i / NVF4_STAGES) & 1), nullptr,
-                    WAIT_LIMIT_NS / 4);
-      }
-    }
-  } else if (warp == 5) {
-    if (lane == 0) {
-      // ---------------- MMA issuer
-      int s = 0;
-      uint32_t ph = 0;
-      int local = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++local) {
-        const int buf = local % S::ACC;
-        const uint32_t use = static_cast<uint32_t>(local / S::ACC);
-        if (!mbar_wait(&tempty[buf], (use & 1) ^ 1, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + buf * BN;
-        for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(&full[s], ph, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          // this stage's scales -> TMEM: A at sf + 4j, B at sf + 16 + (BN / 32) j
-          // (per K = 64 step, 4 columns per 128 rows of the operand)
-          constexpr uint32_t NB = BN / 128;
-          const uint32_t sf = tmem_base + S::TMEM_SF + S::SF_COLS * s;
-          const uint32_t sfa_s = smem_u32(sSFA + s * S::SFA_BYTES);
-          const uint32_t sfb_s = smem_u32(sSFB + s * S::SFB_BYTES);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            tmem_cp_sf(sf + 4 * j, sdesc_kmajor_none(sfa_s + 512 * j, 128));
-#pragma unroll
-            for (uint32_t q = 0; q < NB; ++q)
-              tmem_cp_sf(sf + 16 + 4 * NB * j + 4 * q, sdesc_kmajor_none(sfb_s + 2048 * q + 512 * j, 128));
-          }
-          const uint32_t a_base = smem_u32(sA + s * S::A_BYTES);
-          const uint32_t b_base = smem_u32(sB + s * S::B_BYTES);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {  // K = 64 E2M1 values = 32 bytes per MMA
-            const uint64_t ad = sdesc_kmajor_sw128(a_base + 32 * j);
-            const uint64_t bd = sdesc_kmajor_sw128(b_base + 32 * j);
-            umma_nvf4(d_tmem, ad, bd, IDESC, sf + 4 * j, sf + 16 + 4 * NB * j, (kb | j) != 0);
-          }
-          umma_commit(&empty[s]);
-          if (++s == NVF4_STAGES) {
-            s = 0;
-            ph ^= 1;
-          }
-        }
-        if (ok) umma_commit(&tfull[buf]);
-      }
-      umma_commit(drain);
-      mbar_wait(drain, 0, nullptr, WAIT_LIMIT_NS / 4);
-    }
-  } else {
-    // ---------------- epilogue warps 0..3
-    const int r = warp * 32 + lane;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    int local = 0;
-    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++local) {
-      const int buf = local % S::ACC;
-      const uint32_t use = static_cast<uint32_t>(local / S::ACC);
-      if (!mbar_wait_warp(&tfull[buf], use & 1, abort_flag)) break;
-      tc_fence_after();
-      int mt, nt;
-      tile_coords(t, m_tiles, n_tiles_n, group_m, &mt, &nt);
-      epi(mt * GEMM_BM, nt * BN, tmem_base + lane_base + buf * BN, r);
-      tc_fence_before();
-      mbar_arrive(&tempty[buf]);
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 5) tmem_dealloc(tmem_base, NVF4_TMEM_COLS);
-}
-
-// NVFP4 on CTA pairs: a pair tile is 256 rows x 256 columns (tcgen05.mma
-// cta_group::2, M = 256): each CTA loads its 128 A rows, half of the B rows,
-// its A scale blocks and the scale blocks of all 256 B rows (both CTAs' MMAs
-// read the B scales of every column); all loads complete on the leader's
-// barrier.  Per stage and CTA: 32 KB of codes + 6 KB of scales per 512 MMA
-// clocks at the FP4 rate, the same bytes per clock as the FP8 pair kernel.
-// TMEM: two 256-column accumulators that overlap in 64 columns, acc 0 at
-// [0, 256) and acc 1 at [192, 448), and one 48-column scale region at 448
-// (the scale blocks of k-block g are copied in after the MMAs of k-block
-// g - 1 were issued; tcgen05.cp and tcgen05.mma from one thread run in
-// issue order).  The epilogue of a tile drains the overlapped columns
-// first and releases them (ovl), so the next tile's MMAs start while it
-// converts the remaining 192 columns.
-// DUAL_B (SwiGLU gate/up): B rows of the tile's first 128 columns come from
-// tmB (gate) and of the last 128 from tmB2 (up), both at rows nt * 128, with
-// their scale blocks from tmSFB / tmSFB2 (one 128-row block each); otherwise
-// B rows nt * 256 + [0, 256) come from tmB and their two scale blocks from
-// tmSFB.
-constexpr int NVF4P_STAGES = 5;
-constexpr int NVF4P_A_BYTES = GEMM_BM * 128;
-constexpr int NVF4P_BH_BYTES = 128 * 128;
-constexpr int NVF4P_SFA_BYTES = 2048;
-constexpr int NVF4P_SFB_BYTES = 4096;
-constexpr int NVF4P_STAGE_BYTES = NVF4P_A_BYTES + NVF4P_BH_BYTES + NVF4P_SFA_BYTES + NVF4P_SFB_BYTES;
-constexpr int NVF4P_SMEM_BYTES = NVF4P_STAGES * NVF4P_STAGE_BYTES + 1024 + 256;
-constexpr uint32_t NVF4P_ACC1_COL = 192;
-constexpr uint32_t NVF4P_SF_COL = 448;
-static_assert(NVF4P_ACC1_COL + 256 <= NVF4P_SF_COL && NVF4P_SF_COL + 48 <= 512, "TMEM");
-
-template <bool DUAL_B, class Epi>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
-    gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                          const __grid_constant__ CUtensorMap tmB2,
-                          const __grid_constant__ CUtensorMap tmSFA,
-                          const __grid_constant__ CUtensorMap tmSFB,
-                          const __grid_constant__ CUtensorMap tmSFB2, int M, int n_tiles_n, int K,
-                          int group_m, const Epi epi) {
-  constexpr int BN = 256;
-  constexpr uint32_t IDESC = idesc_nvf4(2 * GEMM_BM, BN);
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = align1024(smem_raw);
-  uint8_t *sA = smem;
-  uint8_t *sB = sA + NVF4P_STAGES * NVF4P_A_BYTES;
-  uint8_t *sSFA = sB + NVF4P_STAGES * NVF4P_BH_BYTES;
-  uint8_t *sSFB = sSFA + NVF4P_STAGES * NVF4P_SFA_BYTES;
-  uint64_t *full = reinterpret_cast<uint64_t *>(sSFB + NVF4P_STAGES * NVF4P_SFB_BYTES);
-  uint64_t *empty = full + NVF4P_STAGES;
-  uint64_t *tfull = empty + NVF4P_STAGES;  // [2]: accumulator ready
-  uint64_t *tempty = tfull + 2;            // [2]: accumulator drained
-  uint64_t *ovl = tempty + 2;              // overlapped columns drained
-  uint64_t *drain = ovl + 1;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();
-  const int pair = blockIdx.x >> 1;
-  const int n_pairs = gridDim.x >> 1;
-  const int m_tiles = (M + 2 * GEMM_BM - 1) / (2 * GEMM_BM);
-  const int n_tiles = m_tiles * n_tiles_n;
-  const int kblocks = K / 256;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < NVF4P_STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 2 * 4);  // one arrival per epilogue warp of the pair
-    }
-    mbar_init(ovl, 2 * 4);
-    mbar_init(drain, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 4 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
-    tma_prefetch_desc(&tmSFA);
-    tma_prefetch_desc(&tmSFB);
-    if (DUAL_B) {
-      tma_prefetch_desc(&tmB2);
-      tma_prefetch_desc(&tmSFB2);
-    }
-  }
-  if (warp == 5) {
-    tmem_alloc_pair(tmem_slot, 512);
-    tmem_relinquish_pair();
-  }
-  tc_fence_before();
-  cluster_sync_all();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-  pdl_wait();
-  pdl_trigger();
-
-  if (warp == 4) {
-    if (lane == 0) {
-      // ---------------- loads (both CTAs), completing on the leader's barrier
-      int s = 0;
-      uint32_t ph = 0;
-      bool ok = true;
-      for (int t = pair; t < n_tiles && ok; t += n_pairs) {
-        int mt, nt;
-        tile_coords(t, m_tiles, n_tiles_n, group_m, &mt, &nt);
-        const int mrow = mt * 2 * GEMM_BM + static_cast<int>(rank) * GEMM_BM;
-        for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait_cluster(&empty[s], ph ^ 1, abort_flag)) {
-            ok = false;
-            break;
-          }
-          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * NVF4P_STAGE_BYTES);
-          const uint32_t bar = map_shared_to_rank(&full[s], 0);
-          tma_load_2d_pair(sA + s * NVF4P_A_BYTES, &tmA, bar, kb * 128, mrow);
-          // scale blocks: [128 words of 4 B] x [4 K chunks] x [row blocks]
-          tma_load_3d_pair(sSFA + s * NVF4P_SFA_BYTES, &tmSFA, bar, 0, 4 * kb, mrow / 128);
-          if constexpr (DUAL_B) {
-            tma_load_2d_pair(sB + s * NVF4P_BH_BYTES, rank ? &tmB2 : &tmB, bar, kb * 128, nt * 128);
-            tma_load_3d_pair(sSFB + s * NVF4P_SFB_BYTES, &tmSFB, bar, 0, 4 * kb, nt);
-            tma_load_3d_pair(sSFB + s * NVF4P_SFB_BYTES + NVF4P_SFB_BYTES / 2, &tmSFB2, bar, 0,
-                             4 * kb, nt);
-          } else {
-            tma_load_2d_pair(sB + s * NVF4P_BH_BYTES, &tmB, bar, kb * 128,
-                             nt * BN + static_cast<int>(rank) * (BN / 2));
-            tma_load_3d_pair(sSFB + s * NVF4P_SFB_BYTES, &tmSFB, bar, 0, 4 * kb, nt * 2);
-          }
-          if (++s == NVF4P_STAGES) {
-            s = 0;
-            ph ^= 1;
-          }
-        }
-      }
-      if (!ok) sleep_ns(50000);  // let the loads already issued land
-    }
-  } else if (warp == 5) {
-    if (lane == 0 && rank == 0) {
-      // ---------------- MMA issuer (leader CTA)
-      int s = 0;
-      uint32_t ph = 0;
-      bool ok = true;
-      const uint32_t sf = tmem_base + NVF4P_SF_COL;
-      for (int t = pair, i = 0; t < n_tiles && ok; t += n_pairs, ++i) {
-        const int acc = i & 1;
-        // this accumulator's own columns: drained by the epilogue of tile i - 2;
-        // the overlapped ones: by the epilogue of tile i - 1
-        if (!mbar_wait_cluster(&tempty[acc], static_cast<uint32_t>((i >> 1) & 1) ^ 1, abort_flag))
-          break;
-        if (i > 0 && !mbar_wait_cluster(ovl, static_cast<uint32_t>((i - 1) & 1), abort_flag)) break;
-        tc_fence_after();
-        const uint32_t d = tmem_base + (acc ? NVF4P_ACC1_COL : 0);
-        for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait_cluster(&full[s], ph, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t sfa_s = smem_u32(sSFA + s * NVF4P_SFA_BYTES);
-          const uint32_t sfb_s = smem_u32(sSFB + s * NVF4P_SFB_BYTES);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            tmem_cp_sf_pair(sf + 4 * j, sdesc_kmajor_none(sfa_s + 512 * j, 128));
-            tmem_cp_sf_pair(sf + 16 + 8 * j, sdesc_kmajor_none(sfb_s + 512 * j, 128));
-            tmem_cp_sf_pair(sf + 16 + 8 * j + 4, sdesc_kmajor_none(sfb_s + 2048 + 512 * j, 128));
-          }
-          const uint32_t a_base = smem_u32(sA + s * NVF4P_A_BYTES);
-          const uint32_t b_base = smem_u32(sB + s * NVF4P_BH_BYTES);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint64_t ad = sdesc_kmajor_sw128(a_base + 32 * j);
-            const uint64_t bd = sdesc_kmajor_sw128(b_base + 32 * j);
-            umma_nvf4_pair(d, ad, bd, IDESC, sf + 4 * j, sf + 16 + 8 * j, (kb | j) != 0);
-          }
-          umma_commit_pair_both(&empty[s]);
-          if (++s == NVF4P_STAGES) {
-            s = 0;
-            ph ^= 1;
-          }
-        }
-        if (ok) umma_commit_pair_both(&tfull[acc]);
-      }
-      umma_commit_pair_both(drain);
-      mbar_wait_cluster(drain, 0, nullptr, WAIT_LIMIT_NS / 4);
-    }
-  } else {
-    // ---------------- epilogue warps 0..3 (both CTAs, own 128 rows)
-    const int r = warp * 32 + lane;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t ovl_leader = map_shared_to_rank(ovl, 0);
-    constexpr int C = Epi::COLS;  // 64 accumulator columns overlap: the top 64 of
-    constexpr int OV = C - 64;    // acc 0's epilogue columns, the bottom 64 of acc 1's
-    for (int t = pair, i = 0; t < n_tiles; t += n_pairs, ++i) {
-      const int acc = i & 1;
-      const bool ok =
-          mbar_wait_cluster(&tfull[acc], static_cast<uint32_t>((i >> 1) & 1), abort_flag);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      tc_fence_after();
-      int mt, nt;
-      tile_coords(t, m_tiles, n_tiles_n, group_m, &mt, &nt);
-      const int m0 = mt * 2 * GEMM_BM + static_cast<int>(rank) * GEMM_BM;
-      const uint32_t tacc = tmem_base + (acc ? NVF4P_ACC1_COL : 0) + lane_base;
-      epi.part(m0, nt * BN, tacc, r, acc ? 0 : OV, acc ? 64 : C);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(ovl_leader);
-      epi.part(m0, nt * BN, tacc, r, acc ? 64 : 0, acc ? C : OV);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(map_shared_to_rank(&tempty[acc], 0));
-    }
-  }
-
-  __syncwarp();
-  tc_fence_before();
-  cluster_sync_all();
-  tc_fence_after();
-  if (warp == 5) tmem_dealloc_pair(tmem_base, 512);
-}
-
-// Scale factors [rows][K/16] (row-major UE4M3 bytes) -> the tensor cores'
-// block order (see gemm_nvf4_kernel); rows padded to a multiple of 128 with
-// zero scales.  One thread per output byte.
-__global__ void nvf4_pack_scales_kernel(const uint8_t *__restrict__ src, uint8_t *__restrict__ dst,
-                                        int rows, int K, long total) {
-  const int kc = K / 64;  // 64-element chunks per row
-  for (long o = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; o < total;
-       o += static_cast<long>(gridDim.x) * blockDim.x) {
-    const long blk = o / 512;
-    const int w = static_cast<int>(o - blk * 512);
-    const long rb = blk / kc;           // 128-row block
-    const int c = static_cast<int>(blk - rb * kc);
-    const int r = static_cast<int>(rb * 128 + (w >> 4) + 32 * ((w >> 2) & 3));
-    const int k16 = c * 4 + (w & 3);
-    dst[o] = r < rows ? src[static_cast<long>(r) * (K / 16) + k16] : 0;
-  }
-}
-
 // ------------------------------------------------------ CTA-pair kernel
 // The same GEMM on a 2-CTA cluster: a pair tile is 256 rows x BN columns
 // (BN = 256, or 192 where 256-wide tiles leave the last wave of pairs mostly
