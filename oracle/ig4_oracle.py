@@ -371,7 +371,8 @@ def block_forward_rows(x, temb, pos, W, H, rows, theta=ROPE_THETA, sections=MROP
 # ---------------------------------------------------------------------------
 
 def stack_forward(x_latent, text, temb, pos, block_weights, n_blocks, w_in, b_in, w_f, b_f,
-                  w_out, b_out, H, theta=ROPE_THETA, sections=MROPE_SECTION, eps=EPS):
+                  w_out, b_out, H, theta=ROPE_THETA, sections=MROPE_SECTION, eps=EPS,
+                  ffn_nvfp4=False, stream_bf16=False):
     """34-block DiT forward of one denoiser step, float64.
 
     Survey page: the DiT is 34 single-stream layers over [text | image]; image
@@ -384,7 +385,11 @@ def stack_forward(x_latent, text, temb, pos, block_weights, n_blocks, w_in, b_in
 
     x_latent: [B, N, C]; text: [B, T, D]; block_weights: callable i -> dict as
     for block_forward (weights are built one block at a time, so they need not
-    all be held at once).  Returns [B, N, C].
+    all be held at once).  ffn_nvfp4: every block's FFN takes NVFP4
+    activations (see block_forward).  stream_bf16: the sequence [text | image]
+    is rounded to bf16 where it is stored, after the in-projection and after
+    every block (the storage precision of a bf16 residual stream; NVFP4's
+    rounding decisions in the next block depend on it).  Returns [B, N, C].
     """
     x_latent = np.asarray(x_latent, dtype=np.float64)
     text = np.asarray(text, dtype=np.float64)
@@ -392,8 +397,11 @@ def stack_forward(x_latent, text, temb, pos, block_weights, n_blocks, w_in, b_in
     T = text.shape[1]
     img = x_latent @ np.asarray(w_in, dtype=np.float64).T + np.asarray(b_in, dtype=np.float64)
     s = np.concatenate([text, img], axis=1)
+    store = bf16_round if stream_bf16 else (lambda a: a)
+    s = store(s)
     for i in range(n_blocks):
-        s = block_forward(s, temb, pos, block_weights(i), H, theta, sections, eps)
+        s = store(block_forward(s, temb, pos, block_weights(i), H, theta, sections, eps,
+                                ffn_nvfp4=ffn_nvfp4))
     shift_f, scale_f = adaln_modulation(temb, w_f, b_f, 2)
     s_f = modulate(s, shift_f, scale_f, eps)
     return s_f[:, T:, :] @ np.asarray(w_out, dtype=np.float64).T + np.asarray(b_out, dtype=np.float64)

@@ -148,15 +148,16 @@ def make_stack_inputs(cfg: Config, seed: int = 0, stress: bool = False) -> dict:
     make_block_weights(cfg, seed, block=i)."""
     D, A, C = cfg.D, cfg.adaln_dim, cfg.latent_ch
     xd = torch.bfloat16 if cfg.x_dtype == "bf16" else torch.float32
+    wd = "e4m3" if cfg.w_dtype == "nvfp4_mixed" else cfg.w_dtype  # only the FFN is NVFP4
     out = {}
     out["x_latent"] = torch.from_numpy(_normal(seed, 0, "x_latent", (cfg.B, cfg.n_img, C))).to(xd)
     out["text"] = torch.from_numpy(_normal(seed, 0, "text", (cfg.B, cfg.T_text, D))).to(xd)
     out["temb"] = torch.from_numpy(_normal(seed, 0, "temb", (cfg.B, A)))
-    out["w_in"], out["s_in"] = _linear(seed, 0, "w_in", D, C, cfg.w_dtype)
+    out["w_in"], out["s_in"] = _linear(seed, 0, "w_in", D, C, wd)
     out["b_in"] = _bias(seed, 0, "b_in", D, stress)
-    out["w_f"], out["s_f"] = _linear(seed, 0, "w_f", 2 * D, A, cfg.w_dtype, std=0.02)
+    out["w_f"], out["s_f"] = _linear(seed, 0, "w_f", 2 * D, A, wd, std=0.02)
     out["b_f"] = _bias(seed, 0, "b_f", 2 * D, stress)
-    out["w_out"], out["s_out"] = _linear(seed, 0, "w_out", C, D, cfg.w_dtype)
+    out["w_out"], out["s_out"] = _linear(seed, 0, "w_out", C, D, wd)
     out["b_out"] = _bias(seed, 0, "b_out", C, stress)
     return out
 

@@ -229,3 +229,36 @@ def test_invalid_arguments_launch_nothing(ig4):
                               torch.empty(ig4.ig4_workspace_size(c), dtype=torch.uint8,
                                           device="cuda"))
     assert e.value.status == ig4.IG4_ERR_INVALID_ARG
+
+
+def test_stack_small_nvfp4_mixed(ig4):
+    """The stack with NVFP4 Mixed weights (3 blocks, B = 2, 160 tokens).  Every
+    block's attention gate is zero and the oracle stores the stream in bf16
+    as the GPU does, so each block's FFN sees the same h2 on both sides and
+    the NVFP4 decisions agree (see the NVFP4 block tests); the stack then
+    checks the assembly, the ping-pong launches and the head."""
+    cfg = CONFIGS["tiny"].with_(name="stack_nvfp4", B=2, T_text=16, grid_h=8, grid_w=8, D=512,
+                                H=2, I=256, x_dtype="bf16", w_dtype="nvfp4_mixed", n_blocks=3)
+    D = cfg.D
+    st = make_stack_inputs(cfg, seed=6, stress=True)
+    wts = []
+    for i in range(3):
+        w = make_block_weights(cfg, seed=6, block=i, stress=True)
+        w["w_ada"].view(torch.uint8)[2 * D:3 * D] = 0
+        w["b_ada"][2 * D:3 * D] = 0.0
+        wts.append(w)
+    got = _stack_gpu(ig4, cfg, st, [ig4.nvfp4_pack_block_scales(to_dev(w)) for w in wts])
+    pos = O.mrope_positions(cfg.T_text, cfg.grid_t, cfg.grid_h, cfg.grid_w)
+    Ws = [block_weights_f64(w) for w in wts]
+    # the library runs the stack's in- and out-projections in bf16 with their
+    # E4M3 weights decoded to bf16; the in-projection's output then feeds the
+    # first block's NVFP4 decisions, so the oracle takes the same bf16 weights
+    ref = O.stack_forward(to_f64(st["x_latent"]), to_f64(st["text"]), to_f64(st["temb"]), pos,
+                          lambda i: Ws[i], 3, O.bf16_round(weight_f64(st["w_in"], st["s_in"])),
+                          to_f64(st["b_in"]), weight_f64(st["w_f"], st["s_f"]),
+                          to_f64(st["b_f"]), O.bf16_round(weight_f64(st["w_out"], st["s_out"])),
+                          to_f64(st["b_out"]), cfg.H, cfg.rope_theta, cfg.sections, cfg.eps,
+                          ffn_nvfp4=True, stream_bf16=True)
+    e = rel_l2(got, ref)
+    print(f"stack nvfp4-mixed, zero attention gates: relL2={e:.3e}")
+    assert e <= 2e-2

@@ -149,3 +149,36 @@ def test_nvfp4_ffn_block_within_quantisation_error():
     rows = np.array([0, 5, 17, 23])
     y_rows = O.block_forward_rows(x, temb, pos, W, H, rows, ffn_nvfp4=True)
     assert np.allclose(y_rows, y_q.reshape(-1, D)[rows], rtol=0, atol=1e-10)
+
+
+def test_nvfp4_stack_is_the_blocks_composed():
+    x, temb, pos, W, H = _tiny_block()
+    B, L, D = x.shape
+    T = 8
+    rng = np.random.default_rng(4)
+    C = 16
+    lat = rng.standard_normal((B, L - T, C))
+    text = x[:, :T]
+    w_in, b_in = rng.standard_normal((D, C)) / 4, rng.standard_normal(D) * 0.1
+    w_f, b_f = rng.standard_normal((2 * D, temb.shape[1])) * 0.02, np.zeros(2 * D)
+    w_out, b_out = rng.standard_normal((C, D)) / 16, np.zeros(C)
+    got = O.stack_forward(lat, text, temb, pos, lambda i: W, 2, w_in, b_in, w_f, b_f, w_out,
+                          b_out, H, ffn_nvfp4=True)
+    s = np.concatenate([text, lat @ w_in.T + b_in], axis=1)
+    for _ in range(2):
+        s = O.block_forward(s, temb, pos, W, H, ffn_nvfp4=True)
+    sh, sc = O.adaln_modulation(temb, w_f, b_f, 2)
+    ref = O.modulate(s, sh, sc)[:, T:] @ w_out.T + b_out
+    assert np.array_equal(got, ref)
+    plain = O.stack_forward(lat, text, temb, pos, lambda i: W, 2, w_in, b_in, w_f, b_f, w_out,
+                            b_out, H)
+    assert not np.array_equal(got, plain)
+    # a bf16-stored stream: rounded after the in-projection and after each block
+    got16 = O.stack_forward(lat, text, temb, pos, lambda i: W, 2, w_in, b_in, w_f, b_f, w_out,
+                            b_out, H, ffn_nvfp4=True, stream_bf16=True)
+    s = O.bf16_round(np.concatenate([text, lat @ w_in.T + b_in], axis=1))
+    for _ in range(2):
+        s = O.bf16_round(O.block_forward(s, temb, pos, W, H, ffn_nvfp4=True))
+    ref16 = O.modulate(s, sh, sc)[:, T:] @ w_out.T + b_out
+    assert np.array_equal(got16, ref16)
+    assert 0 < np.linalg.norm(got16 - got) / np.linalg.norm(got) < 0.2
