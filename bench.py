@@ -50,6 +50,11 @@ KERNEL_SOURCES = {
     "down_residual": ["ig4_gemm.cuh", "ig4_ptx.cuh"],
 }
 SMALL_KERNEL_SOURCES = ["ig4_small.cuh", "ig4_ptx.cuh"]
+# NVFP4 workloads: their FFN GEMMs are the NVFP4 kernels
+NVFP4_KERNEL_SOURCES = {
+    "gate_up_swiglu": ["ig4_gemm.cuh", "ig4_ptx.cuh", "ig4_nvf4.cuh"],
+    "down_residual": ["ig4_gemm.cuh", "ig4_ptx.cuh", "ig4_nvf4.cuh"],
+}
 
 
 def parse():
@@ -114,9 +119,10 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash(kernel):
+def kernel_source_hash(kernel, workload=""):
     h = hashlib.sha256()
-    for name in KERNEL_SOURCES.get(kernel, SMALL_KERNEL_SOURCES):
+    srcs = NVFP4_KERNEL_SOURCES if "nvfp4" in workload else {}
+    for name in srcs.get(kernel, KERNEL_SOURCES.get(kernel, SMALL_KERNEL_SOURCES)):
         with open(os.path.join(ROOT, "stream_diffusion_transformer_fwd_b200", "csrc", name),
                   "rb") as f:
             h.update(f.read())
@@ -132,7 +138,7 @@ def recorded_traffic(kernel, workload):
     with open(path) as f:
         rec = json.load(f)
     ent = rec.get(workload, {}).get(kernel)
-    if not ent or ent.get("source_hash") != kernel_source_hash(kernel):
+    if not ent or ent.get("source_hash") != kernel_source_hash(kernel, workload):
         return None
     return ent.get("dram_bytes_per_launch")
 
@@ -788,7 +794,7 @@ def run_ffn_nvfp4(args, cfg, ig4, rank, world, dev):
                    "l2": "inputs larger than L2", "gflop_per_step": round(flops / 1e9, 1)},
         "roofline": {"bound": "tensor", "achieved": round(ach, 1), "peak": round(peak, 1),
                      "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": None,
-                     "kernel": "gemm_nvf4_kernel (gate/up)",
+                     "kernel": "gemm_nvf4_pair_kernel (gate/up)",
                      "peak_source": f"4 x {tkey} ({peak_src}): nominal fp4/bf16 dense ratio"},
         "kernel_ms": {"gate_up": round(ms_gu, 4), "down": round(ms_dn, 4)},
         "kernel_tflops": {"gate_up": round(ach, 1), "down": round(f_dn / (ms_dn * 1e-3) / 1e12, 1)},
