@@ -111,6 +111,25 @@ def kernel_bytes(cfg, name):
     return None
 
 
+def max_over_ranks(values, device):
+    """Each value's maximum over all ranks (for times: the slowest rank's),
+    through one all-reduce; the values themselves when there is one rank."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return list(values)
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_rate(units_per_rank, world, steps, ms_total, scale=1e12):
+    """Whole-job throughput: the units all ranks processed over `steps` steps
+    divided by the slowest rank's time (ms), in units of `scale` per second."""
+    return world * units_per_rank * steps / (ms_total * 1e-3) / scale
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -363,15 +382,12 @@ def run_ours(args, rank, local_rank, world):
         dist.barrier()
     ms_e2e, h2d, d2h = e2e_pipelined(host_in, y, step_fn, K, max(1, W // 2))
 
-    if world > 1:
-        t = torch.tensor([ms_total, ms_e2e], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total, ms_e2e = t.tolist()
+    ms_total, ms_e2e = max_over_ranks([ms_total, ms_e2e], dev)
 
     flops, per_kernel_flops = block_work(cfg)
     ms_step = ms_total / K
-    value = world * flops * K / (ms_total * 1e-3) / 1e12
-    e2e_value = world * flops * K / (ms_e2e * 1e-3) / 1e12
+    value = job_rate(flops, world, K, ms_total)
+    e2e_value = job_rate(flops, world, K, ms_e2e)
 
     # dominant kernel and its roofline.  The peak is the measured cuBLAS burst
     # figure when the SM clock held its maximum during the timed region, the
@@ -522,16 +538,14 @@ def run_stack(args, cfg, ig4, rank, world, dev):
     if world > 1:
         dist.barrier()
     ms_e2e, h2d, d2h = e2e_pipelined(host_in, out, step_fn, K, 1)
+    ms_total, ms_e2e = max_over_ranks([ms_total, ms_e2e], dev)
     if world > 1:
-        t = torch.tensor([ms_total, ms_e2e], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total, ms_e2e = t.tolist()
         dist.destroy_process_group()
     if rank != 0:
         return 0
     flops = stack_work(cfg)
     blk, per = block_work(cfg)
-    value = world * flops * K / (ms_total * 1e-3) / 1e12
+    value = job_rate(flops, world, K, ms_total)
     peaks, peak_src = load_peaks()
     held_max = bool(clocks) and clocks["sm_mhz"] >= 0.95 * clocks["sm_max_mhz"]
     tkey = "bf16_tflops" if held_max else "bf16_tflops_sustained"
@@ -559,7 +573,7 @@ def run_stack(args, cfg, ig4, rank, world, dev):
                      "kernel": "whole step (GEMMs at 2x and attention at 1x the " + tkey + ")",
                      "peak_source": f"{tkey} ({peak_src}) x nominal fp8/bf16 ratio for the GEMMs"},
         "clocks": clocks, "device_error": ig4.ig4_status_string(err),
-        "e2e": {"value": round(world * flops * K / (ms_e2e * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+        "e2e": {"value": round(job_rate(flops, world, K, ms_e2e), 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(ms_e2e / K, 3)},
         # per block 11 (FP8) or 9 launches, the rotary table only in the first block
@@ -643,10 +657,8 @@ def run_step(args, cfg, ig4, rank, world, dev):
     if world > 1:
         dist.barrier()
     ms_e2e, h2d, d2h = e2e_pipelined(host_in, z, step_fn, K, 1)
+    ms_total, ms_e2e = max_over_ranks([ms_total, ms_e2e], dev)
     if world > 1:
-        tt = torch.tensor([ms_total, ms_e2e], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_total, ms_e2e = tt.tolist()
         dist.destroy_process_group()
     if rank != 0:
         return 0
@@ -662,7 +674,7 @@ def run_step(args, cfg, ig4, rank, world, dev):
         attn_f += cc.n_blocks * per["attention"]
     t_min = gemm_f / ((2.0 if fp8 else 1.0) * bf16_peak * 1e12) + attn_f / (bf16_peak * 1e12)
     mixed_peak = flops / t_min / 1e12
-    value = world * flops * K / (ms_total * 1e-3) / 1e12
+    value = job_rate(flops, world, K, ms_total)
     per_stack = cfg.n_blocks * (10 if fp8 else 8) + 1
     launches = 2 * per_stack + (7 if fp8 else 5) + (6 if fp8 else 4) + 2
     line = {
@@ -685,7 +697,7 @@ def run_step(args, cfg, ig4, rank, world, dev):
                      "kernel": "whole step (GEMMs at 2x and attention at 1x the " + tkey + ")",
                      "peak_source": f"{tkey} ({peak_src}) x nominal fp8/bf16 ratio for the GEMMs"},
         "clocks": clocks, "device_error": ig4.ig4_status_string(err),
-        "e2e": {"value": round(world * flops * K / (ms_e2e * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+        "e2e": {"value": round(job_rate(flops, world, K, ms_e2e), 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(ms_e2e / K, 3)},
         "gpu_launches": K * launches,
@@ -767,17 +779,15 @@ def run_ffn_nvfp4(args, cfg, ig4, rank, world, dev):
         ig4.ig4_nvfp4_linear(din[1], A2[1], A2[2], W2[0], W2[1], W2[2], None, o)
 
     ms_e2e, h2d, d2h = e2e_pipelined(host_in, o2, step_fn, K, 1)
+    ms_total, ms_e2e = max_over_ranks([ms_total, ms_e2e], dev)
     if world > 1:
-        tt = torch.tensor([ms_total, ms_e2e], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_total, ms_e2e = tt.tolist()
         dist.destroy_process_group()
     if rank != 0:
         return 0
     f_gu = 2.0 * M * D * 2 * I
     f_dn = 2.0 * M * I * D
     flops = f_gu + f_dn
-    value = world * flops * K / (ms_total * 1e-3) / 1e12
+    value = job_rate(flops, world, K, ms_total)
     peaks, peak_src = load_peaks()
     held_max = bool(clocks) and clocks["sm_mhz"] >= 0.95 * clocks["sm_max_mhz"]
     tkey = "bf16_tflops" if held_max else "bf16_tflops_sustained"
@@ -799,7 +809,7 @@ def run_ffn_nvfp4(args, cfg, ig4, rank, world, dev):
         "kernel_ms": {"gate_up": round(ms_gu, 4), "down": round(ms_dn, 4)},
         "kernel_tflops": {"gate_up": round(ach, 1), "down": round(f_dn / (ms_dn * 1e-3) / 1e12, 1)},
         "clocks": clocks, "device_error": ig4.ig4_status_string(err),
-        "e2e": {"value": round(world * flops * K / (ms_e2e * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+        "e2e": {"value": round(job_rate(flops, world, K, ms_e2e), 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(ms_e2e / K, 4)},
         "gpu_launches": 2 * K,
@@ -851,16 +861,14 @@ def run_textcond(args, cfg, ig4, rank, world, dev):
     err = ig4.ig4_last_device_error()
     ms_total = start.elapsed_time(end)
     ms_e2e, h2d, d2h = e2e_pipelined([inp["raw"]], out, lambda din, o: call(din[0], o), K, 1)
+    ms_total, ms_e2e = max_over_ranks([ms_total, ms_e2e], dev)
     if world > 1:
-        tt = torch.tensor([ms_total, ms_e2e], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_total, ms_e2e = tt.tolist()
         dist.destroy_process_group()
     if rank != 0:
         return 0
     fp8 = cfg.w_dtype == "e4m3"
     flops = 2.0 * M * K_raw * D
-    value = world * flops * K / (ms_total * 1e-3) / 1e12
+    value = job_rate(flops, world, K, ms_total)
     peaks, peak_src = load_peaks()
     held_max = bool(clocks) and clocks["sm_mhz"] >= 0.95 * clocks["sm_max_mhz"]
     tkey = "bf16_tflops" if held_max else "bf16_tflops_sustained"
@@ -881,7 +889,7 @@ def run_textcond(args, cfg, ig4, rank, world, dev):
                      "kernel": "norm + projection GEMM (GEMM flops only)",
                      "peak_source": f"{'2 x ' if fp8 else ''}{tkey} ({peak_src})"},
         "clocks": clocks, "device_error": ig4.ig4_status_string(err),
-        "e2e": {"value": round(world * flops * K / (ms_e2e * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+        "e2e": {"value": round(job_rate(flops, world, K, ms_e2e), 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(ms_e2e / K, 4)},
         "gpu_launches": 2 * K,
