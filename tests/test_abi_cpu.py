@@ -175,3 +175,24 @@ def test_nvfp4_mixed_config_rules(ig4):
     assert ws(16, 8, 2816, "e4m3") > 0
     assert ws(64, 12, 2944, "nvfp4_mixed") == 0     # I = 23 x 128
     assert ws(64, 12, 2944, "e4m3") > 0
+
+
+def test_nvfp4_validation_returns_before_launch(ig4):
+    lib = ig4.library()
+    p = ctypes.c_void_p(1 << 40)
+    q = ctypes.c_void_p((1 << 40) + 8)  # not 16-byte aligned
+    assert lib.ig4_nvfp4_quantize(4, 96, p, p, p, p, None) == ig4.IG4_ERR_INVALID_ARG  # K % 64
+    assert lib.ig4_nvfp4_quantize(4, 128, q, p, p, p, None) == ig4.IG4_ERR_INVALID_ARG
+    assert lib.ig4_nvfp4_quantize(0, 128, p, p, p, p, None) == ig4.IG4_ERR_INVALID_ARG
+    assert lib.ig4_nvfp4_linear(8, 100, 256, p, p, p, p, p, p, None, p, 0, None) == \
+        ig4.IG4_ERR_INVALID_ARG  # N % 128
+    assert lib.ig4_nvfp4_linear(8, 128, 200, p, p, p, p, p, p, None, p, 0, None) == \
+        ig4.IG4_ERR_INVALID_ARG  # K % 256
+    assert ig4.ig4_nvfp4_scale_bytes(100, 100) == 0
+    assert ig4.ig4_nvfp4_scale_bytes(129, 128) == 2 * 2 * 512
+    # an NVFP4 Mixed block needs the FFN weights' packed scales
+    cfg = ig4.make_config(1, 64, 1, 12, 12, D=1024, H=4, I=2816, w_dtype="nvfp4_mixed")
+    need = ig4.ig4_workspace_size(cfg)
+    w = {name: _Fake((1 << 40) + i * (1 << 20)) for i, (name, _) in
+         enumerate(ig4.BlockWeights._fields_) if name != "sf_up"}
+    assert _call_block(ig4, cfg, ig4.block_weights(w), need) == ig4.IG4_ERR_INVALID_ARG
