@@ -101,7 +101,8 @@ typedef struct ig4_block_weights {
 /* Stack weights: a host array of n_blocks block weight structs, the latent
  * in-projection w_in [D, C] + b_in [D], the final AdaLN w_f [2D, adaln_dim] +
  * b_f [2D] (chunks shift, scale), the out-projection w_out [C, D] + b_out [C].
- * Weights in cfg->w_dtype, s_* scales for E4M3.  C = latent_ch (128). */
+ * Weights in cfg->w_dtype, s_* scales for E4M3 (for IG4_NVFP4_MIXED these three
+ * linears are E4M3 and only the blocks' FFNs NVFP4).  C = latent_ch (128). */
 typedef struct ig4_stack_weights {
   int n_blocks;
   int latent_ch;
