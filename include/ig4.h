@@ -118,7 +118,7 @@ const char *ig4_status_string(int status);
 /* ABI revision of this header (increases on any incompatible change). */
 int ig4_abi_version(void);
 
-/* ---------------------------------------------------------------- a-11 ---
+/* ------------------------------------------------------------ positions ---
  * MRoPE position table (survey page, "单 block 内部": text tokens use a 1D
  * position broadcast to the 3 axes, image tokens use (t, h, w); "条件注入方式":
  * text precedes the image).  Writes int32 pos[3][L] (rows t, h, w), with
@@ -130,7 +130,7 @@ int ig4_abi_version(void);
 ig4_status ig4_mrope_positions(int T_text, int grid_t, int grid_h, int grid_w,
                                int32_t *pos_out, int out_on_device, void *stream);
 
-/* ----------------------------------------------------------------- a-5 ---
+/* --------------------------------------------------------- rotary table ---
  * Rotary tables for a position table: cos_out[l][j] = cos(pos[axis(j)][l] *
  * theta^(-2j/128)), sin_out likewise, fp32 [L][64], angles evaluated in fp64.
  * axis(j) follows `sections` (contiguous chunks t, h, w).  pos: device int32
@@ -139,7 +139,7 @@ ig4_status ig4_mrope_positions(int T_text, int grid_t, int grid_h, int grid_w,
 ig4_status ig4_rope_table(int L, const int32_t *pos, double rope_theta, const int sections[3],
                           float *cos_out, float *sin_out, void *stream);
 
-/* ----------------------------------------------------------------- a-1 ---
+/* ----------------------------------------------------- AdaLN modulation ---
  * AdaLN modulation (survey page, "单 block 内部": AdaLN from the timestep
  * embedding gives the per-block modulation): mod[b][n] = sum_k SiLU(temb[b][k])
  * * W[n][k] (* w_scale[n] for E4M3) + bias[n], fp32 out [B][N].  temb fp32
@@ -149,7 +149,7 @@ ig4_status ig4_adaln_modulation(int B, int A, int N, const float *temb, const vo
                                 int w_dtype, const float *w_scale, const float *bias,
                                 float *mod_out, void *stream);
 
-/* ----------------------------------------------------------------- a-2 ---
+/* ------------------------------------------------------ norm + modulate ---
  * Pre-norm + modulate: h[r] = x[r] * rsqrt(mean(x[r]^2) + eps) * (1 + scale[b])
  * + shift[b] for each token row r of sample b = r / L.  x [B*L][D] in x_dtype
  * (F32 or BF16); shift / scale fp32 with sample stride mod_stride (pointers into
@@ -160,7 +160,7 @@ ig4_status ig4_norm_modulate(int B, int L, int D, const void *x, int x_dtype,
                              const float *shift, const float *scale, int mod_stride, float eps,
                              void *h_out, int h_dtype, float *h_scale_out, void *stream);
 
-/* ------------------------------------------------------- a-3, a-4, a-5 ---
+/* ------------------------------------------------ QKV + QK-norm + MRoPE ---
  * Fused QKV projection with per-head QK-RMSNorm and MRoPE (survey page,
  * "单 block 内部": self-attention with QK-RMSNorm and 3D MRoPE).
  * qkv = h W_qkv^T; q and k are RMS-normalised per (token, head) with g_q / g_k
@@ -175,7 +175,7 @@ ig4_status ig4_qkv_project(int B, int L, int D, int H, const void *h, int h_dtyp
                            const float *rope_cos, const float *rope_sin, void *q_out,
                            void *k_out, void *vt_out, int vt_ld, void *stream);
 
-/* ----------------------------------------------------------------- a-6 ---
+/* ------------------------------------------------------ joint attention ---
  * Joint bidirectional attention over [text | image] (survey page: one
  * self-attention over the single sequence, no separate branches):
  * o[b, l, h*256 + d] = sum_m softmax_m(q[b,h,l] . k[b,h,m] / 16) v[b,h,m,d].
@@ -184,7 +184,7 @@ ig4_status ig4_qkv_project(int B, int L, int D, int H, const void *h, int h_dtyp
 ig4_status ig4_joint_attention(int B, int H, int L, const void *q, const void *k,
                                const void *vt, int vt_ld, void *o_out, void *stream);
 
-/* ----------------------------------------------------------- a-7, a-9 ---
+/* ------------------------------------------------ gated residual linear ---
  * Gated residual linear (survey page, "单 block 内部": AdaLN gates modulate
  * the attention and MLP residual paths): x_out[r][n] = x_res[r][n] +
  * gate[b*gate_stride + n] * sum_k a[r][k] W[n][k] (scaled by a_scale[r] *
@@ -196,7 +196,7 @@ ig4_status ig4_gated_residual_linear(int B, int L, int N, int K, const void *a, 
                                      const float *w_scale, const float *gate, int gate_stride,
                                      const void *x_res, void *x_out, int x_dtype, void *stream);
 
-/* ----------------------------------------------------------------- a-8 ---
+/* --------------------------------------------------------------- SwiGLU ---
  * SwiGLU hidden state (survey page, "单 block 内部": SwiGLU MLP with a SiLU
  * gate): u[r][i] = silu(sum_k h[r][k] Wg[i][k]) * sum_k h[r][k] Wu[i][k]
  * (E4M3: each sum times h_scale[r] * s_gate[i] or s_up[i]).  h [M][K];
@@ -206,7 +206,7 @@ ig4_status ig4_swiglu(int M, int I, int K, const void *h, int h_dtype, const flo
                       const void *w_gate, const void *w_up, int w_dtype, const float *s_gate,
                       const float *s_up, void *u_out, void *stream);
 
-/* ---------------------------------------------------------------- a-10 ---
+/* ------------------------------------------------------ FP8 activations ---
  * Row quantisation of an activation to FP8 E4M3 for the FP8-weight path:
  * scale[r] = max_k |x[r][k]| / 448 (1 if the row is zero), q[r][k] =
  * RNE(x[r][k] / scale[r]) saturated to +-448.  x bf16 [M][K]; q_out E4M3
@@ -254,23 +254,26 @@ ig4_status ig4_block_forward_traced(const ig4_config *cfg, const ig4_block_weigh
  * static device variable: every GPU that loads the library holds those bytes
  * until the process exits.  It allocates nothing and calls no allocating
  * routine.  The caller still passes inputs and outputs as for
- * ig4_block_forward (same layouts and errors).  Configurations whose
- * ig4_workspace_size exceeds the scratch size return IG4_ERR_WORKSPACE
- * without launching anything (e.g. the full-width block up to ~900 tokens,
- * or the 1024-wide block up to ~4000 tokens, fit).
+ * ig4_block_forward (same layouts and errors).  A configuration fits when
+ * ig4_workspace_size(cfg) <= IG4_NOALLOC_SCRATCH_BYTES; larger ones return
+ * IG4_ERR_WORKSPACE before anything is launched.  At B = 1 that is up to 941
+ * tokens of the full-width block (D 4608, I 12288) with bf16 weights, 802
+ * with E4M3 weights and 751 with NVFP4 Mixed weights; 4094, 3491 and 3275
+ * tokens at D 1024, I 2816.
  * The first call on a device looks up the scratch array's device address
- * (a one-time set-up per device, done with that device current); make that
- * first call before any stream capture.  All calls share the one array and
- * it keeps the previous call's contents; no part of it needs to start at
- * zero, because every byte a call reads there was written earlier in the
- * same call.  Calls whose work overlaps on the GPU (different streams, or
- * different host threads without ordering) race on the array: order them. */
+ * (a set-up done with that device current, and done again if the device's
+ * context has changed since, e.g. after a device reset); make that first call
+ * before any stream capture.  All calls share the one array and it keeps the
+ * previous call's contents; no part of it needs to start at zero, because
+ * every byte a call reads there was written earlier in the same call.  Calls
+ * whose work overlaps on the GPU (different streams, or different host
+ * threads without ordering) race on the array: order them. */
 #define IG4_NOALLOC_SCRATCH_BYTES (64ull << 20)
 ig4_status ig4_block_forward_noalloc(const ig4_config *cfg, const ig4_block_weights *w,
                                      const void *x_in, void *x_out, const int32_t *pos,
                                      const float *temb, void *stream);
 
-/* ---------------------------------------------------------------- a-12 ---
+/* ---------------------------------------------------------------- stack ---
  * Bytes of workspace ig4_stack_forward needs (0 if invalid). */
 size_t ig4_stack_workspace_size(const ig4_config *cfg, int latent_ch);
 
@@ -285,6 +288,21 @@ ig4_status ig4_stack_forward(const ig4_config *cfg, const ig4_stack_weights *sw,
                              const void *x_latent, const void *text, void *out_latent,
                              const int32_t *pos, const float *temb, void *workspace,
                              size_t ws_bytes, void *stream);
+
+/* ig4_stack_forward that also copies the sequence [B][L][D] (bf16, the
+ * stack's residual stream [text | image]) entering block tap_blocks[i] into
+ * the caller's device buffer tap_out[i] (16-byte aligned, 2*B*L*D bytes),
+ * for i < n_taps; tap_blocks[i] == n_blocks takes the sequence after the
+ * last block (the final norm's input).  The copies are stream-ordered device
+ * copies between the launches and change nothing else.  For inspecting a
+ * deep stack block by block.  Errors: INVALID_ARG for a block index outside
+ * [0, n_blocks], a NULL or misaligned tap buffer, n_taps < 0; otherwise as
+ * for ig4_stack_forward. */
+ig4_status ig4_stack_forward_tapped(const ig4_config *cfg, const ig4_stack_weights *sw,
+                                    const void *x_latent, const void *text, void *out_latent,
+                                    const int32_t *pos, const float *temb, void *workspace,
+                                    size_t ws_bytes, void *stream, const int *tap_blocks,
+                                    void *const *tap_out, int n_taps);
 
 /* -------------------------------------------------------------- NVFP4 ---
  * Block-scaled 4-bit linear layers ("不用再充会员！Ideogram 4.0 NF4 免费本地部署"

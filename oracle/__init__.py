@@ -34,6 +34,7 @@ from .ig4_oracle import (  # noqa: F401
     e4m3_decode_table,
     e2m1_encode,
     e4m3_encode,
+    final_layer,
     joint_attention,
     merge_heads,
     modulate,
@@ -48,6 +49,7 @@ from .ig4_oracle import (  # noqa: F401
     softmax,
     split_heads,
     stack_forward,
+    stack_input,
     swiglu,
     text_cond_projection,
     TEXT_RAW_LAYERS,

@@ -391,17 +391,33 @@ def stack_forward(x_latent, text, temb, pos, block_weights, n_blocks, w_in, b_in
     every block (the storage precision of a bf16 residual stream; NVFP4's
     rounding decisions in the next block depend on it).  Returns [B, N, C].
     """
-    x_latent = np.asarray(x_latent, dtype=np.float64)
-    text = np.asarray(text, dtype=np.float64)
-    B, N, C = x_latent.shape
-    T = text.shape[1]
-    img = x_latent @ np.asarray(w_in, dtype=np.float64).T + np.asarray(b_in, dtype=np.float64)
-    s = np.concatenate([text, img], axis=1)
+    T = np.asarray(text).shape[1]
     store = bf16_round if stream_bf16 else (lambda a: a)
-    s = store(s)
+    s = store(stack_input(x_latent, text, w_in, b_in))
     for i in range(n_blocks):
         s = store(block_forward(s, temb, pos, block_weights(i), H, theta, sections, eps,
                                 ffn_nvfp4=ffn_nvfp4))
+    return final_layer(s, temb, T, w_f, b_f, w_out, b_out, eps)
+
+
+def stack_input(x_latent, text, w_in, b_in) -> np.ndarray:
+    """The sequence entering the first block: [text | x_latent W_in^T + b_in].
+
+    x_latent [B, N, C] (C = 128 latent channels), text [B, T, D] (already at
+    the transformer's width) -> [B, T + N, D], text tokens first (survey page,
+    "条件注入方式": the text tokens form the prefix of the one sequence).
+    """
+    x_latent = np.asarray(x_latent, dtype=np.float64)
+    text = np.asarray(text, dtype=np.float64)
+    img = x_latent @ np.asarray(w_in, dtype=np.float64).T + np.asarray(b_in, dtype=np.float64)
+    return np.concatenate([text, img], axis=1)
+
+
+def final_layer(s, temb, T, w_f, b_f, w_out, b_out, eps=EPS) -> np.ndarray:
+    """After the last block: weightless RMSNorm with a 2-way AdaLN (shift,
+    scale) from the timestep embedding, then the linear D -> C with bias on the
+    image tokens (the T text tokens are dropped).  s [B, L, D] -> [B, L - T, C]."""
+    s = np.asarray(s, dtype=np.float64)
     shift_f, scale_f = adaln_modulation(temb, w_f, b_f, 2)
     s_f = modulate(s, shift_f, scale_f, eps)
     return s_f[:, T:, :] @ np.asarray(w_out, dtype=np.float64).T + np.asarray(b_out, dtype=np.float64)

@@ -1133,10 +1133,17 @@ size_t ig4_stack_workspace_size(const ig4_config *cfg, int latent_ch) {
   return stack_ws_layout(cfg, latent_ch, nullptr).bytes;
 }
 
-ig4_status ig4_stack_forward(const ig4_config *cfg, const ig4_stack_weights *sw,
-                             const void *x_latent, const void *text, void *out_latent,
-                             const int32_t *pos, const float *temb, void *workspace,
-                             size_t ws_bytes, void *stream) {
+}  // extern "C"
+
+namespace {
+
+// The stack on the caller's arguments; taps (may be empty) copy the sequence
+// entering the listed blocks into caller buffers.
+ig4_status stack_forward_checked(const ig4_config *cfg, const ig4_stack_weights *sw,
+                                 const void *x_latent, const void *text, void *out_latent,
+                                 const int32_t *pos, const float *temb, void *workspace,
+                                 size_t ws_bytes, void *stream, const int *tap_blocks,
+                                 void *const *tap_out, int n_taps) {
   IG4_TRY(check_config(cfg));
   if (!sw || !x_latent || !out_latent || !pos || !temb || !workspace) return IG4_ERR_INVALID_ARG;
   if (cfg->x_dtype != IG4_BF16) return IG4_ERR_UNSUPPORTED;
@@ -1155,6 +1162,10 @@ ig4_status ig4_stack_forward(const ig4_config *cfg, const ig4_stack_weights *sw,
   if (!aligned16(x_latent) || !aligned16(out_latent) || !aligned16(temb) ||
       (text && !aligned16(text)))
     return IG4_ERR_INVALID_ARG;
+  if (n_taps < 0 || (n_taps > 0 && (!tap_blocks || !tap_out))) return IG4_ERR_INVALID_ARG;
+  for (int t = 0; t < n_taps; ++t)
+    if (tap_blocks[t] < 0 || tap_blocks[t] > sw->n_blocks || !tap_out[t] || !aligned16(tap_out[t]))
+      return IG4_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return IG4_ERR_WORKSPACE;
   const StackWs ws = stack_ws_layout(cfg, C, static_cast<uint8_t *>(workspace));
   if (ws_bytes < ws.bytes) return IG4_ERR_WORKSPACE;
@@ -1163,6 +1174,15 @@ ig4_status ig4_stack_forward(const ig4_config *cfg, const ig4_stack_weights *sw,
   const int L = T + N;
   const int D = cfg->D;
   const int B = cfg->B;
+  const size_t seq_bytes = 2ull * B * L * D;  // the stack's stream is bf16
+  // copy the sequence entering block i (i == n_blocks: after the last block)
+  auto tap = [&](int i, const void *seq) -> ig4_status {
+    for (int t = 0; t < n_taps; ++t)
+      if (tap_blocks[t] == i &&
+          cudaMemcpyAsync(tap_out[t], seq, seq_bytes, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+        return IG4_ERR_CUDA;
+    return IG4_OK;
+  };
   // [text | image] sequence in s0: the text prefix, then the latent in-projection.
   if (T > 0) {
     const int vpr = D * 2 / 16;
@@ -1190,10 +1210,12 @@ ig4_status ig4_stack_forward(const ig4_config *cfg, const ig4_stack_weights *sw,
   void *cur = ws.s0;
   void *nxt = ws.s1;
   for (int i = 0; i < sw->n_blocks; ++i) {
+    IG4_TRY(tap(i, cur));
     IG4_TRY(block_forward_impl(cfg, &sw->blocks[i], cur, nxt, pos, temb, ws.blk, st, nullptr,
                                i > 0));
     std::swap(cur, nxt);
   }
+  IG4_TRY(tap(sw->n_blocks, cur));
   // Final layer on the image tokens: RMSNorm + (shift, scale), then D -> C.
   IG4_TRY(launch_adaln(B, cfg->adaln_dim, 2 * D, temb, sw->w_f, cfg->w_dtype, sw->s_f, sw->b_f,
                        ws.mod_f, st));
@@ -1202,6 +1224,27 @@ ig4_status ig4_stack_forward(const ig4_config *cfg, const ig4_stack_weights *sw,
   IG4_TRY(launch_linear_store(B * N, C, D, ws.hf, false, nullptr, w_out, nullptr, sw->b_out,
                               out_latent, IG4_BF16, C, 0, 0, 0, st));
   return IG4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+ig4_status ig4_stack_forward(const ig4_config *cfg, const ig4_stack_weights *sw,
+                             const void *x_latent, const void *text, void *out_latent,
+                             const int32_t *pos, const float *temb, void *workspace,
+                             size_t ws_bytes, void *stream) {
+  return stack_forward_checked(cfg, sw, x_latent, text, out_latent, pos, temb, workspace,
+                               ws_bytes, stream, nullptr, nullptr, 0);
+}
+
+ig4_status ig4_stack_forward_tapped(const ig4_config *cfg, const ig4_stack_weights *sw,
+                                    const void *x_latent, const void *text, void *out_latent,
+                                    const int32_t *pos, const float *temb, void *workspace,
+                                    size_t ws_bytes, void *stream, const int *tap_blocks,
+                                    void *const *tap_out, int n_taps) {
+  return stack_forward_checked(cfg, sw, x_latent, text, out_latent, pos, temb, workspace,
+                               ws_bytes, stream, tap_blocks, tap_out, n_taps);
 }
 
 // ----------------------------------------------------------------- NVFP4
@@ -1416,26 +1459,61 @@ ig4_status ig4_denoise_step(const ig4_config *cfg, const ig4_stack_weights *cond
 // Scratch for ig4_block_forward_noalloc: a static device array, so the entry
 // point never allocates.  In host code `g_noalloc_scratch` names a host-side
 // stand-in, not device memory; its device address comes from
-// cudaGetSymbolAddress, looked up once per device.
+// cudaGetSymbolAddress, looked up on the first call for each device (with
+// that device current) and again whenever the device's current context has
+// changed since (a device reset loads the module anew, possibly elsewhere).
 __device__ __align__(256) uint8_t g_noalloc_scratch[IG4_NOALLOC_SCRATCH_BYTES];
 
 namespace {
-void *g_noalloc_ptr[MAX_DEVICES];
+struct NoallocSlot {
+  void *ptr = nullptr;
+  unsigned long long ctx_id = 0;
+};
+NoallocSlot g_noalloc[MAX_DEVICES];
 std::mutex g_noalloc_mu;
 
-// Device address of the scratch array on the current device (set up on the
-// first call for that device).
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+
+// Unique id of the calling thread's current context (0 if there is none or
+// the driver cannot tell).
+unsigned long long current_ctx_id() {
+  static CtxGetCurrentFn get_cur = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  if (!get_cur || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_cur(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Device address of the scratch array on the current device.
 ig4_status noalloc_scratch(uint8_t **out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return IG4_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
+  NoallocSlot &slot = g_noalloc[dev];
+  const unsigned long long id = current_ctx_id();
+  if (slot.ptr == nullptr || id == 0 || id != slot.ctx_id) {
     void *p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
       return IG4_ERR_CUDA;
-    g_noalloc_ptr[dev] = p;
+    slot.ptr = p;
+    slot.ctx_id = current_ctx_id();  // the lookup made the primary context current
   }
-  *out = static_cast<uint8_t *>(g_noalloc_ptr[dev]);
+  *out = static_cast<uint8_t *>(slot.ptr);
   return IG4_OK;
 }
 }  // namespace

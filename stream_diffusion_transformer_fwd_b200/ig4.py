@@ -100,6 +100,9 @@ _sig("ig4_block_forward_noalloc", [ctypes.POINTER(Config), ctypes.POINTER(BlockW
 _sig("ig4_stack_workspace_size", [ctypes.POINTER(Config), _i], ctypes.c_size_t)
 _sig("ig4_stack_forward", [ctypes.POINTER(Config), ctypes.POINTER(StackWeights), _vp, _vp, _vp,
                            _vp, _vp, _vp, ctypes.c_size_t, _vp])
+_sig("ig4_stack_forward_tapped", [ctypes.POINTER(Config), ctypes.POINTER(StackWeights), _vp, _vp,
+                                  _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp, ctypes.POINTER(_i),
+                                  ctypes.POINTER(_vp), _i])
 _sig("ig4_nvfp4_scale_bytes", [_i, _i], ctypes.c_size_t)
 _sig("ig4_nvfp4_pack_scales", [_i, _i, _vp, _vp, _vp])
 _sig("ig4_nvfp4_linear", [_i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp])
@@ -123,7 +126,7 @@ EXPORTED = ("ig4_status_string", "ig4_abi_version", "ig4_mrope_positions", "ig4_
             "ig4_joint_attention", "ig4_gated_residual_linear", "ig4_swiglu",
             "ig4_quantize_rows", "ig4_workspace_size", "ig4_block_forward",
             "ig4_block_forward_traced", "ig4_block_forward_noalloc", "ig4_stack_workspace_size",
-            "ig4_stack_forward", "ig4_nvfp4_scale_bytes", "ig4_nvfp4_pack_scales",
+            "ig4_stack_forward", "ig4_stack_forward_tapped", "ig4_nvfp4_scale_bytes", "ig4_nvfp4_pack_scales",
             "ig4_nvfp4_linear", "ig4_nvfp4_quantize", "ig4_text_cond_workspace_size", "ig4_text_cond_project",
             "ig4_flow_schedule", "ig4_guidance_schedule", "ig4_cfg_euler",
             "ig4_denoise_workspace_size", "ig4_denoise_step", "ig4_last_device_error",
@@ -340,6 +343,20 @@ def ig4_stack_forward(cfg: Config, sw: StackWeights, x_latent, text, out_latent,
                                   _ptr(text), _ptr(out_latent), _ptr(pos), _ptr(temb),
                                   _ptr(workspace), ws_bytes, _stream(stream)),
            "ig4_stack_forward")
+
+
+def ig4_stack_forward_tapped(cfg: Config, sw: StackWeights, x_latent, text, out_latent, pos,
+                             temb, workspace, taps: dict, stream=None):
+    """ig4_stack_forward that copies the bf16 sequence [B, L, D] entering block i
+    into taps[i] (a device tensor) for each key i (i == n_blocks: after the last block)."""
+    ws_bytes = workspace.numel() * workspace.element_size()
+    idx = list(taps)
+    blocks = (_i * max(1, len(idx)))(*idx)
+    outs = (_vp * max(1, len(idx)))(*[taps[i].data_ptr() for i in idx])
+    _check(_lib.ig4_stack_forward_tapped(ctypes.byref(cfg), ctypes.byref(sw), _ptr(x_latent),
+                                         _ptr(text), _ptr(out_latent), _ptr(pos), _ptr(temb),
+                                         _ptr(workspace), ws_bytes, _stream(stream), blocks, outs,
+                                         len(idx)), "ig4_stack_forward_tapped")
 
 
 def ig4_nvfp4_scale_bytes(rows: int, K: int) -> int:

@@ -3,9 +3,9 @@
 The guided Euler kernel element by element; one full step with asymmetric CFG
 (a conditional stack over [text | image] and a separate image-only
 unconditional stack) in full at reduced width, in bf16 and with E4M3
-weights; and the full-size step (34 + 34 blocks, 1024 px, FP8) with zero
-block gates, where both stacks reduce to their in/out layers and the oracle
-stays cheap."""
+weights, and at the full width with two blocks per branch; and the full-size
+step (34 + 34 live blocks, 1024 px, FP8) as the exact composition of two
+stacks whose blocks are checked against the oracle one by one."""
 
 import numpy as np
 import pytest
@@ -16,7 +16,8 @@ from oracle import ig4_sampler as S
 from oracle.inputs import block_weights_f64, to_f64, weight_f64
 from synth import CONFIGS, make_block_weights, make_stack_inputs
 from tests._util import rel_l2
-from tests.gpu_common import lib, to_dev
+from tests.gpu_common import (check_tapped_stack, lib, live_blocks, run_stack_tapped,
+                              tap_ids_for, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -113,27 +114,73 @@ def test_denoise_step_small_full(ig4, wdt):
     assert e <= (6e-2 if wdt == "e4m3" else 2e-2)
 
 
-def test_denoise_step_full_size_zero_gates(ig4):
-    """The full-size step (1024 px, batch 2, FP8, two 34-block stacks): with every
-    block's AdaLN zero both stacks reduce to in-proj -> final norm -> out-proj."""
-    cfg = CONFIGS["stack_1024px_fp8"]
-    st_c = make_stack_inputs(cfg, seed=9, stress=True)
-    st_u = make_stack_inputs(cfg, seed=10, stress=True)
-    blk_c = to_dev(make_block_weights(cfg, seed=9, block=0, zero_adaln=True))
-    blk_u = to_dev(make_block_weights(cfg, seed=10, block=0, zero_adaln=True))
-    t = S.flow_schedule(48, 0.0, 1.5, 1024, 1024)
-    z = torch.randn(cfg.B, cfg.n_img, cfg.latent_ch, generator=torch.Generator().manual_seed(5))
-    got = _run_step(ig4, cfg, st_c, st_u, [blk_c] * cfg.n_blocks, [blk_u] * cfg.n_blocks, z,
-                    float(t[3]), float(t[4]), 7.0)
+@pytest.mark.parametrize("wdt", ["e4m3"])
+def test_denoise_step_full_width_two_blocks(ig4, wdt):
+    """One sampler step at the full width (D 4608, 18 heads, I 12288) with two
+    live blocks per branch, B = 2, 128 text + 32 x 32 image tokens (the
+    unconditional stack sees the 1024 image tokens alone), against the
+    oracle's whole denoise_step on the same seeded inputs."""
+    cfg = CONFIGS["step_1024px_fp8"].with_(name="step_fw2", B=2, T_text=128, grid_h=32,
+                                           grid_w=32, w_dtype=wdt, n_blocks=2)
+    st_c = make_stack_inputs(cfg, seed=14, stress=True)
+    st_u = make_stack_inputs(cfg, seed=15, stress=True)
+    host_c = [make_block_weights(cfg, seed=14, block=i, stress=True) for i in range(2)]
+    host_u = [make_block_weights(cfg, seed=15, block=i, stress=True) for i in range(2)]
+    t = S.flow_schedule(20, 0.0, 1.75, 512, 512)
+    gw = float(S.guidance_schedule(20, 2)[3])
+    z = torch.randn(cfg.B, cfg.n_img, cfg.latent_ch, generator=torch.Generator().manual_seed(6))
+    got = _run_step(ig4, cfg, st_c, st_u, [to_dev(w) for w in host_c],
+                    [to_dev(w) for w in host_u], z, float(t[3]), float(t[4]), gw)
+    Wc = [block_weights_f64(w) for w in host_c]
+    Wu = [block_weights_f64(w) for w in host_u]
+    dc = _stack_dict(cfg, st_c, 14, 2)
+    du = _stack_dict(cfg, st_u, 15, 2)
+    dc["block_weights"] = lambda i: Wc[i]
+    du["block_weights"] = lambda i: Wu[i]
     ref = S.denoise_step(to_f64(z), to_f64(st_c["text"]), to_f64(st_c["temb"]),
-                         to_f64(st_u["temb"]), float(t[3]), float(t[4]), 7.0,
-                         (cfg.grid_t, cfg.grid_h, cfg.grid_w),
-                         _stack_dict(cfg, st_c, 9, cfg.n_blocks, zero_gates=True),
-                         _stack_dict(cfg, st_u, 10, cfg.n_blocks, zero_gates=True), cfg.H)
+                         to_f64(st_u["temb"]), float(t[3]), float(t[4]), gw,
+                         (cfg.grid_t, cfg.grid_h, cfg.grid_w), dc, du, cfg.H,
+                         theta=cfg.rope_theta, sections=cfg.sections, eps=cfg.eps)
     z0 = to_f64(z)
     e = rel_l2(got - z0, ref - z0)
-    print(f"denoise step full size, zero gates: relL2(dz)={e:.3e}")
-    assert e <= 3e-2
+    print(f"denoise step full width, 2 + 2 blocks, {wdt}: relL2(dz)={e:.3e}")
+    assert e <= (3e-2 if wdt == "e4m3" else 1e-2)
+
+
+def test_denoise_step_full_size_live_blocks(ig4):
+    """The full-size step (1024 px, FP8, two 34-block stacks with live
+    weights).  The step's result must equal, bit for bit, the guided Euler
+    update of the two stacks run on their own through the tapped stack entry
+    point on the bf16-rounded latent; those two stack runs are checked against
+    the oracle block by block (tests.gpu_common.check_tapped_stack: stack
+    input, blocks 0 and 33 of each branch on sampled rows, final layer)."""
+    cfg = CONFIGS["step_1024px_fp8"]
+    cfg_u = cfg.with_(name="step_1024px_fp8_uncond", T_text=0)
+    checked = (0, 33)
+    st_c = make_stack_inputs(cfg, seed=16, stress=True)
+    st_u = make_stack_inputs(cfg_u, seed=17, stress=True)
+    host_c = {i: make_block_weights(cfg, seed=16, block=i, stress=True) for i in checked}
+    host_u = {i: make_block_weights(cfg_u, seed=17, block=i, stress=True) for i in checked}
+    blocks_c = live_blocks(cfg, host_c, seed=16)
+    blocks_u = live_blocks(cfg_u, host_u, seed=17)
+    t = S.flow_schedule(48, 0.0, 1.5, 1024, 1024)
+    t_cur, t_next, gw = float(t[3]), float(t[4]), 7.0
+    z = torch.randn(cfg.B, cfg.n_img, cfg.latent_ch, generator=torch.Generator().manual_seed(5))
+    z_step = _run_step(ig4, cfg, st_c, st_u, blocks_c, blocks_u, z, t_cur, t_next, gw)
+
+    z16 = z.to(torch.bfloat16)
+    v_c, seq_c = run_stack_tapped(ig4, cfg, st_c, blocks_c, tap_ids_for(cfg, host_c), z16)
+    v_u, seq_u = run_stack_tapped(ig4, cfg_u, st_u, blocks_u, tap_ids_for(cfg_u, host_u), z16)
+    del blocks_c, blocks_u
+    zd = z.cuda()
+    z_comp = torch.empty_like(zd)
+    ig4.ig4_cfg_euler(v_c, v_u, gw, t_cur - t_next, zd, z_comp, None)
+    torch.cuda.synchronize()
+    assert np.array_equal(to_f64(z_comp.cpu()), z_step)
+
+    z64 = to_f64(z16)
+    check_tapped_stack(cfg, st_c, host_c, seq_c, v_c, z64)
+    check_tapped_stack(cfg_u, st_u, host_u, seq_u, v_u, z64)
 
 
 def test_denoise_step_argument_errors(ig4):

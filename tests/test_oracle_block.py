@@ -245,3 +245,39 @@ def test_block_flops_closed_form():
     g, a, ada = O.block_flops(1, 4608, 4608, 12288)
     assert g == 4608 * (8 * 4608 ** 2 + 6 * 4608 * 12288)
     assert round((g + a) / 1e9, 1) == 2739.7
+
+
+def test_stack_input_and_final_layer_brute_force():
+    """stack_input and final_layer against scalar loops: the text rows pass
+    through unchanged and come first; each image row is the latent row times
+    W_in plus b_in; the final layer normalises each token over D, applies
+    (1 + scale) and shift from SiLU(temb) W_f^T + b_f, and projects only the
+    tokens after the text prefix."""
+    B, T, N, C, D, A = 2, 3, 4, 5, 6, 4
+    lat = RNG.standard_normal((B, N, C))
+    text = RNG.standard_normal((B, T, D))
+    w_in, b_in = RNG.standard_normal((D, C)), RNG.standard_normal(D)
+    s = O.stack_input(lat, text, w_in, b_in)
+    assert s.shape == (B, T + N, D)
+    assert np.array_equal(s[:, :T], text)
+    for b in range(B):
+        for n in range(N):
+            for d in range(D):
+                ref = b_in[d] + sum(lat[b, n, c] * w_in[d, c] for c in range(C))
+                assert abs(s[b, T + n, d] - ref) <= 1e-12 * (1 + abs(ref))
+    temb = RNG.standard_normal((B, A))
+    w_f, b_f = RNG.standard_normal((2 * D, A)), RNG.standard_normal(2 * D)
+    w_out, b_out = RNG.standard_normal((C, D)), RNG.standard_normal(C)
+    out = O.final_layer(s, temb, T, w_f, b_f, w_out, b_out, eps=1e-6)
+    assert out.shape == (B, N, C)
+    for b in range(B):
+        act = [t / (1.0 + np.exp(-t)) for t in temb[b]]
+        mod = [b_f[j] + sum(act[a] * w_f[j, a] for a in range(A)) for j in range(2 * D)]
+        shift, scale = mod[:D], mod[D:]
+        for n in range(N):
+            row = s[b, T + n]
+            r = 1.0 / np.sqrt(sum(v * v for v in row) / D + 1e-6)
+            h = [row[d] * r * (1.0 + scale[d]) + shift[d] for d in range(D)]
+            for c in range(C):
+                ref = b_out[c] + sum(h[d] * w_out[c, d] for d in range(D))
+                assert abs(out[b, n, c] - ref) <= 1e-11 * (1 + abs(ref))
