@@ -111,7 +111,7 @@ def test_denoise_step_small_full(ig4, wdt):
     print(f"denoise step {wdt}: relL2(dz)={e:.3e}")
     # two stacks of two blocks each and their head; the guided difference keeps
     # the per-stack relative error
-    assert e <= (6e-2 if wdt == "e4m3" else 2e-2)
+    assert e <= (3e-2 if wdt == "e4m3" else 1e-2)
 
 
 @pytest.mark.parametrize("wdt", ["e4m3"])
@@ -174,7 +174,9 @@ def test_denoise_step_full_size_live_blocks(ig4):
     del blocks_c, blocks_u
     zd = z.cuda()
     z_comp = torch.empty_like(zd)
-    ig4.ig4_cfg_euler(v_c, v_u, gw, t_cur - t_next, zd, z_comp, None)
+    # the step takes t_cur and t_next as fp32 and subtracts them in fp32
+    dt = float(np.float32(t_cur) - np.float32(t_next))
+    ig4.ig4_cfg_euler(v_c, v_u, gw, dt, zd, z_comp, None)
     torch.cuda.synchronize()
     assert np.array_equal(to_f64(z_comp.cpu()), z_step)
 
