@@ -430,6 +430,97 @@ ig4_status ig4_denoise_step(const ig4_config *cfg, const ig4_stack_weights *cond
                             float t_next, float gw, void *workspace, size_t ws_bytes,
                             void *stream);
 
+/* ------------------------------------------------- multi-GPU layouts ---
+ * Tensor parallelism over heads (TP) and Ulysses sequence parallelism over
+ * the image tokens (SP) of the block ("SGLang cookbook: Ideogram 4",
+ * section 3, tensor and sequence parallelism: TP shards the DiT weights and
+ * its degree must divide the 18 heads; Ulysses SP keeps the weights whole on
+ * every GPU and shards the image-token sequence; both validated on B200 at
+ * 1024 x 1024 with 2 GPUs).  These calls compute one rank's share; the data
+ * each rank must receive from the others between the calls is moved by the
+ * caller (a collective, or peer-mapped pointers for ig4_tp_reduce).  At most
+ * 8 ranks.  All calls are stream-ordered; argument errors are returned before
+ * anything is launched.
+ *
+ * TP, tp_size P dividing H and with (I / P) % 128 == 0, weights BF16 or E4M3
+ * (IG4_NVFP4_MIXED: UNSUPPORTED).  Rank r holds heads [r H/P, (r+1) H/P) and
+ * FFN columns [r I/P, (r+1) I/P); its ig4_block_weights hold: w_ada, s_ada,
+ * b_ada, g_q, g_k whole; w_qkv [3 D/P][D] = the q rows, then the k rows, then
+ * the v rows of its heads (s_qkv likewise); w_o [D][D/P] = the columns of
+ * W_o for its heads (s_o [D] whole); w_gate, w_up [I/P][D] = its rows
+ * (s_gate, s_up [I/P]); w_down [D][I/P] = its columns (s_down [D] whole).
+ * One block on rank r, with y = x_out:
+ *   ig4_block_tp_attention -> partial_r = [r == 0] x + gate_msa * (o_r W_o,r^T)
+ *   x1 = sum over ranks of partial_r         (all-reduce; ig4_tp_reduce)
+ *   ig4_block_tp_mlp       -> partial_r = [r == 0] x1 + gate_mlp * (u_r W_down,r^T)
+ *   y  = sum over ranks of partial_r         (all-reduce; ig4_tp_reduce)
+ * partials are fp32 [B*L][D] (device, 16-byte aligned); the gates commute
+ * with the sum, so the reduced partials are exactly the block's x1 and y up
+ * to fp32 rounding.  ig4_block_tp_mlp reads the AdaLN output that
+ * ig4_block_tp_attention left in the workspace: pass the same workspace,
+ * unchanged in between.  The FP8 path quantises each rank's attention
+ * output and SwiGLU output over its own columns.
+ * ig4_tp_reduce: out[i] = sum_{k < n_src} src[k][i] (fp32, in index order,
+ * so every rank computes the same bits), stored as out_dtype (IG4_F32 or
+ * IG4_BF16); src is a HOST array of n_src device-accessible fp32 pointers
+ * (this GPU's memory, or peer memory mapped into it), n % 8 == 0.
+ *
+ * SP, sp_size P dividing H, at least P image tokens.  Rank r holds the T text
+ * tokens and the image tokens [off_r, off_r + N_r) of the row-major grid
+ * (contiguous shares, the first N % P ranks one token more;
+ * ig4_sp_image_range): its local sequence x_local is [B][T + N_r][D], text
+ * first, with the positions of ig4_sp_positions.  One block on rank r:
+ *   ig4_block_sp_pre       AdaLN, norm, QKV (+QK-norm, MRoPE) of the local
+ *                          tokens; packs the phase-0 send buffer;
+ *   all-to-all, phase 0    (rank s sends chunk (s -> d) to every d)
+ *   ig4_block_sp_attention unpacks q, k, v of head group r
+ *                          [r H/P, (r+1) H/P) over all L tokens (text rows
+ *                          from its own QKV, image rows from every rank),
+ *                          attention, packs the phase-1 send buffer;
+ *   all-to-all, phase 1
+ *   ig4_block_sp_post      unpacks o of the local tokens (all heads),
+ *                          out-projection + gated residual, norm, SwiGLU,
+ *                          down-projection + gated residual -> x_out_local.
+ * The text tokens are computed on every rank, with the same result there.
+ * Chunk (s -> d), bf16, ig4_sp_exchange_bytes(cfg, P, phase, s, d) bytes:
+ *   phase 0: q [B][H/P][N_s][256], then k likewise, then v^T
+ *            [B][H/P][256][N_s], of head group d over s's image tokens;
+ *   phase 1: o [B][T + N_d][H/P * 256] of head group s over d's text and
+ *            image tokens.
+ * A send buffer holds the chunks to d = 0 .. P-1 in order, a receive buffer
+ * the chunks from s = 0 .. P-1 in order (16-byte aligned).  The workspace
+ * (ig4_sp_workspace_size) must be the same for the three calls of a block. */
+size_t ig4_tp_workspace_size(const ig4_config *cfg, int tp_size);
+ig4_status ig4_block_tp_attention(const ig4_config *cfg, int tp_rank, int tp_size,
+                                  const ig4_block_weights *w, const void *x_in,
+                                  const int32_t *pos, const float *temb, float *partial,
+                                  void *workspace, size_t ws_bytes, void *stream);
+ig4_status ig4_block_tp_mlp(const ig4_config *cfg, int tp_rank, int tp_size,
+                            const ig4_block_weights *w, const void *x1, float *partial,
+                            void *workspace, size_t ws_bytes, void *stream);
+ig4_status ig4_tp_reduce(long long n, int n_src, const float *const *src, void *out,
+                         int out_dtype, void *stream);
+ig4_status ig4_sp_image_range(const ig4_config *cfg, int sp_size, int sp_rank, int *img_off,
+                              int *img_count);
+/* int32 [3][T + N_r] positions of rank r's local tokens (host memory written
+ * before returning if out_on_device == 0, else device memory by a kernel). */
+ig4_status ig4_sp_positions(const ig4_config *cfg, int sp_size, int sp_rank, int32_t *pos_out,
+                            int out_on_device, void *stream);
+size_t ig4_sp_workspace_size(const ig4_config *cfg, int sp_size, int sp_rank);
+size_t ig4_sp_exchange_bytes(const ig4_config *cfg, int sp_size, int phase, int src_rank,
+                             int dst_rank);
+ig4_status ig4_block_sp_pre(const ig4_config *cfg, int sp_rank, int sp_size,
+                            const ig4_block_weights *w, const void *x_local,
+                            const int32_t *pos_local, const float *temb, void *send,
+                            void *workspace, size_t ws_bytes, void *stream);
+ig4_status ig4_block_sp_attention(const ig4_config *cfg, int sp_rank, int sp_size,
+                                  const void *recv, void *send_o, void *workspace,
+                                  size_t ws_bytes, void *stream);
+ig4_status ig4_block_sp_post(const ig4_config *cfg, int sp_rank, int sp_size,
+                             const ig4_block_weights *w, const void *x_local, void *x_out_local,
+                             const void *recv_o, void *workspace, size_t ws_bytes,
+                             void *stream);
+
 /* ------------------------------------------------------------ failure ---
  * Synchronises `stream`, then reads and clears the device error word that the
  * kernels set when a bounded wait times out: IG4_ERR_TIMEOUT if set,

@@ -18,6 +18,7 @@
 #include "ig4_attention.cuh"
 #include "ig4_gemm.cuh"
 #include "ig4_nvf4.cuh"
+#include "ig4_parallel.cuh"
 #include "ig4_small.cuh"
 
 using namespace ig4;
@@ -369,6 +370,8 @@ ig4_status launch_quantize(int M, int K, const void *x, void *q, float *scale, c
   return IG4_ERR_UNSUPPORTED;
 }
 
+// q, k, v of H heads (3 * 256 * H weight rows) from h [B*L][D]; a
+// tensor-parallel shard passes its own head count.
 ig4_status launch_qkv(int B, int L, int D, int H, const void *h, int h_dtype, const float *h_scale,
                       const void *w, const float *w_scale, const float *g_q, const float *g_k,
                       float eps, const float *cs, const float *sn, void *q, void *k, void *vt,
@@ -377,7 +380,7 @@ ig4_status launch_qkv(int B, int L, int D, int H, const void *h, int h_dtype, co
   const bool f8 = is_fp8(h_dtype);
   const int esize = f8 ? 1 : 2;
   CUtensorMap ma, mb;
-  IG4_TRY(gemm_maps(&ma, &mb, h, w, esize, M, 3L * D, D, b_box_rows(256, M)));
+  IG4_TRY(gemm_maps(&ma, &mb, h, w, esize, M, 3L * 256 * H, D, b_box_rows(256, M)));
   const int ntn = 3 * H;
   if (f8) {
     EpiQKV<true> e{static_cast<__nv_bfloat16 *>(q), static_cast<__nv_bfloat16 *>(k),
@@ -827,22 +830,19 @@ struct Tracer {
   }
 };
 
-// The block on already validated arguments.
-// rope_ready: ws.cos / ws.sin already hold the table of these positions (the
-// stack computes it for its first block only; every block shares it).
-ig4_status block_forward_impl(const ig4_config *c, const ig4_block_weights *w, const void *x_in,
-                              void *x_out, const int32_t *pos, const float *temb,
-                              const BlockWs &ws, cudaStream_t st, Tracer *tr,
-                              bool rope_ready = false) {
+// The block's steps before attention: AdaLN, rotary table (unless
+// rope_ready: ws.cos / ws.sin already hold the table of these positions, as
+// in the stack's blocks after the first), norm1, QKV with QK-norm and MRoPE
+// into ws.q, ws.k, ws.vt.  Records trace marks 0..4.
+ig4_status block_pre_attention(const ig4_config *c, const ig4_block_weights *w, const void *x_in,
+                               const int32_t *pos, const float *temb, const BlockWs &ws,
+                               cudaStream_t st, Tracer &t, bool rope_ready) {
   const int L = c->T_text + c->grid_t * c->grid_h * c->grid_w;
   const int M = c->B * L;
-  const int D = c->D, I = c->I, H = c->H;
+  const int D = c->D, H = c->H;
   const bool f8 = is_fp8(c->w_dtype);
   const int hdt = f8 ? IG4_E4M3 : IG4_BF16;
   const int ms = 6 * D;
-  Tracer none{nullptr, 0, 0, st};
-  Tracer &t = tr ? *tr : none;
-
   IG4_TRY(t.mark());
   IG4_TRY(launch_adaln(c->B, c->adaln_dim, 6 * D, temb, w->w_ada, c->w_dtype, w->s_ada, w->b_ada,
                        ws.mod, st));
@@ -856,8 +856,20 @@ ig4_status block_forward_impl(const ig4_config *c, const ig4_block_weights *w, c
   IG4_TRY(launch_qkv(c->B, L, D, H, ws.h, hdt, ws.h_scale, w->w_qkv, w->s_qkv, w->g_q, w->g_k,
                      c->eps, ws.cos, ws.sin, ws.q, ws.k, ws.vt, ws.vt_ld, st));
   IG4_TRY(t.mark());
-  IG4_TRY(launch_attention(c->B, H, L, ws.q, ws.k, ws.vt, ws.vt_ld, ws.o, st));
-  IG4_TRY(t.mark());
+  return IG4_OK;
+}
+
+// The block's steps after attention, with o in ws.o: out-projection + gated
+// residual (x_in -> x_out), norm2, SwiGLU, down-projection + gated residual
+// (in place in x_out).  The AdaLN modulation is read from ws.mod.
+ig4_status block_post_attention(const ig4_config *c, const ig4_block_weights *w, const void *x_in,
+                                void *x_out, const BlockWs &ws, cudaStream_t st, Tracer &t) {
+  const int L = c->T_text + c->grid_t * c->grid_h * c->grid_w;
+  const int M = c->B * L;
+  const int D = c->D, I = c->I;
+  const bool f8 = is_fp8(c->w_dtype);
+  const int hdt = f8 ? IG4_E4M3 : IG4_BF16;
+  const int ms = 6 * D;
   if (f8) {
     IG4_TRY(launch_quantize(M, D, ws.o, ws.oq, ws.o_scale, st));
     IG4_TRY(t.mark());
@@ -896,6 +908,22 @@ ig4_status block_forward_impl(const ig4_config *c, const ig4_block_weights *w, c
                        ws.mod + 5 * D, ms, x_out, x_out, c->x_dtype, st));
   IG4_TRY(t.mark());
   return IG4_OK;
+}
+
+// The block on already validated arguments.
+// rope_ready: ws.cos / ws.sin already hold the table of these positions (the
+// stack computes it for its first block only; every block shares it).
+ig4_status block_forward_impl(const ig4_config *c, const ig4_block_weights *w, const void *x_in,
+                              void *x_out, const int32_t *pos, const float *temb,
+                              const BlockWs &ws, cudaStream_t st, Tracer *tr,
+                              bool rope_ready = false) {
+  const int L = c->T_text + c->grid_t * c->grid_h * c->grid_w;
+  Tracer none{nullptr, 0, 0, st};
+  Tracer &t = tr ? *tr : none;
+  IG4_TRY(block_pre_attention(c, w, x_in, pos, temb, ws, st, t, rope_ready));
+  IG4_TRY(launch_attention(c->B, c->H, L, ws.q, ws.k, ws.vt, ws.vt_ld, ws.o, st));
+  IG4_TRY(t.mark());
+  return block_post_attention(c, w, x_in, x_out, ws, st, t);
 }
 
 // Stack workspace: two sequence buffers, the block workspace, final-layer buffers.
@@ -962,7 +990,7 @@ ig4_status ig4_mrope_positions(int T, int gt, int gh, int gw, int32_t *pos, int 
   if (on_device) {
     if (!aligned16(pos)) return IG4_ERR_INVALID_ARG;
     mrope_positions_kernel<<<static_cast<int>((L + 255) / 256), 256, 0, as_stream(stream)>>>(
-        T, gt, gh, gw, pos);
+        T, gt, gh, gw, 0, gt * gh * gw, pos);
     return last_launch_status();
   }
   for (long l = 0; l < T; ++l) pos[l] = pos[L + l] = pos[2 * L + l] = static_cast<int32_t>(l);
@@ -1451,6 +1479,466 @@ ig4_status ig4_denoise_step(const ig4_config *cfg, const ig4_stack_weights *cond
                             ws.stack, stack_bytes, stream));
   // v = v_u + gw (v_c - v_u); z += (t_cur - t_next) v
   return ig4_cfg_euler(n, ws.v_c, ws.v_u, gw, t_cur - t_next, z, z, nullptr, stream);
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------ multi-GPU layouts
+// Tensor parallelism over heads (TP) and Ulysses sequence parallelism over
+// image tokens (SP), "SGLang cookbook: Ideogram 4", section 3.  The library
+// computes each rank's share and packs / reduces the exchanged data; the
+// transfers between GPUs are the caller's collectives (or peer-mapped
+// pointers handed to ig4_tp_reduce).
+namespace {
+
+constexpr int SP_MAX_RANKS = 8;
+
+// Image tokens [*off, *off + *cnt) of Ulysses rank r of P: contiguous shares
+// in the grid's row-major order, the first N % P ranks one token more.
+void sp_range(long N, int P, int r, long *off, long *cnt) {
+  const long base = N / P, rem = N % P;
+  *cnt = base + (r < rem ? 1 : 0);
+  *off = r * base + std::min<long>(r, rem);
+}
+
+ig4_status check_tp(const ig4_config *c, int rank, int size) {
+  IG4_TRY(check_config(c));
+  if (size < 1 || size > TP_MAX_RANKS || rank < 0 || rank >= size) return IG4_ERR_INVALID_ARG;
+  if (c->H % size != 0 || c->I % size != 0 || (c->I / size) % 128 != 0) return IG4_ERR_UNSUPPORTED;
+  if (is_nvf4_mixed(c->w_dtype)) return IG4_ERR_UNSUPPORTED;
+  return IG4_OK;
+}
+
+// A TP shard's block: H / size heads, I / size FFN columns, full width D.
+ig4_config tp_local(const ig4_config *c, int size) {
+  ig4_config t = *c;
+  t.H = c->H / size;
+  t.I = c->I / size;
+  return t;
+}
+
+// TP partial output [B*L][D] fp32: (x_res or 0) + gate * (a W^T), 256-wide tiles.
+template <typename XT>
+ig4_status launch_partial_t(int B, int L, int N, int K, const void *a, bool f8,
+                            const float *a_scale, const void *w, const float *w_scale,
+                            const float *gate, int gate_stride, const void *x_res, float *out,
+                            cudaStream_t st) {
+  const int M = B * L;
+  CUtensorMap ma, mb;
+  IG4_TRY(gemm_maps(&ma, &mb, a, w, f8 ? 1 : 2, M, N, K, b_box_rows(256, M)));
+  if (f8) {
+    EpiResidGate<256, true, XT, float> e{static_cast<const XT *>(x_res), out, gate, gate_stride,
+                                         L, M, N, a_scale, w_scale};
+    return launch_gemm<256, true, false>(ma, mb, mb, M, N / 256, K, e, st);
+  }
+  EpiResidGate<256, false, XT, float> e{static_cast<const XT *>(x_res), out, gate, gate_stride, L,
+                                        M, N, nullptr, nullptr};
+  return launch_gemm<256, false, false>(ma, mb, mb, M, N / 256, K, e, st);
+}
+
+ig4_status launch_partial(int B, int L, int N, int K, const void *a, bool f8, const float *a_scale,
+                          const void *w, const float *w_scale, const float *gate, int gate_stride,
+                          const void *x_res, int x_dtype, float *out, cudaStream_t st) {
+  if (x_dtype == IG4_F32)
+    return launch_partial_t<float>(B, L, N, K, a, f8, a_scale, w, w_scale, gate, gate_stride,
+                                   x_res, out, st);
+  return launch_partial_t<__nv_bfloat16>(B, L, N, K, a, f8, a_scale, w, w_scale, gate,
+                                         gate_stride, x_res, out, st);
+}
+
+ig4_status check_tp_call(const ig4_config *cfg, int rank, int size, const ig4_block_weights *w,
+                         const void *x, const float *partial, const void *workspace,
+                         size_t ws_bytes, BlockWs *ws) {
+  IG4_TRY(check_tp(cfg, rank, size));
+  IG4_TRY(check_block_weights(cfg, w));
+  if (!x || !partial || !workspace || !aligned16(x) || !aligned16(partial))
+    return IG4_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return IG4_ERR_WORKSPACE;
+  const ig4_config t = tp_local(cfg, size);
+  *ws = block_ws_layout(&t, static_cast<uint8_t *>(const_cast<void *>(workspace)));
+  if (ws_bytes < ws->bytes) return IG4_ERR_WORKSPACE;
+  return IG4_OK;
+}
+
+// ----------------------------------------------------------- Ulysses SP
+
+ig4_status check_sp(const ig4_config *c, int rank, int size) {
+  IG4_TRY(check_config(c));
+  if (size < 1 || size > SP_MAX_RANKS || rank < 0 || rank >= size) return IG4_ERR_INVALID_ARG;
+  if (c->H % size != 0) return IG4_ERR_UNSUPPORTED;
+  const long N = static_cast<long>(c->grid_t) * c->grid_h * c->grid_w;
+  if (N < size) return IG4_ERR_UNSUPPORTED;  // every rank holds image tokens
+  return IG4_OK;
+}
+
+// The block a Ulysses rank runs outside attention: the text tokens and its
+// share of the image tokens, as one flat image row.
+ig4_config sp_local(const ig4_config *c, int size, int rank) {
+  long off = 0, cnt = 0;
+  sp_range(static_cast<long>(c->grid_t) * c->grid_h * c->grid_w, size, rank, &off, &cnt);
+  ig4_config t = *c;
+  t.grid_t = 1;
+  t.grid_h = 1;
+  t.grid_w = static_cast<int>(cnt);
+  return t;
+}
+
+struct SpWs {
+  BlockWs loc;            // the local block's buffers (q, k, vt, o of the local tokens)
+  void *qg, *kg, *vtg;    // the rank's head group over all L tokens
+  void *og;               // attention output of the head group [B*L][Hg*256]
+  int vtg_ld;
+  size_t bytes;
+};
+
+SpWs sp_ws_layout(const ig4_config *c, int size, int rank, uint8_t *base) {
+  SpWs w{};
+  const ig4_config t = sp_local(c, size, rank);
+  w.loc = block_ws_layout(&t, base);
+  size_t off = w.loc.bytes;
+  const long L = c->T_text + static_cast<long>(c->grid_t) * c->grid_h * c->grid_w;
+  const long Hg = c->H / size;
+  w.vtg_ld = static_cast<int>(round_up(L, 8));
+  auto take = [&](size_t n) -> uint8_t * {
+    uint8_t *p = base ? base + off : nullptr;
+    off += round_up(n, 256);
+    return p;
+  };
+  w.qg = take(2 * c->B * Hg * L * 256);
+  w.kg = take(2 * c->B * Hg * L * 256);
+  w.vtg = take(2 * c->B * Hg * 256 * static_cast<long>(w.vtg_ld));
+  w.og = take(2 * c->B * L * Hg * 256);
+  w.bytes = off;
+  return w;
+}
+
+// Bytes of one exchange chunk from rank s to rank d.  Phase 0 (before
+// attention): q, k [B][Hg][N_s][256] and v^T [B][Hg][256][N_s] of d's head
+// group over s's image tokens.  Phase 1 (after attention): o [B][T + N_d]
+// [Hg*256] of s's head group over d's text and image tokens.
+size_t sp_chunk_bytes(const ig4_config *c, int size, int phase, int s, int d) {
+  const long N = static_cast<long>(c->grid_t) * c->grid_h * c->grid_w;
+  long off = 0, cnt = 0;
+  sp_range(N, size, phase == 0 ? s : d, &off, &cnt);
+  const long Hg = c->H / size;
+  if (phase == 0) return 3ull * 2 * c->B * Hg * cnt * 256;
+  return 2ull * c->B * (c->T_text + cnt) * Hg * 256;
+}
+
+// Offset of the chunk for (s, d) in s's send buffer (chunks ordered by d)
+// or in d's receive buffer (ordered by s).
+size_t sp_chunk_offset(const ig4_config *c, int size, int phase, int s, int d, bool in_send) {
+  size_t off = 0;
+  for (int k = 0; k < (in_send ? d : s); ++k)
+    off += in_send ? sp_chunk_bytes(c, size, phase, s, k) : sp_chunk_bytes(c, size, phase, k, d);
+  return off;
+}
+
+struct JobList {
+  CopyJobs jobs;
+  int n = 0;
+  bool overflow = false;
+  // element offsets and strides; bases are 2-byte element pointers
+  void add(const void *src, long long src_off, void *dst, long long dst_off, int n_b, int n_h,
+           int rows, int row_elems, long long s_b, long long s_h, long long s_r, long long d_b,
+           long long d_h, long long d_r) {
+    if (n_b < 1 || n_h < 1 || rows < 1 || row_elems < 1) return;
+    if (n >= EXCHANGE_MAX_JOBS) {
+      overflow = true;
+      return;
+    }
+    CopyJob &j = jobs.j[n++];
+    j.src = static_cast<const uint16_t *>(src) + src_off;
+    j.dst = static_cast<uint16_t *>(dst) + dst_off;
+    j.n_b = n_b;
+    j.n_h = n_h;
+    j.rows = rows;
+    j.row_elems = row_elems;
+    j.s_b = s_b;
+    j.s_h = s_h;
+    j.s_r = s_r;
+    j.d_b = d_b;
+    j.d_h = d_h;
+    j.d_r = d_r;
+    const long long all = (s_b | s_h | s_r | d_b | d_h | d_r | row_elems);
+    j.vec = (all % 8 == 0) && aligned16(j.src) && aligned16(j.dst);
+  }
+  ig4_status launch(cudaStream_t st, int sms) const {
+    if (overflow) return IG4_ERR_UNSUPPORTED;
+    if (n == 0) return IG4_OK;
+    long most = 0;
+    for (int i = 0; i < n; ++i) {
+      const CopyJob &j = jobs.j[i];
+      const long units = static_cast<long>(j.n_b) * j.n_h * j.rows * (j.vec ? j.row_elems / 8 : j.row_elems);
+      most = std::max(most, units);
+    }
+    const int gx = static_cast<int>(std::max<long>(1, std::min<long>((most + 255) / 256, 4L * sms)));
+    if (launch_pdl(exchange_copy_kernel, dim3(gx, n), dim3(256), 0, st, jobs) != cudaSuccess)
+      return IG4_ERR_CUDA;
+    return last_launch_status();
+  }
+};
+
+}  // namespace
+
+extern "C" {
+
+size_t ig4_tp_workspace_size(const ig4_config *cfg, int tp_size) {
+  if (check_tp(cfg, 0, tp_size) != IG4_OK) return 0;
+  const ig4_config t = tp_local(cfg, tp_size);
+  return block_ws_layout(&t, nullptr).bytes;
+}
+
+ig4_status ig4_block_tp_attention(const ig4_config *cfg, int tp_rank, int tp_size,
+                                  const ig4_block_weights *w, const void *x_in,
+                                  const int32_t *pos, const float *temb, float *partial,
+                                  void *workspace, size_t ws_bytes, void *stream) {
+  BlockWs ws;
+  IG4_TRY(check_tp_call(cfg, tp_rank, tp_size, w, x_in, partial, workspace, ws_bytes, &ws));
+  if (!pos || !temb || !aligned16(temb)) return IG4_ERR_INVALID_ARG;
+  const ig4_config t = tp_local(cfg, tp_size);
+  const int L = cfg->T_text + cfg->grid_t * cfg->grid_h * cfg->grid_w;
+  const int M = cfg->B * L;
+  const int D = cfg->D;
+  const int Ks = t.H * 256;  // this shard's attention output width
+  const bool f8 = is_fp8(cfg->w_dtype);
+  cudaStream_t st = as_stream(stream);
+  Tracer none{nullptr, 0, 0, st};
+  IG4_TRY(block_pre_attention(&t, w, x_in, pos, temb, ws, st, none, false));
+  IG4_TRY(launch_attention(cfg->B, t.H, L, ws.q, ws.k, ws.vt, ws.vt_ld, ws.o, st));
+  if (f8) IG4_TRY(launch_quantize(M, Ks, ws.o, ws.oq, ws.o_scale, st));
+  return launch_partial(cfg->B, L, D, Ks, f8 ? ws.oq : ws.o, f8, ws.o_scale, w->w_o, w->s_o,
+                        ws.mod + 2 * D, 6 * D, tp_rank == 0 ? x_in : nullptr, cfg->x_dtype,
+                        partial, st);
+}
+
+ig4_status ig4_block_tp_mlp(const ig4_config *cfg, int tp_rank, int tp_size,
+                            const ig4_block_weights *w, const void *x1, float *partial,
+                            void *workspace, size_t ws_bytes, void *stream) {
+  BlockWs ws;
+  IG4_TRY(check_tp_call(cfg, tp_rank, tp_size, w, x1, partial, workspace, ws_bytes, &ws));
+  const ig4_config t = tp_local(cfg, tp_size);
+  const int L = cfg->T_text + cfg->grid_t * cfg->grid_h * cfg->grid_w;
+  const int M = cfg->B * L;
+  const int D = cfg->D, Is = t.I;
+  const bool f8 = is_fp8(cfg->w_dtype);
+  const int hdt = f8 ? IG4_E4M3 : IG4_BF16;
+  cudaStream_t st = as_stream(stream);
+  IG4_TRY(launch_norm(M, L, D, x1, cfg->x_dtype, ws.mod + 3 * D, ws.mod + 4 * D, 6 * D, cfg->eps,
+                      ws.h, hdt, ws.h_scale, 0, 0, 0, st));
+  IG4_TRY(launch_swiglu(M, Is, D, ws.h, f8, ws.h_scale, w->w_gate, w->w_up, w->s_gate, w->s_up,
+                        ws.u, st));
+  if (f8) IG4_TRY(launch_quantize(M, Is, ws.u, ws.uq, ws.u_scale, st));
+  return launch_partial(cfg->B, L, D, Is, f8 ? ws.uq : ws.u, f8, ws.u_scale, w->w_down,
+                        w->s_down, ws.mod + 5 * D, 6 * D, tp_rank == 0 ? x1 : nullptr,
+                        cfg->x_dtype, partial, st);
+}
+
+ig4_status ig4_tp_reduce(long long n, int n_src, const float *const *src, void *out,
+                         int out_dtype, void *stream) {
+  if (n < 0 || n % 8 || n_src < 1 || n_src > TP_MAX_RANKS || !src || !out || !aligned16(out))
+    return IG4_ERR_INVALID_ARG;
+  if (out_dtype != IG4_F32 && out_dtype != IG4_BF16) return IG4_ERR_INVALID_ARG;
+  TpSources ps{};
+  for (int r = 0; r < n_src; ++r) {
+    if (!src[r] || !aligned16(src[r])) return IG4_ERR_INVALID_ARG;
+    ps.p[r] = src[r];
+  }
+  if (n == 0) return IG4_OK;
+  DeviceInfo *di = nullptr;
+  IG4_TRY(device_info(&di));
+  const long n8 = n / 8;
+  const int grid = static_cast<int>(std::min<long>((n8 + 255) / 256, 8L * di->sms));
+  const cudaError_t e =
+      out_dtype == IG4_F32
+          ? launch_pdl(tp_reduce_kernel<float>, dim3(grid), dim3(256), 0, as_stream(stream), ps,
+                       n_src, static_cast<float *>(out), n8)
+          : launch_pdl(tp_reduce_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0,
+                       as_stream(stream), ps, n_src, static_cast<__nv_bfloat16 *>(out), n8);
+  if (e != cudaSuccess) return IG4_ERR_CUDA;
+  return last_launch_status();
+}
+
+ig4_status ig4_sp_image_range(const ig4_config *cfg, int sp_size, int sp_rank, int *img_off,
+                              int *img_count) {
+  IG4_TRY(check_sp(cfg, sp_rank, sp_size));
+  if (!img_off || !img_count) return IG4_ERR_INVALID_ARG;
+  long off = 0, cnt = 0;
+  sp_range(static_cast<long>(cfg->grid_t) * cfg->grid_h * cfg->grid_w, sp_size, sp_rank, &off,
+           &cnt);
+  *img_off = static_cast<int>(off);
+  *img_count = static_cast<int>(cnt);
+  return IG4_OK;
+}
+
+ig4_status ig4_sp_positions(const ig4_config *cfg, int sp_size, int sp_rank, int32_t *pos_out,
+                            int out_on_device, void *stream) {
+  IG4_TRY(check_sp(cfg, sp_rank, sp_size));
+  if (!pos_out) return IG4_ERR_INVALID_ARG;
+  long off = 0, cnt = 0;
+  sp_range(static_cast<long>(cfg->grid_t) * cfg->grid_h * cfg->grid_w, sp_size, sp_rank, &off,
+           &cnt);
+  const int T = cfg->T_text;
+  const long Ls = T + cnt;
+  if (out_on_device) {
+    if (!aligned16(pos_out)) return IG4_ERR_INVALID_ARG;
+    mrope_positions_kernel<<<static_cast<int>((Ls + 255) / 256), 256, 0, as_stream(stream)>>>(
+        T, cfg->grid_t, cfg->grid_h, cfg->grid_w, static_cast<int>(off), static_cast<int>(cnt),
+        pos_out);
+    return last_launch_status();
+  }
+  const long hw = static_cast<long>(cfg->grid_h) * cfg->grid_w;
+  for (long l = 0; l < T; ++l)
+    pos_out[l] = pos_out[Ls + l] = pos_out[2 * Ls + l] = static_cast<int32_t>(l);
+  for (long i = 0; i < cnt; ++i) {
+    const long n = off + i;
+    const long tt = n / hw, rem = n % hw;
+    pos_out[T + i] = static_cast<int32_t>(T + tt);
+    pos_out[Ls + T + i] = static_cast<int32_t>(T + rem / cfg->grid_w);
+    pos_out[2 * Ls + T + i] = static_cast<int32_t>(T + rem % cfg->grid_w);
+  }
+  return IG4_OK;
+}
+
+size_t ig4_sp_workspace_size(const ig4_config *cfg, int sp_size, int sp_rank) {
+  if (check_sp(cfg, sp_rank, sp_size) != IG4_OK) return 0;
+  return sp_ws_layout(cfg, sp_size, sp_rank, nullptr).bytes;
+}
+
+size_t ig4_sp_exchange_bytes(const ig4_config *cfg, int sp_size, int phase, int src_rank,
+                             int dst_rank) {
+  if (check_sp(cfg, 0, sp_size) != IG4_OK || (phase != 0 && phase != 1) || src_rank < 0 ||
+      src_rank >= sp_size || dst_rank < 0 || dst_rank >= sp_size)
+    return 0;
+  return sp_chunk_bytes(cfg, sp_size, phase, src_rank, dst_rank);
+}
+
+ig4_status ig4_block_sp_pre(const ig4_config *cfg, int sp_rank, int sp_size,
+                            const ig4_block_weights *w, const void *x_local,
+                            const int32_t *pos_local, const float *temb, void *send,
+                            void *workspace, size_t ws_bytes, void *stream) {
+  IG4_TRY(check_sp(cfg, sp_rank, sp_size));
+  IG4_TRY(check_block_weights(cfg, w));
+  if (!x_local || !pos_local || !temb || !send || !workspace) return IG4_ERR_INVALID_ARG;
+  if (!aligned16(x_local) || !aligned16(temb) || !aligned16(send)) return IG4_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return IG4_ERR_WORKSPACE;
+  const SpWs ws = sp_ws_layout(cfg, sp_size, sp_rank, static_cast<uint8_t *>(workspace));
+  if (ws_bytes < ws.bytes) return IG4_ERR_WORKSPACE;
+  DeviceInfo *di = nullptr;
+  IG4_TRY(device_info(&di));
+  cudaStream_t st = as_stream(stream);
+  const ig4_config t = sp_local(cfg, sp_size, sp_rank);
+  Tracer none{nullptr, 0, 0, st};
+  IG4_TRY(block_pre_attention(&t, w, x_local, pos_local, temb, ws.loc, st, none, false));
+  // pack: to rank d, head group d of q, k, v^T over this rank's image tokens
+  const int T = cfg->T_text, B = cfg->B, H = cfg->H, Hg = H / sp_size;
+  const long Ls = T + t.grid_w, Ns = t.grid_w;
+  const long vld = ws.loc.vt_ld;
+  JobList jl;
+  for (int d = 0; d < sp_size; ++d) {
+    uint8_t *ch = static_cast<uint8_t *>(send) + sp_chunk_offset(cfg, sp_size, 0, sp_rank, d, true);
+    const long part = static_cast<long>(B) * Hg * Ns * 256;  // elements per part
+    for (int which = 0; which < 2; ++which)
+      jl.add(which == 0 ? ws.loc.q : ws.loc.k, (static_cast<long>(d) * Hg * Ls + T) * 256,
+             ch + which * 2 * part, 0, B, Hg, static_cast<int>(Ns), 256, H * Ls * 256, Ls * 256,
+             256, Hg * Ns * 256, Ns * 256, 256);
+    jl.add(ws.loc.vt, static_cast<long>(d) * Hg * 256 * vld + T, ch + 2 * 2 * part, 0, B, Hg, 256,
+           static_cast<int>(Ns), H * 256 * vld, 256 * vld, vld, Hg * 256 * Ns, 256 * Ns, Ns);
+  }
+  return jl.launch(st, di->sms);
+}
+
+ig4_status ig4_block_sp_attention(const ig4_config *cfg, int sp_rank, int sp_size,
+                                  const void *recv, void *send_o, void *workspace,
+                                  size_t ws_bytes, void *stream) {
+  IG4_TRY(check_sp(cfg, sp_rank, sp_size));
+  if (!recv || !send_o || !workspace || !aligned16(recv) || !aligned16(send_o))
+    return IG4_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return IG4_ERR_WORKSPACE;
+  const SpWs ws = sp_ws_layout(cfg, sp_size, sp_rank, static_cast<uint8_t *>(workspace));
+  if (ws_bytes < ws.bytes) return IG4_ERR_WORKSPACE;
+  DeviceInfo *di = nullptr;
+  IG4_TRY(device_info(&di));
+  cudaStream_t st = as_stream(stream);
+  const int T = cfg->T_text, B = cfg->B, H = cfg->H, Hg = H / sp_size, r = sp_rank;
+  const long N = static_cast<long>(cfg->grid_t) * cfg->grid_h * cfg->grid_w;
+  const long L = T + N;
+  const ig4_config t = sp_local(cfg, sp_size, r);
+  const long Ls = T + t.grid_w;
+  const long vld = ws.loc.vt_ld, gld = ws.vtg_ld;
+  // unpack: text rows from this rank's own q, k, v^T (head group r), image
+  // rows of every source rank from its chunk
+  JobList jl;
+  for (int which = 0; which < 2; ++which)
+    jl.add(which == 0 ? ws.loc.q : ws.loc.k, static_cast<long>(r) * Hg * Ls * 256,
+           which == 0 ? ws.qg : ws.kg, 0, B, Hg, T, 256, H * Ls * 256, Ls * 256, 256,
+           Hg * L * 256, L * 256, 256);
+  jl.add(ws.loc.vt, static_cast<long>(r) * Hg * 256 * vld, ws.vtg, 0, B, Hg, 256, T,
+         H * 256 * vld, 256 * vld, vld, Hg * 256 * gld, 256 * gld, gld);
+  for (int s = 0; s < sp_size; ++s) {
+    long off = 0, Ns = 0;
+    sp_range(N, sp_size, s, &off, &Ns);
+    const uint8_t *ch =
+        static_cast<const uint8_t *>(recv) + sp_chunk_offset(cfg, sp_size, 0, s, r, false);
+    const long part = static_cast<long>(B) * Hg * Ns * 256;
+    for (int which = 0; which < 2; ++which)
+      jl.add(ch + which * 2 * part, 0, which == 0 ? ws.qg : ws.kg, (T + off) * 256, B, Hg,
+             static_cast<int>(Ns), 256, Hg * Ns * 256, Ns * 256, 256, Hg * L * 256, L * 256, 256);
+    jl.add(ch + 2 * 2 * part, 0, ws.vtg, T + off, B, Hg, 256, static_cast<int>(Ns),
+           Hg * 256 * Ns, 256 * Ns, Ns, Hg * 256 * gld, 256 * gld, gld);
+  }
+  IG4_TRY(jl.launch(st, di->sms));
+  // attention of head group r over all L tokens
+  IG4_TRY(launch_attention(B, Hg, static_cast<int>(L), ws.qg, ws.kg, ws.vtg, ws.vtg_ld, ws.og,
+                           st));
+  // pack: to rank d, the text rows and d's image rows of o (head group r)
+  JobList jo;
+  const long W = static_cast<long>(Hg) * 256;
+  for (int d = 0; d < sp_size; ++d) {
+    long off = 0, Nd = 0;
+    sp_range(N, sp_size, d, &off, &Nd);
+    uint8_t *ch = static_cast<uint8_t *>(send_o) + sp_chunk_offset(cfg, sp_size, 1, r, d, true);
+    jo.add(ws.og, 0, ch, 0, B, 1, T, static_cast<int>(W), L * W, 0, W, (T + Nd) * W, 0, W);
+    jo.add(ws.og, (T + off) * W, ch, T * W, B, 1, static_cast<int>(Nd), static_cast<int>(W),
+           L * W, 0, W, (T + Nd) * W, 0, W);
+  }
+  return jo.launch(st, di->sms);
+}
+
+ig4_status ig4_block_sp_post(const ig4_config *cfg, int sp_rank, int sp_size,
+                             const ig4_block_weights *w, const void *x_local, void *x_out_local,
+                             const void *recv_o, void *workspace, size_t ws_bytes,
+                             void *stream) {
+  IG4_TRY(check_sp(cfg, sp_rank, sp_size));
+  IG4_TRY(check_block_weights(cfg, w));
+  if (!x_local || !x_out_local || !recv_o || !workspace) return IG4_ERR_INVALID_ARG;
+  if (!aligned16(x_local) || !aligned16(x_out_local) || !aligned16(recv_o))
+    return IG4_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return IG4_ERR_WORKSPACE;
+  const SpWs ws = sp_ws_layout(cfg, sp_size, sp_rank, static_cast<uint8_t *>(workspace));
+  if (ws_bytes < ws.bytes) return IG4_ERR_WORKSPACE;
+  const ig4_config t = sp_local(cfg, sp_size, sp_rank);
+  const long Ls = cfg->T_text + static_cast<long>(t.grid_w);
+  const size_t xbytes = (cfg->x_dtype == IG4_F32 ? 4 : 2) * static_cast<size_t>(cfg->B) * Ls * cfg->D;
+  const uint8_t *xi = static_cast<const uint8_t *>(x_local);
+  const uint8_t *xo = static_cast<const uint8_t *>(x_out_local);
+  if (xi < xo + xbytes && xo < xi + xbytes) return IG4_ERR_INVALID_ARG;
+  DeviceInfo *di = nullptr;
+  IG4_TRY(device_info(&di));
+  cudaStream_t st = as_stream(stream);
+  const int B = cfg->B, Hg = cfg->H / sp_size;
+  const long W = static_cast<long>(Hg) * 256, D = cfg->D;
+  // unpack: o columns of head group s from rank s's chunk
+  JobList jl;
+  for (int s = 0; s < sp_size; ++s) {
+    const uint8_t *ch = static_cast<const uint8_t *>(recv_o) +
+                        sp_chunk_offset(cfg, sp_size, 1, s, sp_rank, false);
+    jl.add(ch, 0, ws.loc.o, s * W, B, 1, static_cast<int>(Ls), static_cast<int>(W), Ls * W, 0, W,
+           Ls * D, 0, D);
+  }
+  IG4_TRY(jl.launch(st, di->sms));
+  Tracer none{nullptr, 0, 0, st};
+  return block_post_attention(&t, w, x_local, x_out_local, ws.loc, st, none);
 }
 
 }  // extern "C"

@@ -200,11 +200,13 @@ struct EpiStore {
 };
 
 // Gated residual: x_out[row, col] = x_res[row, col] + gate[b, col] * acc,
-// b = row / L (the AdaLN gate of the row's sample).
-template <int BN, bool FP8, typename XT>
+// b = row / L (the AdaLN gate of the row's sample).  x_res may be null (no
+// residual: a tensor-parallel shard's partial sum); x_out may have another
+// type than x_res (fp32 partial sums).
+template <int BN, bool FP8, typename XT, typename OT = XT>
 struct EpiResidGate {
   const XT *x_res;
-  XT *x_out;
+  OT *x_out;
   const float *gate;
   int gate_stride;
   int L, M, N;
@@ -232,10 +234,15 @@ struct EpiResidGate {
       float g[32], x[32];
       load32_f32_ldg(grow + c, g);
       const long off = static_cast<long>(row) * N + n0 + c;
-      load32_x<XT>(x_res + off, x);
+      if (x_res != nullptr) {
+        load32_x<XT>(x_res + off, x);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[i] = 0.0f;
+      }
 #pragma unroll
       for (int i = 0; i < 32; ++i) x[i] = fmaf(g[i], v[i], x[i]);
-      store32_x<XT>(x_out + off, x);
+      store32_x<OT>(x_out + off, x);
     }
   }
 };

@@ -372,15 +372,18 @@ __global__ void dequant_e4m3_rows_kernel(const uint8_t *__restrict__ q, const fl
 }
 
 // ---------------------------------------------------------- positions
-__global__ void mrope_positions_kernel(int T, int gt, int gh, int gw, int32_t *__restrict__ pos) {
-  const int L = T + gt * gh * gw;
+// Positions of the T text tokens and of the n_img image tokens starting at
+// image index img_off (the whole grid: img_off = 0, n_img = gt * gh * gw).
+__global__ void mrope_positions_kernel(int T, int gt, int gh, int gw, int img_off, int n_img,
+                                       int32_t *__restrict__ pos) {
+  const int L = T + n_img;
   const int l = blockIdx.x * blockDim.x + threadIdx.x;
   if (l >= L) return;
   int pt, ph, pw;
   if (l < T) {
     pt = ph = pw = l;
   } else {
-    const int n = l - T;
+    const int n = l - T + img_off;
     const int hw = gh * gw;
     const int t = n / hw;
     const int rem = n - t * hw;

@@ -118,6 +118,22 @@ _sig("ig4_denoise_workspace_size", [ctypes.POINTER(Config), _i], ctypes.c_size_t
 _sig("ig4_denoise_step", [ctypes.POINTER(Config), ctypes.POINTER(StackWeights),
                           ctypes.POINTER(StackWeights), _vp, _vp, _vp, _vp, _vp, _vp, _f, _f, _f,
                           _vp, ctypes.c_size_t, _vp])
+_sig("ig4_tp_workspace_size", [ctypes.POINTER(Config), _i], ctypes.c_size_t)
+_sig("ig4_block_tp_attention", [ctypes.POINTER(Config), _i, _i, ctypes.POINTER(BlockWeights), _vp,
+                                _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp])
+_sig("ig4_block_tp_mlp", [ctypes.POINTER(Config), _i, _i, ctypes.POINTER(BlockWeights), _vp, _vp,
+                          _vp, ctypes.c_size_t, _vp])
+_sig("ig4_tp_reduce", [ctypes.c_longlong, _i, ctypes.POINTER(_vp), _vp, _i, _vp])
+_sig("ig4_sp_image_range", [ctypes.POINTER(Config), _i, _i, ctypes.POINTER(_i), ctypes.POINTER(_i)])
+_sig("ig4_sp_positions", [ctypes.POINTER(Config), _i, _i, _vp, _i, _vp])
+_sig("ig4_sp_workspace_size", [ctypes.POINTER(Config), _i, _i], ctypes.c_size_t)
+_sig("ig4_sp_exchange_bytes", [ctypes.POINTER(Config), _i, _i, _i, _i], ctypes.c_size_t)
+_sig("ig4_block_sp_pre", [ctypes.POINTER(Config), _i, _i, ctypes.POINTER(BlockWeights), _vp, _vp,
+                          _vp, _vp, _vp, ctypes.c_size_t, _vp])
+_sig("ig4_block_sp_attention", [ctypes.POINTER(Config), _i, _i, _vp, _vp, _vp, ctypes.c_size_t,
+                                _vp])
+_sig("ig4_block_sp_post", [ctypes.POINTER(Config), _i, _i, ctypes.POINTER(BlockWeights), _vp, _vp,
+                           _vp, _vp, ctypes.c_size_t, _vp])
 _sig("ig4_last_device_error", [_vp])
 _sig("ig4_selftest_timeout", [_i, _vp])
 
@@ -129,8 +145,11 @@ EXPORTED = ("ig4_status_string", "ig4_abi_version", "ig4_mrope_positions", "ig4_
             "ig4_stack_forward", "ig4_stack_forward_tapped", "ig4_nvfp4_scale_bytes", "ig4_nvfp4_pack_scales",
             "ig4_nvfp4_linear", "ig4_nvfp4_quantize", "ig4_text_cond_workspace_size", "ig4_text_cond_project",
             "ig4_flow_schedule", "ig4_guidance_schedule", "ig4_cfg_euler",
-            "ig4_denoise_workspace_size", "ig4_denoise_step", "ig4_last_device_error",
-            "ig4_selftest_timeout")
+            "ig4_denoise_workspace_size", "ig4_denoise_step", "ig4_tp_workspace_size",
+            "ig4_block_tp_attention", "ig4_block_tp_mlp", "ig4_tp_reduce", "ig4_sp_image_range",
+            "ig4_sp_positions", "ig4_sp_workspace_size", "ig4_sp_exchange_bytes",
+            "ig4_block_sp_pre", "ig4_block_sp_attention", "ig4_block_sp_post",
+            "ig4_last_device_error", "ig4_selftest_timeout")
 
 
 def library():
@@ -449,3 +468,86 @@ def ig4_last_device_error(stream=None) -> int:
 
 def ig4_selftest_timeout(wait_us: int, stream=None):
     _check(_lib.ig4_selftest_timeout(wait_us, _stream(stream)), "ig4_selftest_timeout")
+
+
+# ------------------------------------------------------- multi-GPU layouts
+
+def ig4_tp_workspace_size(cfg: Config, tp_size: int) -> int:
+    return int(_lib.ig4_tp_workspace_size(ctypes.byref(cfg), tp_size))
+
+
+def ig4_block_tp_attention(cfg: Config, tp_rank: int, tp_size: int, w: BlockWeights, x_in, pos,
+                           temb, partial, workspace, stream=None):
+    """partial (fp32 [B*L, D]) = [rank 0] x + gate_msa * (o_r W_o,r^T) of this head shard."""
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(_lib.ig4_block_tp_attention(ctypes.byref(cfg), tp_rank, tp_size, ctypes.byref(w),
+                                       _ptr(x_in), _ptr(pos), _ptr(temb), _ptr(partial),
+                                       _ptr(workspace), ws_bytes, _stream(stream)),
+           "ig4_block_tp_attention")
+
+
+def ig4_block_tp_mlp(cfg: Config, tp_rank: int, tp_size: int, w: BlockWeights, x1, partial,
+                     workspace, stream=None):
+    """partial = [rank 0] x1 + gate_mlp * (u_r W_down,r^T) of this FFN shard."""
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(_lib.ig4_block_tp_mlp(ctypes.byref(cfg), tp_rank, tp_size, ctypes.byref(w), _ptr(x1),
+                                 _ptr(partial), _ptr(workspace), ws_bytes, _stream(stream)),
+           "ig4_block_tp_mlp")
+
+
+def ig4_tp_reduce(srcs: list, out, stream=None):
+    """out = sum of the fp32 tensors in srcs (device-accessible), in list order."""
+    arr = (_vp * len(srcs))(*[t.data_ptr() for t in srcs])
+    _check(_lib.ig4_tp_reduce(out.numel(), len(srcs), arr, _ptr(out), dtype_code(out),
+                              _stream(stream)), "ig4_tp_reduce")
+
+
+def ig4_sp_image_range(cfg: Config, sp_size: int, sp_rank: int) -> tuple:
+    off, cnt = _i(), _i()
+    _check(_lib.ig4_sp_image_range(ctypes.byref(cfg), sp_size, sp_rank, ctypes.byref(off),
+                                   ctypes.byref(cnt)), "ig4_sp_image_range")
+    return off.value, cnt.value
+
+
+def ig4_sp_positions(cfg: Config, sp_size: int, sp_rank: int, device=None, stream=None):
+    """int32 [3, T + N_r] positions of rank sp_rank's local tokens."""
+    _, cnt = ig4_sp_image_range(cfg, sp_size, sp_rank)
+    out = torch.empty((3, cfg.T_text + cnt), dtype=torch.int32,
+                      device=device if device is not None else "cpu")
+    on_dev = 1 if out.is_cuda else 0
+    _check(_lib.ig4_sp_positions(ctypes.byref(cfg), sp_size, sp_rank, _ptr(out), on_dev,
+                                 _stream(stream) if on_dev else None), "ig4_sp_positions")
+    return out
+
+
+def ig4_sp_workspace_size(cfg: Config, sp_size: int, sp_rank: int) -> int:
+    return int(_lib.ig4_sp_workspace_size(ctypes.byref(cfg), sp_size, sp_rank))
+
+
+def ig4_sp_exchange_bytes(cfg: Config, sp_size: int, phase: int, src_rank: int,
+                          dst_rank: int) -> int:
+    return int(_lib.ig4_sp_exchange_bytes(ctypes.byref(cfg), sp_size, phase, src_rank, dst_rank))
+
+
+def ig4_block_sp_pre(cfg: Config, sp_rank: int, sp_size: int, w: BlockWeights, x_local,
+                     pos_local, temb, send, workspace, stream=None):
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(_lib.ig4_block_sp_pre(ctypes.byref(cfg), sp_rank, sp_size, ctypes.byref(w),
+                                 _ptr(x_local), _ptr(pos_local), _ptr(temb), _ptr(send),
+                                 _ptr(workspace), ws_bytes, _stream(stream)), "ig4_block_sp_pre")
+
+
+def ig4_block_sp_attention(cfg: Config, sp_rank: int, sp_size: int, recv, send_o, workspace,
+                           stream=None):
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(_lib.ig4_block_sp_attention(ctypes.byref(cfg), sp_rank, sp_size, _ptr(recv),
+                                       _ptr(send_o), _ptr(workspace), ws_bytes, _stream(stream)),
+           "ig4_block_sp_attention")
+
+
+def ig4_block_sp_post(cfg: Config, sp_rank: int, sp_size: int, w: BlockWeights, x_local,
+                      x_out_local, recv_o, workspace, stream=None):
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(_lib.ig4_block_sp_post(ctypes.byref(cfg), sp_rank, sp_size, ctypes.byref(w),
+                                  _ptr(x_local), _ptr(x_out_local), _ptr(recv_o), _ptr(workspace),
+                                  ws_bytes, _stream(stream)), "ig4_block_sp_post")
