@@ -280,12 +280,19 @@ ig4_status launch_adaln(int B, int A, int N, const float *temb, const void *w, i
   const int rows_per_cta = (ADALN_THREADS / 32) * ADALN_ROWS_PER_WARP;
   const int grid = (N + rows_per_cta - 1) / rows_per_cta;
   const int smem = B * A * 4;
-  const cudaError_t e =
-      is_fp8(w_dtype)
-          ? launch_pdl(adaln_kernel<true>, dim3(grid), dim3(ADALN_THREADS), smem, st, temb, w,
-                       w_scale, bias, mod, B, A, N)
-          : launch_pdl(adaln_kernel<false>, dim3(grid), dim3(ADALN_THREADS), smem, st, temb, w,
-                       w_scale, bias, mod, B, A, N);
+  const bool f8 = is_fp8(w_dtype);
+  const int mv = (A * (f8 ? 1 : 2) + 511) / 512;  // 16-byte vectors per lane and row
+  cudaError_t e;
+  if (f8)
+    e = mv <= 1 ? launch_pdl(adaln_kernel<true, 1>, dim3(grid), dim3(ADALN_THREADS), smem, st,
+                             temb, w, w_scale, bias, mod, B, A, N)
+                : launch_pdl(adaln_kernel<true, 2>, dim3(grid), dim3(ADALN_THREADS), smem, st,
+                             temb, w, w_scale, bias, mod, B, A, N);
+  else
+    e = mv <= 2 ? launch_pdl(adaln_kernel<false, 2>, dim3(grid), dim3(ADALN_THREADS), smem, st,
+                             temb, w, w_scale, bias, mod, B, A, N)
+                : launch_pdl(adaln_kernel<false, 4>, dim3(grid), dim3(ADALN_THREADS), smem, st,
+                             temb, w, w_scale, bias, mod, B, A, N);
   if (e != cudaSuccess) return IG4_ERR_CUDA;
   return last_launch_status();
 }
@@ -308,6 +315,27 @@ ig4_status launch_norm_t(int rows, int L, int D, const void *x, const float *shi
   if (smem > 48 * 1024) return IG4_ERR_UNSUPPORTED;
   const int nv = (D / 8 + 31) / 32;
   const XT *xp = static_cast<const XT *>(x);
+  if constexpr (sizeof(XT) == 2) {
+    // bf16 stream up to D = 4608: 16 warps per CTA, a row per warp
+    const long per_cta2 = (static_cast<long>(rows) + di->sms - 1) / di->sms;
+    const int rpc2 = static_cast<int>(std::max<long>(NORM2_WARPS, per_cta2));
+    const dim3 grid2((nb + rpc2 - 1) / rpc2, B);
+    const size_t smem2 = 4ull * (D / 8) * sizeof(float4);
+#define IG4_NORM2_CASE(NV)                                                                      \
+  if (nv <= NV) {                                                                              \
+    if (launch_pdl(norm_modulate_rows_kernel<FP8, NV>, grid2, dim3(NORM2_THREADS), smem2, st,  \
+                   xp, shift, scale, mod_stride, L, D, eps, h, hs, remap_n, remap_L,           \
+                   remap_off, rpc2) != cudaSuccess)                                            \
+      return IG4_ERR_CUDA;                                                                     \
+    return last_launch_status();                                                               \
+  }
+    IG4_NORM2_CASE(2)
+    IG4_NORM2_CASE(4)
+    IG4_NORM2_CASE(8)
+    IG4_NORM2_CASE(12)
+    IG4_NORM2_CASE(18)
+#undef IG4_NORM2_CASE
+  }
 #define IG4_NORM_CASE(NV)                                                                        \
   if (nv <= NV) {                                                                                \
     if (launch_pdl(norm_modulate_kernel<XT, FP8, NV>, grid, dim3(NORM_THREADS), smem, st, xp,   \

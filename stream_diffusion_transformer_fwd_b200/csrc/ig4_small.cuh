@@ -12,29 +12,32 @@ namespace ig4 {
 // mod[b][n] = sum_k SiLU(temb[b][k]) W[n][k] (* s[n]) + bias[n].
 // One warp per group of 4 output rows: the warp first issues the loads of all
 // 4 weight rows (up to 4 16-byte vectors per lane and row, A * esize <= 2048
-// bytes), then reduces them, so 16 loads per lane are in flight at once.
-// B <= 8 samples share each weight read; SiLU(temb) sits in shared memory.
+// bytes), so 16 loads per lane are in flight at once; then, sample by sample,
+// it reads the activations its lanes need once (as float4, from SiLU(temb)
+// in shared memory) and applies them to all 4 rows.  B <= 8 samples share
+// each weight read.
 constexpr int ADALN_THREADS = 256;
 constexpr int ADALN_ROWS_PER_WARP = 4;
-constexpr int ADALN_MAXV = 4;
 
-template <bool FP8>
+// MAXV: 16-byte weight vectors per lane and row, ceil(A * esize / 512)
+template <bool FP8, int ADALN_MAXV>
 __global__ void __launch_bounds__(ADALN_THREADS)
     adaln_kernel(const float *__restrict__ temb, const void *__restrict__ w,
                  const float *__restrict__ w_scale, const float *__restrict__ bias,
                  float *__restrict__ mod, int B, int A, int N) {
   pdl_wait();
   pdl_trigger();
-  extern __shared__ float s_act[];  // [B][A]
+  extern __shared__ float4 s_act4[];  // [B][A / 4]
+  float *s_act = reinterpret_cast<float *>(s_act4);
   for (int i = threadIdx.x; i < B * A; i += blockDim.x) s_act[i] = silu_f(temb[i]);
   __syncthreads();
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int n_base = (blockIdx.x * (ADALN_THREADS / 32) + warp) * ADALN_ROWS_PER_WARP;
   // bytes per weight row = A * esize; each lane takes 16-byte vectors lane, lane+32, ...
-  const int esize = FP8 ? 1 : 2;
+  constexpr int esize = FP8 ? 1 : 2;
+  constexpr int EPV = 16 / esize;  // weights per 16-byte vector
   const int vec_per_row = A * esize / 16;
-  const int elems_per_vec = 16 / esize;
   uint4 q[ADALN_ROWS_PER_WARP][ADALN_MAXV];
 #pragma unroll
   for (int rr = 0; rr < ADALN_ROWS_PER_WARP; ++rr) {
@@ -47,53 +50,58 @@ __global__ void __launch_bounds__(ADALN_THREADS)
       if (n < N && v < vec_per_row) q[rr][j] = __ldg(row + v);
     }
   }
+  float sc[ADALN_ROWS_PER_WARP], bn[ADALN_ROWS_PER_WARP];
 #pragma unroll
   for (int rr = 0; rr < ADALN_ROWS_PER_WARP; ++rr) {
     const int n = n_base + rr;
-    if (n >= N) break;
-    float acc[8];
+    sc[rr] = (FP8 && n < N) ? __ldg(w_scale + n) : 1.0f;
+    bn[rr] = (bias != nullptr && n < N) ? __ldg(bias + n) : 0.0f;
+  }
+  for (int b = 0; b < B; ++b) {
+    float acc[ADALN_ROWS_PER_WARP];
 #pragma unroll
-    for (int b = 0; b < 8; ++b) acc[b] = 0.0f;
+    for (int rr = 0; rr < ADALN_ROWS_PER_WARP; ++rr) acc[rr] = 0.0f;
 #pragma unroll
     for (int j = 0; j < ADALN_MAXV; ++j) {
       const int v = lane + 32 * j;
       if (v >= vec_per_row) break;
-      float wv[16];
-      if (FP8) {
-        const uint8_t *c = reinterpret_cast<const uint8_t *>(&q[rr][j]);
+      // the activations of this lane's vector: EPV consecutive floats
+      float a[EPV];
+      const float4 *a4 = s_act4 + (b * A + v * EPV) / 4;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) wv[e] = e4m3_to_f(c[e]);
-      } else {
-        const uint32_t u[4] = {q[rr][j].x, q[rr][j].y, q[rr][j].z, q[rr][j].w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          wv[2 * e] = __uint_as_float(u[e] << 16);
-          wv[2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
-        }
+      for (int e = 0; e < EPV / 4; ++e) {
+        const float4 t = a4[e];
+        a[4 * e] = t.x;
+        a[4 * e + 1] = t.y;
+        a[4 * e + 2] = t.z;
+        a[4 * e + 3] = t.w;
       }
-      const int k0 = v * elems_per_vec;
 #pragma unroll
-      for (int b = 0; b < 8; ++b) {
-        if (b >= B) break;
-        const float *a = s_act + b * A + k0;
-        float s = 0.0f;
-        if (FP8) {
+      for (int rr = 0; rr < ADALN_ROWS_PER_WARP; ++rr) {
+        float wv[EPV];
+        if constexpr (FP8) {
+          const uint8_t *c = reinterpret_cast<const uint8_t *>(&q[rr][j]);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) s = fmaf(wv[e], a[e], s);
+          for (int e = 0; e < 16; ++e) wv[e] = e4m3_to_f(c[e]);
         } else {
+          const uint32_t u[4] = {q[rr][j].x, q[rr][j].y, q[rr][j].z, q[rr][j].w};
 #pragma unroll
-          for (int e = 0; e < 8; ++e) s = fmaf(wv[e], a[e], s);
+          for (int e = 0; e < 4; ++e) {
+            wv[2 * e] = __uint_as_float(u[e] << 16);
+            wv[2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
+          }
         }
-        acc[b] += s;
+        float s2 = 0.0f;
+#pragma unroll
+        for (int e = 0; e < EPV; ++e) s2 = fmaf(wv[e], a[e], s2);
+        acc[rr] += s2;
       }
     }
-    const float sc = FP8 ? __ldg(w_scale + n) : 1.0f;
-    const float bn = bias ? __ldg(bias + n) : 0.0f;
 #pragma unroll
-    for (int b = 0; b < 8; ++b) {
-      if (b >= B) break;
-      const float t = warp_sum(acc[b]);
-      if (lane == 0) mod[static_cast<long>(b) * N + n] = fmaf(t, sc, bn);
+    for (int rr = 0; rr < ADALN_ROWS_PER_WARP; ++rr) {
+      const int n = n_base + rr;
+      const float t = warp_sum(acc[rr]);
+      if (lane == 0 && n < N) mod[static_cast<long>(b) * N + n] = fmaf(t, sc[rr], bn[rr]);
     }
   }
 }
@@ -288,6 +296,135 @@ __global__ void rope_table_kernel(const int32_t *__restrict__ pos, int L, double
   sincos(ang, &s, &c);
   cos_out[idx] = static_cast<float>(c);
   sin_out[idx] = static_cast<float>(s);
+}
+
+// RMSNorm + modulate for a bf16 stream, the block's layout: 16 warps per
+// CTA, one row per warp at a time, the row held in registers (NV 16-byte
+// vectors per lane, no prefetch: the 16 warps keep 16 rows of loads in
+// flight per SM).  (1 + scale) and shift are staged in shared memory as four
+// planes of float4 -- elements 8v..8v+3 and 8v+4..8v+7 of each -- so the
+// lanes of a warp read consecutive 16-byte words (no bank conflicts).
+constexpr int NORM2_THREADS = 512;
+constexpr int NORM2_WARPS = NORM2_THREADS / 32;
+
+template <bool OUT_FP8, int NV>
+__global__ void __launch_bounds__(NORM2_THREADS, 1)
+    norm_modulate_rows_kernel(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ shift,
+                              const float *__restrict__ scale, int mod_stride, int L, int D,
+                              float eps, void *__restrict__ h_out, float *__restrict__ h_scale,
+                              int remap_n, int remap_L, int remap_off, int rows_per_cta) {
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ float4 smod[];  // planes: scale lo, scale hi, shift lo, shift hi [D/8]
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int nb = remap_n > 0 ? remap_n : L;  // rows per sample
+  const int b = blockIdx.y;
+  const int r_begin = blockIdx.x * rows_per_cta;
+  const int r_end = min(r_begin + rows_per_cta, nb);
+  if (r_begin >= nb) return;
+  const int nvec = D / 8;
+  const float4 *sc4 = reinterpret_cast<const float4 *>(scale + static_cast<long>(b) * mod_stride);
+  const float4 *sh4 = reinterpret_cast<const float4 *>(shift + static_cast<long>(b) * mod_stride);
+  for (int i = threadIdx.x; i < D / 4; i += NORM2_THREADS) {
+    float4 s = __ldg(sc4 + i);
+    s.x += 1.0f;
+    s.y += 1.0f;
+    s.z += 1.0f;
+    s.w += 1.0f;
+    const int v = i >> 1, hi = i & 1;
+    smod[hi * nvec + v] = s;
+    smod[(2 + hi) * nvec + v] = __ldg(sh4 + i);
+  }
+  __syncthreads();
+  for (int rr = r_begin + warp; rr < r_end; rr += NORM2_WARPS) {
+    const long in_row = remap_n > 0 ? static_cast<long>(b) * remap_L + remap_off + rr
+                                    : static_cast<long>(b) * L + rr;
+    const uint4 *xr = reinterpret_cast<const uint4 *>(x + in_row * D);
+    uint4 q[NV];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int vi = lane + 32 * i;
+      if (vi < nvec) q[i] = __ldg(xr + vi);
+    }
+    float ss = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      if (lane + 32 * i < nvec) {
+        const uint32_t u[4] = {q[i].x, q[i].y, q[i].z, q[i].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float a = __uint_as_float(u[e] << 16);
+          const float c = __uint_as_float(u[e] & 0xFFFF0000u);
+          ss = fmaf(a, a, ss);
+          ss = fmaf(c, c, ss);
+        }
+      }
+    }
+    ss = warp_sum(ss);
+    const float rstd = rsqrtf(ss / static_cast<float>(D) + eps);
+    const long r = static_cast<long>(b) * nb + rr;  // output row
+    // h of vector i of this row
+    auto modulated = [&](int i, float (&h)[8]) {
+      const int vi = lane + 32 * i;
+      const uint32_t u[4] = {q[i].x, q[i].y, q[i].z, q[i].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        h[2 * e] = __uint_as_float(u[e] << 16);
+        h[2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
+      }
+      const float4 s0 = smod[vi], s1 = smod[nvec + vi];
+      const float4 t0 = smod[2 * nvec + vi], t1 = smod[3 * nvec + vi];
+      const float scv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+      const float shv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) h[e] = fmaf(h[e] * rstd, scv[e], shv[e]);
+    };
+    if constexpr (OUT_FP8) {
+      float amax = 0.0f;
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        if (lane + 32 * i < nvec) {
+          float h[8];
+          modulated(i, h);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(h[e]));
+        }
+      }
+      amax = warp_max(amax);
+      const float qs = amax > 0.0f ? amax / 448.0f : 1.0f;
+      const float inv = 1.0f / qs;
+      uint8_t *hr = static_cast<uint8_t *>(h_out) + r * D;
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        const int vi = lane + 32 * i;
+        if (vi < nvec) {
+          float h[8];
+          modulated(i, h);
+          uint2 w;
+          w.x = static_cast<uint32_t>(pack_e4m3x2(h[0] * inv, h[1] * inv)) |
+                (static_cast<uint32_t>(pack_e4m3x2(h[2] * inv, h[3] * inv)) << 16);
+          w.y = static_cast<uint32_t>(pack_e4m3x2(h[4] * inv, h[5] * inv)) |
+                (static_cast<uint32_t>(pack_e4m3x2(h[6] * inv, h[7] * inv)) << 16);
+          reinterpret_cast<uint2 *>(hr)[vi] = w;
+        }
+      }
+      if (lane == 0) h_scale[r] = qs;
+    } else {
+      __nv_bfloat16 *hr = static_cast<__nv_bfloat16 *>(h_out) + r * D;
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        const int vi = lane + 32 * i;
+        if (vi < nvec) {
+          float h[8];
+          modulated(i, h);
+          reinterpret_cast<uint4 *>(hr)[vi] =
+              make_uint4(pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]),
+                         pack_bf16x2(h[4], h[5]), pack_bf16x2(h[6], h[7]));
+        }
+      }
+    }
+  }
 }
 
 // ------------------------------------------------------ FP8 row quantiser
