@@ -184,6 +184,19 @@ ig4_status ig4_qkv_project(int B, int L, int D, int H, const void *h, int h_dtyp
 ig4_status ig4_joint_attention(int B, int H, int L, const void *q, const void *k,
                                const void *vt, int vt_ld, void *o_out, void *stream);
 
+/* ig4_joint_attention with a workspace (256-byte aligned, at least
+ * ig4_joint_attention_workspace_size(B, H, L) bytes; 0 when no workspace is
+ * needed).  With it, a persistent grid of one CTA per SM takes equal shares
+ * of all (query tile, key tile) pairs, whatever the number of (b, h, query
+ * tile) items, and the items split between CTAs are merged by a second
+ * kernel (pieces in a fixed order, so the result is deterministic); the
+ * block entry points work this way.  Without it (workspace NULL) every item
+ * is one CTA. */
+size_t ig4_joint_attention_workspace_size(int B, int H, int L);
+ig4_status ig4_joint_attention_ws(int B, int H, int L, const void *q, const void *k,
+                                  const void *vt, int vt_ld, void *o_out, void *workspace,
+                                  size_t ws_bytes, void *stream);
+
 /* ------------------------------------------------ gated residual linear ---
  * Gated residual linear (survey page, "单 block 内部": AdaLN gates modulate
  * the attention and MLP residual paths): x_out[r][n] = x_res[r][n] +

@@ -422,8 +422,40 @@ ig4_status launch_qkv(int B, int L, int D, int H, const void *h, int h_dtype, co
   return launch_gemm<256, false, false>(ma, mb, mb, M, ntn, D, e, st);
 }
 
+// The attention kernel's grid: one CTA per (b, h, query tile) item when
+// there are no more items than CTAs (or no partial slots), else one CTA per
+// SM taking the items round-robin, with the last partial round's items split
+// into pieces of key tiles (the kernel's AttSched).
+long att_items(int B, int H, int L) {
+  return static_cast<long>(B) * H * ((L + ATT_BN - 1) / ATT_BN);
+}
+int att_grid(int B, int H, int L, int sms, bool have_part) {
+  const long items = att_items(B, H, L);
+  const int g = std::min(sms, ATT_MAX_CTAS);
+  if (!have_part || items <= g) return static_cast<int>(items);
+  return g;
+}
+// Tail items split into pieces (0: none), as the kernel's AttSched computes it.
+int att_split_items(int B, int H, int L, int grid) {
+  const long items = att_items(B, H, L);
+  const int nkv = (L + ATT_BN - 1) / ATT_BN;
+  const long rem = items % grid;
+  if (rem == 0) return 0;
+  const long k = std::max<long>(1, std::min<long>(nkv, grid / rem));
+  return k > 1 ? static_cast<int>(rem) : 0;
+}
+// Bytes of partial slots the grid may need: one per CTA (0 when no item can
+// be split: a single key tile per item).
+size_t att_part_bytes(int B, int H, int L) {
+  const long nkv = (L + ATT_BN - 1) / ATT_BN;
+  if (nkv <= 1 || att_items(B, H, L) <= 1) return 0;
+  return static_cast<size_t>(ATT_MAX_CTAS) * ATT_PART_BYTES;
+}
+
+// part: att_part_bytes(B, H, L) bytes of workspace for the balanced grid, or
+// nullptr (one CTA per item).
 ig4_status launch_attention(int B, int H, int L, const void *q, const void *k, const void *vt,
-                            int vt_ld, void *o, cudaStream_t st) {
+                            int vt_ld, void *o, void *part, cudaStream_t st) {
   CUtensorMap mq, mk, mv;
   const long BH = static_cast<long>(B) * H;
   IG4_TRY(map_3d_bf16(&mq, q, 256, L, BH, 256, static_cast<long>(L) * 256, 64, ATT_BM));
@@ -432,11 +464,29 @@ ig4_status launch_attention(int B, int H, int L, const void *q, const void *k, c
   // 128-key tile takes two of them.
   IG4_TRY(map_3d_bf16(&mv, vt, L, 256, BH, vt_ld, 256L * vt_ld, 64, 256));
   IG4_TRY(allow_smem(attention_kernel, ATT_SMEM_BYTES));
-  dim3 grid((L + ATT_BM - 1) / ATT_BM, H, B);
-  if (launch_pdl(attention_kernel, grid, dim3(ATT_THREADS), ATT_SMEM_BYTES, st, mq, mk, mv,
-                 static_cast<__nv_bfloat16 *>(o), L, H) != cudaSuccess)
+  DeviceInfo *di = nullptr;
+  IG4_TRY(device_info(&di));
+  const bool have_part = part != nullptr && att_part_bytes(B, H, L) > 0;
+  const long items = att_items(B, H, L);
+  const int grid = att_grid(B, H, L, di->sms, have_part);
+  if (BH > (1L << 30) || items > (1L << 30)) return IG4_ERR_UNSUPPORTED;
+  __nv_bfloat16 *op = static_cast<__nv_bfloat16 *>(o);
+  uint8_t *pp = static_cast<uint8_t *>(part);
+  if (launch_pdl(attention_kernel, dim3(grid), dim3(ATT_THREADS), ATT_SMEM_BYTES, st, mq, mk, mv,
+                 op, L, H, static_cast<int>(BH), pp) != cudaSuccess)
     return IG4_ERR_CUDA;
-  return last_launch_status();
+  IG4_TRY(last_launch_status());
+  const int split = att_split_items(B, H, L, grid);
+  if (split > 0) {
+    // merge the pieces of the split tail items
+    if (launch_pdl(attention_combine_kernel, dim3(split, ATT_BM / ATT_COMBINE_ROWS),
+                   dim3(ATT_COMBINE_THREADS), 0, st,
+                   static_cast<const uint8_t *>(pp), op, L, H, static_cast<int>(BH), grid) !=
+        cudaSuccess)
+      return IG4_ERR_CUDA;
+    IG4_TRY(last_launch_status());
+  }
+  return IG4_OK;
 }
 
 // Tile width for an output of N columns: the candidate (256, 192, 128 that
@@ -783,6 +833,7 @@ struct BlockWs {
   void *uq;       // e4m3 [M][I]
   float *u_scale;
   void *h_sf, *u_sf;  // packed NVFP4 scales of h2 and u (NVFP4-mixed FFN)
+  void *att_part;     // attention partial slots: the u buffer (u is written after attention)
   int vt_ld;
   size_t bytes;
 };
@@ -813,7 +864,9 @@ BlockWs block_ws_layout(const ig4_config *c, uint8_t *base) {
   w.o = take(2 * M * D);
   w.oq = take(f8 ? M * D : 0);
   w.o_scale = reinterpret_cast<float *>(take(f8 ? sizeof(float) * M : 0));
-  w.u = take(2 * M * I);
+  w.u = take(std::max<size_t>(2 * M * I, att_part_bytes(c->B, static_cast<int>(H),
+                                                         static_cast<int>(L))));
+  w.att_part = att_part_bytes(c->B, static_cast<int>(H), static_cast<int>(L)) ? w.u : nullptr;
   w.uq = take(f8 ? M * I : 0);
   w.u_scale = reinterpret_cast<float *>(take(f8 ? sizeof(float) * M : 0));
   // NVFP4 FFN: h2 codes reuse oq (M D / 2 bytes), u codes reuse uq
@@ -949,7 +1002,7 @@ ig4_status block_forward_impl(const ig4_config *c, const ig4_block_weights *w, c
   Tracer none{nullptr, 0, 0, st};
   Tracer &t = tr ? *tr : none;
   IG4_TRY(block_pre_attention(c, w, x_in, pos, temb, ws, st, t, rope_ready));
-  IG4_TRY(launch_attention(c->B, c->H, L, ws.q, ws.k, ws.vt, ws.vt_ld, ws.o, st));
+  IG4_TRY(launch_attention(c->B, c->H, L, ws.q, ws.k, ws.vt, ws.vt_ld, ws.o, ws.att_part, st));
   IG4_TRY(t.mark());
   return block_post_attention(c, w, x_in, x_out, ws, st, t);
 }
@@ -1090,12 +1143,27 @@ ig4_status ig4_qkv_project(int B, int L, int D, int H, const void *h, int h_dtyp
 
 ig4_status ig4_joint_attention(int B, int H, int L, const void *q, const void *k, const void *vt,
                                int vt_ld, void *o_out, void *stream) {
+  return ig4_joint_attention_ws(B, H, L, q, k, vt, vt_ld, o_out, nullptr, 0, stream);
+}
+
+size_t ig4_joint_attention_workspace_size(int B, int H, int L) {
+  if (B < 1 || H < 1 || L < 1) return 0;
+  return att_part_bytes(B, H, L);
+}
+
+ig4_status ig4_joint_attention_ws(int B, int H, int L, const void *q, const void *k,
+                                  const void *vt, int vt_ld, void *o_out, void *workspace,
+                                  size_t ws_bytes, void *stream) {
   if (B < 1 || H < 1 || L < 1 || !q || !k || !vt || !o_out || vt_ld < L || vt_ld % 8)
     return IG4_ERR_INVALID_ARG;
   if (H > 65535 || B > 65535) return IG4_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(vt) || !aligned16(o_out))
     return IG4_ERR_INVALID_ARG;
-  return launch_attention(B, H, L, q, k, vt, vt_ld, o_out, as_stream(stream));
+  if (workspace != nullptr) {
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return IG4_ERR_WORKSPACE;
+    if (ws_bytes < att_part_bytes(B, H, L)) return IG4_ERR_WORKSPACE;
+  }
+  return launch_attention(B, H, L, q, k, vt, vt_ld, o_out, workspace, as_stream(stream));
 }
 
 ig4_status ig4_gated_residual_linear(int B, int L, int N, int K, const void *a, int a_dtype,
@@ -1615,6 +1683,7 @@ struct SpWs {
   BlockWs loc;            // the local block's buffers (q, k, vt, o of the local tokens)
   void *qg, *kg, *vtg;    // the rank's head group over all L tokens
   void *og;               // attention output of the head group [B*L][Hg*256]
+  void *part;             // its attention partial slots (or nullptr)
   int vtg_ld;
   size_t bytes;
 };
@@ -1636,6 +1705,8 @@ SpWs sp_ws_layout(const ig4_config *c, int size, int rank, uint8_t *base) {
   w.kg = take(2 * c->B * Hg * L * 256);
   w.vtg = take(2 * c->B * Hg * 256 * static_cast<long>(w.vtg_ld));
   w.og = take(2 * c->B * L * Hg * 256);
+  const size_t pb = att_part_bytes(c->B, static_cast<int>(Hg), static_cast<int>(L));
+  w.part = pb ? take(pb) : nullptr;
   w.bytes = off;
   return w;
 }
@@ -1733,7 +1804,7 @@ ig4_status ig4_block_tp_attention(const ig4_config *cfg, int tp_rank, int tp_siz
   cudaStream_t st = as_stream(stream);
   Tracer none{nullptr, 0, 0, st};
   IG4_TRY(block_pre_attention(&t, w, x_in, pos, temb, ws, st, none, false));
-  IG4_TRY(launch_attention(cfg->B, t.H, L, ws.q, ws.k, ws.vt, ws.vt_ld, ws.o, st));
+  IG4_TRY(launch_attention(cfg->B, t.H, L, ws.q, ws.k, ws.vt, ws.vt_ld, ws.o, ws.att_part, st));
   if (f8) IG4_TRY(launch_quantize(M, Ks, ws.o, ws.oq, ws.o_scale, st));
   return launch_partial(cfg->B, L, D, Ks, f8 ? ws.oq : ws.o, f8, ws.o_scale, w->w_o, w->s_o,
                         ws.mod + 2 * D, 6 * D, tp_rank == 0 ? x_in : nullptr, cfg->x_dtype,
@@ -1918,7 +1989,7 @@ ig4_status ig4_block_sp_attention(const ig4_config *cfg, int sp_rank, int sp_siz
   IG4_TRY(jl.launch(st, di->sms));
   // attention of head group r over all L tokens
   IG4_TRY(launch_attention(B, Hg, static_cast<int>(L), ws.qg, ws.kg, ws.vtg, ws.vtg_ld, ws.og,
-                           st));
+                           ws.part, st));
   // pack: to rank d, the text rows and d's image rows of o (head group r)
   JobList jo;
   const long W = static_cast<long>(Hg) * 256;

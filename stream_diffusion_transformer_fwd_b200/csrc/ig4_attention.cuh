@@ -1,7 +1,18 @@
 // ig4_attention.cuh - fused flash-style joint attention, head_dim 256, sm_100a.
 //
-// One CTA computes o for 128 query rows of one (sample, head), walking the
-// keys in tiles of 128:
+// Work: for every (sample, head) and every 128-row query tile (an "item"),
+// the 128-key tiles of the whole sequence.  A persistent grid of G CTAs (one
+// per SM) takes the items round-robin, whole: in round r CTA c takes item
+// r G + c, so the CTAs running at the same time share the K and V of a few
+// heads through L2.  The rem items of the last, partial round are split
+// into k = min(key tiles, G / rem) pieces of consecutive key tiles, piece p
+// of tail item j on CTA j k + p, so the last round keeps the SMs busy too.
+// A piece stores its unnormalised O (bf16), row maximum m and row sum l into
+// a partial slot, and attention_combine_kernel merges the pieces of each tail
+// item afterwards, in piece order (deterministic).  With fewer items than
+// SMs (or no workspace for partial slots) every CTA takes one whole item.
+//
+// Per key tile of a segment:
 //   S_j = Q K_j^T     16 tcgen05.mma (M=128, N=128, K=16), Q and K_j from
 //                     shared memory, fp32 scores into TMEM;
 //   softmax           one thread per query row, exp2 domain, in registers;
@@ -16,13 +27,16 @@
 // PV_{j-1}: it only needs PV_{j-2} (long done) before it overwrites P_{j%2},
 // and PV_{j-1} only when it has to rescale O.
 //
-// Shared memory: Q (64 KB, loaded once) and a ring of five 32 KB slots that
-// TMA fills with half tiles in the order the MMAs consume them - K_0, K_1,
-// V_0, K_2, V_1, K_3, V_2, ... - each split in two halves (K: head dims
-// [0,128) and [128,256); V: keys [0,64) and [64,128)), so a slot is released
-// as soon as the MMAs of its half have run.  V arrives transposed ([256,
-// keys], keys contiguous), so every shared-memory operand is K-major with the
-// 128-byte swizzle.
+// Shared memory: Q (64 KB) and a ring of five 32 KB slots that TMA fills with
+// half tiles in the order the MMAs consume them - per segment K_0, K_1, V_0,
+// K_2, V_1, K_3, V_2, ... - each split in two halves (K: head dims [0,128)
+// and [128,256); V: keys [0,64) and [64,128)), so a slot is released as soon
+// as the MMAs of its half have run.  V arrives transposed ([256, keys], keys
+// contiguous), so every shared-memory operand is K-major with the 128-byte
+// swizzle.  Across segments the pipeline keeps running: the producer loads
+// the next segment's Q as soon as the last S MMA of the current one has read
+// Q, the next segment's S MMAs run while the softmax warps drain O, and the
+// next segment's first PV waits only for that drain.
 //
 // The running maximum used for the exponentials only moves when a row's
 // maximum grows by more than 8 (a factor 2^8), so O is rescaled rarely;
@@ -34,10 +48,19 @@
 // on different events (scores read out vs. probabilities written), so one
 // keeps the tensor pipe fed while the other waits.
 //
-// Barrier parity: every barrier a role waits on completes at most one phase
-// ahead of that wait, so try_wait.parity never mistakes a later phase for the
-// awaited one (this is why P-ready and PV-done exist once per P buffer).
-// Every wait is bounded.
+// Barrier parity: try_wait.parity only tells the awaited phase from the one
+// before it, so every wait must start when the barrier is at most one phase
+// ahead of, and not behind, the awaited phase (this is why P-ready and
+// PV-done exist once per P buffer).  The ring's full barriers have two
+// consumers (K halves for the S issuer, V halves for the PV issuer) and TMA
+// loads may land out of order, so one consumer could otherwise start waiting
+// for half h while the load of half h - 5 into the same slot (for the other
+// consumer) is still in flight, and take the completed phase of half h - 10
+// for the one it awaits.  The producer therefore publishes in shared memory
+// how many halves it has passed its empty wait for; a consumer waits for
+// that count to exceed h before it waits on full: the slot's previous phase
+// has then completed.  Phases count tiles (and segments) over the whole
+// range.  Every wait is bounded.
 #pragma once
 
 #include "ig4_ptx.cuh"
@@ -61,10 +84,16 @@ constexpr uint32_t ATT_TMEM_O = 256;
 // log2(e) / sqrt(256)
 constexpr float ATT_SCALE_LOG2 = 0.09016844005556021f;
 constexpr float ATT_RESCALE_THRESHOLD = 8.0f;
+// The largest persistent grid (one partial slot per CTA is reserved).
+constexpr int ATT_MAX_CTAS = 160;
+// A partial slot: unnormalised O bf16 [128][256], then m and l fp32 [128] each.
+constexpr long ATT_PART_O_BYTES = static_cast<long>(ATT_BM) * ATT_DH * 2;
+constexpr long ATT_PART_BYTES = ATT_PART_O_BYTES + 2L * ATT_BM * 4;
 
-// The order in which the ring receives whole tiles ("items"): K_0; K_1 (if
-// any); then, for each tile j, V_j followed by K_{j+2} (if that tile
-// exists).  Each item travels as two 32 KB halves.
+// The order in which the ring receives a segment's whole tiles ("items"):
+// K_0; K_1 (if any); then, for each tile j, V_j followed by K_{j+2} (if that
+// tile exists).  Tile indices are relative to the segment.  Each item
+// travels as two 32 KB halves.
 struct AttRing {
   int nkv;
   __device__ __forceinline__ int items() const { return 2 * nkv; }
@@ -88,10 +117,62 @@ struct AttRing {
   __device__ __forceinline__ int item_v(int t) const { return min(2 * t + 2, 2 * nkv - 1); }
 };
 
+// One segment of a CTA's work: key tiles [t0, t0 + n) of item `item`;
+// `slot` is the partial slot of a tail piece (-1 for a whole item).
+struct AttSeg {
+  int item, t0, n, slot;
+};
+
+// The persistent grid's schedule (computed the same way by the host).
+struct AttSched {
+  int n_items, G, nkv;
+  int rounds;  // whole rounds: items [0, rounds * G)
+  int rem;     // items of the last, partial round
+  int k;       // pieces per tail item (1: tail items run whole)
+  __device__ __forceinline__ AttSched(int n_items_, int G_, int nkv_)
+      : n_items(n_items_), G(G_), nkv(nkv_) {
+    rounds = n_items / G;
+    rem = n_items - rounds * G;
+    k = rem > 0 ? max(1, min(nkv, G / rem)) : 1;
+  }
+  __device__ __forceinline__ int segments(int c) const { return rounds + (c < rem * k ? 1 : 0); }
+  __device__ __forceinline__ AttSeg seg(int c, int s) const {
+    if (s < rounds) return AttSeg{s * G + c, 0, nkv, -1};
+    const int j = c / k, p = c - j * k;
+    const int t0 = p * nkv / k, t1 = (p + 1) * nkv / k;
+    return AttSeg{rounds * G + j, t0, t1 - t0, k > 1 ? c : -1};
+  }
+  // key tiles of the CTA's segments before segment s (every earlier one is whole)
+  __device__ __forceinline__ long tiles_before(int s) const {
+    return static_cast<long>(min(s, rounds)) * nkv;
+  }
+};
+
+// Wait (bounded, like mbar_wait) until the producer has passed its empty
+// wait for half h of the ring, i.e. *passed > h.
+__device__ __forceinline__ bool att_wait_passed(const volatile int *passed, long h,
+                                                volatile int *abort_flag) {
+  if (*passed > h) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 8; ++i) {
+      if (*passed > h) return true;
+      __nanosleep(32);  // leave the issue slots to the softmax warp of this SMSP
+    }
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+      atomicOr(&g_device_error, DEVERR_TIMEOUT);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
 __global__ void __launch_bounds__(ATT_THREADS, 1)
     attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, __nv_bfloat16 *__restrict__ o_out,
-                     int L, int H) {
+                     int L, int H, int n_bh, uint8_t *__restrict__ part) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -99,24 +180,25 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + ATT_OFF_BAR);
   uint64_t *full = bars + 0;      // [ATT_SLOTS]
   uint64_t *empty = bars + 5;     // [ATT_SLOTS]
-  uint64_t *q_full = bars + 10;   // Q landed
+  uint64_t *q_full = bars + 10;   // Q of a segment landed
   uint64_t *s_full = bars + 11;   // S_j in TMEM
   uint64_t *s_free = bars + 12;   // S_j read out of TMEM (one arrival per softmax warp)
   uint64_t *p_full = bars + 13;   // [2] P_j in TMEM buffer j%2 (one arrival per softmax warp)
   uint64_t *pv_done = bars + 15;  // [2] PV_j complete (buffer j%2)
   uint64_t *drain_s = bars + 17;
   uint64_t *drain_pv = bars + 18;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 20);
+  uint64_t *q_empty = bars + 19;  // the last S MMA of a segment has read Q
+  uint64_t *o_free = bars + 20;   // O of a segment drained (one arrival per softmax warp)
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 22);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  volatile int *passed = reinterpret_cast<volatile int *>(tmem_slot + 2);  // halves past empty
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int q0 = blockIdx.x * ATT_BM;
-  const int h = blockIdx.y;
-  const int b = blockIdx.z;
-  const int bh = b * H + h;
-  const int nkv = (L + ATT_BN - 1) / ATT_BN;
-  const AttRing ring_order{nkv};
+  const int nkv = (L + ATT_BN - 1) / ATT_BN;  // key tiles = query tiles
+  const AttSched sched(n_bh * nkv, static_cast<int>(gridDim.x), nkv);
+  const int cta = blockIdx.x;
+  const int n_seg = sched.segments(cta);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < ATT_SLOTS; ++s) {
@@ -132,7 +214,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     mbar_init(&pv_done[1], 1);
     mbar_init(drain_s, 1);
     mbar_init(drain_pv, 1);
+    mbar_init(q_empty, 1);
+    mbar_init(o_free, 4);
     *abort_flag = 0;
+    *passed = 0;
     fence_mbar_init();
   }
   if (warp == 4 && lane == 0) {
@@ -154,31 +239,50 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   if (warp == 4) {
     if (lane == 0) {
       // ------------------------------------------------ TMA producer
-      mbar_arrive_expect_tx(q_full, ATT_Q_BYTES);
-      for (int c = 0; c < 4; ++c) tma_load_3d(smem + c * 16384, &tmQ, q_full, c * 64, q0, bh);
-      const int n = 2 * ring_order.items();  // half items
-      int i = 0;
+      long i = 0;  // half items issued over the range
       bool ok = true;
-      for (; i < n; ++i) {
-        const int slot = i % ATT_SLOTS;
-        const uint32_t ph = static_cast<uint32_t>(i / ATT_SLOTS) & 1;
-        if (!mbar_wait(&empty[slot], ph ^ 1, abort_flag)) { ok = false; break; }
-        mbar_arrive_expect_tx(&full[slot], ATT_SLOT_BYTES);
-        uint8_t *dst = ring + slot * ATT_SLOT_BYTES;
-        const int half = i & 1;
-        int t = 0;
-        if (ring_order.kind(i >> 1, &t) == 1) {
-          for (int c = 0; c < 2; ++c)
-            tma_load_3d(dst + c * 16384, &tmK, &full[slot], (2 * half + c) * 64, t * ATT_BN, bh);
-        } else {
-          tma_load_3d(dst, &tmV, &full[slot], t * ATT_BN + half * 64, 0, bh);
+      int k = 0;
+      int q_issued = -1;  // the last segment whose Q load was issued
+      for (; k < n_seg && ok; ++k) {
+        const AttSeg sg = sched.seg(cta, k);
+        const int bh = sg.item / nkv;
+        const int q0 = (sg.item - bh * nkv) * ATT_BM;
+        // Q: free once the last S MMA of the previous segment has run
+        if (k > 0 && !mbar_wait(q_empty, static_cast<uint32_t>(k - 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(q_full, ATT_Q_BYTES);
+        for (int c = 0; c < 4; ++c) tma_load_3d(smem + c * 16384, &tmQ, q_full, c * 64, q0, bh);
+        q_issued = k;
+        const AttRing ro{sg.n};
+        const int n = 2 * ro.items();  // half items of this segment
+        for (int hi = 0; hi < n; ++hi, ++i) {
+          const int slot = static_cast<int>(i % ATT_SLOTS);
+          const uint32_t ph = static_cast<uint32_t>(i / ATT_SLOTS) & 1;
+          if (!mbar_wait(&empty[slot], ph ^ 1, abort_flag)) { ok = false; break; }
+          // half i - 5 is consumed, so full[slot] has completed its phase
+          __threadfence_block();
+          *passed = static_cast<int>(i + 1);
+          mbar_arrive_expect_tx(&full[slot], ATT_SLOT_BYTES);
+          uint8_t *dst = ring + slot * ATT_SLOT_BYTES;
+          const int half = hi & 1;
+          int t = 0;
+          if (ro.kind(hi >> 1, &t) == 1) {
+            for (int c = 0; c < 2; ++c)
+              tma_load_3d(dst + c * 16384, &tmK, &full[slot], (2 * half + c) * 64,
+                          (sg.t0 + t) * ATT_BN, bh);
+          } else {
+            tma_load_3d(dst, &tmV, &full[slot], (sg.t0 + t) * ATT_BN + half * 64, 0, bh);
+          }
         }
       }
       if (!ok) {
         // let the loads already issued land before the shared memory goes away
-        mbar_wait(q_full, 0, nullptr, WAIT_LIMIT_NS / 4);
-        for (int k = (i > ATT_SLOTS ? i - ATT_SLOTS : 0); k < i; ++k)
-          mbar_wait(&full[k % ATT_SLOTS], static_cast<uint32_t>(k / ATT_SLOTS) & 1, nullptr,
+        if (q_issued >= 0)
+          mbar_wait(q_full, static_cast<uint32_t>(q_issued) & 1, nullptr, WAIT_LIMIT_NS / 4);
+        for (long j = (i > ATT_SLOTS ? i - ATT_SLOTS : 0); j < i; ++j)
+          mbar_wait(&full[j % ATT_SLOTS], static_cast<uint32_t>(j / ATT_SLOTS) & 1, nullptr,
                     WAIT_LIMIT_NS / 4);
       }
     }
@@ -187,30 +291,43 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       // ------------------------------------------------ S issuer: S_t = Q K_t^T
       constexpr uint32_t IDESC_S = idesc_bf16(ATT_BM, ATT_BN);
       const uint32_t q_base = smem_u32(smem);
-      bool ok = mbar_wait(q_full, 0, abort_flag);
-      for (int t = 0; t < nkv && ok; ++t) {
-        // the S buffer is free once the softmax has read S_{t-1}
-        if (t > 0 && !mbar_wait(s_free, static_cast<uint32_t>(t - 1) & 1, abort_flag)) break;
-        const int u = ring_order.item_k(t);
-        for (int half = 0; half < 2 && ok; ++half) {
-          const int i = 2 * u + half;
-          const int slot = i % ATT_SLOTS;
-          if (!mbar_wait(&full[slot], static_cast<uint32_t>(i / ATT_SLOTS) & 1, abort_flag)) {
+      bool ok = true;
+      long gt = 0;  // tiles over the CTA's segments
+      for (int k = 0; k < n_seg && ok; ++k) {
+        const AttSeg sg = sched.seg(cta, k);
+        const AttRing ro{sg.n};
+        const long ibase = 4 * sched.tiles_before(k);  // half items before this segment
+        if (!mbar_wait(q_full, static_cast<uint32_t>(k) & 1, abort_flag)) break;
+        for (int t = 0; t < sg.n && ok; ++t, ++gt) {
+          // the S buffer is free once the softmax has read S_{gt-1}
+          if (gt > 0 && !mbar_wait(s_free, static_cast<uint32_t>(gt - 1) & 1, abort_flag)) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          const uint32_t k_base = smem_u32(ring + slot * ATT_SLOT_BYTES);
+          const int it = ro.item_k(t);
+          for (int half = 0; half < 2 && ok; ++half) {
+            const long i = ibase + 2 * it + half;
+            const int slot = static_cast<int>(i % ATT_SLOTS);
+            if (!att_wait_passed(passed, i, abort_flag) ||
+                !mbar_wait(&full[slot], static_cast<uint32_t>(i / ATT_SLOTS) & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t k_base = smem_u32(ring + slot * ATT_SLOT_BYTES);
 #pragma unroll
-          for (int kq = 0; kq < 8; ++kq) {
-            const int kk = half * 8 + kq;  // K step of 16 head dims
-            const uint64_t ad = sdesc_kmajor_sw128(q_base + (kk >> 2) * 16384 + (kk & 3) * 32);
-            const uint64_t bd = sdesc_kmajor_sw128(k_base + (kq >> 2) * 16384 + (kq & 3) * 32);
-            umma_bf16(tmem + ATT_TMEM_S, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+            for (int kq = 0; kq < 8; ++kq) {
+              const int kk = half * 8 + kq;  // K step of 16 head dims
+              const uint64_t ad = sdesc_kmajor_sw128(q_base + (kk >> 2) * 16384 + (kk & 3) * 32);
+              const uint64_t bd = sdesc_kmajor_sw128(k_base + (kq >> 2) * 16384 + (kq & 3) * 32);
+              umma_bf16(tmem + ATT_TMEM_S, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(&empty[slot]);
           }
-          umma_commit(&empty[slot]);
+          if (ok) umma_commit(s_full);
         }
-        if (ok) umma_commit(s_full);
+        // Q may be replaced once these MMAs have run
+        if (ok) umma_commit(q_empty);
       }
       umma_commit(drain_s);
       mbar_wait(drain_s, 0, nullptr, WAIT_LIMIT_NS / 4);
@@ -220,30 +337,46 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       // ------------------------------------------------ PV issuer: O += P_j V_j
       constexpr uint32_t IDESC_PV = idesc_bf16(ATT_BM, ATT_DH);
       bool ok = true;
-      for (int j = 0; j < nkv && ok; ++j) {
-        const int pb = j & 1;
-        if (!mbar_wait(&p_full[pb], static_cast<uint32_t>(j >> 1) & 1, abort_flag)) break;
-        tc_fence_after();
-        const int u = ring_order.item_v(j);
-        for (int half = 0; half < 2 && ok; ++half) {
-          const int i = 2 * u + half;
-          const int slot = i % ATT_SLOTS;
-          if (!mbar_wait(&full[slot], static_cast<uint32_t>(i / ATT_SLOTS) & 1, abort_flag)) {
+      long gt = 0;
+      for (int k = 0; k < n_seg && ok; ++k) {
+        const AttSeg sg = sched.seg(cta, k);
+        const AttRing ro{sg.n};
+        const long ibase = 4 * sched.tiles_before(k);
+        for (int j = 0; j < sg.n && ok; ++j, ++gt) {
+          const int pb = static_cast<int>(gt & 1);
+          if (!mbar_wait(&p_full[pb], static_cast<uint32_t>(gt >> 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          // the first PV of a segment overwrites O: the previous one's O drained
+          if (j == 0 && k > 0 &&
+              !mbar_wait(o_free, static_cast<uint32_t>(k - 1) & 1, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t v_base = smem_u32(ring + slot * ATT_SLOT_BYTES);
+          const int it = ro.item_v(j);
+          for (int half = 0; half < 2 && ok; ++half) {
+            const long i = ibase + 2 * it + half;
+            const int slot = static_cast<int>(i % ATT_SLOTS);
+            if (!att_wait_passed(passed, i, abort_flag) ||
+                !mbar_wait(&full[slot], static_cast<uint32_t>(i / ATT_SLOTS) & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t v_base = smem_u32(ring + slot * ATT_SLOT_BYTES);
 #pragma unroll
-          for (int kq = 0; kq < 4; ++kq) {
-            const int kk = half * 4 + kq;  // K step of 16 keys
-            const uint64_t bd = sdesc_kmajor_sw128(v_base + kq * 32);
-            umma_bf16_ts(tmem + ATT_TMEM_O, tmem + ATT_TMEM_P + 64 * pb + kk * 8, bd, IDESC_PV,
-                         (j > 0 || kk > 0) ? 1u : 0u);
+            for (int kq = 0; kq < 4; ++kq) {
+              const int kk = half * 4 + kq;  // K step of 16 keys
+              const uint64_t bd = sdesc_kmajor_sw128(v_base + kq * 32);
+              umma_bf16_ts(tmem + ATT_TMEM_O, tmem + ATT_TMEM_P + 64 * pb + kk * 8, bd, IDESC_PV,
+                           (j > 0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit(&empty[slot]);
           }
-          umma_commit(&empty[slot]);
+          if (ok) umma_commit(&pv_done[pb]);
         }
-        if (ok) umma_commit(&pv_done[pb]);
       }
       umma_commit(drain_pv);
       mbar_wait(drain_pv, 0, nullptr, WAIT_LIMIT_NS / 4);
@@ -252,142 +385,172 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     // -------------------------------------------- softmax warps 0..3
     const int r = warp * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    float m_used = -INFINITY;
-    float l_sum = 0.0f;
-    bool ok = true;
     const uint64_t scale2 = f2_pack(ATT_SCALE_LOG2, ATT_SCALE_LOG2);
-
-    for (int j = 0; j < nkv && ok; ++j) {
-      if (!mbar_wait_warp(s_full, static_cast<uint32_t>(j) & 1, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      float t[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float a[32];
-        tmem_ld32(tmem + lane_base + ATT_TMEM_S + c * 32, a);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) t[32 * c + i] = a[i];
-      }
-      // S_j is in registers: the S buffer may take S_{j+1}.
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_free);
-
-      const int kbase = j * ATT_BN;
-      if (kbase + ATT_BN > L) {
-#pragma unroll
-        for (int i = 0; i < 128; ++i)
-          if (kbase + i >= L) t[i] = -INFINITY;
-      }
-      float m4[4] = {t[0], t[1], t[2], t[3]};
-#pragma unroll
-      for (int i = 4; i < 128; i += 8) {
-        m4[0] = fmax3(m4[0], t[i + 0], t[i + 1]);
-        m4[1] = fmax3(m4[1], t[i + 2], t[i + 3]);
-        m4[2] = fmax3(m4[2], t[i + 4], t[i + 5]);
-        m4[3] = fmax3(m4[3], t[i + 6], t[i + 7]);
-      }
-      const float mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * ATT_SCALE_LOG2;
-
-      // Running maximum for this tile (moved only when it grows by more than
-      // the threshold) and the factor that rescales what came before.
-      float m_new = m_used;
-      float f = 1.0f;
-      bool need = false;
-      if (j == 0) {
-        m_new = mx;
-      } else if (mx > m_used + ATT_RESCALE_THRESHOLD) {
-        need = true;
-        m_new = mx;
-        f = exp2_approx(m_used - mx);
-      }
-      const bool any_need = __any_sync(0xffffffffu, need);
-
-      // p = 2^(s * scale - m), packed to bf16 pairs; row sum in fp32 pairs
-      const uint64_t negm2 = f2_pack(-m_new, -m_new);
-      uint32_t pk[64];
-      uint64_t acc[4] = {0, 0, 0, 0};
-#pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const uint64_t x2 = ffma2(f2_pack(t[2 * i], t[2 * i + 1]), scale2, negm2);
-        const float p0 = exp2_approx(f2_lo(x2));
-        const float p1 = exp2_approx(f2_hi(x2));
-        const uint64_t p2 = f2_pack(p0, p1);
-        acc[i & 3] = fadd2(acc[i & 3], p2);
-        pk[i] = pack_bf16x2(p0, p1);
-      }
-      const uint64_t s2 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
-      const float rowsum = f2_lo(s2) + f2_hi(s2);
-
-      const int pb = j & 1;
-      if (j >= 2) {
-        // PV_{j-2} read this P buffer
-        if (!mbar_wait_warp(&pv_done[pb], static_cast<uint32_t>((j >> 1) - 1) & 1, abort_flag)) {
-          ok = false;
-          break;
-        }
-      }
-      if (any_need) {
-        // PV_{j-1} must be done: it writes O
-        if (!mbar_wait_warp(&pv_done[pb ^ 1], static_cast<uint32_t>((j - 1) >> 1) & 1,
-                            abort_flag)) {
-          ok = false;
-          break;
-        }
+    bool ok = true;
+    long gt = 0;
+    for (int k = 0; k < n_seg && ok; ++k) {
+      const AttSeg sg = sched.seg(cta, k);
+      float m_used = -INFINITY;
+      float l_sum = 0.0f;
+      for (int j = 0; j < sg.n; ++j, ++gt) {
+        if (!mbar_wait_warp(s_full, static_cast<uint32_t>(gt) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-#pragma unroll 1
-        for (int c = 0; c < ATT_DH; c += 32) {
-          float o[32];
-          tmem_ld32(tmem + lane_base + ATT_TMEM_O + c, o);
+        float t[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float a[32];
+          tmem_ld32(tmem + lane_base + ATT_TMEM_S + c * 32, a);
           tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= f;
-          tmem_st32(tmem + lane_base + ATT_TMEM_O + c, o);
+          for (int i = 0; i < 32; ++i) t[32 * c + i] = a[i];
         }
+        // S_j is in registers: the S buffer may take S_{j+1}.
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free);
+
+        const int kbase = (sg.t0 + j) * ATT_BN;
+        if (kbase + ATT_BN > L) {
+#pragma unroll
+          for (int i = 0; i < 128; ++i)
+            if (kbase + i >= L) t[i] = -INFINITY;
+        }
+        float m4[4] = {t[0], t[1], t[2], t[3]};
+#pragma unroll
+        for (int i = 4; i < 128; i += 8) {
+          m4[0] = fmax3(m4[0], t[i + 0], t[i + 1]);
+          m4[1] = fmax3(m4[1], t[i + 2], t[i + 3]);
+          m4[2] = fmax3(m4[2], t[i + 4], t[i + 5]);
+          m4[3] = fmax3(m4[3], t[i + 6], t[i + 7]);
+        }
+        const float mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * ATT_SCALE_LOG2;
+
+        // Running maximum for this tile (moved only when it grows by more than
+        // the threshold) and the factor that rescales what came before.
+        float m_new = m_used;
+        float f = 1.0f;
+        bool need = false;
+        if (j == 0) {
+          m_new = mx;
+        } else if (mx > m_used + ATT_RESCALE_THRESHOLD) {
+          need = true;
+          m_new = mx;
+          f = exp2_approx(m_used - mx);
+        }
+        const bool any_need = __any_sync(0xffffffffu, need);
+
+        // p = 2^(s * scale - m), packed to bf16 pairs; row sum in fp32 pairs
+        const uint64_t negm2 = f2_pack(-m_new, -m_new);
+        uint32_t pk[64];
+        uint64_t acc[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const uint64_t x2 = ffma2(f2_pack(t[2 * i], t[2 * i + 1]), scale2, negm2);
+          const float p0 = exp2_approx(f2_lo(x2));
+          const float p1 = exp2_approx(f2_hi(x2));
+          const uint64_t p2 = f2_pack(p0, p1);
+          acc[i & 3] = fadd2(acc[i & 3], p2);
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        const uint64_t s2 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
+        const float rowsum = f2_lo(s2) + f2_hi(s2);
+
+        const int pb = static_cast<int>(gt & 1);
+        if (gt >= 2) {
+          // PV_{gt-2} read this P buffer
+          if (!mbar_wait_warp(&pv_done[pb], static_cast<uint32_t>((gt >> 1) - 1) & 1,
+                              abort_flag)) {
+            ok = false;
+            break;
+          }
+        }
+        if (any_need) {
+          // PV_{gt-1} (same segment, j > 0) must be done: it writes O
+          if (!mbar_wait_warp(&pv_done[pb ^ 1], static_cast<uint32_t>((gt - 1) >> 1) & 1,
+                              abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < ATT_DH; c += 32) {
+            float o[32];
+            tmem_ld32(tmem + lane_base + ATT_TMEM_O + c, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= f;
+            tmem_st32(tmem + lane_base + ATT_TMEM_O + c, o);
+          }
+        }
+        tc_fence_after();
+        {
+          uint32_t w[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) w[i] = pk[i];
+          tmem_st32_u(tmem + lane_base + ATT_TMEM_P + 64 * pb, w);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) w[i] = pk[32 + i];
+          tmem_st32_u(tmem + lane_base + ATT_TMEM_P + 64 * pb + 32, w);
+        }
+        tmem_st_wait();
+        l_sum = l_sum * f + rowsum;
+        m_used = m_new;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[pb]);
+      }
+      if (!ok) break;
+      // ---- the segment's output: O / l (bf16) or the partial (O, m, l)
+      const long gl = gt - 1;
+      if (!mbar_wait_warp(&pv_done[gl & 1], static_cast<uint32_t>(gl >> 1) & 1, abort_flag)) {
+        ok = false;
+        break;
       }
       tc_fence_after();
-      {
-        uint32_t w[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) w[i] = pk[i];
-        tmem_st32_u(tmem + lane_base + ATT_TMEM_P + 64 * pb, w);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) w[i] = pk[32 + i];
-        tmem_st32_u(tmem + lane_base + ATT_TMEM_P + 64 * pb + 32, w);
-      }
-      tmem_st_wait();
-      l_sum = l_sum * f + rowsum;
-      m_used = m_new;
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[pb]);
-    }
-    const int jl = nkv - 1;
-    if (ok && mbar_wait_warp(&pv_done[jl & 1], static_cast<uint32_t>(jl >> 1) & 1, abort_flag)) {
-      tc_fence_after();
+      const int bh = sg.item / nkv;
+      const int q0 = (sg.item - bh * nkv) * ATT_BM;
+      const int b = bh / H, h = bh - (bh / H) * H;
       const int lq = q0 + r;
       const bool valid = lq < L;
-      const float inv = 1.0f / l_sum;
-      __nv_bfloat16 *dst = o_out + (static_cast<long>(b) * L + lq) * (static_cast<long>(H) * ATT_DH) +
-                           h * ATT_DH;
+      const float inv = sg.slot < 0 ? 1.0f / l_sum : 1.0f;
+      __nv_bfloat16 *dst;
+      if (sg.slot < 0) {
+        dst = o_out + (static_cast<long>(b) * L + lq) * (static_cast<long>(H) * ATT_DH) +
+              h * ATT_DH;
+      } else {
+        uint8_t *sp = part + static_cast<long>(sg.slot) * ATT_PART_BYTES;
+        dst = reinterpret_cast<__nv_bfloat16 *>(sp) + static_cast<long>(r) * ATT_DH;
+        float *ml = reinterpret_cast<float *>(sp + ATT_PART_O_BYTES);
+        ml[r] = m_used;
+        ml[ATT_BM + r] = l_sum;
+      }
+      const bool store = valid || sg.slot >= 0;
+      // O in two halves of 128 columns: four TMEM loads in flight per wait
 #pragma unroll 1
-      for (int c = 0; c < ATT_DH; c += 32) {
-        float o[32];
-        tmem_ld32(tmem + lane_base + ATT_TMEM_O + c, o);
-        tmem_ld_wait();
-        if (!valid) continue;
-        uint4 *d = reinterpret_cast<uint4 *>(dst + c);
+      for (int hc = 0; hc < ATT_DH; hc += 128) {
+        float o[4][32];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint4 w;
-          w.x = pack_bf16x2(o[8 * q + 0] * inv, o[8 * q + 1] * inv);
-          w.y = pack_bf16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv);
-          w.z = pack_bf16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv);
-          w.w = pack_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv);
-          d[q] = w;
+        for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_base + ATT_TMEM_O + hc + 32 * c, o[c]);
+        tmem_ld_wait();
+        if (!store) continue;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint4 *d = reinterpret_cast<uint4 *>(dst + hc + 32 * c);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 w;
+            w.x = pack_bf16x2(o[c][8 * q + 0] * inv, o[c][8 * q + 1] * inv);
+            w.y = pack_bf16x2(o[c][8 * q + 2] * inv, o[c][8 * q + 3] * inv);
+            w.z = pack_bf16x2(o[c][8 * q + 4] * inv, o[c][8 * q + 5] * inv);
+            w.w = pack_bf16x2(o[c][8 * q + 6] * inv, o[c][8 * q + 7] * inv);
+            d[q] = w;
+          }
         }
       }
+      // O is in registers or memory: the next segment's first PV may overwrite it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(o_free);
     }
   }
 
@@ -395,6 +558,73 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 5) tmem_dealloc(tmem, ATT_TMEM_COLS);
+}
+
+// Merge of the split tail items: block (j, y) takes rows 8y .. 8y+7 of tail
+// item j, one warp per row; the item's k pieces sit in partial slots
+// j k .. j k + k - 1.  m = max m_p, l = sum l_p 2^(m_p - m),
+// o = sum O_p 2^(m_p - m) / l (pieces in order), stored as bf16.  Lane p
+// holds m and l of piece p (32 pieces at a time) and passes its weight by
+// shuffle; lane i accumulates head dims 8i .. 8i+7.
+constexpr int ATT_COMBINE_THREADS = 256;
+constexpr int ATT_COMBINE_ROWS = ATT_COMBINE_THREADS / 32;
+
+__global__ void __launch_bounds__(ATT_COMBINE_THREADS)
+    attention_combine_kernel(const uint8_t *__restrict__ part, __nv_bfloat16 *__restrict__ o_out,
+                             int L, int H, int n_bh, int G) {
+  pdl_wait();
+  pdl_trigger();
+  const int nkv = (L + ATT_BN - 1) / ATT_BN;
+  const AttSched sched(n_bh * nkv, G, nkv);
+  const int j = blockIdx.x;
+  const int k = sched.k;
+  if (j >= sched.rem || k < 2) return;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int r = blockIdx.y * ATT_COMBINE_ROWS + warp;
+  const int item = sched.rounds * G + j;
+  const int bh = item / nkv;
+  const int q0 = (item - bh * nkv) * ATT_BM;
+  const int lq = q0 + r;
+  if (r >= ATT_BM || lq >= L) return;
+  const int b = bh / H, h = bh - (bh / H) * H;
+  const uint8_t *first = part + static_cast<long>(j) * k * ATT_PART_BYTES;
+  auto ml_of = [&](int p) {
+    return reinterpret_cast<const float *>(first + static_cast<long>(p) * ATT_PART_BYTES +
+                                           ATT_PART_O_BYTES);
+  };
+  float m = -INFINITY;
+  for (int p0 = 0; p0 < k; p0 += 32)
+    if (p0 + lane < k) m = fmaxf(m, ml_of(p0 + lane)[r]);
+  m = warp_max(m);
+  float l = 0.0f, acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  for (int p0 = 0; p0 < k; p0 += 32) {
+    float wgt = 0.0f;
+    if (p0 + lane < k) {
+      const float *ml = ml_of(p0 + lane);
+      wgt = exp2f(ml[r] - m);
+      l = fmaf(ml[ATT_BM + r], wgt, l);
+    }
+    const int n = min(32, k - p0);
+#pragma unroll 4
+    for (int q = 0; q < n; ++q) {
+      const float w = __shfl_sync(0xffffffffu, wgt, q);
+      const uint4 v = reinterpret_cast<const uint4 *>(
+          first + static_cast<long>(p0 + q) * ATT_PART_BYTES + static_cast<long>(r) * ATT_DH * 2)[lane];
+      const uint32_t u4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        acc[2 * e] = fmaf(__uint_as_float(u4[e] << 16), w, acc[2 * e]);
+        acc[2 * e + 1] = fmaf(__uint_as_float(u4[e] & 0xFFFF0000u), w, acc[2 * e + 1]);
+      }
+    }
+  }
+  const float inv = 1.0f / warp_sum(l);
+  __nv_bfloat16 *dst = o_out + (static_cast<long>(b) * L + lq) * (static_cast<long>(H) * ATT_DH) +
+                       h * ATT_DH + 8 * lane;
+  *reinterpret_cast<uint4 *>(dst) =
+      make_uint4(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv),
+                 pack_bf16x2(acc[4] * inv, acc[5] * inv), pack_bf16x2(acc[6] * inv, acc[7] * inv));
 }
 
 }  // namespace ig4

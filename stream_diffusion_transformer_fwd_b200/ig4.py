@@ -86,6 +86,8 @@ _sig("ig4_norm_modulate", [_i, _i, _i, _vp, _i, _vp, _vp, _i, _f, _vp, _i, _vp, 
 _sig("ig4_qkv_project", [_i, _i, _i, _i, _vp, _i, _vp, _vp, _i, _vp, _vp, _vp, _f, _vp, _vp,
                          _vp, _vp, _vp, _i, _vp])
 _sig("ig4_joint_attention", [_i, _i, _i, _vp, _vp, _vp, _i, _vp, _vp])
+_sig("ig4_joint_attention_workspace_size", [_i, _i, _i], ctypes.c_size_t)
+_sig("ig4_joint_attention_ws", [_i, _i, _i, _vp, _vp, _vp, _i, _vp, _vp, ctypes.c_size_t, _vp])
 _sig("ig4_gated_residual_linear", [_i, _i, _i, _i, _vp, _i, _vp, _vp, _i, _vp, _vp, _i, _vp,
                                    _vp, _i, _vp])
 _sig("ig4_swiglu", [_i, _i, _i, _vp, _i, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp])
@@ -139,7 +141,8 @@ _sig("ig4_selftest_timeout", [_i, _vp])
 
 EXPORTED = ("ig4_status_string", "ig4_abi_version", "ig4_mrope_positions", "ig4_rope_table",
             "ig4_adaln_modulation", "ig4_norm_modulate", "ig4_qkv_project",
-            "ig4_joint_attention", "ig4_gated_residual_linear", "ig4_swiglu",
+            "ig4_joint_attention", "ig4_joint_attention_workspace_size", "ig4_joint_attention_ws",
+            "ig4_gated_residual_linear", "ig4_swiglu",
             "ig4_quantize_rows", "ig4_workspace_size", "ig4_block_forward",
             "ig4_block_forward_traced", "ig4_block_forward_noalloc", "ig4_stack_workspace_size",
             "ig4_stack_forward", "ig4_stack_forward_tapped", "ig4_nvfp4_scale_bytes", "ig4_nvfp4_pack_scales",
@@ -280,6 +283,19 @@ def ig4_qkv_project(B, L, D, H, h, h_scale, w_qkv, w_scale, g_q, g_k, eps, rope_
 def ig4_joint_attention(B, H, L, q, k, vt, vt_ld, o_out, stream=None):
     _check(_lib.ig4_joint_attention(B, H, L, _ptr(q), _ptr(k), _ptr(vt), vt_ld, _ptr(o_out),
                                     _stream(stream)), "ig4_joint_attention")
+
+
+def ig4_joint_attention_workspace_size(B: int, H: int, L: int) -> int:
+    return int(_lib.ig4_joint_attention_workspace_size(B, H, L))
+
+
+def ig4_joint_attention_ws(B, H, L, q, k, vt, vt_ld, o_out, workspace, stream=None):
+    """ig4_joint_attention on the balanced persistent grid (workspace from
+    ig4_joint_attention_workspace_size; may be empty)."""
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(_lib.ig4_joint_attention_ws(B, H, L, _ptr(q), _ptr(k), _ptr(vt), vt_ld, _ptr(o_out),
+                                       _ptr(workspace) if ws_bytes else None, ws_bytes,
+                                       _stream(stream)), "ig4_joint_attention_ws")
 
 
 def ig4_gated_residual_linear(B, L, N, K, a, a_scale, w, w_scale, gate, gate_stride, x_res,

@@ -278,3 +278,32 @@ def test_joint_attention(ig4, B, H, L, qscale):
     # P is rounded to bf16 before the PV product and o once on output
     assert rel_l2(got, ref) <= 1e-2
     assert np.max(np.abs(got - ref)) <= 2e-2 * np.max(np.abs(ref)) + 1e-3
+
+
+# the balanced persistent grid: more (b, h, query tile) items than SMs, so
+# key-tile ranges split items between CTAs (partial O merged afterwards);
+# ragged tails; a single item spread over many CTAs; one item per CTA
+@pytest.mark.parametrize("B,H,L,qscale", [(1, 18, 1152, 1.0), (2, 5, 2000, 1.0),
+                                          (1, 37, 640, 8.0), (1, 1, 2560, 1.0),
+                                          (1, 3, 129, 1.0), (3, 2, 100, 1.0)])
+def test_joint_attention_balanced_grid(ig4, B, H, L, qscale):
+    q = randn("bq", (B, H, L, 256)) * qscale
+    k = randn("bk", (B, H, L, 256))
+    v = randn("bv", (B, H, L, 256))
+    vt_ld = (L + 7) // 8 * 8
+    vt = torch.zeros((B, H, 256, vt_ld), dtype=torch.bfloat16)
+    vt[..., :L] = v.transpose(2, 3)
+    ws = torch.empty(ig4.ig4_joint_attention_workspace_size(B, H, L), dtype=torch.uint8,
+                     device="cuda")
+    o = torch.empty((B * L, H * 256), dtype=torch.bfloat16, device="cuda")
+    qd, kd, vd = q.cuda(), k.cuda(), vt.cuda()
+    ig4.ig4_joint_attention_ws(B, H, L, qd, kd, vd, vt_ld, o, ws)
+    o2 = torch.empty_like(o)
+    ig4.ig4_joint_attention_ws(B, H, L, qd, kd, vd, vt_ld, o2, ws)
+    torch.cuda.synchronize()
+    assert ig4.ig4_last_device_error() == ig4.IG4_OK
+    assert torch.equal(o, o2)  # the merge order is fixed
+    ref = O.merge_heads(O.joint_attention(f64(q), f64(k), f64(v))).reshape(B * L, H * 256)
+    got = f64(o.cpu())
+    assert rel_l2(got, ref) <= 1e-2
+    assert np.max(np.abs(got - ref)) <= 2e-2 * np.max(np.abs(ref)) + 1e-3
