@@ -65,6 +65,8 @@ def parse():
     p.add_argument("--config", default="1024px")
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--fp8-peak", action="store_true",
+                   help="measure the cuBLAS e4m3 GEMM rate (8192^3) and print it")
     return p.parse_args()
 
 
@@ -136,6 +138,61 @@ def load_peaks():
         with open(path) as f:
             return json.load(f), "measured"
     return dict(FALLBACK_PEAKS), "fallback"
+
+
+def fp8_peak(bf16_peak, sustained):
+    """Dense FP8 (e4m3) tensor peak for an FP8 GEMM roofline: the cuBLAS
+    e4m3 rate measured on this machine (profiles/fp8_peak.json, written from
+    `bench.py --fp8-peak`), else 2x the bf16 figure (the nominal dense
+    ratio).  Returns (TFLOP/s, note)."""
+    path = os.path.join(ROOT, "profiles", "fp8_peak.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            rec = json.load(f)
+        key = "e4m3_tflops_sustained" if sustained else "e4m3_tflops"
+        if key in rec:
+            return float(rec[key]), f"cuBLAS e4m3 {'sustained' if sustained else 'burst'} (measured, profiles/fp8_peak.json)"
+    return 2.0 * bf16_peak, "2 x bf16: nominal fp8/bf16 dense ratio"
+
+
+def measure_fp8_peak():
+    """cuBLAS e4m3 GEMM rate (torch._scaled_mm, 8192^3, bf16 out, per-tensor
+    scales) timed with CUDA events: a burst of 20 calls after warm-up, and a
+    ~4 s loop for the power-capped sustained rate.  Prints one JSON line."""
+    import torch
+    torch.cuda.set_device(0)
+    n = 8192
+    g = torch.Generator(device="cuda").manual_seed(0)
+    a = torch.randn(n, n, device="cuda", generator=g).to(torch.float8_e4m3fn)
+    b = torch.randn(n, n, device="cuda", generator=g).to(torch.float8_e4m3fn)
+    one = torch.ones((), device="cuda")
+    def mm():
+        return torch._scaled_mm(a, b.t(), scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+    for _ in range(10):
+        mm()
+    torch.cuda.synchronize()
+    flops = 2.0 * n ** 3
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(20):
+        mm()
+    e1.record()
+    torch.cuda.synchronize()
+    burst = flops * 20 / (e0.elapsed_time(e1) * 1e-3) / 1e12
+    sampler = ClockSampler(0)
+    sampler.start()
+    reps = max(20, int(4.0 / (flops / (burst * 1e12))))
+    e0.record()
+    for _ in range(reps):
+        mm()
+    e1.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    sustained = flops * reps / (e0.elapsed_time(e1) * 1e-3) / 1e12
+    print(json.dumps({"e4m3_tflops": round(burst, 1), "e4m3_tflops_sustained": round(sustained, 1),
+                      "shape": [n, n, n], "op": "torch._scaled_mm e4m3 x e4m3 -> bf16",
+                      "sustained_reps": reps, "clocks": clocks}), flush=True)
+    return 0
 
 
 def kernel_source_hash(kernel, workload=""):
@@ -411,8 +468,7 @@ def run_ours(args, rank, local_rank, world):
             peak = 4.0 * tensor_peak
             peak_note = f"4 x {tnote}: nominal fp4/bf16 dense ratio"
         elif fp8 and dom_name != "attention":
-            peak = 2.0 * tensor_peak
-            peak_note = f"2 x {tnote}: nominal fp8/bf16 dense ratio"
+            peak, peak_note = fp8_peak(tensor_peak, not held_max)
         else:
             peak = tensor_peak
             peak_note = tnote
@@ -562,7 +618,8 @@ def run_stack(args, cfg, ig4, rank, world, dev):
     # mixed bound: the GEMMs at the FP8 rate (2x bf16), attention at the bf16 rate
     gemm_f = cfg.n_blocks * (blk - per["attention"] - per["adaln"])
     attn_f = cfg.n_blocks * per["attention"]
-    t_min = gemm_f / ((2.0 if fp8 else 1.0) * bf16_peak * 1e12) + attn_f / (bf16_peak * 1e12)
+    gemm_peak = fp8_peak(bf16_peak, not held_max)[0] if fp8 else bf16_peak
+    t_min = gemm_f / (gemm_peak * 1e12) + attn_f / (bf16_peak * 1e12)
     mixed_peak = flops / t_min / 1e12
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
@@ -579,8 +636,9 @@ def run_stack(args, cfg, ig4, rank, world, dev):
         "roofline": {"bound": "tensor", "achieved": round(value / world, 1),
                      "peak": round(mixed_peak, 1), "unit": "TFLOP/s",
                      "frac": round(value / world / mixed_peak, 4), "traffic": None,
-                     "kernel": "whole step (GEMMs at 2x and attention at 1x the " + tkey + ")",
-                     "peak_source": f"{tkey} ({peak_src}) x nominal fp8/bf16 ratio for the GEMMs"},
+                     "kernel": "whole step (GEMMs at the FP8 and attention at the bf16 rate)",
+                     "peak_source": (f"attention: {tkey} ({peak_src}); GEMMs: "
+                                     f"{fp8_peak(bf16_peak, not held_max)[1] if fp8 else tkey}")},
         "clocks": clocks, "device_error": ig4.ig4_status_string(err),
         "e2e": {"value": round(job_rate(flops, world, K, ms_e2e), 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -681,7 +739,8 @@ def run_step(args, cfg, ig4, rank, world, dev):
         blk, per = block_work(cc)
         gemm_f += cc.n_blocks * (blk - per["attention"] - per["adaln"])
         attn_f += cc.n_blocks * per["attention"]
-    t_min = gemm_f / ((2.0 if fp8 else 1.0) * bf16_peak * 1e12) + attn_f / (bf16_peak * 1e12)
+    gemm_peak = fp8_peak(bf16_peak, not held_max)[0] if fp8 else bf16_peak
+    t_min = gemm_f / (gemm_peak * 1e12) + attn_f / (bf16_peak * 1e12)
     mixed_peak = flops / t_min / 1e12
     value = job_rate(flops, world, K, ms_total)
     per_stack = cfg.n_blocks * (10 if fp8 else 8) + 1
@@ -703,8 +762,9 @@ def run_step(args, cfg, ig4, rank, world, dev):
         "roofline": {"bound": "tensor", "achieved": round(value / world, 1),
                      "peak": round(mixed_peak, 1), "unit": "TFLOP/s",
                      "frac": round(value / world / mixed_peak, 4), "traffic": None,
-                     "kernel": "whole step (GEMMs at 2x and attention at 1x the " + tkey + ")",
-                     "peak_source": f"{tkey} ({peak_src}) x nominal fp8/bf16 ratio for the GEMMs"},
+                     "kernel": "whole step (GEMMs at the FP8 and attention at the bf16 rate)",
+                     "peak_source": (f"attention: {tkey} ({peak_src}); GEMMs: "
+                                     f"{fp8_peak(bf16_peak, not held_max)[1] if fp8 else tkey}")},
         "clocks": clocks, "device_error": ig4.ig4_status_string(err),
         "e2e": {"value": round(job_rate(flops, world, K, ms_e2e), 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -1006,6 +1066,8 @@ def run_reference(args, rank, world):
 
 def main():
     args = parse()
+    if args.fp8_peak:
+        return measure_fp8_peak()
     rank, local_rank, world = dist_env()
     if args.impl == "reference":
         return run_reference(args, rank, world)
