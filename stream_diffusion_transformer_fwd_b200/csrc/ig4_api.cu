@@ -422,68 +422,100 @@ ig4_status launch_qkv(int B, int L, int D, int H, const void *h, int h_dtype, co
   return launch_gemm<256, false, false>(ma, mb, mb, M, ntn, D, e, st);
 }
 
-// The attention kernel's grid: one CTA per (b, h, query tile) item when
-// there are no more items than CTAs (or no partial slots), else one CTA per
-// SM taking the items round-robin, with the last partial round's items split
-// into pieces of key tiles (the kernel's AttSched).
-long att_items(int B, int H, int L) {
-  return static_cast<long>(B) * H * ((L + ATT_BN - 1) / ATT_BN);
-}
-int att_grid(int B, int H, int L, int sms, bool have_part) {
-  const long items = att_items(B, H, L);
-  const int g = std::min(sms, ATT_MAX_CTAS);
-  if (!have_part || items <= g) return static_cast<int>(items);
-  return g;
-}
-// Tail items split into pieces (0: none), as the kernel's AttSched computes it.
-int att_split_items(int B, int H, int L, int grid) {
-  const long items = att_items(B, H, L);
+// The attention kernel's launch.  With two or more query tiles the kernel
+// runs on CTA pairs (an item is two query tiles of one (b, h)), else on
+// single CTAs (an item is the one query tile).  Workers (pairs or CTAs): one
+// per item when there are no more items than workers fit on the device (or
+// no partial slots), else one per SM (pair) taking the items round-robin,
+// with the last partial round's items split into pieces of key tiles (the
+// kernel's AttSched).
+struct AttPlan {
+  bool pair;
+  long items;
+  int workers;  // pairs or CTAs
+  int split;    // tail items split into pieces (0: none)
+};
+AttPlan att_plan(int B, int H, int L, int sms, bool have_part) {
+  AttPlan p{};
   const int nkv = (L + ATT_BN - 1) / ATT_BN;
-  const long rem = items % grid;
-  if (rem == 0) return 0;
-  const long k = std::max<long>(1, std::min<long>(nkv, grid / rem));
-  return k > 1 ? static_cast<int>(rem) : 0;
+  p.pair = nkv >= 2;
+  const int ctas = p.pair ? 2 : 1;
+  p.items = static_cast<long>(B) * H * (p.pair ? (nkv + 1) / 2 : nkv);
+  const int g = std::max(1, std::min(sms, ATT_MAX_CTAS) / ctas);
+  p.workers = (!have_part || p.items <= g) ? static_cast<int>(p.items) : g;
+  const long rem = p.items % p.workers;
+  const long k = rem ? std::max<long>(1, std::min<long>(nkv, p.workers / rem)) : 1;
+  p.split = k > 1 ? static_cast<int>(rem) : 0;
+  return p;
 }
 // Bytes of partial slots the grid may need: one per CTA (0 when no item can
 // be split: a single key tile per item).
 size_t att_part_bytes(int B, int H, int L) {
   const long nkv = (L + ATT_BN - 1) / ATT_BN;
-  if (nkv <= 1 || att_items(B, H, L) <= 1) return 0;
+  if (nkv <= 1 || static_cast<long>(B) * H * nkv <= 1) return 0;
   return static_cast<size_t>(ATT_MAX_CTAS) * ATT_PART_BYTES;
 }
 
 // part: att_part_bytes(B, H, L) bytes of workspace for the balanced grid, or
-// nullptr (one CTA per item).
+// nullptr (one worker per item).
 ig4_status launch_attention(int B, int H, int L, const void *q, const void *k, const void *vt,
                             int vt_ld, void *o, void *part, cudaStream_t st) {
-  CUtensorMap mq, mk, mv;
-  const long BH = static_cast<long>(B) * H;
-  IG4_TRY(map_3d_bf16(&mq, q, 256, L, BH, 256, static_cast<long>(L) * 256, 64, ATT_BM));
-  IG4_TRY(map_3d_bf16(&mk, k, 256, L, BH, 256, static_cast<long>(L) * 256, 64, ATT_BN));
-  // V^T boxes are 64 keys (128 bytes, the swizzle span) x 256 head dims; a
-  // 128-key tile takes two of them.
-  IG4_TRY(map_3d_bf16(&mv, vt, L, 256, BH, vt_ld, 256L * vt_ld, 64, 256));
-  IG4_TRY(allow_smem(attention_kernel, ATT_SMEM_BYTES));
   DeviceInfo *di = nullptr;
   IG4_TRY(device_info(&di));
+  const long BH = static_cast<long>(B) * H;
   const bool have_part = part != nullptr && att_part_bytes(B, H, L) > 0;
-  const long items = att_items(B, H, L);
-  const int grid = att_grid(B, H, L, di->sms, have_part);
-  if (BH > (1L << 30) || items > (1L << 30)) return IG4_ERR_UNSUPPORTED;
+  const AttPlan plan = att_plan(B, H, L, di->sms, have_part);
+  if (BH > (1L << 30) || plan.items > (1L << 29)) return IG4_ERR_UNSUPPORTED;
+  CUtensorMap mq, mk, mv;
+  IG4_TRY(map_3d_bf16(&mq, q, 256, L, BH, 256, static_cast<long>(L) * 256, 64, ATT_BM));
+  // K boxes: 64 head dims (128 bytes, the swizzle span) x the keys one CTA
+  // loads per tile (all 128, or its 64 of a pair's tile).  V^T boxes: 64 keys
+  // x the head dims one CTA loads (all 256, or its 128 of a pair's).
+  IG4_TRY(map_3d_bf16(&mk, k, 256, L, BH, 256, static_cast<long>(L) * 256, 64,
+                      plan.pair ? ATT_BN / 2 : ATT_BN));
+  IG4_TRY(map_3d_bf16(&mv, vt, L, 256, BH, vt_ld, 256L * vt_ld, 64,
+                      plan.pair ? ATT_DH / 2 : ATT_DH));
   __nv_bfloat16 *op = static_cast<__nv_bfloat16 *>(o);
   uint8_t *pp = static_cast<uint8_t *>(part);
-  if (launch_pdl(attention_kernel, dim3(grid), dim3(ATT_THREADS), ATT_SMEM_BYTES, st, mq, mk, mv,
-                 op, L, H, static_cast<int>(BH), pp) != cudaSuccess)
-    return IG4_ERR_CUDA;
-  IG4_TRY(last_launch_status());
-  const int split = att_split_items(B, H, L, grid);
-  if (split > 0) {
-    // merge the pieces of the split tail items
-    if (launch_pdl(attention_combine_kernel, dim3(split, ATT_BM / ATT_COMBINE_ROWS),
-                   dim3(ATT_COMBINE_THREADS), 0, st,
-                   static_cast<const uint8_t *>(pp), op, L, H, static_cast<int>(BH), grid) !=
-        cudaSuccess)
+  if (plan.pair) {
+    IG4_TRY(allow_smem(attention_kernel<true>, ATT_SMEM_BYTES));
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(2 * plan.workers);
+    lc.blockDim = dim3(ATT_THREADS);
+    lc.dynamicSmemBytes = ATT_SMEM_BYTES;
+    lc.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 2;
+    if (cudaLaunchKernelEx(&lc, attention_kernel<true>, mq, mk, mv, op, L, H,
+                           static_cast<int>(BH), pp) != cudaSuccess)
       return IG4_ERR_CUDA;
+  } else {
+    IG4_TRY(allow_smem(attention_kernel<false>, ATT_SMEM_BYTES));
+    if (launch_pdl(attention_kernel<false>, dim3(plan.workers), dim3(ATT_THREADS),
+                   ATT_SMEM_BYTES, st, mq, mk, mv, op, L, H, static_cast<int>(BH),
+                   pp) != cudaSuccess)
+      return IG4_ERR_CUDA;
+  }
+  IG4_TRY(last_launch_status());
+  if (plan.split > 0) {
+    // merge the pieces of the split tail items
+    const int rows = (plan.pair ? 2 : 1) * ATT_BM;
+    const dim3 grid(plan.split, rows / ATT_COMBINE_ROWS);
+    const cudaError_t e =
+        plan.pair ? launch_pdl(attention_combine_kernel<true>, grid, dim3(ATT_COMBINE_THREADS), 0,
+                               st, static_cast<const uint8_t *>(pp), op, L, H,
+                               static_cast<int>(BH), plan.workers)
+                  : launch_pdl(attention_combine_kernel<false>, grid, dim3(ATT_COMBINE_THREADS),
+                               0, st, static_cast<const uint8_t *>(pp), op, L, H,
+                               static_cast<int>(BH), plan.workers);
+    if (e != cudaSuccess) return IG4_ERR_CUDA;
     IG4_TRY(last_launch_status());
   }
   return IG4_OK;

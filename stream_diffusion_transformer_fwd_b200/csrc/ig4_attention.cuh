@@ -42,9 +42,28 @@
 // maximum grows by more than 8 (a factor 2^8), so O is rescaled rarely;
 // numerator and denominator use the same maximum, so the result is unchanged.
 //
+// CTA pairs.  With two or more query tiles the kernel runs on 2-CTA
+// clusters (tcgen05.mma.cta_group::2, M = 256): an item is then two query
+// tiles of one (sample, head), rank r of the pair holding query tile
+// 2 u + r (an odd count leaves rank 1 of the last item a tile past the
+// sequence, computed on zero-filled Q and not stored).  Each CTA keeps its
+// own 128 query rows, S, P and O in its own TMEM, and loads only HALF of
+// every key tile: K of its 64 keys (4 chunks [64 keys x 128 B]) and V^T of
+// its 128 head dims (2 chunks [128 dims x 128 B]), 32 KB each, one ring slot
+// per K or V item.  The leader issues S_j = Q K_j^T as 16 MMAs of N = 128
+// and O += P_j V_j as 8 MMAs of N = 256 with A = P read from both CTAs'
+// TMEM.  So per key tile each SM moves 64 KB of K and V instead of 128 KB
+// (the single-CTA kernel's L2 traffic starves the ring), and the ring holds
+// two and a half tiles instead of one and a quarter.  Both CTAs' loads
+// complete on the leader's full barriers (the leader posts the bytes of
+// both); the leader's commits arrive on both CTAs' empty / S-ready / PV-done
+// barriers; the softmax warps of both CTAs arrive on the leader's S-free,
+// P-ready and O-free barriers (8 arrivals).
+//
 // Warp roles (224 threads): warps 0-3 softmax + output (warp w owns TMEM
 // lanes / query rows 32w..32w+31), warp 4 TMA producer, warp 5 TMEM
-// allocation and the S MMAs, warp 6 the PV MMAs.  The two MMA threads wait
+// allocation and the S MMAs, warp 6 the PV MMAs (the MMA roles only in the
+// leader of a pair).  The two MMA threads wait
 // on different events (scores read out vs. probabilities written), so one
 // keeps the tensor pipe fed while the other waits.
 //
@@ -169,10 +188,46 @@ __device__ __forceinline__ bool att_wait_passed(const volatile int *passed, long
   }
 }
 
+// Waits and arrivals of the pipeline.  In a pair the hand-offs between the
+// CTAs carry no data through ordinary memory (only tensor memory, ordered by
+// the tcgen05 fences around them), so they keep the CTA-scope semantics.
+template <bool PAIR>
+__device__ __forceinline__ bool att_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                         unsigned long long limit_ns = WAIT_LIMIT_NS) {
+  return mbar_wait(bar, parity, abort_flag, limit_ns);
+}
+
+template <bool PAIR>
+__device__ __forceinline__ bool att_wait_warp(uint64_t *bar, uint32_t parity,
+                                              volatile int *abort_flag) {
+  return __all_sync(0xffffffffu, att_wait<PAIR>(bar, parity, abort_flag));
+}
+
+// Commit of the MMAs issued so far to a barrier (in both CTAs of a pair).
+template <bool PAIR>
+__device__ __forceinline__ void att_commit(uint64_t *bar) {
+  if constexpr (PAIR)
+    umma_commit_pair_both(bar);
+  else
+    umma_commit(bar);
+}
+
+// Arrive on a barrier that the leader CTA holds (the CTA itself when single).
+template <bool PAIR>
+__device__ __forceinline__ void att_arrive_leader(uint64_t *bar) {
+  if constexpr (PAIR)
+    mbar_arrive_remote(map_shared_to_rank(bar, 0));
+  else
+    mbar_arrive(bar);
+}
+
+template <bool PAIR>
 __global__ void __launch_bounds__(ATT_THREADS, 1)
     attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, __nv_bfloat16 *__restrict__ o_out,
                      int L, int H, int n_bh, uint8_t *__restrict__ part) {
+  constexpr int CTAS = PAIR ? 2 : 1;
+  constexpr int UPI = PAIR ? 1 : 2;  // ring units (slots) per item
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -191,14 +246,17 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   uint64_t *o_free = bars + 20;   // O of a segment drained (one arrival per softmax warp)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 22);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-  volatile int *passed = reinterpret_cast<volatile int *>(tmem_slot + 2);  // halves past empty
+  volatile int *passed = reinterpret_cast<volatile int *>(tmem_slot + 2);  // ring units past empty
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int nkv = (L + ATT_BN - 1) / ATT_BN;  // key tiles = query tiles
-  const AttSched sched(n_bh * nkv, static_cast<int>(gridDim.x), nkv);
-  const int cta = blockIdx.x;
-  const int n_seg = sched.segments(cta);
+  const int rank = PAIR ? static_cast<int>(cluster_ctarank()) : 0;
+  const bool leader = rank == 0;
+  const int nkv = (L + ATT_BN - 1) / ATT_BN;          // key tiles = query tiles
+  const int n_units = PAIR ? (nkv + 1) / 2 : nkv;     // items per (sample, head)
+  const AttSched sched(n_bh * n_units, static_cast<int>(gridDim.x) / CTAS, nkv);
+  const int worker = blockIdx.x / CTAS;
+  const int n_seg = sched.segments(worker);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < ATT_SLOTS; ++s) {
@@ -207,15 +265,15 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     }
     mbar_init(q_full, 1);
     mbar_init(s_full, 1);
-    mbar_init(s_free, 4);
-    mbar_init(&p_full[0], 4);
-    mbar_init(&p_full[1], 4);
+    mbar_init(s_free, 4 * CTAS);
+    mbar_init(&p_full[0], 4 * CTAS);
+    mbar_init(&p_full[1], 4 * CTAS);
     mbar_init(&pv_done[0], 1);
     mbar_init(&pv_done[1], 1);
     mbar_init(drain_s, 1);
     mbar_init(drain_pv, 1);
     mbar_init(q_empty, 1);
-    mbar_init(o_free, 4);
+    mbar_init(o_free, 4 * CTAS);
     *abort_flag = 0;
     *passed = 0;
     fence_mbar_init();
@@ -226,11 +284,19 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     tma_prefetch_desc(&tmV);
   }
   if (warp == 5) {
-    tmem_alloc(tmem_slot, ATT_TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, ATT_TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, ATT_TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR)
+    cluster_sync_all();
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   pdl_wait();
@@ -238,176 +304,229 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 
   if (warp == 4) {
     if (lane == 0) {
-      // ------------------------------------------------ TMA producer
-      long i = 0;  // half items issued over the range
+      // ------------------------------------------------ TMA producer (each CTA its own part)
+      long i = 0;  // ring units issued over the range
       bool ok = true;
       int k = 0;
       int q_issued = -1;  // the last segment whose Q load was issued
       for (; k < n_seg && ok; ++k) {
-        const AttSeg sg = sched.seg(cta, k);
-        const int bh = sg.item / nkv;
-        const int q0 = (sg.item - bh * nkv) * ATT_BM;
+        const AttSeg sg = sched.seg(worker, k);
+        const int bh = sg.item / n_units;
+        const int q0 = ((sg.item - bh * n_units) * CTAS + rank) * ATT_BM;
         // Q: free once the last S MMA of the previous segment has run
-        if (k > 0 && !mbar_wait(q_empty, static_cast<uint32_t>(k - 1) & 1, abort_flag)) {
+        if (k > 0 && !att_wait<PAIR>(q_empty, static_cast<uint32_t>(k - 1) & 1, abort_flag)) {
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(q_full, ATT_Q_BYTES);
-        for (int c = 0; c < 4; ++c) tma_load_3d(smem + c * 16384, &tmQ, q_full, c * 64, q0, bh);
+        if (leader) mbar_arrive_expect_tx(q_full, CTAS * ATT_Q_BYTES);
+        for (int c = 0; c < 4; ++c) {
+          if constexpr (PAIR)
+            tma_load_3d_pair(smem + c * 16384, &tmQ, map_shared_to_rank(q_full, 0), c * 64, q0, bh);
+          else
+            tma_load_3d(smem + c * 16384, &tmQ, q_full, c * 64, q0, bh);
+        }
         q_issued = k;
         const AttRing ro{sg.n};
-        const int n = 2 * ro.items();  // half items of this segment
+        const int n = UPI * ro.items();  // ring units of this segment
         for (int hi = 0; hi < n; ++hi, ++i) {
           const int slot = static_cast<int>(i % ATT_SLOTS);
           const uint32_t ph = static_cast<uint32_t>(i / ATT_SLOTS) & 1;
-          if (!mbar_wait(&empty[slot], ph ^ 1, abort_flag)) { ok = false; break; }
-          // half i - 5 is consumed, so full[slot] has completed its phase
-          __threadfence_block();
-          *passed = static_cast<int>(i + 1);
-          mbar_arrive_expect_tx(&full[slot], ATT_SLOT_BYTES);
+          if (!att_wait<PAIR>(&empty[slot], ph ^ 1, abort_flag)) { ok = false; break; }
+          if (leader) {
+            // unit i - 5 is consumed, so full[slot] has completed its phase
+            __threadfence_block();
+            *passed = static_cast<int>(i + 1);
+            mbar_arrive_expect_tx(&full[slot], CTAS * ATT_SLOT_BYTES);
+          }
           uint8_t *dst = ring + slot * ATT_SLOT_BYTES;
-          const int half = hi & 1;
           int t = 0;
-          if (ro.kind(hi >> 1, &t) == 1) {
-            for (int c = 0; c < 2; ++c)
-              tma_load_3d(dst + c * 16384, &tmK, &full[slot], (2 * half + c) * 64,
-                          (sg.t0 + t) * ATT_BN, bh);
+          const int kind = ro.kind(hi / UPI, &t);
+          const int key0 = (sg.t0 + t) * ATT_BN;
+          if constexpr (PAIR) {
+            // this CTA's half of the pair's tile: keys [64 rank, +64) of K,
+            // head dims [128 rank, +128) of V^T
+            const uint32_t fb = map_shared_to_rank(&full[slot], 0);
+            if (kind == 1) {
+              for (int c = 0; c < 4; ++c)
+                tma_load_3d_pair(dst + c * 8192, &tmK, fb, c * 64, key0 + 64 * rank, bh);
+            } else {
+              for (int c = 0; c < 2; ++c)
+                tma_load_3d_pair(dst + c * 16384, &tmV, fb, key0 + 64 * c, 128 * rank, bh);
+            }
           } else {
-            tma_load_3d(dst, &tmV, &full[slot], (sg.t0 + t) * ATT_BN + half * 64, 0, bh);
+            const int half = hi & 1;
+            if (kind == 1) {
+              for (int c = 0; c < 2; ++c)
+                tma_load_3d(dst + c * 16384, &tmK, &full[slot], (2 * half + c) * 64, key0, bh);
+            } else {
+              tma_load_3d(dst, &tmV, &full[slot], key0 + half * 64, 0, bh);
+            }
           }
         }
       }
       if (!ok) {
         // let the loads already issued land before the shared memory goes away
-        if (q_issued >= 0)
-          mbar_wait(q_full, static_cast<uint32_t>(q_issued) & 1, nullptr, WAIT_LIMIT_NS / 4);
-        for (long j = (i > ATT_SLOTS ? i - ATT_SLOTS : 0); j < i; ++j)
-          mbar_wait(&full[j % ATT_SLOTS], static_cast<uint32_t>(j / ATT_SLOTS) & 1, nullptr,
-                    WAIT_LIMIT_NS / 4);
+        if constexpr (PAIR) {
+          // (a pair's loads complete on the leader's barriers)
+          sleep_ns(50000);
+        } else {
+          if (q_issued >= 0)
+            mbar_wait(q_full, static_cast<uint32_t>(q_issued) & 1, nullptr, WAIT_LIMIT_NS / 4);
+          for (long j = (i > ATT_SLOTS ? i - ATT_SLOTS : 0); j < i; ++j)
+            mbar_wait(&full[j % ATT_SLOTS], static_cast<uint32_t>(j / ATT_SLOTS) & 1, nullptr,
+                      WAIT_LIMIT_NS / 4);
+        }
       }
     }
   } else if (warp == 5) {
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       // ------------------------------------------------ S issuer: S_t = Q K_t^T
-      constexpr uint32_t IDESC_S = idesc_bf16(ATT_BM, ATT_BN);
-      const uint32_t q_base = smem_u32(smem);
+      constexpr uint32_t IDESC_S = idesc_bf16(CTAS * ATT_BM, ATT_BN);
+      const uint64_t qd = sdesc_kmajor_sw128(smem_u32(smem));
       bool ok = true;
       long gt = 0;  // tiles over the CTA's segments
       for (int k = 0; k < n_seg && ok; ++k) {
-        const AttSeg sg = sched.seg(cta, k);
+        const AttSeg sg = sched.seg(worker, k);
         const AttRing ro{sg.n};
-        const long ibase = 4 * sched.tiles_before(k);  // half items before this segment
-        if (!mbar_wait(q_full, static_cast<uint32_t>(k) & 1, abort_flag)) break;
+        const long ibase = 2 * UPI * sched.tiles_before(k);  // ring units before this segment
+        if (!att_wait<PAIR>(q_full, static_cast<uint32_t>(k) & 1, abort_flag)) break;
         for (int t = 0; t < sg.n && ok; ++t, ++gt) {
           // the S buffer is free once the softmax has read S_{gt-1}
-          if (gt > 0 && !mbar_wait(s_free, static_cast<uint32_t>(gt - 1) & 1, abort_flag)) {
+          if (gt > 0 && !att_wait<PAIR>(s_free, static_cast<uint32_t>(gt - 1) & 1, abort_flag)) {
             ok = false;
             break;
           }
           const int it = ro.item_k(t);
-          for (int half = 0; half < 2 && ok; ++half) {
-            const long i = ibase + 2 * it + half;
+          for (int u = 0; u < UPI && ok; ++u) {
+            const long i = ibase + UPI * it + u;
             const int slot = static_cast<int>(i % ATT_SLOTS);
             if (!att_wait_passed(passed, i, abort_flag) ||
-                !mbar_wait(&full[slot], static_cast<uint32_t>(i / ATT_SLOTS) & 1, abort_flag)) {
+                !att_wait<PAIR>(&full[slot], static_cast<uint32_t>(i / ATT_SLOTS) & 1,
+                                abort_flag)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint32_t k_base = smem_u32(ring + slot * ATT_SLOT_BYTES);
+            // descriptors of the slot's and Q's first chunk; a K step adds its
+            // byte offset / 16 to the start-address field (no carry out of it:
+            // shared memory addresses stay below 2^18)
+            const uint64_t kd = sdesc_kmajor_sw128(smem_u32(ring + slot * ATT_SLOT_BYTES));
+            if constexpr (PAIR) {
+              // 64 keys x 256 head dims in each CTA: 4 chunks [64 keys x 128 B]
 #pragma unroll
-            for (int kq = 0; kq < 8; ++kq) {
-              const int kk = half * 8 + kq;  // K step of 16 head dims
-              const uint64_t ad = sdesc_kmajor_sw128(q_base + (kk >> 2) * 16384 + (kk & 3) * 32);
-              const uint64_t bd = sdesc_kmajor_sw128(k_base + (kq >> 2) * 16384 + (kq & 3) * 32);
-              umma_bf16(tmem + ATT_TMEM_S, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+              for (int kk = 0; kk < 16; ++kk)
+                umma_bf16_pair(tmem + ATT_TMEM_S, qd + ((kk >> 2) * 16384 + (kk & 3) * 32) / 16,
+                               kd + ((kk >> 2) * 8192 + (kk & 3) * 32) / 16, IDESC_S,
+                               kk > 0 ? 1u : 0u);
+            } else {
+#pragma unroll
+              for (int kq = 0; kq < 8; ++kq) {
+                const int kk = u * 8 + kq;  // K step of 16 head dims
+                umma_bf16(tmem + ATT_TMEM_S, qd + ((kk >> 2) * 16384 + (kk & 3) * 32) / 16,
+                          kd + ((kq >> 2) * 16384 + (kq & 3) * 32) / 16, IDESC_S,
+                          kk > 0 ? 1u : 0u);
+              }
             }
-            umma_commit(&empty[slot]);
+            att_commit<PAIR>(&empty[slot]);
           }
-          if (ok) umma_commit(s_full);
+          if (ok) att_commit<PAIR>(s_full);
         }
         // Q may be replaced once these MMAs have run
-        if (ok) umma_commit(q_empty);
+        if (ok) att_commit<PAIR>(q_empty);
       }
-      umma_commit(drain_s);
-      mbar_wait(drain_s, 0, nullptr, WAIT_LIMIT_NS / 4);
+      att_commit<PAIR>(drain_s);
+      att_wait<PAIR>(drain_s, 0, nullptr, WAIT_LIMIT_NS / 4);
     }
   } else if (warp == 6) {
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       // ------------------------------------------------ PV issuer: O += P_j V_j
-      constexpr uint32_t IDESC_PV = idesc_bf16(ATT_BM, ATT_DH);
+      constexpr uint32_t IDESC_PV = idesc_bf16(CTAS * ATT_BM, ATT_DH);
       bool ok = true;
       long gt = 0;
       for (int k = 0; k < n_seg && ok; ++k) {
-        const AttSeg sg = sched.seg(cta, k);
+        const AttSeg sg = sched.seg(worker, k);
         const AttRing ro{sg.n};
-        const long ibase = 4 * sched.tiles_before(k);
+        const long ibase = 2 * UPI * sched.tiles_before(k);
         for (int j = 0; j < sg.n && ok; ++j, ++gt) {
           const int pb = static_cast<int>(gt & 1);
-          if (!mbar_wait(&p_full[pb], static_cast<uint32_t>(gt >> 1) & 1, abort_flag)) {
+          if (!att_wait<PAIR>(&p_full[pb], static_cast<uint32_t>(gt >> 1) & 1, abort_flag)) {
             ok = false;
             break;
           }
           // the first PV of a segment overwrites O: the previous one's O drained
           if (j == 0 && k > 0 &&
-              !mbar_wait(o_free, static_cast<uint32_t>(k - 1) & 1, abort_flag)) {
+              !att_wait<PAIR>(o_free, static_cast<uint32_t>(k - 1) & 1, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const int it = ro.item_v(j);
-          for (int half = 0; half < 2 && ok; ++half) {
-            const long i = ibase + 2 * it + half;
+          for (int u = 0; u < UPI && ok; ++u) {
+            const long i = ibase + UPI * it + u;
             const int slot = static_cast<int>(i % ATT_SLOTS);
             if (!att_wait_passed(passed, i, abort_flag) ||
-                !mbar_wait(&full[slot], static_cast<uint32_t>(i / ATT_SLOTS) & 1, abort_flag)) {
+                !att_wait<PAIR>(&full[slot], static_cast<uint32_t>(i / ATT_SLOTS) & 1,
+                                abort_flag)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint32_t v_base = smem_u32(ring + slot * ATT_SLOT_BYTES);
+            const uint64_t vd = sdesc_kmajor_sw128(smem_u32(ring + slot * ATT_SLOT_BYTES));
+            const uint32_t p_col = tmem + ATT_TMEM_P + 64 * pb;
+            if constexpr (PAIR) {
+              // 128 head dims x 128 keys in each CTA: 2 chunks [128 dims x 128 B]
 #pragma unroll
-            for (int kq = 0; kq < 4; ++kq) {
-              const int kk = half * 4 + kq;  // K step of 16 keys
-              const uint64_t bd = sdesc_kmajor_sw128(v_base + kq * 32);
-              umma_bf16_ts(tmem + ATT_TMEM_O, tmem + ATT_TMEM_P + 64 * pb + kk * 8, bd, IDESC_PV,
-                           (j > 0 || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < 8; ++kk)  // K step of 16 keys
+                umma_bf16_ts_pair(tmem + ATT_TMEM_O, p_col + kk * 8,
+                                  vd + ((kk >> 2) * 16384 + (kk & 3) * 32) / 16, IDESC_PV,
+                                  (j > 0 || kk > 0) ? 1u : 0u);
+            } else {
+#pragma unroll
+              for (int kq = 0; kq < 4; ++kq) {
+                const int kk = u * 4 + kq;  // K step of 16 keys
+                umma_bf16_ts(tmem + ATT_TMEM_O, p_col + kk * 8, vd + (kq * 32) / 16, IDESC_PV,
+                             (j > 0 || kk > 0) ? 1u : 0u);
+              }
             }
-            umma_commit(&empty[slot]);
+            att_commit<PAIR>(&empty[slot]);
           }
-          if (ok) umma_commit(&pv_done[pb]);
+          if (ok) att_commit<PAIR>(&pv_done[pb]);
         }
       }
-      umma_commit(drain_pv);
-      mbar_wait(drain_pv, 0, nullptr, WAIT_LIMIT_NS / 4);
+      att_commit<PAIR>(drain_pv);
+      att_wait<PAIR>(drain_pv, 0, nullptr, WAIT_LIMIT_NS / 4);
     }
   } else {
-    // -------------------------------------------- softmax warps 0..3
+    // -------------------------------------------- softmax warps 0..3 (each CTA its own rows)
     const int r = warp * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     const uint64_t scale2 = f2_pack(ATT_SCALE_LOG2, ATT_SCALE_LOG2);
     bool ok = true;
     long gt = 0;
     for (int k = 0; k < n_seg && ok; ++k) {
-      const AttSeg sg = sched.seg(cta, k);
+      const AttSeg sg = sched.seg(worker, k);
       float m_used = -INFINITY;
       float l_sum = 0.0f;
       for (int j = 0; j < sg.n; ++j, ++gt) {
-        if (!mbar_wait_warp(s_full, static_cast<uint32_t>(gt) & 1, abort_flag)) { ok = false; break; }
+        if (!att_wait_warp<PAIR>(s_full, static_cast<uint32_t>(gt) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
+        // all 128 scores in flight before one wait
+        float sc[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_base + ATT_TMEM_S + c * 32, sc[c]);
+        tmem_ld_wait();
         float t[128];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float a[32];
-          tmem_ld32(tmem + lane_base + ATT_TMEM_S + c * 32, a);
-          tmem_ld_wait();
+        for (int c = 0; c < 4; ++c)
 #pragma unroll
-          for (int i = 0; i < 32; ++i) t[32 * c + i] = a[i];
-        }
+          for (int i = 0; i < 32; ++i) t[32 * c + i] = sc[c][i];
         // S_j is in registers: the S buffer may take S_{j+1}.
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(s_free);
+        if (lane == 0) att_arrive_leader<PAIR>(s_free);
 
         const int kbase = (sg.t0 + j) * ATT_BN;
         if (kbase + ATT_BN > L) {
@@ -458,16 +577,16 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         const int pb = static_cast<int>(gt & 1);
         if (gt >= 2) {
           // PV_{gt-2} read this P buffer
-          if (!mbar_wait_warp(&pv_done[pb], static_cast<uint32_t>((gt >> 1) - 1) & 1,
-                              abort_flag)) {
+          if (!att_wait_warp<PAIR>(&pv_done[pb], static_cast<uint32_t>((gt >> 1) - 1) & 1,
+                                   abort_flag)) {
             ok = false;
             break;
           }
         }
         if (any_need) {
           // PV_{gt-1} (same segment, j > 0) must be done: it writes O
-          if (!mbar_wait_warp(&pv_done[pb ^ 1], static_cast<uint32_t>((gt - 1) >> 1) & 1,
-                              abort_flag)) {
+          if (!att_wait_warp<PAIR>(&pv_done[pb ^ 1], static_cast<uint32_t>((gt - 1) >> 1) & 1,
+                                   abort_flag)) {
             ok = false;
             break;
           }
@@ -497,18 +616,19 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         m_used = m_new;
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[pb]);
+        if (lane == 0) att_arrive_leader<PAIR>(&p_full[pb]);
       }
       if (!ok) break;
       // ---- the segment's output: O / l (bf16) or the partial (O, m, l)
       const long gl = gt - 1;
-      if (!mbar_wait_warp(&pv_done[gl & 1], static_cast<uint32_t>(gl >> 1) & 1, abort_flag)) {
+      if (!att_wait_warp<PAIR>(&pv_done[gl & 1], static_cast<uint32_t>(gl >> 1) & 1,
+                               abort_flag)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const int bh = sg.item / nkv;
-      const int q0 = (sg.item - bh * nkv) * ATT_BM;
+      const int bh = sg.item / n_units;
+      const int q0 = ((sg.item - bh * n_units) * CTAS + rank) * ATT_BM;
       const int b = bh / H, h = bh - (bh / H) * H;
       const int lq = q0 + r;
       const bool valid = lq < L;
@@ -518,7 +638,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         dst = o_out + (static_cast<long>(b) * L + lq) * (static_cast<long>(H) * ATT_DH) +
               h * ATT_DH;
       } else {
-        uint8_t *sp = part + static_cast<long>(sg.slot) * ATT_PART_BYTES;
+        uint8_t *sp = part + static_cast<long>(sg.slot * CTAS + rank) * ATT_PART_BYTES;
         dst = reinterpret_cast<__nv_bfloat16 *>(sp) + static_cast<long>(r) * ATT_DH;
         float *ml = reinterpret_cast<float *>(sp + ATT_PART_O_BYTES);
         ml[r] = m_used;
@@ -550,49 +670,64 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       // O is in registers or memory: the next segment's first PV may overwrite it
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(o_free);
+      if (lane == 0) att_arrive_leader<PAIR>(o_free);
     }
   }
 
+  __syncwarp();
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR)
+    cluster_sync_all();
+  else
+    __syncthreads();
   tc_fence_after();
-  if (warp == 5) tmem_dealloc(tmem, ATT_TMEM_COLS);
+  if (warp == 5) {
+    if constexpr (PAIR)
+      tmem_dealloc_pair(tmem, ATT_TMEM_COLS);
+    else
+      tmem_dealloc(tmem, ATT_TMEM_COLS);
+  }
 }
 
 // Merge of the split tail items: block (j, y) takes rows 8y .. 8y+7 of tail
-// item j, one warp per row; the item's k pieces sit in partial slots
-// j k .. j k + k - 1.  m = max m_p, l = sum l_p 2^(m_p - m),
+// item j (128 rows, or 256 for a pair item: rows [128 r, 128 r + 128) come
+// from rank r), one warp per row; piece p of the item sits in partial slot
+// j k + p (for pairs, 2 (j k + p) + r).  m = max m_p, l = sum l_p 2^(m_p - m),
 // o = sum O_p 2^(m_p - m) / l (pieces in order), stored as bf16.  Lane p
 // holds m and l of piece p (32 pieces at a time) and passes its weight by
 // shuffle; lane i accumulates head dims 8i .. 8i+7.
 constexpr int ATT_COMBINE_THREADS = 256;
 constexpr int ATT_COMBINE_ROWS = ATT_COMBINE_THREADS / 32;
 
+template <bool PAIR>
 __global__ void __launch_bounds__(ATT_COMBINE_THREADS)
     attention_combine_kernel(const uint8_t *__restrict__ part, __nv_bfloat16 *__restrict__ o_out,
                              int L, int H, int n_bh, int G) {
+  constexpr int CTAS = PAIR ? 2 : 1;
   pdl_wait();
   pdl_trigger();
   const int nkv = (L + ATT_BN - 1) / ATT_BN;
-  const AttSched sched(n_bh * nkv, G, nkv);
+  const int n_units = PAIR ? (nkv + 1) / 2 : nkv;
+  const AttSched sched(n_bh * n_units, G, nkv);
   const int j = blockIdx.x;
   const int k = sched.k;
   if (j >= sched.rem || k < 2) return;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int r = blockIdx.y * ATT_COMBINE_ROWS + warp;
+  const int rp = blockIdx.y * ATT_COMBINE_ROWS + warp;  // row of the item
+  if (rp >= CTAS * ATT_BM) return;
+  const int rank = rp / ATT_BM;
+  const int r = rp - rank * ATT_BM;
   const int item = sched.rounds * G + j;
-  const int bh = item / nkv;
-  const int q0 = (item - bh * nkv) * ATT_BM;
+  const int bh = item / n_units;
+  const int q0 = ((item - bh * n_units) * CTAS + rank) * ATT_BM;
   const int lq = q0 + r;
-  if (r >= ATT_BM || lq >= L) return;
+  if (lq >= L) return;
   const int b = bh / H, h = bh - (bh / H) * H;
-  const uint8_t *first = part + static_cast<long>(j) * k * ATT_PART_BYTES;
-  auto ml_of = [&](int p) {
-    return reinterpret_cast<const float *>(first + static_cast<long>(p) * ATT_PART_BYTES +
-                                           ATT_PART_O_BYTES);
+  auto slot_of = [&](int p) {
+    return part + static_cast<long>((j * k + p) * CTAS + rank) * ATT_PART_BYTES;
   };
+  auto ml_of = [&](int p) { return reinterpret_cast<const float *>(slot_of(p) + ATT_PART_O_BYTES); };
   float m = -INFINITY;
   for (int p0 = 0; p0 < k; p0 += 32)
     if (p0 + lane < k) m = fmaxf(m, ml_of(p0 + lane)[r]);
@@ -609,8 +744,8 @@ __global__ void __launch_bounds__(ATT_COMBINE_THREADS)
 #pragma unroll 4
     for (int q = 0; q < n; ++q) {
       const float w = __shfl_sync(0xffffffffu, wgt, q);
-      const uint4 v = reinterpret_cast<const uint4 *>(
-          first + static_cast<long>(p0 + q) * ATT_PART_BYTES + static_cast<long>(r) * ATT_DH * 2)[lane];
+      const uint4 v = reinterpret_cast<const uint4 *>(slot_of(p0 + q) +
+                                                      static_cast<long>(r) * ATT_DH * 2)[lane];
       const uint32_t u4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {

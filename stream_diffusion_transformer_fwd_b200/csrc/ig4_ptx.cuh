@@ -401,6 +401,19 @@ __device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a_desc,
       : "memory");
 }
 
+// D(tmem of both CTAs) (+)= A (both CTAs' TMEM, 128 rows each at the same
+// address) * B^T (halves in both CTAs' smem), bf16 inputs, fp32 accumulate.
+__device__ __forceinline__ void umma_bf16_ts_pair(uint32_t d_tmem, uint32_t a_tmem,
+                                                  uint64_t b_desc, uint32_t idesc,
+                                                  uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive once on the mbarrier at this shared offset in both CTAs of the pair
 // when every MMA this thread issued so far has completed.
 __device__ __forceinline__ void umma_commit_pair_both(uint64_t *bar) {
@@ -470,6 +483,14 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
                : "memory");
 }
 
+// Arrive on the mbarrier at a shared::cluster address with the default
+// (CTA-scope release) semantics.  For hand-offs whose data travels through
+// tensor memory and tcgen05 fences, not through ordinary memory: a
+// cluster-scope release costs the arriving thread about a thousand cycles.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -500,6 +521,14 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity
       return false;
     }
   }
+}
+
+// mbar_wait_cluster for roles where the whole warp waits (same answer in
+// every lane).
+__device__ __forceinline__ bool mbar_wait_cluster_warp(uint64_t *bar, uint32_t parity,
+                                                       volatile int *abort_flag) {
+  const bool ok = mbar_wait_cluster(bar, parity, abort_flag);
+  return __all_sync(0xffffffffu, ok);
 }
 
 __device__ __forceinline__ void sleep_ns(unsigned int ns) {
