@@ -558,18 +558,20 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         }
         const bool any_need = __any_sync(0xffffffffu, need);
 
-        // p = 2^(s * scale - m), packed to bf16 pairs; row sum in fp32 pairs
+        // p = 2^(s * scale - m), packed to bf16 pairs; row sum in fp32 pairs.
+        // One pair in eight takes the FMA-pipe exponential, which the MUFU
+        // unit (the softmax's bottleneck) does not serve.
         const uint64_t negm2 = f2_pack(-m_new, -m_new);
         uint32_t pk[64];
         uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
           const uint64_t x2 = ffma2(f2_pack(t[2 * i], t[2 * i + 1]), scale2, negm2);
-          const float p0 = exp2_approx(f2_lo(x2));
-          const float p1 = exp2_approx(f2_hi(x2));
-          const uint64_t p2 = f2_pack(p0, p1);
+          const uint64_t p2 = (i & 7) == 0
+                                  ? exp2_poly2(x2)
+                                  : f2_pack(exp2_approx(f2_lo(x2)), exp2_approx(f2_hi(x2)));
           acc[i & 3] = fadd2(acc[i & 3], p2);
-          pk[i] = pack_bf16x2(p0, p1);
+          pk[i] = pack_bf16x2(f2_lo(p2), f2_hi(p2));
         }
         const uint64_t s2 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
         const float rowsum = f2_lo(s2) + f2_hi(s2);

@@ -547,6 +547,38 @@ __device__ __forceinline__ float exp2_approx(float x) {
 }
 
 // max of three fp32 values in one instruction (sm_100)
+// 2^x for a pair of floats on the FMA pipe, to take load off the MUFU unit
+// (ex2.approx) in the softmax.  Cody-Waite range reduction (Cody and Waite,
+// Software Manual for the Elementary Functions, 1980): x = n + f with
+// n = rint(x) (adding 1.5 * 2^23 rounds to an integer in the low mantissa
+// bits) and f in [-1/2, 1/2]; 2^f by a cubic whose coefficients were fitted
+// here by weighted least squares on Chebyshev nodes (max relative error
+// 7.5e-5 on [-1/2, 1/2], far below the bf16 rounding of P); n is added to the
+// exponent field.  x is clamped at -125 so that the result stays a normal
+// number (about 2e-38 where ex2 gives 0 - invisible once P is summed or
+// rounded to bf16).
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+  const float x0 = fmaxf(__uint_as_float(static_cast<uint32_t>(x2)), -125.0f);
+  const float x1 = fmaxf(__uint_as_float(static_cast<uint32_t>(x2 >> 32)), -125.0f);
+  uint64_t xc, y, r, f, p;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(xc) : "f"(x0), "f"(x1));
+  const uint64_t magic = 0x4B4000004B400000ull;   // 1.5 * 2^23, twice
+  const uint64_t nmagic = 0xCB400000CB400000ull;  // -1.5 * 2^23, twice
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(y) : "l"(xc), "l"(magic));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(y), "l"(nmagic));
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(f) : "l"(xc), "l"(r));
+  const uint64_t c3 = 0x3D61FBA03D61FBA0ull;  // 0.055171609
+  const uint64_t c2 = 0x3E786F0C3E786F0Cull;  // 0.242611110
+  const uint64_t c1 = 0x3F31798D3F31798Dull;  // 0.693260968
+  const uint64_t c0 = 0x3F7FFB493F7FFB49ull;  // 0.999928057
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(c3), "l"(f), "l"(c2));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(p), "l"(f), "l"(c1));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(p), "l"(f), "l"(c0));
+  const uint32_t lo = static_cast<uint32_t>(p) + (static_cast<uint32_t>(y) << 23);
+  const uint32_t hi = static_cast<uint32_t>(p >> 32) + (static_cast<uint32_t>(y >> 32) << 23);
+  return static_cast<uint64_t>(lo) | (static_cast<uint64_t>(hi) << 32);
+}
+
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
