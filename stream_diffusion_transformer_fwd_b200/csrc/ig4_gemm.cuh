@@ -558,6 +558,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 // 128-clock MMA each SM reads 8 KB of operands instead of 12 KB, and each SM
 // loads a third fewer bytes per flop.
 //
+// K-snake: a pair's odd-numbered tiles sweep K from the last k-block down.
+// All pairs move from tile to tile at about the same time, so each round of
+// tiles starts on the k-blocks the previous round read last, which are still
+// in L2 where the two rounds share A rows or B rows.
+//
 // Barriers: full[s] in the leader (its producer posts the bytes of both
 // CTAs; both CTAs' loads complete on it); empty[s] and tfull[b] in both CTAs
 // (arrived by the leader's multicast commits); tempty[b] in the leader (one
@@ -644,10 +649,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
-      for (int t = pair; t < n_tiles && ok; t += n_pairs) {
+      int local = 0;
+      for (int t = pair; t < n_tiles && ok; t += n_pairs, ++local) {
         int mt, nt;
         tile_coords(t, m_tiles, n_tiles_n, group_m, &mt, &nt);
-        for (int kb = 0; kb < kblocks; ++kb) {
+        for (int it = 0; it < kblocks; ++it) {
+          const int kb = (local & 1) ? kblocks - 1 - it : it;  // K-snake
           if (!mbar_wait_cluster(&empty[s], ph ^ 1, abort_flag)) {
             ok = false;
             break;
@@ -683,7 +690,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         if (!mbar_wait_cluster(&tempty[buf], (use & 1) ^ 1, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * BN;
-        for (int kb = 0; kb < kblocks; ++kb) {
+        for (int it = 0; it < kblocks; ++it) {  // k-blocks in the producer's order
           if (!mbar_wait_cluster(&full[s], ph, abort_flag)) {
             ok = false;
             break;
@@ -696,9 +703,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             const uint64_t ad = sdesc_kmajor_sw128(a_base + kk * UK_BYTES);
             const uint64_t bd = sdesc_kmajor_sw128(b_base + kk * UK_BYTES);
             if (FP8)
-              umma_f8_pair(d_tmem, ad, bd, IDESC, (kb | kk) != 0);
+              umma_f8_pair(d_tmem, ad, bd, IDESC, (it | kk) != 0);
             else
-              umma_bf16_pair(d_tmem, ad, bd, IDESC, (kb | kk) != 0);
+              umma_bf16_pair(d_tmem, ad, bd, IDESC, (it | kk) != 0);
           }
           umma_commit_pair_both(&empty[s]);
           if (++s == PAIR_STAGES) {

@@ -324,6 +324,20 @@ __global__ void __launch_bounds__(NORM2_THREADS, 1)
   const int r_end = min(r_begin + rows_per_cta, nb);
   if (r_begin >= nb) return;
   const int nvec = D / 8;
+  auto load_row = [&](int rr, uint4 (&q)[NV]) {
+    const long in_row = remap_n > 0 ? static_cast<long>(b) * remap_L + remap_off + rr
+                                    : static_cast<long>(b) * L + rr;
+    const uint4 *xr = reinterpret_cast<const uint4 *>(x + in_row * D);
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int vi = lane + 32 * i;
+      if (vi < nvec) q[i] = __ldg(xr + vi);
+    }
+  };
+  // the warp's first row is in flight while the modulation vectors are staged
+  uint4 q[NV];
+  int rr = r_begin + warp;
+  if (rr < r_end) load_row(rr, q);
   const float4 *sc4 = reinterpret_cast<const float4 *>(scale + static_cast<long>(b) * mod_stride);
   const float4 *sh4 = reinterpret_cast<const float4 *>(shift + static_cast<long>(b) * mod_stride);
   for (int i = threadIdx.x; i < D / 4; i += NORM2_THREADS) {
@@ -337,75 +351,65 @@ __global__ void __launch_bounds__(NORM2_THREADS, 1)
     smod[(2 + hi) * nvec + v] = __ldg(sh4 + i);
   }
   __syncthreads();
-  for (int rr = r_begin + warp; rr < r_end; rr += NORM2_WARPS) {
-    const long in_row = remap_n > 0 ? static_cast<long>(b) * remap_L + remap_off + rr
-                                    : static_cast<long>(b) * L + rr;
-    const uint4 *xr = reinterpret_cast<const uint4 *>(x + in_row * D);
-    uint4 q[NV];
-#pragma unroll
-    for (int i = 0; i < NV; ++i) {
-      const int vi = lane + 32 * i;
-      if (vi < nvec) q[i] = __ldg(xr + vi);
-    }
-    float ss = 0.0f;
+  const uint64_t *smod2 = reinterpret_cast<const uint64_t *>(smod);  // pairs of floats
+  for (; rr < r_end; rr += NORM2_WARPS) {
+    // sum of squares over the row: two elements per packed FMA
+    uint64_t ss2 = 0;
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
       if (lane + 32 * i < nvec) {
         const uint32_t u[4] = {q[i].x, q[i].y, q[i].z, q[i].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float a = __uint_as_float(u[e] << 16);
-          const float c = __uint_as_float(u[e] & 0xFFFF0000u);
-          ss = fmaf(a, a, ss);
-          ss = fmaf(c, c, ss);
+          const uint64_t v = bf16x2_to_f2(u[e]);
+          ss2 = ffma2(v, v, ss2);
         }
       }
     }
-    ss = warp_sum(ss);
+    const float ss = warp_sum(f2_lo(ss2) + f2_hi(ss2));
     const float rstd = rsqrtf(ss / static_cast<float>(D) + eps);
+    const uint64_t rstd2 = f2_pack(rstd, rstd);
     const long r = static_cast<long>(b) * nb + rr;  // output row
-    // h of vector i of this row
-    auto modulated = [&](int i, float (&h)[8]) {
+    // h = x rstd (1 + scale) + shift of vector i of this row, as 4 pairs
+    auto modulated = [&](int i, uint64_t (&h)[4]) {
       const int vi = lane + 32 * i;
       const uint32_t u[4] = {q[i].x, q[i].y, q[i].z, q[i].w};
+      const uint64_t sc[4] = {smod2[2 * vi], smod2[2 * vi + 1], smod2[2 * (nvec + vi)],
+                              smod2[2 * (nvec + vi) + 1]};
+      const uint64_t sh[4] = {smod2[2 * (2 * nvec + vi)], smod2[2 * (2 * nvec + vi) + 1],
+                              smod2[2 * (3 * nvec + vi)], smod2[2 * (3 * nvec + vi) + 1]};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        h[2 * e] = __uint_as_float(u[e] << 16);
-        h[2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
-      }
-      const float4 s0 = smod[vi], s1 = smod[nvec + vi];
-      const float4 t0 = smod[2 * nvec + vi], t1 = smod[3 * nvec + vi];
-      const float scv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-      const float shv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
-#pragma unroll
-      for (int e = 0; e < 8; ++e) h[e] = fmaf(h[e] * rstd, scv[e], shv[e]);
+      for (int e = 0; e < 4; ++e) h[e] = ffma2(fmul2(bf16x2_to_f2(u[e]), rstd2), sc[e], sh[e]);
     };
     if constexpr (OUT_FP8) {
       float amax = 0.0f;
 #pragma unroll
       for (int i = 0; i < NV; ++i) {
         if (lane + 32 * i < nvec) {
-          float h[8];
+          uint64_t h[4];
           modulated(i, h);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(h[e]));
+          for (int e = 0; e < 4; ++e) amax = fmax3(amax, fabsf(f2_lo(h[e])), fabsf(f2_hi(h[e])));
         }
       }
       amax = warp_max(amax);
       const float qs = amax > 0.0f ? amax / 448.0f : 1.0f;
       const float inv = 1.0f / qs;
+      const uint64_t inv2 = f2_pack(inv, inv);
       uint8_t *hr = static_cast<uint8_t *>(h_out) + r * D;
 #pragma unroll
       for (int i = 0; i < NV; ++i) {
         const int vi = lane + 32 * i;
         if (vi < nvec) {
-          float h[8];
+          uint64_t h[4];
           modulated(i, h);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) h[e] = fmul2(h[e], inv2);
           uint2 w;
-          w.x = static_cast<uint32_t>(pack_e4m3x2(h[0] * inv, h[1] * inv)) |
-                (static_cast<uint32_t>(pack_e4m3x2(h[2] * inv, h[3] * inv)) << 16);
-          w.y = static_cast<uint32_t>(pack_e4m3x2(h[4] * inv, h[5] * inv)) |
-                (static_cast<uint32_t>(pack_e4m3x2(h[6] * inv, h[7] * inv)) << 16);
+          w.x = static_cast<uint32_t>(pack_e4m3x2(f2_lo(h[0]), f2_hi(h[0]))) |
+                (static_cast<uint32_t>(pack_e4m3x2(f2_lo(h[1]), f2_hi(h[1]))) << 16);
+          w.y = static_cast<uint32_t>(pack_e4m3x2(f2_lo(h[2]), f2_hi(h[2]))) |
+                (static_cast<uint32_t>(pack_e4m3x2(f2_lo(h[3]), f2_hi(h[3]))) << 16);
           reinterpret_cast<uint2 *>(hr)[vi] = w;
         }
       }
@@ -416,14 +420,15 @@ __global__ void __launch_bounds__(NORM2_THREADS, 1)
       for (int i = 0; i < NV; ++i) {
         const int vi = lane + 32 * i;
         if (vi < nvec) {
-          float h[8];
+          uint64_t h[4];
           modulated(i, h);
-          reinterpret_cast<uint4 *>(hr)[vi] =
-              make_uint4(pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]),
-                         pack_bf16x2(h[4], h[5]), pack_bf16x2(h[6], h[7]));
+          reinterpret_cast<uint4 *>(hr)[vi] = make_uint4(
+              pack_bf16x2(f2_lo(h[0]), f2_hi(h[0])), pack_bf16x2(f2_lo(h[1]), f2_hi(h[1])),
+              pack_bf16x2(f2_lo(h[2]), f2_hi(h[2])), pack_bf16x2(f2_lo(h[3]), f2_hi(h[3])));
         }
       }
     }
+    if (rr + NORM2_WARPS < r_end) load_row(rr + NORM2_WARPS, q);
   }
 }
 
