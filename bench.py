@@ -32,10 +32,13 @@ sys.path.insert(0, ROOT)
 METRIC = ("DiT block fwd TFLOP/s & ms at 1024px (4608d, 4096+512 tok), % of B200 tensor peak")
 KERNEL_NAMES = ["adaln", "rope_table", "norm1", "qkv_norm_rope", "attention", "out_proj_residual",
                 "norm2", "gate_up_swiglu", "down_residual"]
-KERNEL_NAMES_FP8 = ["adaln", "rope_table", "norm1", "qkv_norm_rope", "attention", "quantize_o",
-                    "out_proj_residual", "norm2", "gate_up_swiglu", "quantize_u", "down_residual"]
+# FP8: the attention and SwiGLU epilogues write their outputs as MX8 (E4M3
+# with a scale per 32 elements), so the two trace intervals that held the
+# activation quantisers stay empty ("*_none": no kernel launches there).
+KERNEL_NAMES_FP8 = ["adaln", "rope_table", "norm1", "qkv_norm_rope", "attention", "o_mx8_none",
+                    "out_proj_residual", "norm2", "gate_up_swiglu", "u_mx8_none", "down_residual"]
 # NVFP4 Mixed: norm2 and the NVFP4 quantiser of h2 share one trace interval
-KERNEL_NAMES_NVFP4 = ["adaln", "rope_table", "norm1", "qkv_norm_rope", "attention", "quantize_o",
+KERNEL_NAMES_NVFP4 = ["adaln", "rope_table", "norm1", "qkv_norm_rope", "attention", "o_mx8_none",
                       "out_proj_residual", "norm2_quantize", "gate_up_swiglu", "quantize_u",
                       "down_residual"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -102,11 +105,9 @@ def kernel_bytes(cfg, name):
         return M * D * (xs + hs)
     if name == "rope_table":
         return L * (3 * 4 + 2 * 64 * 4)
-    if name == "quantize_o":
-        return M * D * 3
     if name == "quantize_u":
-        # NVFP4: bf16 in, codes (1/2 B) and scales (1/16 B) out; FP8: bf16 in, byte out
-        return M * cfg.I * (2.5625 if cfg.w_dtype == "nvfp4_mixed" else 3)
+        # NVFP4: bf16 in, codes (1/2 B) and scales (1/16 B) out
+        return M * cfg.I * 2.5625
     if name == "norm2_quantize":
         # x in, bf16 h2 out and back in, NVFP4 codes and scales out
         return M * D * (xs + 4.5625)
@@ -535,7 +536,8 @@ def run_ours(args, rank, local_rank, world):
         "device_error": ig4.ig4_status_string(err),
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e / K, 4)},
-        "gpu_launches": (n_launch + (1 if nv4 else 0)) * K,  # NVFP4: norm2 + quantiser share a slot
+        # empty intervals launch nothing; NVFP4: norm2 + quantiser share a slot
+        "gpu_launches": (sum(1 for n in names if not n.endswith("_none")) + (1 if nv4 else 0)) * K,
         "kernel_ms_basis": "CUDA events between the kernels of K further traced calls",
         "cpu_baseline": cpu_base,
     }

@@ -227,6 +227,23 @@ ig4_status ig4_swiglu(int M, int I, int K, const void *h, int h_dtype, const flo
 ig4_status ig4_quantize_rows(int M, int K, const void *x, void *q_out, float *scale_out,
                              void *stream);
 
+/* Block quantisation of an activation to MX8, the form the FP8 block feeds
+ * its out- and down-projections (block-scaled E4M3, tcgen05 kind::mxf8f6f4;
+ * the release weights' FP8 E4M3 format is from "Ideogram 4 快速开始",
+ * hardware and precision section; the 32-element blocks are this library's
+ * choice): for every 32 consecutive elements of a row with amax = max |x|,
+ * e = ceil(log2(float(amax / 448))) (at least -126; 0 for a zero block),
+ * codes = RNE_E4M3(x * 2^-e) saturated to +-448, scale byte = e + 127.
+ * x bf16 [M][K]; codes_out E4M3 [M][K]; sf_out receives the scale bytes in
+ * the tensor cores' order: the 4 scales of row r and 128-element k-block kb
+ * at byte 512 ((r / 128) (K / 128) + kb) + 16 (r % 32) + 4 ((r % 128) / 32),
+ * ig4_mx8_scale_bytes(M, K) bytes (rows padded to a multiple of 128; the
+ * padding is not written).  K % 128 == 0, K <= 65536; x and codes_out
+ * 16-byte aligned.  Errors: IG4_ERR_INVALID_ARG. */
+ig4_status ig4_quantize_mx8(int M, int K, const void *x, void *codes_out, void *sf_out,
+                            void *stream);
+size_t ig4_mx8_scale_bytes(int M, int K);
+
 /* --------------------------------------------------------- whole block ---
  * Bytes of workspace ig4_block_forward needs for cfg (0 if cfg is invalid). */
 size_t ig4_workspace_size(const ig4_config *cfg);

@@ -40,6 +40,9 @@ from .ig4_oracle import (  # noqa: F401
     modulate,
     nvfp4_activation_values,
     quantize_nvfp4_activations,
+    quantize_mx8_activations,
+    mx8_values,
+    MX8_BLOCK,
     mrope_angles,
     mrope_axis_of_pair,
     mrope_positions,

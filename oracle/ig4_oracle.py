@@ -546,6 +546,48 @@ def quantize_nvfp4_activations(x):
     return e2m1_encode(q), sc, s
 
 
+MX8_BLOCK = 32            # elements per scale of the FP8 block's MX8 activations
+
+
+def quantize_mx8_activations(x):
+    """Activation rows -> MX8: (E4M3 codes uint8 [M, K], scale bytes uint8
+    [M, K/32]) with x[m, k] ~= 2^(scale[m, k/32] - 127) * e4m3(code[m, k]).
+
+    The FP8 block's out- and down-projections take their activations in this
+    form (the release weights are FP8 E4M3, "Ideogram 4 快速开始", section on
+    hardware and precision; sharing a power-of-two scale per 32 elements is
+    the implementation's reading, not the pages').  Per block of 32
+    consecutive elements of a row:
+      amax = max |x|;
+      e    = ceil(log2(float32(amax / 448))), at least -126; 0 for amax = 0;
+      code = RNE_E4M3(x * 2^-e), saturating at +-448;
+      scale byte = e + 127.
+    The quotient amax / 448 is rounded to float32 (the precision the
+    quantising kernel takes the decision in); x * 2^-e is exact.
+    """
+    x = np.asarray(x, dtype=np.float32)
+    M, K = x.shape
+    assert K % MX8_BLOCK == 0
+    blocks = x.reshape(M, K // MX8_BLOCK, MX8_BLOCK).astype(np.float64)
+    amax = np.abs(x).reshape(M, K // MX8_BLOCK, MX8_BLOCK).max(axis=2)
+    v = (amax / np.float32(E4M3_MAX)).astype(np.float32).astype(np.float64)
+    e = np.zeros(amax.shape, dtype=np.int64)
+    nz = v > 0
+    mant, ex = np.frexp(v[nz])                 # v = mant * 2^ex, mant in [0.5, 1)
+    e[nz] = np.where(mant == 0.5, ex - 1, ex)  # ceil(log2 v)
+    e = np.where(amax > 0, np.maximum(e, -126), 0)
+    codes = e4m3_encode(blocks * np.ldexp(1.0, -e)[..., None]).reshape(M, K)
+    return codes, (e + 127).astype(np.uint8)
+
+
+def mx8_values(codes, scales) -> np.ndarray:
+    """float64 values of MX8 codes and scale bytes."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    M, K = codes.shape
+    vals = e4m3_decode_table()[codes].reshape(M, K // MX8_BLOCK, MX8_BLOCK)
+    return (vals * np.ldexp(1.0, np.asarray(scales, dtype=np.int64) - 127)[..., None]).reshape(M, K)
+
+
 def nvfp4_activation_values(x) -> np.ndarray:
     """float64 values of the NVFP4 quantisation of bf16 activations:
     s[m] * decode_E4M3(sc[m, k / 16]) * decode_E2M1(code[m, k]), taken of the

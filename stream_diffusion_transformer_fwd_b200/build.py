@@ -20,6 +20,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libig4.so")
 SOURCES = ["ig4_api.cu"]
 DEPS = ["ig4_api.cu", "ig4_ptx.cuh", "ig4_gemm.cuh", "ig4_attention.cuh", "ig4_small.cuh",
+        "ig4_mx8.cuh",
         "ig4_nvf4.cuh", "ig4_parallel.cuh"]
 
 

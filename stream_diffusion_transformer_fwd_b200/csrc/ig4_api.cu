@@ -17,6 +17,7 @@
 #include "ig4.h"
 #include "ig4_attention.cuh"
 #include "ig4_gemm.cuh"
+#include "ig4_mx8.cuh"
 #include "ig4_nvf4.cuh"
 #include "ig4_parallel.cuh"
 #include "ig4_small.cuh"
@@ -460,9 +461,11 @@ size_t att_part_bytes(int B, int H, int L) {
 }
 
 // part: att_part_bytes(B, H, L) bytes of workspace for the balanced grid, or
-// nullptr (one worker per item).
+// nullptr (one worker per item).  o_sf != nullptr: o receives MX8 (E4M3
+// codes [B*L][H*256] and the packed scales in o_sf) instead of bf16.
 ig4_status launch_attention(int B, int H, int L, const void *q, const void *k, const void *vt,
-                            int vt_ld, void *o, void *part, cudaStream_t st) {
+                            int vt_ld, void *o, void *part, cudaStream_t st,
+                            void *o_sf = nullptr) {
   DeviceInfo *di = nullptr;
   IG4_TRY(device_info(&di));
   const long BH = static_cast<long>(B) * H;
@@ -497,13 +500,13 @@ ig4_status launch_attention(int B, int H, int L, const void *q, const void *k, c
     lc.attrs = attr;
     lc.numAttrs = 2;
     if (cudaLaunchKernelEx(&lc, attention_kernel<true>, mq, mk, mv, op, L, H,
-                           static_cast<int>(BH), pp) != cudaSuccess)
+                           static_cast<int>(BH), pp, static_cast<uint8_t *>(o_sf)) != cudaSuccess)
       return IG4_ERR_CUDA;
   } else {
     IG4_TRY(allow_smem(attention_kernel<false>, ATT_SMEM_BYTES));
     if (launch_pdl(attention_kernel<false>, dim3(plan.workers), dim3(ATT_THREADS),
-                   ATT_SMEM_BYTES, st, mq, mk, mv, op, L, H, static_cast<int>(BH),
-                   pp) != cudaSuccess)
+                   ATT_SMEM_BYTES, st, mq, mk, mv, op, L, H, static_cast<int>(BH), pp,
+                   static_cast<uint8_t *>(o_sf)) != cudaSuccess)
       return IG4_ERR_CUDA;
   }
   IG4_TRY(last_launch_status());
@@ -514,10 +517,10 @@ ig4_status launch_attention(int B, int H, int L, const void *q, const void *k, c
     const cudaError_t e =
         plan.pair ? launch_pdl(attention_combine_kernel<true>, grid, dim3(ATT_COMBINE_THREADS), 0,
                                st, static_cast<const uint8_t *>(pp), op, L, H,
-                               static_cast<int>(BH), plan.workers)
+                               static_cast<int>(BH), plan.workers, static_cast<uint8_t *>(o_sf))
                   : launch_pdl(attention_combine_kernel<false>, grid, dim3(ATT_COMBINE_THREADS),
                                0, st, static_cast<const uint8_t *>(pp), op, L, H,
-                               static_cast<int>(BH), plan.workers);
+                               static_cast<int>(BH), plan.workers, static_cast<uint8_t *>(o_sf));
     if (e != cudaSuccess) return IG4_ERR_CUDA;
     IG4_TRY(last_launch_status());
   }
@@ -618,6 +621,132 @@ ig4_status launch_swiglu(int M, int I, int K, const void *h, bool f8, const floa
   }
   EpiSwiGLU<false> e{static_cast<__nv_bfloat16 *>(u), I, M, nullptr, nullptr, nullptr};
   return launch_gemm<256, false, true>(ma, mg, mu, M, I / 128, K, e, st);
+}
+
+// ------------------------------------------------- MX8 (FP8, 1x32 scales)
+// The FP8 block feeds the out- and down-projections MX8 activations (E4M3
+// with a UE8M0 scale per 32 elements, written by the attention and SwiGLU
+// epilogues) through the block-scaled pair GEMM.  K % 128 == 0, N % 192 == 0
+// or N % 256 == 0.
+inline bool mx8_ok(long N, long K) { return K % 128 == 0 && (N % 192 == 0 || N % 256 == 0); }
+
+// bytes of packed MX8 scales of an [M][K] operand (rows padded to 128)
+inline size_t mx8_sf_bytes(long M, long K) { return static_cast<size_t>((M + 127) / 128) * (K / 128) * 512; }
+
+ig4_status launch_mx8_quantize(int M, int K, const void *x, void *codes, void *sf,
+                               cudaStream_t st) {
+  if (K % 128) return IG4_ERR_UNSUPPORTED;
+  const int rows_per_cta = MX8Q_THREADS / 32;
+  if (launch_pdl(quantize_mx8_kernel, dim3((M + rows_per_cta - 1) / rows_per_cta),
+                 dim3(MX8Q_THREADS), 0, st, static_cast<const __nv_bfloat16 *>(x), M, K,
+                 static_cast<uint8_t *>(codes), static_cast<uint8_t *>(sf)) != cudaSuccess)
+    return IG4_ERR_CUDA;
+  return last_launch_status();
+}
+
+// scale chunks [row blocks][K/128][128 words]; a box is one chunk
+ig4_status map_mx8_sf(CUtensorMap *m, const void *base, long rows, long K) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return IG4_ERR_CUDA;
+  const long rb = (rows + 127) / 128;
+  cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(K / 128), static_cast<cuuint64_t>(rb)};
+  cuuint64_t strides[2] = {512, static_cast<cuuint64_t>(K / 128) * 512};
+  cuuint32_t box[3] = {128, 1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void *>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? IG4_OK : IG4_ERR_CUDA;
+}
+
+// Block-scaled pair GEMM with A in MX8: 192-wide tiles (gemm_pair_kernel's
+// MX8A variant) where N % 192 == 0 - on N = 4608 they fill the last wave of
+// pairs better than 256-wide ones and keep the accumulators apart - else
+// 256-wide tiles with overlapping accumulators (gemm_mx8_pair_kernel).
+template <int BN, class Epi>
+ig4_status launch_mx8_gemm(const void *a_codes, const void *a_sf, const void *w, int M, int N,
+                           int K, const Epi &ep, cudaStream_t st) {
+  static_assert(BN == 192 || BN == 256, "MX8 tile width");
+  if (K % 128 || N % BN) return IG4_ERR_UNSUPPORTED;
+  CUtensorMap ma, mb, msa;
+  IG4_TRY(map_2d(&ma, a_codes, 1, M, K, K, GEMM_BM, 128));
+  IG4_TRY(map_2d(&mb, w, 1, N, K, K, BN / 2, 128));
+  IG4_TRY(map_mx8_sf(&msa, a_sf, M, K));
+  DeviceInfo *di = nullptr;
+  IG4_TRY(device_info(&di));
+  const int n_tiles_n = N / BN;
+  const long tiles = static_cast<long>((M + 2 * GEMM_BM - 1) / (2 * GEMM_BM)) * n_tiles_n;
+  const int pairs = static_cast<int>(std::min<long>(tiles, di->sms / 2));
+  const int group_m = gemm_group_m(M, K, 1);
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(2 * pairs);
+  lc.blockDim = dim3(GEMM_THREADS);
+  lc.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 2;
+  cudaError_t e;
+  if constexpr (BN == 192) {
+    auto kern = gemm_pair_kernel<192, true, false, Epi, true>;
+    constexpr int SMEM = PairShape<192, true>::SMEM_BYTES;
+    IG4_TRY(allow_smem(kern, SMEM));
+    lc.dynamicSmemBytes = SMEM;
+    e = cudaLaunchKernelEx(&lc, kern, ma, mb, msa, M, n_tiles_n, K, group_m, ep);
+  } else {
+    auto kern = gemm_mx8_pair_kernel<Epi>;
+    IG4_TRY(allow_smem(kern, MX8P_SMEM_BYTES));
+    lc.dynamicSmemBytes = MX8P_SMEM_BYTES;
+    e = cudaLaunchKernelEx(&lc, kern, ma, mb, msa, M, n_tiles_n, K, group_m, ep);
+  }
+  if (e != cudaSuccess) return IG4_ERR_CUDA;
+  return last_launch_status();
+}
+
+template <int BN, typename XT>
+ig4_status launch_mx8_resid_bn(int B, int L, int N, int K, const void *a_codes, const void *a_sf,
+                               const void *w, const float *w_scale, const float *gate,
+                               int gate_stride, const void *x_res, void *x_out, cudaStream_t st) {
+  const int M = B * L;
+  EpiResidGate<BN, true, XT> e{static_cast<const XT *>(x_res), static_cast<XT *>(x_out), gate,
+                               gate_stride, L, M, N, nullptr, w_scale};
+  return launch_mx8_gemm<BN>(a_codes, a_sf, w, M, N, K, e, st);
+}
+
+// x_out = x_res + gate * (w_scale (A W^T)) with A in MX8.
+ig4_status launch_mx8_resid(int B, int L, int N, int K, const void *a_codes, const void *a_sf,
+                            const void *w, const float *w_scale, const float *gate,
+                            int gate_stride, const void *x_res, void *x_out, int x_dtype,
+                            cudaStream_t st) {
+  const bool f32 = x_dtype == IG4_F32;
+  if (N % 192 == 0)
+    return f32 ? launch_mx8_resid_bn<192, float>(B, L, N, K, a_codes, a_sf, w, w_scale, gate,
+                                                 gate_stride, x_res, x_out, st)
+               : launch_mx8_resid_bn<192, __nv_bfloat16>(B, L, N, K, a_codes, a_sf, w, w_scale,
+                                                         gate, gate_stride, x_res, x_out, st);
+  return f32 ? launch_mx8_resid_bn<256, float>(B, L, N, K, a_codes, a_sf, w, w_scale, gate,
+                                               gate_stride, x_res, x_out, st)
+             : launch_mx8_resid_bn<256, __nv_bfloat16>(B, L, N, K, a_codes, a_sf, w, w_scale,
+                                                       gate, gate_stride, x_res, x_out, st);
+}
+
+// FP8 SwiGLU writing u as MX8 (codes [M][I], packed scales).  I % 128 == 0.
+ig4_status launch_swiglu_mx8(int M, int I, int K, const void *h, const float *h_scale,
+                             const void *wg, const void *wu, const float *sg, const float *su,
+                             void *uq, void *usf, cudaStream_t st) {
+  if (I % 128) return IG4_ERR_UNSUPPORTED;
+  CUtensorMap ma, mg, mu;
+  IG4_TRY(map_2d(&ma, h, 1, M, K, K, GEMM_BM, 128));
+  IG4_TRY(map_2d(&mg, wg, 1, I, K, K, 128, 128));
+  IG4_TRY(map_2d(&mu, wu, 1, I, K, K, 128, 128));
+  EpiSwiGLUMx8 e{static_cast<uint8_t *>(uq), static_cast<uint8_t *>(usf), I, M, h_scale, sg, su};
+  return launch_gemm<256, true, true>(ma, mg, mu, M, I / 128, K, e, st);
 }
 
 // E4M3 weight [N][K] with per-row scale -> bf16 [N][K].  K % 16 == 0.
@@ -867,11 +996,20 @@ struct BlockWs {
   void *u;        // bf16 [M][I]
   void *uq;       // e4m3 [M][I]
   float *u_scale;
-  void *h_sf, *u_sf;  // packed NVFP4 scales of h2 and u (NVFP4-mixed FFN)
+  void *h_sf, *u_sf;  // packed NVFP4 scales of h2 and u (NVFP4-mixed FFN); u_sf: MX8 scales of u (FP8)
+  void *o_sf;         // MX8 scales of the attention output (FP8 weights)
   void *att_part;     // attention partial slots: the u buffer (u is written after attention)
   int vt_ld;
   size_t bytes;
 };
+
+// The FP8 block's MX8 stages: the attention output into the out-projection
+// (N = K = D), u into the down-projection (N = D, K = I; not with the NVFP4
+// FFN).
+inline bool mx8_attn_out(const ig4_config *c) { return is_fp8(c->w_dtype) && mx8_ok(c->D, c->D); }
+inline bool mx8_ffn(const ig4_config *c) {
+  return is_fp8(c->w_dtype) && !is_nvf4_mixed(c->w_dtype) && mx8_ok(c->D, c->I);
+}
 
 // Lays the block's buffers out from `base` (nullptr: only count bytes).
 BlockWs block_ws_layout(const ig4_config *c, uint8_t *base) {
@@ -907,7 +1045,8 @@ BlockWs block_ws_layout(const ig4_config *c, uint8_t *base) {
   // NVFP4 FFN: h2 codes reuse oq (M D / 2 bytes), u codes reuse uq
   const long rb = (M + 127) / 128;
   w.h_sf = take(nv4 ? rb * (D / 64) * 512 : 0);
-  w.u_sf = take(nv4 ? rb * (I / 64) * 512 : 0);
+  w.u_sf = take(nv4 ? rb * (I / 64) * 512 : (mx8_ffn(c) ? mx8_sf_bytes(M, I) : 0));
+  w.o_sf = take(mx8_attn_out(c) ? mx8_sf_bytes(M, D) : 0);
   w.bytes = off;
   return w;
 }
@@ -979,19 +1118,28 @@ ig4_status block_pre_attention(const ig4_config *c, const ig4_block_weights *w, 
 // residual (x_in -> x_out), norm2, SwiGLU, down-projection + gated residual
 // (in place in x_out).  The AdaLN modulation is read from ws.mod.
 ig4_status block_post_attention(const ig4_config *c, const ig4_block_weights *w, const void *x_in,
-                                void *x_out, const BlockWs &ws, cudaStream_t st, Tracer &t) {
+                                void *x_out, const BlockWs &ws, cudaStream_t st, Tracer &t,
+                                bool o_is_mx8 = false) {
   const int L = c->T_text + c->grid_t * c->grid_h * c->grid_w;
   const int M = c->B * L;
   const int D = c->D, I = c->I;
   const bool f8 = is_fp8(c->w_dtype);
   const int hdt = f8 ? IG4_E4M3 : IG4_BF16;
   const int ms = 6 * D;
-  if (f8) {
-    IG4_TRY(launch_quantize(M, D, ws.o, ws.oq, ws.o_scale, st));
+  if (f8 && mx8_attn_out(c)) {
+    // MX8 attention output: written by the attention epilogue, or encoded here
+    if (!o_is_mx8) IG4_TRY(launch_mx8_quantize(M, D, ws.o, ws.oq, ws.o_sf, st));
     IG4_TRY(t.mark());
+    IG4_TRY(launch_mx8_resid(c->B, L, D, D, ws.oq, ws.o_sf, w->w_o, w->s_o, ws.mod + 2 * D, ms,
+                             x_in, x_out, c->x_dtype, st));
+  } else {
+    if (f8) {
+      IG4_TRY(launch_quantize(M, D, ws.o, ws.oq, ws.o_scale, st));
+      IG4_TRY(t.mark());
+    }
+    IG4_TRY(launch_resid(c->B, L, D, D, f8 ? ws.oq : ws.o, f8, ws.o_scale, w->w_o, w->s_o,
+                         ws.mod + 2 * D, ms, x_in, x_out, c->x_dtype, st));
   }
-  IG4_TRY(launch_resid(c->B, L, D, D, f8 ? ws.oq : ws.o, f8, ws.o_scale, w->w_o, w->s_o,
-                       ws.mod + 2 * D, ms, x_in, x_out, c->x_dtype, st));
   IG4_TRY(t.mark());
   if (is_nvf4_mixed(c->w_dtype)) {
     // FFN in NVFP4: h2 (bf16) and u (bf16) are quantised to NVFP4 for the
@@ -1013,6 +1161,17 @@ ig4_status block_post_attention(const ig4_config *c, const ig4_block_weights *w,
   IG4_TRY(launch_norm(M, L, D, x_out, c->x_dtype, ws.mod + 3 * D, ws.mod + 4 * D, ms, c->eps,
                       ws.h, hdt, ws.h_scale, 0, 0, 0, st));
   IG4_TRY(t.mark());
+  if (mx8_ffn(c)) {
+    // u leaves the SwiGLU epilogue as MX8 (its trace slot after it stays empty)
+    IG4_TRY(launch_swiglu_mx8(M, I, D, ws.h, ws.h_scale, w->w_gate, w->w_up, w->s_gate, w->s_up,
+                              ws.uq, ws.u_sf, st));
+    IG4_TRY(t.mark());
+    IG4_TRY(t.mark());
+    IG4_TRY(launch_mx8_resid(c->B, L, D, I, ws.uq, ws.u_sf, w->w_down, w->s_down, ws.mod + 5 * D,
+                             ms, x_out, x_out, c->x_dtype, st));
+    IG4_TRY(t.mark());
+    return IG4_OK;
+  }
   IG4_TRY(launch_swiglu(M, I, D, ws.h, f8, ws.h_scale, w->w_gate, w->w_up, w->s_gate, w->s_up,
                         ws.u, st));
   IG4_TRY(t.mark());
@@ -1037,9 +1196,11 @@ ig4_status block_forward_impl(const ig4_config *c, const ig4_block_weights *w, c
   Tracer none{nullptr, 0, 0, st};
   Tracer &t = tr ? *tr : none;
   IG4_TRY(block_pre_attention(c, w, x_in, pos, temb, ws, st, t, rope_ready));
-  IG4_TRY(launch_attention(c->B, c->H, L, ws.q, ws.k, ws.vt, ws.vt_ld, ws.o, ws.att_part, st));
+  const bool mx8 = mx8_attn_out(c);  // FP8: the attention epilogue writes MX8
+  IG4_TRY(launch_attention(c->B, c->H, L, ws.q, ws.k, ws.vt, ws.vt_ld, mx8 ? ws.oq : ws.o,
+                           ws.att_part, st, mx8 ? ws.o_sf : nullptr));
   IG4_TRY(t.mark());
-  return block_post_attention(c, w, x_in, x_out, ws, st, t);
+  return block_post_attention(c, w, x_in, x_out, ws, st, t, mx8);
 }
 
 // Stack workspace: two sequence buffers, the block workspace, final-layer buffers.
@@ -1241,6 +1402,19 @@ ig4_status ig4_quantize_rows(int M, int K, const void *x, void *q_out, float *sc
     return IG4_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(q_out)) return IG4_ERR_INVALID_ARG;
   return launch_quantize(M, K, x, q_out, scale_out, as_stream(stream));
+}
+
+ig4_status ig4_quantize_mx8(int M, int K, const void *x, void *codes_out, void *sf_out,
+                            void *stream) {
+  if (M < 1 || K < 128 || K % 128 || K > 65536 || !x || !codes_out || !sf_out)
+    return IG4_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes_out)) return IG4_ERR_INVALID_ARG;
+  return launch_mx8_quantize(M, K, x, codes_out, sf_out, as_stream(stream));
+}
+
+size_t ig4_mx8_scale_bytes(int M, int K) {
+  if (M < 1 || K < 128 || K % 128) return 0;
+  return mx8_sf_bytes(M, K);
 }
 
 size_t ig4_workspace_size(const ig4_config *cfg) {

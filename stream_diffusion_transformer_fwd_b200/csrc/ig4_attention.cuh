@@ -82,6 +82,7 @@
 // range.  Every wait is bounded.
 #pragma once
 
+#include "ig4_mx8.cuh"
 #include "ig4_ptx.cuh"
 
 namespace ig4 {
@@ -225,7 +226,8 @@ template <bool PAIR>
 __global__ void __launch_bounds__(ATT_THREADS, 1)
     attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, __nv_bfloat16 *__restrict__ o_out,
-                     int L, int H, int n_bh, uint8_t *__restrict__ part) {
+                     int L, int H, int n_bh, uint8_t *__restrict__ part,
+                     uint8_t *__restrict__ o_sf) {
   constexpr int CTAS = PAIR ? 2 : 1;
   constexpr int UPI = PAIR ? 1 : 2;  // ring units (slots) per item
   extern __shared__ uint8_t smem_raw[];
@@ -647,6 +649,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         ml[ATT_BM + r] = l_sum;
       }
       const bool store = valid || sg.slot >= 0;
+      // MX8 output (o_sf != nullptr): E4M3 codes in o_out's bytes, a scale per 32 dims
+      const bool mx8 = o_sf != nullptr && sg.slot < 0;
       // O in two halves of 128 columns: four TMEM loads in flight per wait
 #pragma unroll 1
       for (int hc = 0; hc < ATT_DH; hc += 128) {
@@ -655,6 +659,23 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_base + ATT_TMEM_O + hc + 32 * c, o[c]);
         tmem_ld_wait();
         if (!store) continue;
+        if (mx8) {
+          const long grow = static_cast<long>(b) * L + lq;
+          const int HD = H * ATT_DH;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[c][i] *= inv;
+            uint4 q[2];
+            const uint8_t sb = mx8_encode32(o[c], q);
+            const int col = h * ATT_DH + hc + 32 * c;
+            uint4 *d = reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(o_out) + grow * HD + col);
+            d[0] = q[0];
+            d[1] = q[1];
+            o_sf[mx8_sf_offset(static_cast<int>(grow), col / MX8_BLOCK, HD)] = sb;
+          }
+          continue;
+        }
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint4 *d = reinterpret_cast<uint4 *>(dst + hc + 32 * c);
@@ -704,7 +725,7 @@ constexpr int ATT_COMBINE_ROWS = ATT_COMBINE_THREADS / 32;
 template <bool PAIR>
 __global__ void __launch_bounds__(ATT_COMBINE_THREADS)
     attention_combine_kernel(const uint8_t *__restrict__ part, __nv_bfloat16 *__restrict__ o_out,
-                             int L, int H, int n_bh, int G) {
+                             int L, int H, int n_bh, int G, uint8_t *__restrict__ o_sf) {
   constexpr int CTAS = PAIR ? 2 : 1;
   pdl_wait();
   pdl_trigger();
@@ -757,6 +778,31 @@ __global__ void __launch_bounds__(ATT_COMBINE_THREADS)
     }
   }
   const float inv = 1.0f / warp_sum(l);
+  if (o_sf != nullptr) {
+    // MX8 output: lanes 4j .. 4j + 3 hold a block of 32 head dims
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      acc[i] = bf16_round(acc[i] * inv);  // the bf16 output's value, encoded
+      amax = fmaxf(amax, fabsf(acc[i]));
+    }
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    const int e = mx8_exponent(amax);
+    const float is = mx8_inv_scale(e);
+    const long grow = static_cast<long>(b) * L + lq;
+    const int HD = H * ATT_DH;
+    const int col = h * ATT_DH + 8 * lane;
+    uint2 w;
+    w.x = static_cast<uint32_t>(pack_e4m3x2(acc[0] * is, acc[1] * is)) |
+          (static_cast<uint32_t>(pack_e4m3x2(acc[2] * is, acc[3] * is)) << 16);
+    w.y = static_cast<uint32_t>(pack_e4m3x2(acc[4] * is, acc[5] * is)) |
+          (static_cast<uint32_t>(pack_e4m3x2(acc[6] * is, acc[7] * is)) << 16);
+    *reinterpret_cast<uint2 *>(reinterpret_cast<uint8_t *>(o_out) + grow * HD + col) = w;
+    if ((lane & 3) == 0)
+      o_sf[mx8_sf_offset(static_cast<int>(grow), col / MX8_BLOCK, HD)] = static_cast<uint8_t>(e + 127);
+    return;
+  }
   __nv_bfloat16 *dst = o_out + (static_cast<long>(b) * L + lq) * (static_cast<long>(H) * ATT_DH) +
                        h * ATT_DH + 8 * lane;
   *reinterpret_cast<uint4 *>(dst) =

@@ -222,7 +222,8 @@ struct EpiResidGate {
     const int row = m0 + r;
     const bool valid = row < M;
     const int b = valid ? row / L : 0;
-    const float rs = (FP8 && valid) ? __ldg(a_scale + row) : 1.0f;
+    // a_scale == nullptr: A's scales were applied by the tensor cores (MX8)
+    const float rs = (FP8 && valid && a_scale != nullptr) ? __ldg(a_scale + row) : 1.0f;
     const float *grow = gate + static_cast<long>(b) * gate_stride + n0;
 #pragma unroll 1
     for (int c = lo; c < hi; c += 32) {
@@ -567,23 +568,32 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 // CTAs; both CTAs' loads complete on it); empty[s] and tfull[b] in both CTAs
 // (arrived by the leader's multicast commits); tempty[b] in the leader (one
 // arrival per epilogue warp of the pair).
-template <int BN>
+template <int BN, bool MX8A = false>
 struct PairShape {
   static_assert(BN == 256 || BN == 192, "pair tile width");
   static constexpr int A_BYTES = GEMM_BM * 128;          // 16 KB
   static constexpr int BH_BYTES = (BN / 2) * 128;        // 16 KB or 12 KB (a multiple of 1 KB)
-  static constexpr int STAGE_BYTES = A_BYTES + BH_BYTES;
+  static constexpr int SF_BYTES = MX8A ? 512 : 0;        // A's scale chunk (MX8)
+  static constexpr int STAGE_BYTES = A_BYTES + BH_BYTES + SF_BYTES;
   static constexpr int STAGES = BN == 256 ? 6 : 7;       // ~200 KB of shared memory
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 };
 
-template <int BN, bool FP8, bool DUAL_B, class Epi>
+// MX8A: A in MX8 (E4M3 with a UE8M0 scale per 32 elements, see ig4_mx8.cuh)
+// and B in E4M3 with unit block scales: tcgen05.mma kind::mxf8f6f4 with
+// block_scale; tmB2 then maps A's 512-byte scale chunks, which the leader
+// copies into TMEM once per k-block (one tcgen05.cp); B's scales (byte 127)
+// are written into TMEM once.  192-wide tiles only: the two accumulators
+// (384 columns) leave room for the scales.
+template <int BN, bool FP8, bool DUAL_B, class Epi, bool MX8A = false>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmB2, int M, int n_tiles_n, int K,
                      int group_m, const Epi epi) {
   static_assert(!DUAL_B || BN == 256, "SwiGLU pairs split 128 gate / 128 up rows");
-  using P = PairShape<BN>;
+  static_assert(!MX8A || (FP8 && !DUAL_B && BN == 192), "MX8 A: FP8, single B, 192-wide tiles");
+  using P = PairShape<BN, MX8A>;
+  constexpr uint32_t SFA_COL = 448, SFB_COL = 464;  // MX8A scale columns (after 2 x 192)
   constexpr int PAIR_STAGES = P::STAGES;
   constexpr int PAIR_STAGE_BYTES = P::STAGE_BYTES;
   constexpr int A_BYTES = P::A_BYTES;
@@ -597,6 +607,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   uint8_t *smem = align1024(smem_raw);
   uint8_t *sA = smem;
   uint8_t *sB = smem + PAIR_STAGES * A_BYTES;
+  uint8_t *sSF = sB + PAIR_STAGES * BH_BYTES;  // MX8A only
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + PAIR_STAGES * PAIR_STAGE_BYTES);
   uint64_t *empty = full + PAIR_STAGES;
   uint64_t *tfull = empty + PAIR_STAGES;
@@ -640,6 +651,19 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  if constexpr (MX8A) {
+    // B's unit scales (byte 127) in every lane of the B scale columns
+    if (warp < 4) {
+      uint32_t ones[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) ones[i] = 0x7F7F7F7Fu;
+      tmem_st32_u(tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + SFB_COL, ones);
+      tmem_st_wait();
+    }
+    tc_fence_before();
+    cluster_sync_all();
+    tc_fence_after();
+  }
   pdl_wait();
   pdl_trigger();
 
@@ -669,6 +693,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           else
             tma_load_2d_pair(sB + s * BH_BYTES, &tmB, bar, kb * BK,
                              nt * BN + static_cast<int>(rank) * (BN / 2));
+          if constexpr (MX8A)
+            tma_load_3d_pair(sSF + s * 512, &tmB2, bar, 0, kb,
+                             mt * 2 + static_cast<int>(rank));
           if (++s == PAIR_STAGES) {
             s = 0;
             ph ^= 1;
@@ -698,11 +725,16 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           tc_fence_after();
           const uint32_t a_base = smem_u32(sA + s * A_BYTES);
           const uint32_t b_base = smem_u32(sB + s * BH_BYTES);
+          if constexpr (MX8A)
+            tmem_cp_sf_pair(tmem_base + SFA_COL, sdesc_kmajor_none(smem_u32(sSF + s * 512), 128));
 #pragma unroll
           for (int kk = 0; kk < 128 / UK_BYTES; ++kk) {
             const uint64_t ad = sdesc_kmajor_sw128(a_base + kk * UK_BYTES);
             const uint64_t bd = sdesc_kmajor_sw128(b_base + kk * UK_BYTES);
-            if (FP8)
+            if constexpr (MX8A)
+              umma_mx8_pair(d_tmem, ad, bd, idesc_mx8(2 * GEMM_BM, BN, kk), tmem_base + SFA_COL,
+                            tmem_base + SFB_COL, (it | kk) != 0);
+            else if (FP8)
               umma_f8_pair(d_tmem, ad, bd, IDESC, (it | kk) != 0);
             else
               umma_bf16_pair(d_tmem, ad, bd, IDESC, (it | kk) != 0);

@@ -469,6 +469,26 @@ __device__ __forceinline__ void umma_nvf4_pair(uint32_t d_tmem, uint64_t a_desc,
       : "memory");
 }
 
+// Instruction descriptor of a block-scaled FP8 MMA: A, B E4M3 (format 0),
+// UE8M0 scales (bit 23), K-major, dense K = 32; scale factor ids of A in
+// bits [29,31) and of B in [4,6).
+__host__ __device__ constexpr uint32_t idesc_mx8(int M, int N, int a_sf_id) {
+  return (1u << 23) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24) | (static_cast<uint32_t>(a_sf_id) << 29);
+}
+
+__device__ __forceinline__ void umma_mx8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                              uint32_t idesc, uint32_t sfa_tmem,
+                                              uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], "
+      "p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
 // tcgen05.cp 32x128b.warpx4 for a CTA pair: issued by the leader, it copies
 // the 512-byte block at the same shared-memory offset of each CTA into that
 // CTA's TMEM.

@@ -92,6 +92,8 @@ _sig("ig4_gated_residual_linear", [_i, _i, _i, _i, _vp, _i, _vp, _vp, _i, _vp, _
                                    _vp, _i, _vp])
 _sig("ig4_swiglu", [_i, _i, _i, _vp, _i, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp])
 _sig("ig4_quantize_rows", [_i, _i, _vp, _vp, _vp, _vp])
+_sig("ig4_quantize_mx8", [_i, _i, _vp, _vp, _vp, _vp])
+_sig("ig4_mx8_scale_bytes", [_i, _i], ctypes.c_size_t)
 _sig("ig4_workspace_size", [ctypes.POINTER(Config)], ctypes.c_size_t)
 _sig("ig4_block_forward", [ctypes.POINTER(Config), ctypes.POINTER(BlockWeights), _vp, _vp, _vp,
                            _vp, _vp, ctypes.c_size_t, _vp])
@@ -143,7 +145,8 @@ EXPORTED = ("ig4_status_string", "ig4_abi_version", "ig4_mrope_positions", "ig4_
             "ig4_adaln_modulation", "ig4_norm_modulate", "ig4_qkv_project",
             "ig4_joint_attention", "ig4_joint_attention_workspace_size", "ig4_joint_attention_ws",
             "ig4_gated_residual_linear", "ig4_swiglu",
-            "ig4_quantize_rows", "ig4_workspace_size", "ig4_block_forward",
+            "ig4_quantize_rows", "ig4_quantize_mx8", "ig4_mx8_scale_bytes", "ig4_workspace_size",
+            "ig4_block_forward",
             "ig4_block_forward_traced", "ig4_block_forward_noalloc", "ig4_stack_workspace_size",
             "ig4_stack_forward", "ig4_stack_forward_tapped", "ig4_nvfp4_scale_bytes", "ig4_nvfp4_pack_scales",
             "ig4_nvfp4_linear", "ig4_nvfp4_quantize", "ig4_text_cond_workspace_size", "ig4_text_cond_project",
@@ -316,6 +319,15 @@ def ig4_swiglu(M, I, K, h, h_scale, w_gate, w_up, s_gate, s_up, u_out, stream=No
 def ig4_quantize_rows(M, K, x, q_out, scale_out, stream=None):
     _check(_lib.ig4_quantize_rows(M, K, _ptr(x), _ptr(q_out), _ptr(scale_out), _stream(stream)),
            "ig4_quantize_rows")
+
+
+def ig4_quantize_mx8(M, K, x, codes_out, sf_out, stream=None):
+    _check(_lib.ig4_quantize_mx8(M, K, _ptr(x), _ptr(codes_out), _ptr(sf_out), _stream(stream)),
+           "ig4_quantize_mx8")
+
+
+def ig4_mx8_scale_bytes(M, K) -> int:
+    return int(_lib.ig4_mx8_scale_bytes(M, K))
 
 
 def ig4_workspace_size(cfg: Config) -> int:
