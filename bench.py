@@ -46,11 +46,11 @@ REFERENCE_ROWS = 32
 # The source files that define each kernel's device code (a recorded DRAM
 # traffic figure is only reported while these are unchanged).
 KERNEL_SOURCES = {
-    "attention": ["ig4_attention.cuh", "ig4_ptx.cuh"],
+    "attention": ["ig4_attention.cuh", "ig4_ptx.cuh", "ig4_mx8.cuh"],
     "qkv_norm_rope": ["ig4_gemm.cuh", "ig4_ptx.cuh"],
-    "out_proj_residual": ["ig4_gemm.cuh", "ig4_ptx.cuh"],
-    "gate_up_swiglu": ["ig4_gemm.cuh", "ig4_ptx.cuh"],
-    "down_residual": ["ig4_gemm.cuh", "ig4_ptx.cuh"],
+    "out_proj_residual": ["ig4_gemm.cuh", "ig4_ptx.cuh", "ig4_mx8.cuh"],
+    "gate_up_swiglu": ["ig4_gemm.cuh", "ig4_ptx.cuh", "ig4_mx8.cuh"],
+    "down_residual": ["ig4_gemm.cuh", "ig4_ptx.cuh", "ig4_mx8.cuh"],
 }
 SMALL_KERNEL_SOURCES = ["ig4_small.cuh", "ig4_ptx.cuh"]
 # NVFP4 workloads: their FFN GEMMs are the NVFP4 kernels
