@@ -324,9 +324,10 @@ ig4_status launch_norm_t(int rows, int L, int D, const void *x, const float *shi
     const long per_cta2 = (static_cast<long>(rows) + di->sms - 1) / di->sms;
     const int rpc2 = static_cast<int>(std::max<long>(NORM2_WARPS, per_cta2));
     const dim3 grid2((nb + rpc2 - 1) / rpc2, B);
-    const size_t smem2 = 4ull * (D / 8) * sizeof(float4);
+    const size_t smem2 = norm2_smem_bytes(D);
 #define IG4_NORM2_CASE(NV)                                                                      \
   if (nv <= NV) {                                                                              \
+    IG4_TRY(allow_smem(norm_modulate_rows_kernel<FP8, NV>, static_cast<int>(smem2)));          \
     if (launch_pdl(norm_modulate_rows_kernel<FP8, NV>, grid2, dim3(NORM2_THREADS), smem2, st,  \
                    xp, shift, scale, mod_stride, L, D, eps, h, hs, remap_n, remap_L,           \
                    remap_off, rpc2) != cudaSuccess)                                            \

@@ -298,14 +298,25 @@ __global__ void rope_table_kernel(const int32_t *__restrict__ pos, int L, double
   sin_out[idx] = static_cast<float>(s);
 }
 
-// RMSNorm + modulate for a bf16 stream, the block's layout: 16 warps per
-// CTA, one row per warp at a time, the row held in registers (NV 16-byte
-// vectors per lane, no prefetch: the 16 warps keep 16 rows of loads in
-// flight per SM).  (1 + scale) and shift are staged in shared memory as four
-// planes of float4 -- elements 8v..8v+3 and 8v+4..8v+7 of each -- so the
-// lanes of a warp read consecutive 16-byte words (no bank conflicts).
-constexpr int NORM2_THREADS = 512;
-constexpr int NORM2_WARPS = NORM2_THREADS / 32;
+// RMSNorm + modulate for a bf16 stream, the block's layout: each CTA takes
+// rows_per_cta rows of one sample.  A producer warp streams the rows into a
+// ring of NORM2_SLOTS shared-memory slots with bulk copies (cp.async.bulk,
+// one row each), so ~150 KB of loads per SM are in flight regardless of the
+// SM's limit on outstanding load misses (which kept the register-loading
+// version of this kernel near 2 TB/s); 8 consumer warps take rows j,
+// j + 8, ... of the CTA, read each from its slot into registers (NV 16-byte
+// vectors per lane), free the slot and compute.  (1 + scale) and shift are
+// staged in shared memory as four planes of float4 -- elements 8v..8v+3 and
+// 8v+4..8v+7 of each -- so the lanes of a warp read consecutive 16-byte
+// words (no bank conflicts).
+constexpr int NORM2_CWARPS = 8;
+constexpr int NORM2_THREADS = 32 * (NORM2_CWARPS + 1);
+constexpr int NORM2_WARPS = NORM2_CWARPS;
+constexpr int NORM2_SLOTS = 16;
+// shared memory of a launch: modulation planes, row slots, barriers
+__host__ __device__ constexpr size_t norm2_smem_bytes(int D) {
+  return 4ull * (D / 8) * 16 + static_cast<size_t>(NORM2_SLOTS) * D * 2 + 2 * NORM2_SLOTS * 8 + 16;
+}
 
 template <bool OUT_FP8, int NV>
 __global__ void __launch_bounds__(NORM2_THREADS, 1)
@@ -323,24 +334,45 @@ __global__ void __launch_bounds__(NORM2_THREADS, 1)
   const int r_begin = blockIdx.x * rows_per_cta;
   const int r_end = min(r_begin + rows_per_cta, nb);
   if (r_begin >= nb) return;
+  const int nrows = r_end - r_begin;
   const int nvec = D / 8;
-  auto load_row = [&](int rr, uint4 (&q)[NV]) {
-    const long in_row = remap_n > 0 ? static_cast<long>(b) * remap_L + remap_off + rr
-                                    : static_cast<long>(b) * L + rr;
-    const uint4 *xr = reinterpret_cast<const uint4 *>(x + in_row * D);
-#pragma unroll
-    for (int i = 0; i < NV; ++i) {
-      const int vi = lane + 32 * i;
-      if (vi < nvec) q[i] = __ldg(xr + vi);
+  const uint32_t row_bytes = static_cast<uint32_t>(D) * 2;
+  uint8_t *slots = reinterpret_cast<uint8_t *>(smod + 4 * nvec);
+  uint64_t *full = reinterpret_cast<uint64_t *>(slots + static_cast<size_t>(NORM2_SLOTS) * row_bytes);
+  uint64_t *empty = full + NORM2_SLOTS;
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + NORM2_SLOTS);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NORM2_SLOTS; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
     }
-  };
-  // the warp's first row is in flight while the modulation vectors are staged
-  uint4 q[NV];
-  int rr = r_begin + warp;
-  if (rr < r_end) load_row(rr, q);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (warp == NORM2_CWARPS) {
+    // ------------------------------------------------ producer: one row per slot
+    if (lane == 0) {
+      int j = 0;
+      for (; j < nrows; ++j) {
+        const int slot = j % NORM2_SLOTS;
+        const uint32_t ph = static_cast<uint32_t>(j / NORM2_SLOTS) & 1;
+        if (j >= NORM2_SLOTS && !mbar_wait(&empty[slot], ph ^ 1, abort_flag)) break;
+        const int rr = r_begin + j;
+        const long in_row = remap_n > 0 ? static_cast<long>(b) * remap_L + remap_off + rr
+                                        : static_cast<long>(b) * L + rr;
+        mbar_arrive_expect_tx(&full[slot], row_bytes);
+        bulk_load(slots + static_cast<size_t>(slot) * row_bytes, x + in_row * D, row_bytes,
+                  &full[slot]);
+      }
+      if (j < nrows) sleep_ns(20000);  // let the copies already issued land
+    }
+    return;
+  }
+  // ---------------------------------------------------- consumers
   const float4 *sc4 = reinterpret_cast<const float4 *>(scale + static_cast<long>(b) * mod_stride);
   const float4 *sh4 = reinterpret_cast<const float4 *>(shift + static_cast<long>(b) * mod_stride);
-  for (int i = threadIdx.x; i < D / 4; i += NORM2_THREADS) {
+  for (int i = threadIdx.x; i < D / 4; i += 32 * NORM2_CWARPS) {
     float4 s = __ldg(sc4 + i);
     s.x += 1.0f;
     s.y += 1.0f;
@@ -350,9 +382,9 @@ __global__ void __launch_bounds__(NORM2_THREADS, 1)
     smod[hi * nvec + v] = s;
     smod[(2 + hi) * nvec + v] = __ldg(sh4 + i);
   }
-  __syncthreads();
+  named_barrier_sync(1, 32 * NORM2_CWARPS);
   const uint64_t *smod2 = reinterpret_cast<const uint64_t *>(smod);  // pairs of floats
-  for (; rr < r_end; rr += NORM2_WARPS) {
+  auto process = [&](int rr, const uint4 (&q)[NV]) {
     // sum of squares over the row: two elements per packed FMA
     uint64_t ss2 = 0;
 #pragma unroll
@@ -428,7 +460,22 @@ __global__ void __launch_bounds__(NORM2_THREADS, 1)
         }
       }
     }
-    if (rr + NORM2_WARPS < r_end) load_row(rr + NORM2_WARPS, q);
+  };
+  uint4 q[NV];
+  for (int j = warp; j < nrows; j += NORM2_CWARPS) {
+    const int slot = j % NORM2_SLOTS;
+    if (!mbar_wait_warp(&full[slot], static_cast<uint32_t>(j / NORM2_SLOTS) & 1, abort_flag))
+      break;
+    const uint4 *src = reinterpret_cast<const uint4 *>(slots + static_cast<size_t>(slot) * row_bytes);
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int vi = lane + 32 * i;
+      if (vi < nvec) q[i] = src[vi];
+    }
+    // the row is in registers: the slot may take the row NORM2_SLOTS further on
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[slot]);
+    process(r_begin + j, q);
   }
 }
 
