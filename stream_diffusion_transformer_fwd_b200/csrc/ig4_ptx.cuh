@@ -551,12 +551,6 @@ __device__ __forceinline__ bool mbar_wait_cluster_warp(uint64_t *bar, uint32_t p
   return __all_sync(0xffffffffu, ok);
 }
 
-// Barrier among `count` threads (a multiple of 32) under hardware barrier id
-// `id` (1..15; id 0 is __syncthreads').
-__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
 __device__ __forceinline__ void sleep_ns(unsigned int ns) {
   const unsigned long long t0 = globaltimer_ns();
   while (globaltimer_ns() - t0 < ns) __nanosleep(1000);

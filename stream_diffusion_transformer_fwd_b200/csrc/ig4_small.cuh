@@ -309,6 +309,12 @@ __global__ void rope_table_kernel(const int32_t *__restrict__ pos, int L, double
 // staged in shared memory as four planes of float4 -- elements 8v..8v+3 and
 // 8v+4..8v+7 of each -- so the lanes of a warp read consecutive 16-byte
 // words (no bank conflicts).
+// Barrier among `count` threads (a multiple of 32) under hardware barrier id
+// `id` (1..15; id 0 is __syncthreads').
+__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 constexpr int NORM2_CWARPS = 8;
 constexpr int NORM2_THREADS = 32 * (NORM2_CWARPS + 1);
 constexpr int NORM2_WARPS = NORM2_CWARPS;
