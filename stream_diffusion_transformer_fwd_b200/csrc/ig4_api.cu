@@ -177,7 +177,7 @@ ig4_status map_3d_bf16(CUtensorMap *m, const void *base, long d0, long d1, long 
 // 256- and 192-wide tiles over more than one 128-row block run on CTA pairs
 // (M = 256 per pair tile, B rows split between the two CTAs); the B tensor
 // map's box is then BN / 2 rows.
-inline bool use_pair(int BN, int M) { return (BN == 256 || BN == 192) && M > GEMM_BM; }
+inline bool use_pair(int BN, int M) { return (BN == 256 || BN == 240 || BN == 192) && M > GEMM_BM; }
 inline int b_box_rows(int BN, int M) { return use_pair(BN, M) ? BN / 2 : BN; }
 
 // Tile order of the persistent GEMMs: plain m-fastest while A fits easily in
@@ -198,7 +198,7 @@ ig4_status launch_gemm(const CUtensorMap &A, const CUtensorMap &B, const CUtenso
   DeviceInfo *di = nullptr;
   IG4_TRY(device_info(&di));
   const int group_m = gemm_group_m(M, K, FP8 ? 1 : 2);
-  if constexpr (BN == 256 || BN == 192) {
+  if constexpr (BN == 256 || BN == 240 || BN == 192) {
     if (use_pair(BN, M)) {
       auto kern = gemm_pair_kernel<BN, FP8, DUAL_B, Epi>;
       constexpr int PAIR_SMEM_BYTES = PairShape<BN>::SMEM_BYTES;
@@ -224,6 +224,9 @@ ig4_status launch_gemm(const CUtensorMap &A, const CUtensorMap &B, const CUtenso
       return last_launch_status();
     }
   }
+  if constexpr (BN == 240) {
+    return IG4_ERR_UNSUPPORTED;  // 240-wide tiles run on CTA pairs only
+  } else {
   auto kern = gemm_tc_kernel<BN, FP8, DUAL_B, Epi>;
   constexpr int SMEM = GemmShape<BN>::SMEM_BYTES;
   IG4_TRY(allow_smem(kern, SMEM));
@@ -233,6 +236,7 @@ ig4_status launch_gemm(const CUtensorMap &A, const CUtensorMap &B, const CUtenso
                  group_m, epi) != cudaSuccess)
     return IG4_ERR_CUDA;
   return last_launch_status();
+  }
 }
 
 // A [M][K] and W [N][K] maps for one GEMM (esize 2 = bf16, 1 = e4m3).
@@ -528,33 +532,41 @@ ig4_status launch_attention(int B, int H, int L, const void *q, const void *k, c
   return IG4_OK;
 }
 
-// Tile width for an output of N columns: the candidate (256, 192, 128 that
-// divides N) with the best product of wave efficiency (tiles / (waves *
-// workers), where a worker is a CTA pair for 256 and 192 over more than 128
-// rows and a single CTA otherwise) and per-tile MMA efficiency (single-CTA
-// 192- and 128-wide tiles read more shared memory per flop; measured on the
-// 4608 x 4608 x 4608 out-projection, single-CTA 192-wide tiles ran 10% slower
-// per tile than 256-wide ones; on the 4608 x 4608 out- and down-projections
-// 192-wide pair tiles ran at 0.79 of the 256-wide pair rate per flop, so they
-// only win where 256-wide tiles leave most of a wave of pairs idle).
-int choose_bn(int M, int N, int sms) {
-  const int cand[3] = {256, 192, 128};
-  const double mma_eff_single[3] = {1.0, 0.88, 0.8};
-  const double mma_eff_pair[3] = {1.0, 0.8, 0.0};
+// Tile width for an output of N columns: the candidate with the best product
+// of wave efficiency (tiles / (waves * workers), where a worker is a CTA pair
+// for the 256-, 240- and 192-wide tiles over more than 128 rows and a single
+// CTA otherwise), useful columns (240-wide tiles need not divide N: the last
+// one is partial) and per-tile MMA efficiency.  Single-CTA 192- and 128-wide
+// tiles read more shared memory per flop (measured on the 4608 x 4608 x 4608
+// out-projection, single-CTA 192-wide tiles ran 10% slower per tile than
+// 256-wide ones); 192-wide pair tiles ran at 0.79 of the 256-wide pair rate
+// per flop on the 4608 x 4608 out- and down-projections (a pair tile of 192
+// needs ~75 operand bytes per cycle per SM from L2 against 64 at 256); 240
+// needs ~66.  On N = 4608 the 256-wide tiles leave the last of 4.4 rounds of
+// 74 pairs 62% idle, the 240-wide ones (20 column tiles, 4% of them past N)
+// the last of 4.86 rounds 14% idle.
+// allow240: the epilogue handles a partial last tile (the gated residual).
+int choose_bn(int M, int N, int sms, bool allow240 = false) {
+  const int cand[4] = {256, 240, 192, 128};
+  const double mma_eff_single[4] = {1.0, 0.0, 0.88, 0.8};
+  const double mma_eff_pair[4] = {1.0, 0.97, 0.8, 0.0};
   int best = 0;
   double best_score = -1.0;
-  for (int i = 0; i < 3; ++i) {
-    if (N % cand[i]) continue;
-    const bool pair = use_pair(cand[i], M);
+  for (int i = 0; i < 4; ++i) {
+    const int bn = cand[i];
+    const bool pair = use_pair(bn, M);
+    if (bn == 240 ? (!allow240 || !pair || N % 16) : (N % bn)) continue;
     const int bm = pair ? 2 * GEMM_BM : GEMM_BM;
     const int workers = pair ? sms / 2 : sms;
-    const long tiles = static_cast<long>((M + bm - 1) / bm) * (N / cand[i]);
+    const long tiles_n = (N + bn - 1) / bn;
+    const long tiles = static_cast<long>((M + bm - 1) / bm) * tiles_n;
     const long waves = (tiles + workers - 1) / workers;
     const double eff = pair ? mma_eff_pair[i] : mma_eff_single[i];
-    const double score = eff * static_cast<double>(tiles) / static_cast<double>(waves * workers);
+    const double useful = static_cast<double>(N) / static_cast<double>(tiles_n * bn);
+    const double score = eff * useful * static_cast<double>(tiles) / static_cast<double>(waves * workers);
     if (score > best_score + 1e-9) {
       best_score = score;
-      best = cand[i];
+      best = bn;
     }
   }
   return best;
@@ -570,11 +582,11 @@ ig4_status launch_resid_bn(int B, int L, int N, int K, const void *a, bool f8, c
   if (f8) {
     EpiResidGate<BN, true, XT> e{static_cast<const XT *>(x_res), static_cast<XT *>(x_out), gate,
                                   gate_stride, L, M, N, a_scale, w_scale};
-    return launch_gemm<BN, true, false>(ma, mb, mb, M, N / BN, K, e, st);
+    return launch_gemm<BN, true, false>(ma, mb, mb, M, (N + BN - 1) / BN, K, e, st);
   }
   EpiResidGate<BN, false, XT> e{static_cast<const XT *>(x_res), static_cast<XT *>(x_out), gate,
                                  gate_stride, L, M, N, nullptr, nullptr};
-  return launch_gemm<BN, false, false>(ma, mb, mb, M, N / BN, K, e, st);
+  return launch_gemm<BN, false, false>(ma, mb, mb, M, (N + BN - 1) / BN, K, e, st);
 }
 
 template <typename XT>
@@ -583,9 +595,12 @@ ig4_status launch_resid_t(int B, int L, int N, int K, const void *a, bool f8, co
                           const void *x_res, void *x_out, cudaStream_t st) {
   DeviceInfo *di = nullptr;
   IG4_TRY(device_info(&di));
-  switch (choose_bn(B * L, N, di->sms)) {
+  switch (choose_bn(B * L, N, di->sms, true)) {
     case 256:
       return launch_resid_bn<256, XT>(B, L, N, K, a, f8, a_scale, w, w_scale, gate, gate_stride,
+                                      x_res, x_out, st);
+    case 240:
+      return launch_resid_bn<240, XT>(B, L, N, K, a, f8, a_scale, w, w_scale, gate, gate_stride,
                                       x_res, x_out, st);
     case 192:
       return launch_resid_bn<192, XT>(B, L, N, K, a, f8, a_scale, w, w_scale, gate, gate_stride,
@@ -627,9 +642,8 @@ ig4_status launch_swiglu(int M, int I, int K, const void *h, bool f8, const floa
 // ------------------------------------------------- MX8 (FP8, 1x32 scales)
 // The FP8 block feeds the out- and down-projections MX8 activations (E4M3
 // with a UE8M0 scale per 32 elements, written by the attention and SwiGLU
-// epilogues) through the block-scaled pair GEMM.  K % 128 == 0, N % 192 == 0
-// or N % 256 == 0.
-inline bool mx8_ok(long N, long K) { return K % 128 == 0 && (N % 192 == 0 || N % 256 == 0); }
+// epilogues) through the block-scaled pair GEMM.  K % 128 == 0, N % 16 == 0.
+inline bool mx8_ok(long N, long K) { return K % 128 == 0 && N % 16 == 0; }
 
 // bytes of packed MX8 scales of an [M][K] operand (rows padded to 128)
 inline size_t mx8_sf_bytes(long M, long K) { return static_cast<size_t>((M + 127) / 128) * (K / 128) * 512; }
@@ -661,28 +675,31 @@ ig4_status map_mx8_sf(CUtensorMap *m, const void *base, long rows, long K) {
   return r == CUDA_SUCCESS ? IG4_OK : IG4_ERR_CUDA;
 }
 
-// Block-scaled pair GEMM with A in MX8: 192-wide tiles (gemm_pair_kernel's
-// MX8A variant) where N % 192 == 0 - on N = 4608 they fill the last wave of
-// pairs better than 256-wide ones and keep the accumulators apart - else
-// 256-wide tiles with overlapping accumulators (gemm_mx8_pair_kernel).
+// Block-scaled pair GEMM with A in MX8: gemm_pair_kernel's MX8A variant on
+// 240-wide tiles (or 192-wide where the tile chooser prefers them): two
+// accumulators of at most 240 columns leave TMEM room for the scales.
 template <int BN, class Epi>
 ig4_status launch_mx8_gemm(const void *a_codes, const void *a_sf, const void *w, int M, int N,
                            int K, const Epi &ep, cudaStream_t st) {
-  static_assert(BN == 192 || BN == 256, "MX8 tile width");
-  if (K % 128 || N % BN) return IG4_ERR_UNSUPPORTED;
+  static_assert(BN == 192 || BN == 240, "MX8 tile width");
+  if (K % 128 || N % 16 || (BN == 192 && N % 192)) return IG4_ERR_UNSUPPORTED;
   CUtensorMap ma, mb, msa;
   IG4_TRY(map_2d(&ma, a_codes, 1, M, K, K, GEMM_BM, 128));
   IG4_TRY(map_2d(&mb, w, 1, N, K, K, BN / 2, 128));
   IG4_TRY(map_mx8_sf(&msa, a_sf, M, K));
   DeviceInfo *di = nullptr;
   IG4_TRY(device_info(&di));
-  const int n_tiles_n = N / BN;
+  const int n_tiles_n = (N + BN - 1) / BN;
   const long tiles = static_cast<long>((M + 2 * GEMM_BM - 1) / (2 * GEMM_BM)) * n_tiles_n;
   const int pairs = static_cast<int>(std::min<long>(tiles, di->sms / 2));
   const int group_m = gemm_group_m(M, K, 1);
+  auto kern = gemm_pair_kernel<BN, true, false, Epi, true>;
+  constexpr int SMEM = PairShape<BN, true>::SMEM_BYTES;
+  IG4_TRY(allow_smem(kern, SMEM));
   cudaLaunchConfig_t lc = {};
   lc.gridDim = dim3(2 * pairs);
   lc.blockDim = dim3(GEMM_THREADS);
+  lc.dynamicSmemBytes = SMEM;
   lc.stream = st;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -693,20 +710,8 @@ ig4_status launch_mx8_gemm(const void *a_codes, const void *a_sf, const void *w,
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = attr;
   lc.numAttrs = 2;
-  cudaError_t e;
-  if constexpr (BN == 192) {
-    auto kern = gemm_pair_kernel<192, true, false, Epi, true>;
-    constexpr int SMEM = PairShape<192, true>::SMEM_BYTES;
-    IG4_TRY(allow_smem(kern, SMEM));
-    lc.dynamicSmemBytes = SMEM;
-    e = cudaLaunchKernelEx(&lc, kern, ma, mb, msa, M, n_tiles_n, K, group_m, ep);
-  } else {
-    auto kern = gemm_mx8_pair_kernel<Epi>;
-    IG4_TRY(allow_smem(kern, MX8P_SMEM_BYTES));
-    lc.dynamicSmemBytes = MX8P_SMEM_BYTES;
-    e = cudaLaunchKernelEx(&lc, kern, ma, mb, msa, M, n_tiles_n, K, group_m, ep);
-  }
-  if (e != cudaSuccess) return IG4_ERR_CUDA;
+  if (cudaLaunchKernelEx(&lc, kern, ma, mb, msa, M, n_tiles_n, K, group_m, ep) != cudaSuccess)
+    return IG4_ERR_CUDA;
   return last_launch_status();
 }
 
@@ -726,14 +731,18 @@ ig4_status launch_mx8_resid(int B, int L, int N, int K, const void *a_codes, con
                             int gate_stride, const void *x_res, void *x_out, int x_dtype,
                             cudaStream_t st) {
   const bool f32 = x_dtype == IG4_F32;
-  if (N % 192 == 0)
+  DeviceInfo *di = nullptr;
+  IG4_TRY(device_info(&di));
+  // 192-wide where it divides N and the chooser prefers it, else 240-wide
+  const int M = B * L;
+  if (M > GEMM_BM && choose_bn(M, N, di->sms, true) == 192)
     return f32 ? launch_mx8_resid_bn<192, float>(B, L, N, K, a_codes, a_sf, w, w_scale, gate,
                                                  gate_stride, x_res, x_out, st)
                : launch_mx8_resid_bn<192, __nv_bfloat16>(B, L, N, K, a_codes, a_sf, w, w_scale,
                                                          gate, gate_stride, x_res, x_out, st);
-  return f32 ? launch_mx8_resid_bn<256, float>(B, L, N, K, a_codes, a_sf, w, w_scale, gate,
+  return f32 ? launch_mx8_resid_bn<240, float>(B, L, N, K, a_codes, a_sf, w, w_scale, gate,
                                                gate_stride, x_res, x_out, st)
-             : launch_mx8_resid_bn<256, __nv_bfloat16>(B, L, N, K, a_codes, a_sf, w, w_scale,
+             : launch_mx8_resid_bn<240, __nv_bfloat16>(B, L, N, K, a_codes, a_sf, w, w_scale,
                                                        gate, gate_stride, x_res, x_out, st);
 }
 

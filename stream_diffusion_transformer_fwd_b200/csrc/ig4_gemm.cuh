@@ -152,6 +152,62 @@ __device__ __forceinline__ void apply_scales(float (&v)[32], float rs, const flo
   }
 }
 
+// W-wide (16 or 32) versions of the loads and stores above, for the chunks
+// of the gated-residual epilogue (a 240-wide tile ends in a 16-column chunk).
+template <int W>
+__device__ __forceinline__ void load_f32_w(const float *src, float (&v)[32]) {
+  const float4 *s = reinterpret_cast<const float4 *>(src);
+#pragma unroll
+  for (int q = 0; q < W / 4; ++q) {
+    const float4 w = __ldg(s + q);
+    v[4 * q] = w.x;
+    v[4 * q + 1] = w.y;
+    v[4 * q + 2] = w.z;
+    v[4 * q + 3] = w.w;
+  }
+}
+template <int W, typename T>
+__device__ __forceinline__ void load_x_w(const T *src, float (&v)[32]) {
+  if constexpr (sizeof(T) == 4) {
+    const float4 *s = reinterpret_cast<const float4 *>(src);
+#pragma unroll
+    for (int q = 0; q < W / 4; ++q) {
+      const float4 w = s[q];
+      v[4 * q] = w.x;
+      v[4 * q + 1] = w.y;
+      v[4 * q + 2] = w.z;
+      v[4 * q + 3] = w.w;
+    }
+  } else {
+    const uint4 *s = reinterpret_cast<const uint4 *>(src);
+#pragma unroll
+    for (int q = 0; q < W / 8; ++q) {
+      const uint4 w = s[q];
+      const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        v[8 * q + 2 * e] = __uint_as_float(u[e] << 16);
+        v[8 * q + 2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
+      }
+    }
+  }
+}
+template <int W, typename T>
+__device__ __forceinline__ void store_x_w(T *dst, const float (&v)[32]) {
+  if constexpr (sizeof(T) == 4) {
+    float4 *d = reinterpret_cast<float4 *>(dst);
+#pragma unroll
+    for (int q = 0; q < W / 4; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+  } else {
+    uint4 *d = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+    for (int q = 0; q < W / 8; ++q)
+      d[q] = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                        pack_bf16x2(v[8 * q + 4], v[8 * q + 5]),
+                        pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+  }
+}
+
 // ------------------------------------------------------------- epilogues
 // Each epilogue is called by the 128 epilogue threads for one output tile;
 // `tacc` is the TMEM address of this warp's 32 lanes at column 0 of the
@@ -217,7 +273,8 @@ struct EpiResidGate {
     part(m0, n0, tacc, r, 0, BN);
   }
 
-  // columns [lo, hi) of the tile (multiples of 32)
+  // columns [lo, hi) of the tile (multiples of 16); columns at or past N (the
+  // last tile of a 240-wide tiling) are skipped
   __device__ __forceinline__ void part(int m0, int n0, uint32_t tacc, int r, int lo, int hi) const {
     const int row = m0 + r;
     const bool valid = row < M;
@@ -225,26 +282,41 @@ struct EpiResidGate {
     // a_scale == nullptr: A's scales were applied by the tensor cores (MX8)
     const float rs = (FP8 && valid && a_scale != nullptr) ? __ldg(a_scale + row) : 1.0f;
     const float *grow = gate + static_cast<long>(b) * gate_stride + n0;
+    const int cmax = min(hi, N - n0);
 #pragma unroll 1
-    for (int c = lo; c < hi; c += 32) {
-      float v[32];
-      tmem_ld32(tacc + c, v);
-      tmem_ld_wait();
-      if (!valid) continue;
-      apply_scales<FP8>(v, rs, b_scale + n0 + c);
-      float g[32], x[32];
-      load32_f32_ldg(grow + c, g);
-      const long off = static_cast<long>(row) * N + n0 + c;
-      if (x_res != nullptr) {
-        load32_x<XT>(x_res + off, x);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) x[i] = 0.0f;
-      }
-#pragma unroll
-      for (int i = 0; i < 32; ++i) x[i] = fmaf(g[i], v[i], x[i]);
-      store32_x<OT>(x_out + off, x);
+    for (int c = lo; c < cmax; c += 32) {
+      if (cmax - c >= 32)
+        chunk<32>(n0, tacc, row, valid, rs, grow, c);
+      else
+        chunk<16>(n0, tacc, row, valid, rs, grow, c);
     }
+  }
+
+  template <int W>
+  __device__ __forceinline__ void chunk(int n0, uint32_t tacc, int row, bool valid, float rs,
+                                        const float *grow, int c) const {
+    float v[32];
+    tmem_ld32(tacc + c, v);  // (a 16-wide chunk reads 16 spare columns)
+    tmem_ld_wait();
+    if (!valid) return;
+    if constexpr (FP8) {
+      float sc[32];
+      load_f32_w<W>(b_scale + n0 + c, sc);
+#pragma unroll
+      for (int i = 0; i < W; ++i) v[i] *= rs * sc[i];
+    }
+    float g[32], x[32];
+    load_f32_w<W>(grow + c, g);
+    const long off = static_cast<long>(row) * N + n0 + c;
+    if (x_res != nullptr) {
+      load_x_w<W>(x_res + off, x);
+    } else {
+#pragma unroll
+      for (int i = 0; i < W; ++i) x[i] = 0.0f;
+    }
+#pragma unroll
+    for (int i = 0; i < W; ++i) x[i] = fmaf(g[i], v[i], x[i]);
+    store_x_w<W>(x_out + off, x);
   }
 };
 
@@ -570,12 +642,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 // arrival per epilogue warp of the pair).
 template <int BN, bool MX8A = false>
 struct PairShape {
-  static_assert(BN == 256 || BN == 192, "pair tile width");
+  static_assert(BN == 256 || BN == 240 || BN == 192, "pair tile width");
   static constexpr int A_BYTES = GEMM_BM * 128;          // 16 KB
-  static constexpr int BH_BYTES = (BN / 2) * 128;        // 16 KB or 12 KB (a multiple of 1 KB)
+  static constexpr int BH_BYTES = (BN / 2) * 128;        // 16, 15 or 12 KB (a multiple of 1 KB)
   static constexpr int SF_BYTES = MX8A ? 512 : 0;        // A's scale chunk (MX8)
   static constexpr int STAGE_BYTES = A_BYTES + BH_BYTES + SF_BYTES;
-  static constexpr int STAGES = BN == 256 ? 6 : 7;       // ~200 KB of shared memory
+  static constexpr int STAGES = BN == 256 ? 6 : 7;       // 190-227 KB of shared memory
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 };
 
@@ -591,9 +663,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                      const __grid_constant__ CUtensorMap tmB2, int M, int n_tiles_n, int K,
                      int group_m, const Epi epi) {
   static_assert(!DUAL_B || BN == 256, "SwiGLU pairs split 128 gate / 128 up rows");
-  static_assert(!MX8A || (FP8 && !DUAL_B && BN == 192), "MX8 A: FP8, single B, 192-wide tiles");
+  static_assert(!MX8A || (FP8 && !DUAL_B && (BN == 192 || BN == 240)),
+                "MX8 A: FP8, single B, 192- or 240-wide tiles");
   using P = PairShape<BN, MX8A>;
-  constexpr uint32_t SFA_COL = 448, SFB_COL = 464;  // MX8A scale columns (after 2 x 192)
+  // TMEM: accumulator b at column b * ACC_STRIDE (a 240-wide tile's second
+  // accumulator starts at 256); MX8A scale columns after both
+  constexpr uint32_t ACC_STRIDE = BN == 240 ? 256 : BN;
+  constexpr uint32_t SFA_COL = BN == 240 ? 496 : 448;
+  constexpr uint32_t SFB_COL = BN == 240 ? 500 : 464;
+  constexpr uint32_t SF_INIT_COL = BN == 240 ? 480 : 464;  // 32 columns of byte 127
   constexpr int PAIR_STAGES = P::STAGES;
   constexpr int PAIR_STAGE_BYTES = P::STAGE_BYTES;
   constexpr int A_BYTES = P::A_BYTES;
@@ -657,7 +735,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       uint32_t ones[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) ones[i] = 0x7F7F7F7Fu;
-      tmem_st32_u(tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + SFB_COL, ones);
+      tmem_st32_u(tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + SF_INIT_COL, ones);
       tmem_st_wait();
     }
     tc_fence_before();
@@ -716,7 +794,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         const uint32_t use = static_cast<uint32_t>(local >> 1);
         if (!mbar_wait_cluster(&tempty[buf], (use & 1) ^ 1, abort_flag)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + buf * BN;
+        const uint32_t d_tmem = tmem_base + buf * ACC_STRIDE;
         for (int it = 0; it < kblocks; ++it) {  // k-blocks in the producer's order
           if (!mbar_wait_cluster(&full[s], ph, abort_flag)) {
             ok = false;
@@ -766,7 +844,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       int mt, nt;
       tile_coords(t, m_tiles, n_tiles_n, group_m, &mt, &nt);
       epi(mt * 2 * GEMM_BM + static_cast<int>(rank) * GEMM_BM, nt * BN,
-          tmem_base + lane_base + buf * BN, r);
+          tmem_base + lane_base + buf * ACC_STRIDE, r);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(buf ? tempty_leader1 : tempty_leader0);

@@ -1,7 +1,9 @@
 // ig4_mx8.cuh - FP8 activations with 1x32 block scales (MX format) for the
 // FP8 path's two activation-side GEMM inputs (the attention output feeding
-// the out-projection, u feeding the down-projection), and the block-scaled
-// FP8 GEMM on CTA pairs (tcgen05 kind::mxf8f6f4) that consumes them.
+// the out-projection, u feeding the down-projection): the encoding, the row
+// quantiser and the SwiGLU epilogue that writes it.  The block-scaled GEMM
+// that consumes it is gemm_pair_kernel's MX8A variant (tcgen05
+// kind::mxf8f6f4).
 //
 // Source: "Ideogram 4 快速开始", section on hardware and precision: the
 // release weights are FP8 E4M3 with per-output-channel scales.  How the
@@ -168,207 +170,5 @@ struct EpiSwiGLUMx8 {
     }
   }
 };
-
-// ------------------------------------------------- block-scaled FP8 GEMM
-// The CTA-pair GEMM (see gemm_pair_kernel) with A in MX8 (E4M3 codes and a
-// UE8M0 scale per 32 elements) and B in E4M3 with unit block scales (the
-// weights' per-channel fp32 scale stays in the epilogue): tcgen05.mma
-// kind::mxf8f6f4 with block_scale.  Per 128-element k-block a stage holds
-// A (128 rows x 128 B), half of B (128 rows x 128 B) and A's 512-byte
-// scale chunk; the leader copies that chunk into TMEM (one tcgen05.cp) and
-// issues 4 MMAs of K = 32, the j-th reading scale byte j of each row (scale
-// factor id j).  B's scales are the constant 1.0 (byte 127), written into
-// TMEM once.  The two 256-column accumulators overlap by 64 columns to leave
-// room for the scales: accumulator 1 starts at column 192, and the epilogue
-// of a tile drains the overlapped columns first and reports it (barrier
-// ovl), so the next tile's MMAs may start while the rest drains.  K-snake
-// as in gemm_pair_kernel.
-constexpr int MX8P_STAGES = 6;
-constexpr int MX8P_A_BYTES = GEMM_BM * 128;
-constexpr int MX8P_BH_BYTES = 128 * 128;
-constexpr int MX8P_SFA_BYTES = 512;
-constexpr int MX8P_STAGE_BYTES = MX8P_A_BYTES + MX8P_BH_BYTES + MX8P_SFA_BYTES;
-constexpr int MX8P_SMEM_BYTES = MX8P_STAGES * MX8P_STAGE_BYTES + 1024 + 256;
-constexpr uint32_t MX8P_ACC1_COL = 192;
-constexpr uint32_t MX8P_SFA_COL = 448;  // 4 columns
-constexpr uint32_t MX8P_SFB_COL = 464;  // 32 columns of byte 127
-static_assert(MX8P_ACC1_COL + 256 <= MX8P_SFA_COL && MX8P_SFB_COL + 32 <= 512, "TMEM");
-
-template <class Epi>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
-    gemm_mx8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                         const __grid_constant__ CUtensorMap tmSFA, int M, int n_tiles_n, int K,
-                         int group_m, const Epi epi) {
-  constexpr int BN = 256;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = align1024(smem_raw);
-  uint8_t *sA = smem;
-  uint8_t *sB = sA + MX8P_STAGES * MX8P_A_BYTES;
-  uint8_t *sSFA = sB + MX8P_STAGES * MX8P_BH_BYTES;
-  uint64_t *full = reinterpret_cast<uint64_t *>(sSFA + MX8P_STAGES * MX8P_SFA_BYTES);
-  uint64_t *empty = full + MX8P_STAGES;
-  uint64_t *tfull = empty + MX8P_STAGES;  // [2]: accumulator ready
-  uint64_t *tempty = tfull + 2;           // [2]: accumulator drained
-  uint64_t *ovl = tempty + 2;             // overlapped columns drained
-  uint64_t *drain = ovl + 1;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();
-  const int pair = blockIdx.x >> 1;
-  const int n_pairs = gridDim.x >> 1;
-  const int m_tiles = (M + 2 * GEMM_BM - 1) / (2 * GEMM_BM);
-  const int n_tiles = m_tiles * n_tiles_n;
-  const int kblocks = K / 128;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < MX8P_STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 2 * 4);  // one arrival per epilogue warp of the pair
-    }
-    mbar_init(ovl, 2 * 4);
-    mbar_init(drain, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 4 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
-    tma_prefetch_desc(&tmSFA);
-  }
-  if (warp == 5) {
-    tmem_alloc_pair(tmem_slot, 512);
-    tmem_relinquish_pair();
-  }
-  tc_fence_before();
-  cluster_sync_all();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-  if (warp < 4) {
-    // B's unit scales (byte 127) in every lane of the B scale columns
-    uint32_t ones[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) ones[i] = 0x7F7F7F7Fu;
-    tmem_st32_u(tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + MX8P_SFB_COL, ones);
-    tmem_st_wait();
-  }
-  tc_fence_before();
-  cluster_sync_all();
-  tc_fence_after();
-  pdl_wait();
-  pdl_trigger();
-
-  if (warp == 4) {
-    if (lane == 0) {
-      // ---------------- loads (both CTAs), completing on the leader's barrier
-      int s = 0;
-      uint32_t ph = 0;
-      bool ok = true;
-      int local = 0;
-      for (int t = pair; t < n_tiles && ok; t += n_pairs, ++local) {
-        int mt, nt;
-        tile_coords(t, m_tiles, n_tiles_n, group_m, &mt, &nt);
-        const int mrow = mt * 2 * GEMM_BM + static_cast<int>(rank) * GEMM_BM;
-        for (int it = 0; it < kblocks; ++it) {
-          const int kb = (local & 1) ? kblocks - 1 - it : it;  // K-snake
-          if (!mbar_wait_cluster(&empty[s], ph ^ 1, abort_flag)) {
-            ok = false;
-            break;
-          }
-          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * MX8P_STAGE_BYTES);
-          const uint32_t bar = map_shared_to_rank(&full[s], 0);
-          tma_load_2d_pair(sA + s * MX8P_A_BYTES, &tmA, bar, kb * 128, mrow);
-          tma_load_3d_pair(sSFA + s * MX8P_SFA_BYTES, &tmSFA, bar, 0, kb, mrow / 128);
-          tma_load_2d_pair(sB + s * MX8P_BH_BYTES, &tmB, bar, kb * 128,
-                           nt * BN + static_cast<int>(rank) * (BN / 2));
-          if (++s == MX8P_STAGES) {
-            s = 0;
-            ph ^= 1;
-          }
-        }
-      }
-      if (!ok) sleep_ns(50000);  // let the loads already issued land
-    }
-  } else if (warp == 5) {
-    if (lane == 0 && rank == 0) {
-      // ---------------- MMA issuer (leader CTA)
-      int s = 0;
-      uint32_t ph = 0;
-      bool ok = true;
-      const uint32_t sfa = tmem_base + MX8P_SFA_COL;
-      const uint32_t sfb = tmem_base + MX8P_SFB_COL;
-      for (int t = pair, i = 0; t < n_tiles && ok; t += n_pairs, ++i) {
-        const int acc = i & 1;
-        // this accumulator's own columns: drained by the epilogue of tile i - 2;
-        // the overlapped ones: by the epilogue of tile i - 1
-        if (!mbar_wait_cluster(&tempty[acc], static_cast<uint32_t>((i >> 1) & 1) ^ 1, abort_flag))
-          break;
-        if (i > 0 && !mbar_wait_cluster(ovl, static_cast<uint32_t>((i - 1) & 1), abort_flag)) break;
-        tc_fence_after();
-        const uint32_t d = tmem_base + (acc ? MX8P_ACC1_COL : 0);
-        for (int it = 0; it < kblocks; ++it) {  // k-blocks in the producer's order
-          if (!mbar_wait_cluster(&full[s], ph, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          tmem_cp_sf_pair(sfa, sdesc_kmajor_none(smem_u32(sSFA + s * MX8P_SFA_BYTES), 128));
-          const uint64_t ad = sdesc_kmajor_sw128(smem_u32(sA + s * MX8P_A_BYTES));
-          const uint64_t bd = sdesc_kmajor_sw128(smem_u32(sB + s * MX8P_BH_BYTES));
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            umma_mx8_pair(d, ad + 2 * j, bd + 2 * j, idesc_mx8(2 * GEMM_BM, BN, j), sfa, sfb,
-                          (it | j) != 0);
-          umma_commit_pair_both(&empty[s]);
-          if (++s == MX8P_STAGES) {
-            s = 0;
-            ph ^= 1;
-          }
-        }
-        if (ok) umma_commit_pair_both(&tfull[acc]);
-      }
-      umma_commit_pair_both(drain);
-      mbar_wait_cluster(drain, 0, nullptr, WAIT_LIMIT_NS / 4);
-    }
-  } else {
-    // ---------------- epilogue warps 0..3 (both CTAs, own 128 rows)
-    const int r = warp * 32 + lane;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t ovl_leader = map_shared_to_rank(ovl, 0);
-    constexpr int C = Epi::COLS;  // 64 accumulator columns overlap: the top 64 of
-    constexpr int OV = C - 64;    // acc 0's epilogue columns, the bottom 64 of acc 1's
-    for (int t = pair, i = 0; t < n_tiles; t += n_pairs, ++i) {
-      const int acc = i & 1;
-      const bool ok =
-          mbar_wait_cluster(&tfull[acc], static_cast<uint32_t>((i >> 1) & 1), abort_flag);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      tc_fence_after();
-      int mt, nt;
-      tile_coords(t, m_tiles, n_tiles_n, group_m, &mt, &nt);
-      const int m0 = mt * 2 * GEMM_BM + static_cast<int>(rank) * GEMM_BM;
-      const uint32_t tacc = tmem_base + (acc ? MX8P_ACC1_COL : 0) + lane_base;
-      epi.part(m0, nt * BN, tacc, r, acc ? 0 : OV, acc ? 64 : C);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(ovl_leader);
-      epi.part(m0, nt * BN, tacc, r, acc ? 64 : 0, acc ? C : OV);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(map_shared_to_rank(&tempty[acc], 0));
-    }
-  }
-
-  __syncwarp();
-  tc_fence_before();
-  cluster_sync_all();
-  tc_fence_after();
-  if (warp == 5) tmem_dealloc_pair(tmem_base, 512);
-}
 
 }  // namespace ig4

@@ -138,7 +138,10 @@ def test_quantize_rows(ig4, M, K):
     (1, 300, 1024, 2816, "bf16", "e4m3"),
     (1, 200, 384, 512, "f32", "bf16"),      # 128-wide single-CTA tiles
     (1, 200, 640, 512, "f32", "bf16"),      # 128-wide tiles
-    (1, 4608, 4608, 256, "f32", "bf16"),    # the block's out-projection shape (256-wide pair tiles)
+    (1, 4608, 4608, 256, "f32", "bf16"),    # the block's out-projection shape (240-wide pair
+                                            # tiles, the last of 20 column tiles 48 wide)
+    (1, 4608, 4608, 512, "f32", "e4m3"),    # the same with E4M3 operands
+    (2, 2304, 4608, 128, "bf16", "bf16"),   # 240-wide tiles, batch boundary, bf16 stream
     (1, 1100, 4608, 256, "bf16", "bf16"),   # 192-wide pair tiles, ragged last pair tile
     (1, 1152, 4608, 256, "f32", "e4m3"),    # 192-wide pair tiles, E4M3 (512px shape)
     (1, 4864, 4608, 512, "bf16", "bf16"),   # 256-wide pair tiles (2048x352 shape)
