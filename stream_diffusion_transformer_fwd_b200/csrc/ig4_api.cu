@@ -181,15 +181,16 @@ inline bool use_pair(int BN, int M) { return (BN == 256 || BN == 240 || BN == 19
 inline int b_box_rows(int BN, int M) { return use_pair(BN, M) ? BN / 2 : BN; }
 
 // Tile order of the persistent GEMMs: plain m-fastest while A fits easily in
-// L2 (the 126 MB L2 then serves every re-read of A), groups of 12 m tiles
+// L2 (the 126 MB L2 then serves every re-read of A), groups of 10 m tiles
 // once A is larger, so that consecutive rounds of pair tiles share A rows
 // (which the pair kernel's K-snake then finds in L2).  DRAM reads of the
-// 1024 px down-projection (A = 113 MB), ncu, K-snake on: groups of 4 m
-// tiles 599 MB, 6 565 MB, 8 567 MB, 12 536 MB, m-fastest 571 MB (649 MB for
-// groups of 8 before the K-snake); the other GEMMs of the block moved by
-// less than 1%.
+// 1024 px down-projection (A = 113 MB, 240-wide pair tiles), ncu: groups of
+// 4 m tiles 634 MB, 6 576 MB, 8 610 MB, 10 542 MB, 12 570 MB, m-fastest 578
+// MB (with 256-wide tiles, groups of 12: 536 MB; 649 MB for groups of 8
+// before the K-snake); times within 1%, and the other GEMMs of the block
+// moved by less than 1%.
 inline int gemm_group_m(long M, long K, int esize) {
-  return M * K * esize <= (64L << 20) ? (1 << 30) : 12;
+  return M * K * esize <= (64L << 20) ? (1 << 30) : 10;
 }
 
 template <int BN, bool FP8, bool DUAL_B, class Epi>
