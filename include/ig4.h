@@ -287,8 +287,8 @@ ig4_status ig4_block_forward_traced(const ig4_config *cfg, const ig4_block_weigh
  * ig4_block_forward (same layouts and errors).  A configuration fits when
  * ig4_workspace_size(cfg) <= IG4_NOALLOC_SCRATCH_BYTES; larger ones return
  * IG4_ERR_WORKSPACE before anything is launched.  At B = 1 that is up to 941
- * tokens of the full-width block (D 4608, I 12288) with bf16 weights, 802
- * with E4M3 weights and 751 with NVFP4 Mixed weights; 4094, 3491 and 3275
+ * tokens of the full-width block (D 4608, I 12288) with bf16 weights, 796
+ * with E4M3 weights and 750 with NVFP4 Mixed weights; 4094, 3469 and 3270
  * tokens at D 1024, I 2816.
  * The first call on a device looks up the scratch array's device address
  * (a set-up done with that device current, and done again if the device's
