@@ -393,22 +393,26 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         const long ibase = 2 * UPI * sched.tiles_before(k);  // ring units before this segment
         if (!att_wait<PAIR>(q_full, static_cast<uint32_t>(k) & 1, abort_flag)) break;
         for (int t = 0; t < sg.n && ok; ++t, ++gt) {
+          const int it = ro.item_k(t);
+          // K_t resident first: its slot checks then stay off the path from the
+          // softmax's release of S to the next S MMA (K_t's load waits only on
+          // items consumed before it, so this order adds no dependency)
+          for (int u = 0; u < UPI && ok; ++u) {
+            const long i = ibase + UPI * it + u;
+            ok = att_wait_passed(passed, i, abort_flag) &&
+                 att_wait<PAIR>(&full[i % ATT_SLOTS], static_cast<uint32_t>(i / ATT_SLOTS) & 1,
+                                abort_flag);
+          }
           // the S buffer is free once the softmax has read S_{gt-1}
-          if (gt > 0 && !att_wait<PAIR>(s_free, static_cast<uint32_t>(gt - 1) & 1, abort_flag)) {
+          if (!ok ||
+              (gt > 0 && !att_wait<PAIR>(s_free, static_cast<uint32_t>(gt - 1) & 1, abort_flag))) {
             ok = false;
             break;
           }
-          const int it = ro.item_k(t);
-          for (int u = 0; u < UPI && ok; ++u) {
+          tc_fence_after();
+          for (int u = 0; u < UPI; ++u) {
             const long i = ibase + UPI * it + u;
             const int slot = static_cast<int>(i % ATT_SLOTS);
-            if (!att_wait_passed(passed, i, abort_flag) ||
-                !att_wait<PAIR>(&full[slot], static_cast<uint32_t>(i / ATT_SLOTS) & 1,
-                                abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
             // descriptors of the slot's and Q's first chunk; a K step adds its
             // byte offset / 16 to the start-address field (no carry out of it:
             // shared memory addresses stay below 2^18)
@@ -451,7 +455,16 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         const long ibase = 2 * UPI * sched.tiles_before(k);
         for (int j = 0; j < sg.n && ok; ++j, ++gt) {
           const int pb = static_cast<int>(gt & 1);
-          if (!att_wait<PAIR>(&p_full[pb], static_cast<uint32_t>(gt >> 1) & 1, abort_flag)) {
+          const int it = ro.item_v(j);
+          // V_j resident before waiting for P_j (V_j's load waits only on items
+          // consumed before it), so P_j's arrival is followed by the MMAs alone
+          for (int u = 0; u < UPI && ok; ++u) {
+            const long i = ibase + UPI * it + u;
+            ok = att_wait_passed(passed, i, abort_flag) &&
+                 att_wait<PAIR>(&full[i % ATT_SLOTS], static_cast<uint32_t>(i / ATT_SLOTS) & 1,
+                                abort_flag);
+          }
+          if (!ok || !att_wait<PAIR>(&p_full[pb], static_cast<uint32_t>(gt >> 1) & 1, abort_flag)) {
             ok = false;
             break;
           }
@@ -462,17 +475,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             break;
           }
           tc_fence_after();
-          const int it = ro.item_v(j);
-          for (int u = 0; u < UPI && ok; ++u) {
+          for (int u = 0; u < UPI; ++u) {
             const long i = ibase + UPI * it + u;
             const int slot = static_cast<int>(i % ATT_SLOTS);
-            if (!att_wait_passed(passed, i, abort_flag) ||
-                !att_wait<PAIR>(&full[slot], static_cast<uint32_t>(i / ATT_SLOTS) & 1,
-                                abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
             const uint64_t vd = sdesc_kmajor_sw128(smem_u32(ring + slot * ATT_SLOT_BYTES));
             const uint32_t p_col = tmem + ATT_TMEM_P + 64 * pb;
             if constexpr (PAIR) {
