@@ -29,7 +29,8 @@
  * Memory: every pointer argument documented as "device" must be device
  * memory of the current device; the caller owns every buffer.  The library
  * never allocates, frees, or synchronises a stream, except
- * ig4_last_device_error, which synchronises the stream it is given.
+ * ig4_last_device_error and ig4_sm_clock_mhz, which synchronise the stream
+ * they are given.
  * Linear weights are row-major [out, in] (K contiguous).  All calls are
  * asynchronous on the given cudaStream_t (passed as void*, NULL = legacy
  * default stream); argument errors are returned synchronously and nothing is
@@ -564,6 +565,17 @@ ig4_status ig4_last_device_error(void *stream);
  * returns IG4_ERR_TIMEOUT and the context stays usable.  No paper
  * counterpart: it exercises the timeout path every other kernel relies on. */
 ig4_status ig4_selftest_timeout(int wait_us, void *stream);
+
+/* ---------------------------------------------------------- measurement ---
+ * SM clock as a kernel sees it: launches a one-thread kernel on `stream`
+ * that counts SM cycles over window_us microseconds (1 .. 100,000) of the
+ * GPU's global timer, synchronises the stream and writes cycles / time in
+ * MHz to *mhz (host).  Queued after other work it reads the clock at the
+ * moment that work ends, e.g. a power-capped clock after sustained tensor
+ * work.  IG4_ERR_INVALID_ARG for a window out of range or a null mhz;
+ * IG4_ERR_CUDA if the launch or the synchronisation fails.  No paper
+ * counterpart: an instrument for reading timings. */
+ig4_status ig4_sm_clock_mhz(int window_us, void *stream, double *mhz);
 
 #ifdef __cplusplus
 }

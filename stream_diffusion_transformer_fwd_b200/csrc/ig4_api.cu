@@ -2325,6 +2325,27 @@ ig4_status noalloc_scratch(uint8_t **out) {
 }
 }  // namespace
 
+// ------------------------------------------------------------ SM clock
+// One thread counts SM cycles across a window of the global nanosecond
+// timer; cycles / ns is the SM clock of that moment.  Under a power cap the
+// clock drops within a millisecond of heavy tensor work, faster than a
+// polled driver reading follows.  The loop is bounded by an iteration cap as
+// well as by the window.
+__device__ unsigned long long g_clock_probe[2];
+
+__global__ void sm_clock_probe_kernel(unsigned long long window_ns) {
+  unsigned long long t0, t1;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+  const long long c0 = clock64();
+  long it = 0;
+  do {
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t1));
+  } while (t1 - t0 < window_ns && ++it < (1L << 26));
+  const long long c1 = clock64();
+  g_clock_probe[0] = static_cast<unsigned long long>(c1 - c0);
+  g_clock_probe[1] = t1 - t0;
+}
+
 extern "C" {
 
 ig4_status ig4_block_forward_noalloc(const ig4_config *cfg, const ig4_block_weights *w,
@@ -2357,6 +2378,21 @@ ig4_status ig4_last_device_error(void *stream) {
       return IG4_ERR_CUDA;
     return IG4_ERR_TIMEOUT;
   }
+  return IG4_OK;
+}
+
+ig4_status ig4_sm_clock_mhz(int window_us, void *stream, double *mhz) {
+  if (window_us < 1 || window_us > 100000 || mhz == nullptr) return IG4_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  sm_clock_probe_kernel<<<1, 1, 0, st>>>(static_cast<unsigned long long>(window_us) * 1000ull);
+  IG4_TRY(last_launch_status());
+  unsigned long long v[2] = {0, 0};
+  if (cudaMemcpyFromSymbolAsync(v, g_clock_probe, sizeof(v), 0, cudaMemcpyDeviceToHost, st) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return IG4_ERR_CUDA;
+  if (v[1] == 0) return IG4_ERR_CUDA;
+  *mhz = 1e3 * static_cast<double>(v[0]) / static_cast<double>(v[1]);
   return IG4_OK;
 }
 

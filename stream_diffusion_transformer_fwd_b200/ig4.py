@@ -140,6 +140,7 @@ _sig("ig4_block_sp_post", [ctypes.POINTER(Config), _i, _i, ctypes.POINTER(BlockW
                            _vp, _vp, ctypes.c_size_t, _vp])
 _sig("ig4_last_device_error", [_vp])
 _sig("ig4_selftest_timeout", [_i, _vp])
+_sig("ig4_sm_clock_mhz", [_i, _vp, ctypes.POINTER(ctypes.c_double)])
 
 EXPORTED = ("ig4_status_string", "ig4_abi_version", "ig4_mrope_positions", "ig4_rope_table",
             "ig4_adaln_modulation", "ig4_norm_modulate", "ig4_qkv_project",
@@ -155,7 +156,7 @@ EXPORTED = ("ig4_status_string", "ig4_abi_version", "ig4_mrope_positions", "ig4_
             "ig4_block_tp_attention", "ig4_block_tp_mlp", "ig4_tp_reduce", "ig4_sp_image_range",
             "ig4_sp_positions", "ig4_sp_workspace_size", "ig4_sp_exchange_bytes",
             "ig4_block_sp_pre", "ig4_block_sp_attention", "ig4_block_sp_post",
-            "ig4_last_device_error", "ig4_selftest_timeout")
+            "ig4_last_device_error", "ig4_selftest_timeout", "ig4_sm_clock_mhz")
 
 
 def library():
@@ -496,6 +497,13 @@ def ig4_last_device_error(stream=None) -> int:
 
 def ig4_selftest_timeout(wait_us: int, stream=None):
     _check(_lib.ig4_selftest_timeout(wait_us, _stream(stream)), "ig4_selftest_timeout")
+
+
+def ig4_sm_clock_mhz(window_us: int = 20, stream=None) -> float:
+    """SM clock (MHz) read by a kernel queued on the stream (synchronises it)."""
+    v = ctypes.c_double(0.0)
+    _check(_lib.ig4_sm_clock_mhz(window_us, _stream(stream), ctypes.byref(v)), "ig4_sm_clock_mhz")
+    return v.value
 
 
 # ------------------------------------------------------- multi-GPU layouts

@@ -160,6 +160,10 @@ def test_op_validation_returns_before_launch(ig4):
     assert lib.ig4_joint_attention(1, 1, 10, p, p, p, 4, p, None) == ig4.IG4_ERR_INVALID_ARG
     assert lib.ig4_quantize_rows(4, 20000, p, p, p, None) == ig4.IG4_ERR_INVALID_ARG
     assert lib.ig4_selftest_timeout(0, None) == ig4.IG4_ERR_INVALID_ARG
+    mhz = ctypes.c_double(0.0)
+    assert lib.ig4_sm_clock_mhz(0, None, ctypes.byref(mhz)) == ig4.IG4_ERR_INVALID_ARG
+    assert lib.ig4_sm_clock_mhz(100001, None, ctypes.byref(mhz)) == ig4.IG4_ERR_INVALID_ARG
+    assert lib.ig4_sm_clock_mhz(20, None, None) == ig4.IG4_ERR_INVALID_ARG
     assert lib.ig4_adaln_modulation(9, 512, 8, p, p, 1, None, None, p, None) == \
         ig4.IG4_ERR_INVALID_ARG
 

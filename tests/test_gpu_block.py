@@ -246,6 +246,13 @@ def test_timeout_selftest_reports_and_context_survives(ig4):
     assert rel_l2(y.reshape(y_ref.shape), y_ref) <= 1e-2
 
 
+def test_sm_clock_probe_reads_a_plausible_clock(ig4):
+    """The clock probe's cycles / global-timer ratio lies between idle and
+    boost clocks of the part (a wrong unit would be off by 10^3)."""
+    mhz = [ig4.ig4_sm_clock_mhz(50) for _ in range(3)]
+    assert all(100.0 < m < 3500.0 for m in mhz), mhz
+
+
 def test_invalid_arguments_launch_nothing(ig4):
     cfg = CONFIGS["tiny"]
     c = ig4.config_from(cfg)
