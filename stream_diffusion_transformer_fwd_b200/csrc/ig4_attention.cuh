@@ -213,6 +213,16 @@ __device__ __forceinline__ void att_commit(uint64_t *bar) {
     umma_commit(bar);
 }
 
+// 32-byte global store (sm_100 and later; the address 32-byte aligned).  A
+// softmax thread writes its own output row, rows H * 512 bytes apart, so a
+// warp's store touches 32 lines: 32-byte pieces halve the store instructions
+// and write whole sectors.
+__device__ __forceinline__ void st_global_v8(void *p, const uint32_t (&w)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]),
+               "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+
 // Arrive on a barrier that the leader CTA holds (the CTA itself when single).
 template <bool PAIR>
 __device__ __forceinline__ void att_arrive_leader(uint64_t *bar) {
@@ -656,6 +666,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       const bool store = valid || sg.slot >= 0;
       // MX8 output (o_sf != nullptr): E4M3 codes in o_out's bytes, a scale per 32 dims
       const bool mx8 = o_sf != nullptr && sg.slot < 0;
+      // every row start and 32-column step is a multiple of 32 bytes from the
+      // base, so one test of the base covers all threads' stores
+      const bool a32 = ((reinterpret_cast<uintptr_t>(mx8 ? static_cast<void *>(o_out)
+                                                          : static_cast<void *>(dst)) &
+                         31) == 0);
       // O in two halves of 128 columns: four TMEM loads in flight per wait
 #pragma unroll 1
       for (int hc = 0; hc < ATT_DH; hc += 128) {
@@ -675,9 +690,28 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             const uint8_t sb = mx8_encode32(o[c], q);
             const int col = h * ATT_DH + hc + 32 * c;
             uint4 *d = reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(o_out) + grow * HD + col);
-            d[0] = q[0];
-            d[1] = q[1];
+            if (a32) {
+              const uint32_t w[8] = {q[0].x, q[0].y, q[0].z, q[0].w, q[1].x, q[1].y, q[1].z, q[1].w};
+              st_global_v8(d, w);
+            } else {
+              d[0] = q[0];
+              d[1] = q[1];
+            }
             o_sf[mx8_sf_offset(static_cast<int>(grow), col / MX8_BLOCK, HD)] = sb;
+          }
+          continue;
+        }
+        if (a32) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              uint32_t w[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                w[i] = pack_bf16x2(o[c][16 * q + 2 * i] * inv, o[c][16 * q + 2 * i + 1] * inv);
+              st_global_v8(dst + hc + 32 * c + 16 * q, w);
+            }
           }
           continue;
         }
