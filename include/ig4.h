@@ -180,8 +180,11 @@ ig4_status ig4_qkv_project(int B, int L, int D, int H, const void *h, int h_dtyp
  * Joint bidirectional attention over [text | image] (survey page: one
  * self-attention over the single sequence, no separate branches):
  * o[b, l, h*256 + d] = sum_m softmax_m(q[b,h,l] . k[b,h,m] / 16) v[b,h,m,d].
- * q, k bf16 [B][H][L][256]; vt bf16 [B][H][256][vt_ld]; o_out bf16 [B*L][H*256].
- * Errors: INVALID_ARG (NULL, L < 1, vt_ld < L or vt_ld % 8). */
+ * q, k bf16 [B][H][L][256]; vt bf16 [B][H][256][vt_ld]; o_out bf16 [B*L][H*256];
+ * all device, 16-byte aligned (an o_out 32-byte aligned is written with
+ * 32-byte stores, one otherwise 16-byte aligned with 16-byte stores: the same
+ * values).  Errors: INVALID_ARG (NULL, misaligned, L < 1, vt_ld < L or
+ * vt_ld % 8). */
 ig4_status ig4_joint_attention(int B, int H, int L, const void *q, const void *k,
                                const void *vt, int vt_ld, void *o_out, void *stream);
 

@@ -283,6 +283,35 @@ def test_joint_attention(ig4, B, H, L, qscale):
     assert np.max(np.abs(got - ref)) <= 2e-2 * np.max(np.abs(ref)) + 1e-3
 
 
+# an output only 16-byte aligned takes 16-byte stores instead of 32-byte
+# ones: the same values, bit for bit (with and without the workspace grid)
+@pytest.mark.parametrize("B,H,L,use_ws", [(1, 3, 300, True), (1, 2, 200, False),
+                                          (1, 18, 1152, True)])
+def test_joint_attention_output_16_byte_aligned(ig4, B, H, L, use_ws):
+    q = randn("gq", (B, H, L, 256)).cuda()
+    k = randn("gk", (B, H, L, 256)).cuda()
+    vt_ld = (L + 7) // 8 * 8
+    vt = torch.zeros((B, H, 256, vt_ld), dtype=torch.bfloat16)
+    vt[..., :L] = randn("gv", (B, H, L, 256)).transpose(2, 3)
+    vt = vt.cuda()
+    n = B * L * H * 256
+    o = torch.empty((B * L, H * 256), dtype=torch.bfloat16, device="cuda")
+    buf = torch.empty(n + 16, dtype=torch.bfloat16, device="cuda")
+    o16 = buf[8:8 + n].view(B * L, H * 256)
+    assert o.data_ptr() % 32 == 0 and o16.data_ptr() % 32 == 16
+    if use_ws:
+        ws = torch.empty(ig4.ig4_joint_attention_workspace_size(B, H, L), dtype=torch.uint8,
+                         device="cuda")
+        ig4.ig4_joint_attention_ws(B, H, L, q, k, vt, vt_ld, o, ws)
+        ig4.ig4_joint_attention_ws(B, H, L, q, k, vt, vt_ld, o16, ws)
+    else:
+        ig4.ig4_joint_attention(B, H, L, q, k, vt, vt_ld, o)
+        ig4.ig4_joint_attention(B, H, L, q, k, vt, vt_ld, o16)
+    torch.cuda.synchronize()
+    assert ig4.ig4_last_device_error() == ig4.IG4_OK
+    assert torch.equal(o, o16)
+
+
 # the balanced persistent grid: more (b, h, query tile) items than SMs, so
 # key-tile ranges split items between CTAs (partial O merged afterwards);
 # ragged tails; a single item spread over many CTAs; one item per CTA
