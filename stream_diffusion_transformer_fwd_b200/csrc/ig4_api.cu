@@ -860,7 +860,7 @@ ig4_status launch_nvf4_pair_maps(const CUtensorMap &ma, const CUtensorMap &mb,
   const int group_m = gemm_group_m(M, K / 2, 1);
   cudaLaunchConfig_t lc = {};
   lc.gridDim = dim3(2 * pairs);
-  lc.blockDim = dim3(GEMM_THREADS);
+  lc.blockDim = dim3(NVF4P_THREADS);
   lc.dynamicSmemBytes = NVF4P_SMEM_BYTES;
   lc.stream = st;
   cudaLaunchAttribute attr[2];

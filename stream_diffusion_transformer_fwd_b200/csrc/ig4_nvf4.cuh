@@ -316,31 +316,36 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 // read the B scales of every column); all loads complete on the leader's
 // barrier.  Per stage and CTA: 32 KB of codes + 6 KB of scales per 512 MMA
 // clocks at the FP4 rate, the same bytes per clock as the FP8 pair kernel.
-// TMEM: two 256-column accumulators that overlap in 64 columns, acc 0 at
-// [0, 256) and acc 1 at [192, 448), and one 48-column scale region at 448
-// (the scale blocks of k-block g are copied in after the MMAs of k-block
-// g - 1 were issued; tcgen05.cp and tcgen05.mma from one thread run in
-// issue order).  The epilogue of a tile drains the overlapped columns
-// first and releases them (ovl), so the next tile's MMAs start while it
-// converts the remaining 192 columns.
+// TMEM: two 256-column accumulators that overlap in 96 columns, acc 0 at
+// [0, 256) and acc 1 at [160, 416), and two 48-column scale regions at 416
+// and 464.  A copy warp moves each k-block's scale blocks into region g % 2
+// (twelve tcgen05.cp of 512 bytes; each holds its issuing thread for ~64
+// cycles, more than the k-block's 512 cycles of FP4 MMAs, so they stay off
+// the MMA thread) and signals the MMA thread through sf_ready; it refills a
+// region once the MMAs of k-block g - 2 that read it have completed (the
+// stage's empty barrier).  The epilogue of a tile drains the overlapped
+// columns first and releases them (ovl), so the next tile's MMAs start while
+// it converts the rest.
 // DUAL_B (SwiGLU gate/up): B rows of the tile's first 128 columns come from
 // tmB (gate) and of the last 128 from tmB2 (up), both at rows nt * 128, with
 // their scale blocks from tmSFB / tmSFB2 (one 128-row block each); otherwise
 // B rows nt * 256 + [0, 256) come from tmB and their two scale blocks from
 // tmSFB.
 constexpr int NVF4P_STAGES = 5;
+constexpr int NVF4P_THREADS = 224;  // epilogue warps 0-3, TMA 4, MMA 5, scale copies 6
 constexpr int NVF4P_A_BYTES = GEMM_BM * 128;
 constexpr int NVF4P_BH_BYTES = 128 * 128;
 constexpr int NVF4P_SFA_BYTES = 2048;
 constexpr int NVF4P_SFB_BYTES = 4096;
 constexpr int NVF4P_STAGE_BYTES = NVF4P_A_BYTES + NVF4P_BH_BYTES + NVF4P_SFA_BYTES + NVF4P_SFB_BYTES;
 constexpr int NVF4P_SMEM_BYTES = NVF4P_STAGES * NVF4P_STAGE_BYTES + 1024 + 256;
-constexpr uint32_t NVF4P_ACC1_COL = 192;
-constexpr uint32_t NVF4P_SF_COL = 448;
-static_assert(NVF4P_ACC1_COL + 256 <= NVF4P_SF_COL && NVF4P_SF_COL + 48 <= 512, "TMEM");
+constexpr uint32_t NVF4P_ACC1_COL = 160;
+constexpr int NVF4P_OVL = 256 - static_cast<int>(NVF4P_ACC1_COL);  // overlapped columns
+constexpr uint32_t NVF4P_SF_COL = 416;                             // two regions of 48
+static_assert(NVF4P_ACC1_COL + 256 <= NVF4P_SF_COL && NVF4P_SF_COL + 2 * 48 <= 512, "TMEM");
 
 template <bool DUAL_B, class Epi>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
+__global__ void __launch_bounds__(NVF4P_THREADS, 1)
     gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                           const __grid_constant__ CUtensorMap tmB2,
                           const __grid_constant__ CUtensorMap tmSFA,
@@ -361,7 +366,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   uint64_t *tempty = tfull + 2;            // [2]: accumulator drained
   uint64_t *ovl = tempty + 2;              // overlapped columns drained
   uint64_t *drain = ovl + 1;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  uint64_t *sf_ready = drain + 1;          // [2]: scale region copied
+  uint64_t *cdrain = sf_ready + 2;         // the copy warp's last copies done
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(cdrain + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -384,6 +391,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     mbar_init(ovl, 2 * 4);
     mbar_init(drain, 1);
+    mbar_init(&sf_ready[0], 1);
+    mbar_init(&sf_ready[1], 1);
+    mbar_init(cdrain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -452,7 +462,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
-      const uint32_t sf = tmem_base + NVF4P_SF_COL;
+      long g = 0;  // k-blocks over the tiles
       for (int t = pair, i = 0; t < n_tiles && ok; t += n_pairs, ++i) {
         const int acc = i & 1;
         // this accumulator's own columns: drained by the epilogue of tile i - 2;
@@ -462,20 +472,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         if (i > 0 && !mbar_wait_cluster(ovl, static_cast<uint32_t>((i - 1) & 1), abort_flag)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + (acc ? NVF4P_ACC1_COL : 0);
-        for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait_cluster(&full[s], ph, abort_flag)) {
+        for (int kb = 0; kb < kblocks; ++kb, ++g) {
+          if (!mbar_wait_cluster(&full[s], ph, abort_flag) ||
+              !mbar_wait_cluster(&sf_ready[g & 1], static_cast<uint32_t>((g >> 1) & 1),
+                                 abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sfa_s = smem_u32(sSFA + s * NVF4P_SFA_BYTES);
-          const uint32_t sfb_s = smem_u32(sSFB + s * NVF4P_SFB_BYTES);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            tmem_cp_sf_pair(sf + 4 * j, sdesc_kmajor_none(sfa_s + 512 * j, 128));
-            tmem_cp_sf_pair(sf + 16 + 8 * j, sdesc_kmajor_none(sfb_s + 512 * j, 128));
-            tmem_cp_sf_pair(sf + 16 + 8 * j + 4, sdesc_kmajor_none(sfb_s + 2048 + 512 * j, 128));
-          }
+          const uint32_t sf = tmem_base + NVF4P_SF_COL + 48 * static_cast<uint32_t>(g & 1);
           const uint32_t a_base = smem_u32(sA + s * NVF4P_A_BYTES);
           const uint32_t b_base = smem_u32(sB + s * NVF4P_BH_BYTES);
 #pragma unroll
@@ -495,13 +500,55 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       umma_commit_pair_both(drain);
       mbar_wait_cluster(drain, 0, nullptr, WAIT_LIMIT_NS / 4);
     }
+  } else if (warp == 6) {
+    if (lane == 0 && rank == 0) {
+      // ---------------- scale copies (leader CTA): stage data -> TMEM region g % 2
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      long g = 0;
+      for (int t = pair; t < n_tiles && ok; t += n_pairs) {
+        for (int kb = 0; kb < kblocks; ++kb, ++g) {
+          // the stage has landed; region g % 2 was last read by the MMAs of
+          // k-block g - 2, which completed the empty barrier of their stage
+          bool ready = mbar_wait_cluster(&full[s], ph, abort_flag);
+          if (ready && g >= 2) {
+            const long gp = g - 2;
+            ready = mbar_wait_cluster(&empty[gp % NVF4P_STAGES],
+                                      static_cast<uint32_t>((gp / NVF4P_STAGES) & 1), abort_flag);
+          }
+          if (!ready) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sf = tmem_base + NVF4P_SF_COL + 48 * static_cast<uint32_t>(g & 1);
+          const uint32_t sfa_s = smem_u32(sSFA + s * NVF4P_SFA_BYTES);
+          const uint32_t sfb_s = smem_u32(sSFB + s * NVF4P_SFB_BYTES);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            tmem_cp_sf_pair(sf + 4 * j, sdesc_kmajor_none(sfa_s + 512 * j, 128));
+            tmem_cp_sf_pair(sf + 16 + 8 * j, sdesc_kmajor_none(sfb_s + 512 * j, 128));
+            tmem_cp_sf_pair(sf + 16 + 8 * j + 4, sdesc_kmajor_none(sfb_s + 2048 + 512 * j, 128));
+          }
+          umma_commit_pair_both(&sf_ready[g & 1]);
+          if (++s == NVF4P_STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+      }
+      // no copy of this thread is in flight when TMEM is freed
+      umma_commit_pair_both(cdrain);
+      mbar_wait_cluster(cdrain, 0, nullptr, WAIT_LIMIT_NS / 4);
+    }
   } else {
     // ---------------- epilogue warps 0..3 (both CTAs, own 128 rows)
     const int r = warp * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     const uint32_t ovl_leader = map_shared_to_rank(ovl, 0);
-    constexpr int C = Epi::COLS;  // 64 accumulator columns overlap: the top 64 of
-    constexpr int OV = C - 64;    // acc 0's epilogue columns, the bottom 64 of acc 1's
+    constexpr int C = Epi::COLS;  // NVF4P_OVL accumulator columns overlap: the top ones
+    constexpr int OV = C - NVF4P_OVL;  // of acc 0's epilogue columns, the bottom ones of acc 1's
     for (int t = pair, i = 0; t < n_tiles; t += n_pairs, ++i) {
       const int acc = i & 1;
       const bool ok =
@@ -512,11 +559,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       tile_coords(t, m_tiles, n_tiles_n, group_m, &mt, &nt);
       const int m0 = mt * 2 * GEMM_BM + static_cast<int>(rank) * GEMM_BM;
       const uint32_t tacc = tmem_base + (acc ? NVF4P_ACC1_COL : 0) + lane_base;
-      epi.part(m0, nt * BN, tacc, r, acc ? 0 : OV, acc ? 64 : C);
+      epi.part(m0, nt * BN, tacc, r, acc ? 0 : OV, acc ? NVF4P_OVL : C);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(ovl_leader);
-      epi.part(m0, nt * BN, tacc, r, acc ? 64 : 0, acc ? C : OV);
+      epi.part(m0, nt * BN, tacc, r, acc ? NVF4P_OVL : 0, acc ? C : OV);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(map_shared_to_rank(&tempty[acc], 0));
