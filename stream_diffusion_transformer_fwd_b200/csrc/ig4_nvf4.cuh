@@ -318,12 +318,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 // clocks at the FP4 rate, the same bytes per clock as the FP8 pair kernel.
 // TMEM: two 256-column accumulators that overlap in 96 columns, acc 0 at
 // [0, 256) and acc 1 at [160, 416), and two 48-column scale regions at 416
-// and 464.  A copy warp moves each k-block's scale blocks into region g % 2
-// (twelve tcgen05.cp of 512 bytes; each holds its issuing thread for ~64
-// cycles, more than the k-block's 512 cycles of FP4 MMAs, so they stay off
-// the MMA thread) and signals the MMA thread through sf_ready; it refills a
-// region once the MMAs of k-block g - 2 that read it have completed (the
-// stage's empty barrier).  The epilogue of a tile drains the overlapped
+// and 464.  Two copy warps move each k-block's scale blocks into region g % 2
+// (twelve tcgen05.cp of 512 bytes, six per warp: each holds its issuing
+// thread for ~64 cycles, so twelve in one thread would outlast the k-block's
+// 512 cycles of FP4 MMAs) and signal the MMA thread through sf_ready (two
+// arrivals); a region is refilled once the MMAs of k-block g - 2 that read it
+// have completed (the stage's empty barrier).  The epilogue of a tile drains the overlapped
 // columns first and releases them (ovl), so the next tile's MMAs start while
 // it converts the rest.
 // DUAL_B (SwiGLU gate/up): B rows of the tile's first 128 columns come from
@@ -332,7 +332,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 // B rows nt * 256 + [0, 256) come from tmB and their two scale blocks from
 // tmSFB.
 constexpr int NVF4P_STAGES = 5;
-constexpr int NVF4P_THREADS = 224;  // epilogue warps 0-3, TMA 4, MMA 5, scale copies 6
+constexpr int NVF4P_THREADS = 256;  // epilogue warps 0-3, TMA 4, MMA 5, scale copies 6-7
 constexpr int NVF4P_A_BYTES = GEMM_BM * 128;
 constexpr int NVF4P_BH_BYTES = 128 * 128;
 constexpr int NVF4P_SFA_BYTES = 2048;
@@ -391,9 +391,9 @@ __global__ void __launch_bounds__(NVF4P_THREADS, 1)
     }
     mbar_init(ovl, 2 * 4);
     mbar_init(drain, 1);
-    mbar_init(&sf_ready[0], 1);
-    mbar_init(&sf_ready[1], 1);
-    mbar_init(cdrain, 1);
+    mbar_init(&sf_ready[0], 2);  // one commit per copy warp
+    mbar_init(&sf_ready[1], 2);
+    mbar_init(cdrain, 2);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -500,9 +500,11 @@ __global__ void __launch_bounds__(NVF4P_THREADS, 1)
       umma_commit_pair_both(drain);
       mbar_wait_cluster(drain, 0, nullptr, WAIT_LIMIT_NS / 4);
     }
-  } else if (warp == 6) {
+  } else if (warp == 6 || warp == 7) {
     if (lane == 0 && rank == 0) {
-      // ---------------- scale copies (leader CTA): stage data -> TMEM region g % 2
+      // ---------------- scale copies (leader CTA): stage data -> TMEM region g % 2,
+      // warp 6 the blocks of MMAs 0-1 of the k-block, warp 7 those of MMAs 2-3
+      const int j0 = 2 * (warp - 6);
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
@@ -526,7 +528,7 @@ __global__ void __launch_bounds__(NVF4P_THREADS, 1)
           const uint32_t sfa_s = smem_u32(sSFA + s * NVF4P_SFA_BYTES);
           const uint32_t sfb_s = smem_u32(sSFB + s * NVF4P_SFB_BYTES);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
+          for (int j = j0; j < j0 + 2; ++j) {
             tmem_cp_sf_pair(sf + 4 * j, sdesc_kmajor_none(sfa_s + 512 * j, 128));
             tmem_cp_sf_pair(sf + 16 + 8 * j, sdesc_kmajor_none(sfb_s + 512 * j, 128));
             tmem_cp_sf_pair(sf + 16 + 8 * j + 4, sdesc_kmajor_none(sfb_s + 2048 + 512 * j, 128));
