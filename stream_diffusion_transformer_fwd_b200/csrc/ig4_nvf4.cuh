@@ -318,11 +318,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 // clocks at the FP4 rate, the same bytes per clock as the FP8 pair kernel.
 // TMEM: two 256-column accumulators that overlap in 96 columns, acc 0 at
 // [0, 256) and acc 1 at [160, 416), and two 48-column scale regions at 416
-// and 464.  Two copy warps move each k-block's scale blocks into region g % 2
-// (twelve tcgen05.cp of 512 bytes, six per warp: each holds its issuing
-// thread for ~64 cycles, so twelve in one thread would outlast the k-block's
-// 512 cycles of FP4 MMAs) and signal the MMA thread through sf_ready (two
-// arrivals); a region is refilled once the MMAs of k-block g - 2 that read it
+// and 464.  Four copy warps move each k-block's scale blocks into region
+// g % 2 (twelve tcgen05.cp of 512 bytes, three per warp: a copy holds its
+// issuing thread for ~50 cycles, and copies from different threads run side
+// by side, so twelve in one thread would outlast the k-block's 512 cycles of
+// FP4 MMAs) and signal the MMA thread through sf_ready (one arrival per copy
+// warp); a region is refilled once the MMAs of k-block g - 2 that read it
 // have completed (the stage's empty barrier).  The epilogue of a tile drains the overlapped
 // columns first and releases them (ovl), so the next tile's MMAs start while
 // it converts the rest.
@@ -332,7 +333,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 // B rows nt * 256 + [0, 256) come from tmB and their two scale blocks from
 // tmSFB.
 constexpr int NVF4P_STAGES = 5;
-constexpr int NVF4P_THREADS = 256;  // epilogue warps 0-3, TMA 4, MMA 5, scale copies 6-7
+constexpr int NVF4P_COPY_WARPS = 4;  // one MMA's scale blocks (three copies) per warp
+constexpr int NVF4P_THREADS = 32 * (6 + NVF4P_COPY_WARPS);  // epilogue 0-3, TMA 4, MMA 5, copies
 constexpr int NVF4P_A_BYTES = GEMM_BM * 128;
 constexpr int NVF4P_BH_BYTES = 128 * 128;
 constexpr int NVF4P_SFA_BYTES = 2048;
@@ -343,6 +345,57 @@ constexpr uint32_t NVF4P_ACC1_COL = 160;
 constexpr int NVF4P_OVL = 256 - static_cast<int>(NVF4P_ACC1_COL);  // overlapped columns
 constexpr uint32_t NVF4P_SF_COL = 416;                             // two regions of 48
 static_assert(NVF4P_ACC1_COL + 256 <= NVF4P_SF_COL && NVF4P_SF_COL + 2 * 48 <= 512, "TMEM");
+
+// SwiGLU epilogue of a dual-B pair tile (EpiSwiGLU layout: gate in
+// accumulator columns [0, 128), up in [128, 256)).  The 96 columns shared
+// with the other accumulator (acc 0: up columns [160, 256); acc 1: gate
+// columns [0, 96)) are read into registers and released first, so the next
+// tile's MMAs wait for three TMEM loads rather than for 96 of the 128 output
+// columns; then the four 32-column chunks are converted.
+template <class Epi>
+__device__ __forceinline__ void nvf4_swiglu_epilogue(const Epi &ep, int m0, int n0, uint32_t tacc,
+                                                     int r, int acc, uint32_t ovl_leader,
+                                                     int lane) {
+  float ov[3][32];
+  const uint32_t obase = acc ? 0u : 160u;
+#pragma unroll
+  for (int k = 0; k < 3; ++k) tmem_ld32(tacc + obase + 32 * k, ov[k]);
+  tmem_ld_wait();
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive_cluster(ovl_leader);
+  const int row = m0 + r;
+  const bool valid = row < ep.M;
+  const float rs = valid ? __ldg(ep.a_scale + row) : 1.0f;
+  const int n = n0 / 2;  // tile index * 128
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    float g[32], up[32];
+    if (acc == 0) {  // up of chunks 1..3 preloaded
+      tmem_ld32(tacc + 32 * c, g);
+      if (c == 0) tmem_ld32(tacc + 128, up);
+      tmem_ld_wait();
+      if (c > 0) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) up[i] = ov[c > 0 ? c - 1 : 0][i];
+      }
+    } else {  // gate of chunks 0..2 preloaded
+      tmem_ld32(tacc + 128 + 32 * c, up);
+      if (c == 3) tmem_ld32(tacc + 96, g);
+      tmem_ld_wait();
+      if (c < 3) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) g[i] = ov[c < 3 ? c : 0][i];
+      }
+    }
+    if (!valid) continue;
+    apply_scales<true>(g, rs, ep.s_gate + n + 32 * c);
+    apply_scales<true>(up, rs, ep.s_up + n + 32 * c);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) g[i] = silu_f(g[i]) * up[i];
+    store32_bf16(ep.u + static_cast<long>(row) * ep.I + n + 32 * c, g);
+  }
+}
 
 template <bool DUAL_B, class Epi>
 __global__ void __launch_bounds__(NVF4P_THREADS, 1)
@@ -391,9 +444,9 @@ __global__ void __launch_bounds__(NVF4P_THREADS, 1)
     }
     mbar_init(ovl, 2 * 4);
     mbar_init(drain, 1);
-    mbar_init(&sf_ready[0], 2);  // one commit per copy warp
-    mbar_init(&sf_ready[1], 2);
-    mbar_init(cdrain, 2);
+    mbar_init(&sf_ready[0], NVF4P_COPY_WARPS);  // one commit per copy warp
+    mbar_init(&sf_ready[1], NVF4P_COPY_WARPS);
+    mbar_init(cdrain, NVF4P_COPY_WARPS);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -500,11 +553,11 @@ __global__ void __launch_bounds__(NVF4P_THREADS, 1)
       umma_commit_pair_both(drain);
       mbar_wait_cluster(drain, 0, nullptr, WAIT_LIMIT_NS / 4);
     }
-  } else if (warp == 6 || warp == 7) {
+  } else if (warp >= 6) {
     if (lane == 0 && rank == 0) {
       // ---------------- scale copies (leader CTA): stage data -> TMEM region g % 2,
-      // warp 6 the blocks of MMAs 0-1 of the k-block, warp 7 those of MMAs 2-3
-      const int j0 = 2 * (warp - 6);
+      // warp 6 + c the blocks of MMA j of the k-block for j % NVF4P_COPY_WARPS == c
+      const int j0 = warp - 6;
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
@@ -528,7 +581,7 @@ __global__ void __launch_bounds__(NVF4P_THREADS, 1)
           const uint32_t sfa_s = smem_u32(sSFA + s * NVF4P_SFA_BYTES);
           const uint32_t sfb_s = smem_u32(sSFB + s * NVF4P_SFB_BYTES);
 #pragma unroll
-          for (int j = j0; j < j0 + 2; ++j) {
+          for (int j = j0; j < 4; j += NVF4P_COPY_WARPS) {
             tmem_cp_sf_pair(sf + 4 * j, sdesc_kmajor_none(sfa_s + 512 * j, 128));
             tmem_cp_sf_pair(sf + 16 + 8 * j, sdesc_kmajor_none(sfb_s + 512 * j, 128));
             tmem_cp_sf_pair(sf + 16 + 8 * j + 4, sdesc_kmajor_none(sfb_s + 2048 + 512 * j, 128));
@@ -561,11 +614,15 @@ __global__ void __launch_bounds__(NVF4P_THREADS, 1)
       tile_coords(t, m_tiles, n_tiles_n, group_m, &mt, &nt);
       const int m0 = mt * 2 * GEMM_BM + static_cast<int>(rank) * GEMM_BM;
       const uint32_t tacc = tmem_base + (acc ? NVF4P_ACC1_COL : 0) + lane_base;
-      epi.part(m0, nt * BN, tacc, r, acc ? 0 : OV, acc ? NVF4P_OVL : C);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(ovl_leader);
-      epi.part(m0, nt * BN, tacc, r, acc ? NVF4P_OVL : 0, acc ? C : OV);
+      if constexpr (DUAL_B) {
+        nvf4_swiglu_epilogue(epi, m0, nt * BN, tacc, r, acc, ovl_leader, lane);
+      } else {
+        epi.part(m0, nt * BN, tacc, r, acc ? 0 : OV, acc ? NVF4P_OVL : C);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(ovl_leader);
+        epi.part(m0, nt * BN, tacc, r, acc ? NVF4P_OVL : 0, acc ? C : OV);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(map_shared_to_rank(&tempty[acc], 0));
