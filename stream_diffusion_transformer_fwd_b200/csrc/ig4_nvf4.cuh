@@ -324,9 +324,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 // by side, so twelve in one thread would outlast the k-block's 512 cycles of
 // FP4 MMAs) and signal the MMA thread through sf_ready (one arrival per copy
 // warp); a region is refilled once the MMAs of k-block g - 2 that read it
-// have completed (the stage's empty barrier).  The epilogue of a tile drains the overlapped
-// columns first and releases them (ovl), so the next tile's MMAs start while
-// it converts the rest.
+// have completed (the stage's empty barrier).  The epilogue of a tile drains
+// the overlapped columns first and releases them (ovl), so the next tile's
+// MMAs start while it converts the rest.
 // DUAL_B (SwiGLU gate/up): B rows of the tile's first 128 columns come from
 // tmB (gate) and of the last 128 from tmB2 (up), both at rows nt * 128, with
 // their scale blocks from tmSFB / tmSFB2 (one 128-row block each); otherwise
@@ -334,7 +334,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 // tmSFB.
 constexpr int NVF4P_STAGES = 5;
 constexpr int NVF4P_COPY_WARPS = 4;  // one MMA's scale blocks (three copies) per warp
-constexpr int NVF4P_THREADS = 32 * (6 + NVF4P_COPY_WARPS);  // epilogue 0-3, TMA 4, MMA 5, copies
+// Epilogue warps 0-3, TMA 4, MMA 5, copies 6-9.  Registers are allocated per
+// group of four warps, so ten warps are charged as twelve: 168 per thread.
+constexpr int NVF4P_THREADS = 32 * (6 + NVF4P_COPY_WARPS);
 constexpr int NVF4P_A_BYTES = GEMM_BM * 128;
 constexpr int NVF4P_BH_BYTES = 128 * 128;
 constexpr int NVF4P_SFA_BYTES = 2048;
@@ -420,7 +422,7 @@ __global__ void __launch_bounds__(NVF4P_THREADS, 1)
   uint64_t *ovl = tempty + 2;              // overlapped columns drained
   uint64_t *drain = ovl + 1;
   uint64_t *sf_ready = drain + 1;          // [2]: scale region copied
-  uint64_t *cdrain = sf_ready + 2;         // the copy warp's last copies done
+  uint64_t *cdrain = sf_ready + 2;         // the copy warps' last copies done
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(cdrain + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
